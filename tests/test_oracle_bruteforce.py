@@ -1,0 +1,73 @@
+"""The oracle's paged attention against a dense numpy brute force on tiny inputs.
+
+The brute force builds, per sequence, the full score matrix and a dense mask
+from NumKong's band rule ("Attention with a Pre-Packed KV-Cache": row r of q
+rows over k keys sits at r + k - q and sees keys_before keys before it and
+keys_after = 0 after), applies a masked softmax and returns zeros for rows with
+no visible key. The paged pools are built here from dense K/V with a shuffled
+page assignment, independently of the oracle.
+"""
+
+import numpy as np
+import pytest
+
+import oracle as O
+from test_oracle_pins import paged
+
+
+def dense_reference(q, k_dense, v_dense, q_lens, scale, window):
+    H = q.shape[1]
+    Hk = k_dense[0].shape[1]
+    G = H // Hk
+    out = np.zeros(q.shape, dtype=np.float64)
+    t0 = 0
+    for b, ql in enumerate(q_lens):
+        kl = k_dense[b].shape[0]
+        rows = np.arange(ql)[:, None]
+        keys = np.arange(kl)[None, :]
+        pos = rows + kl - ql
+        mask = keys <= pos
+        if window > 0:
+            mask &= keys >= pos - (window - 1)
+        for h in range(H):
+            qq = q[t0:t0 + ql, h].astype(np.float64)
+            kk = k_dense[b][:, h // G].astype(np.float64)
+            vv = v_dense[b][:, h // G].astype(np.float64)
+            s = scale * (qq @ kk.T)
+            s = np.where(mask, s, -np.inf)
+            m = s.max(axis=1, keepdims=True) if kl else np.full((ql, 1), -np.inf)
+            has = np.isfinite(m[:, 0])
+            w = np.zeros_like(s)
+            w[has] = np.exp(s[has] - m[has])
+            w[has] /= w[has].sum(axis=1, keepdims=True)
+            out[t0:t0 + ql, h] = w @ vv if kl else 0.0
+        t0 += ql
+    return out
+
+
+CASES = [
+    # (q_lens, kv_lens, H, Hk, d, page, window)
+    ([5, 11], [5, 11], 4, 2, 16, 4, 0),
+    ([1, 1, 1], [7, 1, 19], 4, 1, 8, 4, 0),
+    ([3, 8, 2], [10, 8, 20], 6, 3, 8, 3, 0),
+    ([6, 9], [6, 20], 2, 2, 8, 4, 4),
+    ([4, 1], [2, 3], 2, 1, 4, 2, 0),          # rows with no key
+    ([12], [12], 8, 2, 16, 5, 1),             # window 1: only itself
+    ([7, 0, 5], [7, 4, 15], 4, 4, 8, 4, 3),   # an empty sequence
+]
+
+
+@pytest.mark.parametrize("idx", range(len(CASES)))
+def test_oracle_matches_dense_bruteforce(idx):
+    q_lens, kv_lens, H, Hk, d, P, w = CASES[idx]
+    rng = np.random.default_rng(100 + idx)
+    k = [rng.normal(size=(n, Hk, d)).astype(np.float32) for n in kv_lens]
+    v = [rng.normal(size=(n, Hk, d)).astype(np.float32) for n in kv_lens]
+    T = sum(q_lens)
+    q = rng.normal(size=(T, H, d)).astype(np.float32)
+    kp, vp, bt = paged(k, v, page_size=P, seed=len(q_lens))
+    offs = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    scale = 1.0 / np.sqrt(d)
+    got = O.attention(q, offs, kv_lens, kp, vp, bt, Hk, scale, w, n_threads=2)
+    want = dense_reference(q, k, v, q_lens, scale, w)
+    assert np.max(np.abs(got - want)) < 1e-12

@@ -1,0 +1,54 @@
+"""Plant plausible mistakes in copies of the oracle and check the pins catch them.
+
+Each mutation is a one-line change to rpk_oracle.c (a flipped sign, a dropped
+term, a wrong index); the copy is compiled on the CPU into a temporary
+library and the pin and brute-force suites are run against it in a child
+process. Every mutation must make them fail.
+"""
+
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "rpk_oracle.c")
+
+MUTATIONS = {
+    "rotation_sign": ("out[base + i1] = a * c - bb * s;", "out[base + i1] = a * c + bb * s;"),
+    "pairing_swapped": ("int i1 = interleaved ? 2 * j : j;", "int i1 = interleaved ? j : 2 * j;"),
+    "frequency_exponent": ("pow(base, -2.0 * (double)j / (double)rotary_dim)",
+                           "pow(base, -(double)j / (double)rotary_dim)"),
+    "implicit_position": ("if (!position_ids) pos = cache_lens[b] + i;",
+                          "if (!position_ids) pos = i;"),
+    "mrope_section_edge": ("if (j < acc) return s;", "if (j <= acc) return s;"),
+    "scale_dropped": ("double s = J->scale * acc;", "double s = acc;"),
+    "gqa_mapping": ("int kvh = h / group;", "int kvh = h % J->n_kv_heads;"),
+    "window_off_by_one": ("int64_t l = window > 0 ? p - (window - 1) : 0;",
+                          "int64_t l = window > 0 ? p - window : 0;"),
+    "query_alignment": ("int64_t p = (int64_t)r + k_len - q_len;", "int64_t p = (int64_t)r;"),
+    "rounding_ties_away": ("double r = rint(a / ulp) * ulp;",
+                           "double r = floor(a / ulp + 0.5) * ulp;"),
+    "running_sum_not_rescaled": ("*l = *l * alpha + p;", "*l = *l + p;"),
+    "slot_row": ("int32_t row = slot % page_size;", "int32_t row = (slot + 1) % page_size;"),
+    "value_weight_unnormalised": ("double wj = w[j - lo] / den;", "double wj = w[j - lo];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_mutation(name, tmp_path):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not found once: {old!r}"
+    mutated = tmp_path / "rpk_oracle_mut.c"
+    mutated.write_text(src.replace(old, new))
+    so = tmp_path / "librpk_oracle_mut.so"
+    subprocess.run(["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-pthread", str(mutated),
+                    "-o", str(so), "-lm"], check=True)
+    env = dict(os.environ, RPK_ORACLE_LIB=str(so))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_bruteforce.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0, f"mutation {name} survived the pins:\n{r.stdout[-2000:]}"

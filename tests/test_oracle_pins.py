@@ -1,0 +1,530 @@
+"""The fp64 oracle against what the pages and the mathematics fix.
+
+Each test pins one part of the oracle to a value the pages print, a closed
+form, an invariant or a special case, so that a dropped term, a wrong sign or
+index, or a transposed operand fails one of them. No GPU is used.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+# ----------------------------------------------------------------- helpers
+
+
+def paged(k_dense, v_dense, page_size, seed=0, spare=3, dtype=np.float32):
+    """Scatter per-sequence dense K/V ([k_len, Hk, d] each) into a shuffled pool.
+
+    Written here, independently of the oracle, so that tests can compare the
+    oracle's paged reads with dense formulations.
+    """
+    rng = np.random.default_rng(seed)
+    n_pages = [(k.shape[0] + page_size - 1) // page_size for k in k_dense]
+    total = sum(n_pages) + spare
+    perm = rng.permutation(total)
+    Hk, d = k_dense[0].shape[1:]
+    kp = np.full((total, page_size, Hk, d), np.nan, dtype=dtype)
+    vp = np.full((total, page_size, Hk, d), np.nan, dtype=dtype)
+    bt = np.full((len(k_dense), max(1, max(n_pages))), -1, dtype=np.int32)
+    cur = 0
+    for b, (k, v) in enumerate(zip(k_dense, v_dense)):
+        for pg in range(n_pages[b]):
+            bt[b, pg] = perm[cur]
+            rows = k[pg * page_size:(pg + 1) * page_size]
+            kp[perm[cur], :rows.shape[0]] = rows
+            vp[perm[cur], :rows.shape[0]] = v[pg * page_size:(pg + 1) * page_size]
+            cur += 1
+    return kp, vp, bt
+
+
+def one_row_attention(q_vec, keys, values, scale, window=0):
+    """Attention of one query row (q_len = 1) over k_len keys, via the oracle."""
+    q = np.asarray(q_vec, dtype=np.float32)[None, None, :]
+    k = np.asarray(keys, dtype=np.float32)[:, None, :]
+    v = np.asarray(values, dtype=np.float32)[:, None, :]
+    kp, vp, bt = paged([k], [v], page_size=2)
+    out = O.attention(q, [0, 1], [k.shape[0]], kp, vp, bt, 1, scale, window)
+    return out[0, 0]
+
+
+def e(i, d, scale=1.0):
+    x = np.zeros(d, dtype=np.float32)
+    x[i] = scale
+    return x
+
+
+# --------------------------------------------------------- bf16 narrowing
+
+
+def test_bf16_matches_library_rounding_of_fp32_values():
+    # For values exactly representable in fp32, one rounding fp64 -> bf16 is the
+    # same as torch's fp32 -> bf16 (round to nearest, ties to even).
+    rng = np.random.default_rng(1)
+    bits = rng.integers(0, 2**32, size=200_000, dtype=np.uint64).astype(np.uint32)
+    f = bits.view(np.float32)
+    f = f[np.isfinite(f)]
+    # add exact ties: bf16 values plus half an ulp
+    base = (rng.integers(0, 2**16, size=20_000, dtype=np.uint32) << 16).astype(np.uint32)
+    ties = (base | 0x8000).view(np.float32)
+    f = np.concatenate([f, ties[np.isfinite(ties)]])
+    want = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = O.round_to(f.astype(np.float64), O.BF16)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("x,bits", [
+    (1.0 + 2**-8, 0x3F80),                 # tie -> even mantissa (1.0)
+    (1.0 + 3 * 2**-8, 0x3F82),             # tie -> even mantissa (1 + 2^-6)
+    (1.0 + 2**-8 + 2**-40, 0x3F81),        # just above the tie: one rounding goes up
+    (-(1.0 + 2**-8 + 2**-40), 0xBF81),
+    (2.0**-133, 0x0001),                   # smallest subnormal
+    (2.0**-134, 0x0000),                   # tie with zero -> even (zero)
+    (3 * 2.0**-134, 0x0002),               # tie between 1 and 2 units -> 2
+    (2.0**127 * (2 - 2**-7), 0x7F7F),      # largest finite
+    (2.0**127 * (2 - 2**-8), 0x7F80),      # tie above the largest finite -> inf
+    (2.0**127 * (2 - 2**-8) * (1 - 2**-40), 0x7F7F),
+    (-0.0, 0x8000),
+    (float("inf"), 0x7F80),
+    (float("-inf"), 0xFF80),
+])
+def test_bf16_rounding_cases(x, bits):
+    assert O.f64_to_bf16_bits(x) == bits
+
+
+def test_bf16_nan_and_widening():
+    assert O.f64_to_bf16_bits(float("nan")) & 0x7F80 == 0x7F80
+    assert O.f64_to_bf16_bits(float("nan")) & 0x007F != 0
+    assert O.bf16_bits_to_f64(0x3F80) == 1.0
+    assert O.bf16_bits_to_f64(0xC0A0) == -5.0
+    assert O.bf16_bits_to_f64(0x0001) == 2.0**-133
+
+
+# ------------------------------------------------- scores and softmax pins
+
+
+def test_scaled_score_worked_example(golden):
+    # q.k = 8 with d = 64 scores 1.0: against a key scoring 0 the weights are
+    # e/(1+e) and 1/(1+e).
+    g = golden["scaled_score"]
+    d = g["d_k"]
+    keys = [e(0, d), np.zeros(d, np.float32)]
+    out = one_row_attention(e(0, d, g["dot"]), keys, [e(0, d), e(1, d)], 1 / math.sqrt(d))
+    s = g["score"]
+    assert out[0] == pytest.approx(math.exp(s) / (math.exp(s) + 1.0), rel=1e-15)
+    assert out[1] == pytest.approx(1.0 / (math.exp(s) + 1.0), rel=1e-15)
+
+
+def test_cross_attention_score_worked_example(golden):
+    g = golden["cross_attention_score"]
+    d = g["d_k"]
+    out = one_row_attention(e(0, d, g["q"]), [e(0, d, g["k"]), np.zeros(d, np.float32)],
+                            [e(0, d), e(1, d)], 1 / math.sqrt(d))
+    s = g["score"]
+    assert out[0] == pytest.approx(math.exp(s) / (math.exp(s) + 1.0), rel=1e-15)
+
+
+def test_stable_softmax_worked_example(golden):
+    g = golden["stable_softmax"]
+    d = 4
+    keys = [e(0, d, s) for s in g["scores"]]
+    w = one_row_attention(e(0, d), keys, [e(i, d) for i in range(3)], 1.0)
+    assert w[0] == pytest.approx(g["weight0"], rel=1e-15)
+    # sum_exp = 1 / (weight of the max-score key)
+    assert 1.0 / w[2] == pytest.approx(g["sum_exp"], rel=1e-15)
+    assert w.sum() == pytest.approx(1.0, abs=1e-15)
+
+
+def test_two_pass_reproduces_online_worked_example(golden):
+    g = golden["online_softmax"]
+    d = 4
+    out = one_row_attention(e(0, d), [e(0, d, s) for s in g["scores"]],
+                            [e(0, d, v) for v in g["values"]], 1.0)
+    assert out[0] == pytest.approx(g["final"], rel=1e-15)
+    assert np.all(out[1:] == 0.0)
+
+
+def test_online_state_worked_example(golden):
+    # The printed o after key 1 is one fp64 ulp from the correctly rounded
+    # 10 + e^-1 * 20, hence the relative tolerance rather than equality.
+    g = golden["online_softmax"]
+    m, l, o = g["m0"], 0.0, 0.0
+    for s, v, want in zip(g["scores"], g["values"], g["steps"]):
+        m, l, o = O.flash_step(m, l, o, s, v)
+        assert m == want["m"]
+        assert l == pytest.approx(want["l"], rel=1e-15)
+        assert o == pytest.approx(want["o"], rel=5e-16)
+    assert o / l == pytest.approx(g["final"], rel=1e-15)
+
+
+def test_online_state_agrees_with_two_pass_random():
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        n = int(rng.integers(1, 40))
+        d = n
+        scores = rng.normal(0, 3, size=n).astype(np.float32)
+        vals = rng.normal(size=n).astype(np.float32)
+        m, l, o = -math.inf, 0.0, 0.0
+        for s, v in zip(scores, vals):
+            m, l, o = O.flash_step(m, l, o, float(s), float(v))
+        two = one_row_attention(e(0, d), [e(0, d, s) for s in scores],
+                                [e(0, d, v) for v in vals], 1.0)
+        assert o / l == pytest.approx(two[0], rel=1e-13, abs=1e-15)
+
+
+def test_weights_sum_to_one():
+    rng = np.random.default_rng(4)
+    d, n = 32, 20
+    q = rng.normal(size=d).astype(np.float32)
+    keys = rng.normal(size=(n, d)).astype(np.float32)
+    w = one_row_attention(q, keys, [e(i, d) for i in range(n)], 0.3)
+    assert w[:n].sum() == pytest.approx(1.0, abs=1e-14)
+    assert np.all(w[:n] > 0)
+
+
+# ------------------------------------------------------------- the band
+
+
+def test_causal_mask_worked_example(golden):
+    # q_len = k_len = 6 prefill: row r sits at position r.
+    for qpos, kpos in golden["causal_mask"]["attend"]:
+        lo, hi = O.band(qpos, 6, 6, 0)
+        assert lo <= kpos <= hi
+    for qpos, kpos in golden["causal_mask"]["masked"]:
+        lo, hi = O.band(qpos, 6, 6, 0)
+        assert not (lo <= kpos <= hi)
+
+
+def test_causal_mask_functional():
+    # Changing value 5 leaves row 3 bit-identical; changing value 3 moves row 5.
+    rng = np.random.default_rng(5)
+    d, L = 16, 6
+    q = rng.normal(size=(L, 1, d)).astype(np.float32)
+    k = rng.normal(size=(L, 1, d)).astype(np.float32)
+    v = rng.normal(size=(L, 1, d)).astype(np.float32)
+
+    def run(vv):
+        kp, vp, bt = paged([k], [vv], page_size=4)
+        return O.attention(q, [0, L], [L], kp, vp, bt, 1, 0.25, 0)
+
+    base = run(v)
+    v5 = v.copy(); v5[5] += 1.0
+    v3 = v.copy(); v3[3] += 1.0
+    assert np.array_equal(run(v5)[3], base[3])
+    assert not np.array_equal(run(v3)[5], base[5])
+
+
+def test_band_alignment_and_window():
+    # decode: one row over k keys sits at position k - 1
+    assert O.band(0, 1, 10, 0) == (0, 9)
+    # window w: w keys including the row's own
+    assert O.band(0, 1, 10, 4) == (6, 9)
+    # chunked prefill: 3 new rows appended to 7 cached keys
+    assert O.band(0, 3, 10, 0) == (0, 7)
+    assert O.band(2, 3, 10, 0) == (0, 9)
+    # more rows than keys: early rows see nothing
+    lo, hi = O.band(0, 4, 2, 0)
+    assert hi < lo
+
+
+def test_single_visible_key_returns_its_value():
+    rng = np.random.default_rng(6)
+    d, L = 8, 9
+    q = rng.normal(size=(L, 2, d)).astype(np.float32)
+    k = rng.normal(size=(L, 1, d)).astype(np.float32)
+    v = rng.normal(size=(L, 1, d)).astype(np.float32)
+    kp, vp, bt = paged([k], [v], page_size=4)
+    out = O.attention(q, [0, L], [L], kp, vp, bt, 1, 0.5, window=1)
+    for r in range(L):
+        for h in range(2):
+            assert np.array_equal(out[r, h], v[r, 0].astype(np.float64))
+
+
+def test_rows_without_keys_are_zero():
+    rng = np.random.default_rng(7)
+    d = 8
+    q = rng.normal(size=(4, 1, d)).astype(np.float32)
+    k = rng.normal(size=(2, 1, d)).astype(np.float32)
+    v = rng.normal(size=(2, 1, d)).astype(np.float32)
+    kp, vp, bt = paged([k], [v], page_size=4)
+    out = O.attention(q, [0, 4], [2], kp, vp, bt, 1, 0.5, 0)
+    assert np.all(out[0] == 0.0) and np.all(out[1] == 0.0)
+    assert np.array_equal(out[2, 0], v[0, 0].astype(np.float64))   # sees key 0 only
+    assert not np.all(out[3] == 0.0)
+
+
+def test_decode_equals_last_prefill_row():
+    rng = np.random.default_rng(8)
+    d, L, H, Hk = 16, 13, 4, 2
+    q = rng.normal(size=(L, H, d)).astype(np.float32)
+    k = rng.normal(size=(L, Hk, d)).astype(np.float32)
+    v = rng.normal(size=(L, Hk, d)).astype(np.float32)
+    kp, vp, bt = paged([k], [v], page_size=4)
+    for w in (0, 5):
+        full = O.attention(q, [0, L], [L], kp, vp, bt, Hk, 0.3, w)
+        dec = O.attention(q[L - 1:], [0, 1], [L], kp, vp, bt, Hk, 0.3, w)
+        assert np.array_equal(full[L - 1], dec[0])
+
+
+def test_gqa_head_mapping(golden):
+    g = golden["gqa_group"]
+    H, Hk = g["n_heads"], g["n_kv_heads"]
+    assert H // Hk == g["group"]
+    rng = np.random.default_rng(9)
+    d, L = 8, 5
+    q = rng.normal(size=(L, H, d)).astype(np.float32)
+    k = rng.normal(size=(L, Hk, d)).astype(np.float32)
+    v = rng.normal(size=(L, Hk, d)).astype(np.float32)
+    kp, vp, bt = paged([k], [v], page_size=4)
+    gqa = O.attention(q, [0, L], [L], kp, vp, bt, Hk, 0.4, 0)
+    # multi-head attention with each KV head repeated group times
+    kr = np.repeat(k, g["group"], axis=1)
+    vr = np.repeat(v, g["group"], axis=1)
+    kp2, vp2, bt2 = paged([kr], [vr], page_size=4)
+    mha = O.attention(q, [0, L], [L], kp2, vp2, bt2, H, 0.4, 0)
+    assert np.array_equal(gqa, mha)
+    # query head 5 reads KV head 1 (5 // 4)
+    assert np.array_equal(gqa[:, 5], O.attention(
+        q[:, 5:6], [0, L], [L], *paged([k[:, 1:2]], [v[:, 1:2]], page_size=4), 1, 0.4, 0)[:, 0])
+
+
+def test_attention_selected_rows_match_all_rows():
+    rng = np.random.default_rng(10)
+    d, H, Hk = 8, 4, 2
+    lens = [3, 7]
+    k = [rng.normal(size=(n, Hk, d)).astype(np.float32) for n in lens]
+    v = [rng.normal(size=(n, Hk, d)).astype(np.float32) for n in lens]
+    kp, vp, bt = paged(k, v, page_size=4)
+    q = rng.normal(size=(sum(lens), H, d)).astype(np.float32)
+    full = O.attention(q, [0, 3, 10], lens, kp, vp, bt, Hk, 0.3, 0)
+    rows = np.array([[9, 3], [0, 0], [4, 2]])
+    part = O.attention(q, [0, 3, 10], lens, kp, vp, bt, Hk, 0.3, 0, rows=rows)
+    for i, (t, h) in enumerate(rows):
+        assert np.array_equal(part[i], full[t, h])
+
+
+def test_kv_bytes_formula(golden):
+    from ragged_paged_kv_rope_b200 import metrics
+    g = golden["kv_cache_bytes"]
+    assert metrics.kv_cache_bytes(g["layers"], g["heads"], g["head_dim"], g["seq_len"],
+                                  g["batch"], g["bytes_per_elt"]) == g["bytes"]
+
+
+# ------------------------------------------------------------ RoPE table
+
+
+def test_table_pair0_is_position_in_radians(golden):
+    g = golden["sin_position_1"]
+    t = O.freqs_cis(50, 128, 500000.0)
+    assert t[g["position"], 1] == np.float32(g["value"])
+    for p in range(50):
+        assert t[p, 0] == np.float32(math.cos(p)) and t[p, 1] == np.float32(math.sin(p))
+
+
+def test_table_position0_and_known_frequency():
+    R, base = 128, 10000.0
+    t = O.freqs_cis(201, R, base)
+    assert np.all(t[0, 0::2] == 1.0) and np.all(t[0, 1::2] == 0.0)
+    # pair j = R/4 has frequency base^(-1/2) = 0.01: at position 100 the angle is 1
+    j = R // 4
+    assert abs(float(t[100, 2 * j]) - math.cos(1.0)) <= 2 * 2**-24
+    assert abs(float(t[100, 2 * j + 1]) - math.sin(1.0)) <= 2 * 2**-24
+    # the last pair of R = 2 has frequency 1 as well
+    t2 = O.freqs_cis(5, 2, base)
+    assert t2[3, 1] == np.float32(math.sin(3.0))
+    # cos^2 + sin^2 = 1 up to fp32 rounding of both entries
+    c, s = t[:, 0::2].astype(np.float64), t[:, 1::2].astype(np.float64)
+    assert np.max(np.abs(c * c + s * s - 1.0)) < 4 * 2**-24
+
+
+def test_table_frequencies_decrease_geometrically():
+    # ratio of the angles of consecutive pairs is base^(-2/R) everywhere
+    R, base, p = 64, 10000.0, 3
+    t = O.freqs_cis(p + 1, R, base)
+    ang = np.arctan2(t[p, 1::2].astype(np.float64), t[p, 0::2].astype(np.float64))
+    ratio = base ** (-2.0 / R)
+    for j in range(1, R // 2):
+        assert ang[j] / ang[j - 1] == pytest.approx(ratio, rel=1e-5)
+
+
+# ------------------------------------------------------------------ RoPE
+
+
+def _rope(x, offs, cache_lens, table, interleaved, R, pos=None, mrope=None):
+    return O.rope(x, offs, cache_lens, pos, mrope, table, interleaved, R)
+
+
+def test_rope_position0_is_identity():
+    rng = np.random.default_rng(11)
+    x = torch.from_numpy(rng.normal(size=(5, 3, 64)).astype(np.float32)).to(torch.bfloat16)
+    tab = O.freqs_cis(4, 64, 10000.0)
+    for il in (False, True):
+        out = _rope(x, [0, 5], [0], tab, il, 64, pos=np.zeros(5, np.int32))
+        assert np.array_equal(out, O.widen(x))
+
+
+def test_rope_rotation_sign_on_unit_pair():
+    # (1, 0) at position p becomes (cos theta, sin theta): multiplication by e^{i theta}
+    d = R = 8
+    tab = O.freqs_cis(10, R, 100.0)
+    x = np.zeros((1, 1, d), np.float32)
+    x[0, 0, 0] = 1.0
+    out = _rope(x, [0, 1], [7], tab, False, R)
+    assert out[0, 0, 0] == tab[7, 0] and out[0, 0, R // 2] == tab[7, 1]
+    out = _rope(x, [0, 1], [7], tab, True, R)
+    assert out[0, 0, 0] == tab[7, 0] and out[0, 0, 1] == tab[7, 1]
+    # pair j of the half layout is (x[j], x[j + R/2])
+    x = np.zeros((1, 1, d), np.float32)
+    x[0, 0, 3 + R // 2] = 1.0       # second member of pair 3
+    out = _rope(x, [0, 1], [7], tab, False, R)
+    assert out[0, 0, 3] == -tab[7, 7] and out[0, 0, 3 + R // 2] == tab[7, 6]
+
+
+def test_rope_preserves_pair_norms():
+    rng = np.random.default_rng(12)
+    d, R = 128, 128
+    x = rng.normal(size=(20, 4, d)).astype(np.float32)
+    tab = O.freqs_cis(400, R, 500000.0)
+    pos = rng.integers(0, 400, size=20).astype(np.int32)
+    for il in (False, True):
+        out = _rope(x, [0, 20], [0], tab, il, R, pos=pos)
+        xd = x.astype(np.float64)
+        if il:
+            n_in = xd[..., 0::2] ** 2 + xd[..., 1::2] ** 2
+            n_out = out[..., 0::2] ** 2 + out[..., 1::2] ** 2
+        else:
+            n_in = xd[..., :R // 2] ** 2 + xd[..., R // 2:] ** 2
+            n_out = out[..., :R // 2] ** 2 + out[..., R // 2:] ** 2
+        # |(a,b)|^2 (c^2 + s^2): the fp32 table entries give c^2 + s^2 = 1 +- 2^-22
+        assert np.max(np.abs(n_out / n_in - 1.0)) < 4 * 2**-24
+
+
+def test_rope_half_and_interleaved_agree_under_pair_permutation():
+    rng = np.random.default_rng(13)
+    d, R = 64, 48
+    x = rng.normal(size=(6, 2, d)).astype(np.float32)
+    tab = O.freqs_cis(30, R, 10000.0)
+    pos = rng.integers(0, 30, size=6).astype(np.int32)
+    half = R // 2
+    # interleaved channel 2j <- half channel j, 2j+1 <- j + R/2; the rest as is
+    perm = np.arange(d)
+    perm[0:R:2] = np.arange(half)
+    perm[1:R:2] = np.arange(half, R)
+    x_il = x[..., perm]
+    out_half = _rope(x, [0, 6], [0], tab, False, R, pos=pos)
+    out_il = _rope(x_il, [0, 6], [0], tab, True, R, pos=pos)
+    assert np.array_equal(out_il, out_half[..., perm])
+
+
+def test_partial_rope_passes_tail_channels():
+    rng = np.random.default_rng(14)
+    d, R = 256, 128
+    x = torch.from_numpy(rng.normal(size=(4, 3, d)).astype(np.float32)).to(torch.bfloat16)
+    tab = O.freqs_cis(100, R, 10000.0)
+    for il in (False, True):
+        out = _rope(x, [0, 4], [50], tab, il, R)
+        assert np.array_equal(out[..., R:], O.widen(x)[..., R:])
+        assert not np.array_equal(out[..., :R], O.widen(x)[..., :R])
+
+
+def test_rope_composes_by_position():
+    # rotating by a then by b equals rotating by a + b (angle linear in position)
+    rng = np.random.default_rng(15)
+    d = R = 32
+    x = rng.normal(size=(3, 2, d)).astype(np.float32)
+    tab = O.freqs_cis(64, R, 10000.0)
+    a = np.array([3, 10, 0], np.int32)
+    b = np.array([5, 20, 7], np.int32)
+    once = _rope(x, [0, 3], [0], tab, False, R, pos=a)
+    twice = _rope(once.astype(np.float32), [0, 3], [0], tab, False, R, pos=b)
+    direct = _rope(x, [0, 3], [0], tab, False, R, pos=a + b)
+    assert np.max(np.abs(twice - direct)) < 1e-5
+
+
+def test_rope_implicit_positions_from_cache_lens():
+    rng = np.random.default_rng(16)
+    d = R = 16
+    x = rng.normal(size=(7, 2, d)).astype(np.float32)
+    tab = O.freqs_cis(64, R, 10000.0)
+    offs, cl = [0, 3, 7], [10, 20]
+    implicit = _rope(x, offs, cl, tab, False, R)
+    explicit = _rope(x, offs, None, tab, False, R,
+                     pos=np.array([10, 11, 12, 20, 21, 22, 23], np.int32))
+    assert np.array_equal(implicit, explicit)
+
+
+def test_mrope_sections():
+    rng = np.random.default_rng(17)
+    d = R = 128
+    sec = (16, 24, 24)
+    x = rng.normal(size=(5, 2, d)).astype(np.float32)
+    tab = O.freqs_cis(100, R, 10000.0)
+    p = rng.integers(0, 100, size=5).astype(np.int32)
+    same = np.stack([p, p, p])
+    plain = _rope(x, [0, 5], None, tab, False, R, pos=p)
+    m = _rope(x, [0, 5], None, tab, False, R, pos=same, mrope=sec)
+    assert np.array_equal(m, plain)
+    # only section 1 (pairs 16..39) moves when only its positions change
+    moved = same.copy()
+    moved[1] = (p + 9) % 100
+    m2 = _rope(x, [0, 5], None, tab, False, R, pos=moved, mrope=sec)
+    changed = np.any(m2 != m, axis=(0, 1))
+    pairs = np.zeros(d, bool)
+    pairs[16:40] = True
+    pairs[64 + 16:64 + 40] = True
+    assert np.array_equal(changed, pairs)
+    # the section's rotation is the plain rotation at the section's positions
+    plain_moved = _rope(x, [0, 5], None, tab, False, R, pos=moved[1])
+    assert np.array_equal(m2[..., pairs], plain_moved[..., pairs])
+
+
+def test_rope_rejects_out_of_range_position():
+    tab = O.freqs_cis(4, 8, 10000.0)
+    x = np.zeros((1, 1, 8), np.float32)
+    with pytest.raises(ValueError):
+        _rope(x, [0, 1], [4], tab, False, 8)
+
+
+# ----------------------------------------------------------- cache image
+
+
+def test_cache_image_hand_example():
+    # one sequence, page size 2, pages [3, 1, 0], one cached token, two new:
+    # slot 1 -> page 3 row 1, slot 2 -> page 1 row 0
+    Hk, d = 1, 2
+    kp = np.full((4, 2, Hk, d), -7.0, np.float32)
+    vp = np.full((4, 2, Hk, d), -9.0, np.float32)
+    k_rot = np.array([[[1.25, 2.5]], [[3.0, 4.0]]], np.float64)
+    v_new = np.array([[[5.0, 6.0]], [[7.0, 8.0]]], np.float32)
+    k2, v2 = O.cache_image(k_rot, v_new, [0, 2], [1], np.array([[3, 1, 0]]), kp, vp)
+    want_k = kp.copy(); want_v = vp.copy()
+    want_k[3, 1, 0] = [1.25, 2.5]; want_v[3, 1, 0] = [5.0, 6.0]
+    want_k[1, 0, 0] = [3.0, 4.0]; want_v[1, 0, 0] = [7.0, 8.0]
+    assert np.array_equal(k2, want_k) and np.array_equal(v2, want_v)
+
+
+def test_cache_image_logical_order_invariant():
+    from ragged_paged_kv_rope_b200 import workloads as W
+    wl = W.make("mixed_chunked_mrope", seed=2, batch=4, n_heads=4, n_kv_heads=2,
+                head_dim=16, rotary_dim=16, new_tokens=("uniform", 1, 9),
+                cache_tokens=("uniform", 0, 20), page_size=4, mrope_section=(2, 3, 3))
+    k_rot = O.widen(wl.k_new)
+    kp, vp = O.cache_image(k_rot, wl.v_new, wl.q_offsets, wl.cache_lens, wl.block_table,
+                           wl.k_pages, wl.v_pages)
+    kp0 = wl.k_pages.view(torch.int16).numpy()
+    kp_new = kp.view(np.int16)
+    P = 4
+    touched = np.zeros(kp0.shape[:2], bool)
+    for b in range(4):
+        for i in range(int(wl.q_lens[b])):
+            slot = int(wl.cache_lens[b]) + i
+            page = wl.block_table[b, slot // P]
+            touched[page, slot % P] = True
+            t = int(wl.q_offsets[b]) + i
+            assert np.array_equal(vp[page, slot % P], wl.v_new[t].view(torch.int16).numpy().view(np.uint16))
+            assert np.array_equal(kp[page, slot % P], O.round_to(k_rot[t], O.BF16))
+    assert touched.sum() == wl.total_tokens
+    assert np.array_equal(kp_new[~touched], kp0[~touched])
