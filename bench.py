@@ -1,0 +1,473 @@
+"""Benchmark of the fused RoPE + paged-KV + ragged-attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rpk|reference]
+                    [--workload NAME] [--no-prefill] [--no-cpu-baseline]
+
+One step is one pass of the whole path over one batch: rope_qk_paged_ragged
+for the batch's new tokens (RoPE on Q and K, K/V written into the paged
+cache) followed by ragged_paged_attention over the cache. The default
+workload is the Llama-3-8B-shaped decode batch (64 sequences, 1 new token
+each, cached contexts U[512, 8192], 32 q / 8 kv heads, d 128, page 64); its
+metric is the K/V bytes attention reads per second. Every run also measures
+the ragged causal prefill workload (16 sequences of U[128, 4096] tokens) in
+TFLOP/s of visible (query, key) pairs, reported under "prefill".
+
+Under torchrun each rank runs its own batch (a different seed): sequences are
+independent, so the path shards with no exchange (weak scaling); the time is
+the max over ranks.
+
+Prints exactly one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import ragged_paged_kv_rope_b200 as R  # noqa: E402
+from ragged_paged_kv_rope_b200 import metrics as M  # noqa: E402
+from ragged_paged_kv_rope_b200 import workloads as W  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="rpk", choices=["rpk", "reference"])
+    ap.add_argument("--workload", default="llama3_8b_decode", choices=sorted(W.SPECS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- plumbing
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": float(pk["hbm_gbs"]), "bf16_tflops": float(pk["bf16_tflops"]),
+                "bf16_tflops_sustained": float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def load_traffic(kernel: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if the
+    kernel's source is unchanged since the capture (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            table = json.load(f)
+        ent = table[kernel]
+        src = os.path.join(ROOT, "ragged_paged_kv_rope_b200", "csrc", ent["source"])
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        if digest != ent["sha256"]:
+            return None
+        return ent
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------- the GPU path
+
+class Step:
+    """Device-resident inputs of one workload and the two C-ABI calls of a step."""
+
+    def __init__(self, wl: W.Workload, device):
+        sp = wl.spec
+        self.wl, self.sp = wl, sp
+        i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+        self.q = wl.q.to(device)
+        self.k_new = wl.k_new.to(device)
+        self.v_new = wl.v_new.to(device)
+        self.offsets = i32(wl.q_offsets)
+        self.kv_lens = i32(wl.kv_lens)
+        self.position_ids = None if wl.position_ids is None else i32(wl.position_ids)
+        self.error_word = torch.zeros(1, dtype=torch.int32, device=device)
+        self.cache = R.PagedKVCache(wl.k_pages.to(device), wl.v_pages.to(device),
+                                    i32(wl.block_table), i32(wl.cache_lens), self.error_word)
+        self.table = R.freqs_cis(wl.max_position, sp.rotary_dim, sp.theta, device=device)
+        self.q_rot = torch.empty_like(self.q)
+        self.out = torch.empty_like(self.q)
+        n = R.ragged_paged_attention_workspace_size(wl.total_tokens, sp.n_heads, sp.head_dim,
+                                                    sp.batch, wl.max_kv_len, sp.page_size)
+        self.workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+    def rope(self, stream=None):
+        sp = self.sp
+        R.rope_qk_paged_ragged(self.q, self.offsets, self.k_new, self.v_new, self.cache,
+                               self.table, self.position_ids, sp.interleaved, sp.rotary_dim,
+                               self.q_rot, mrope_section=sp.mrope_section, stream=stream)
+
+    def attention(self, stream=None):
+        sp, wl = self.sp, self.wl
+        R.ragged_paged_attention(self.q_rot, self.offsets, self.kv_lens, self.cache, sp.n_heads,
+                                 sp.n_kv_heads, sp.head_dim, sp.softmax_scale, sp.window,
+                                 self.out, max_q_len=wl.max_q_len, max_kv_len=wl.max_kv_len,
+                                 workspace=self.workspace, stream=stream)
+
+    def launches_per_step(self) -> int:
+        """Kernels of this library launched per step: RoPE, then attention
+        (the decode path adds a combine kernel when a sequence can span
+        several 512-key splits)."""
+        sp, wl = self.sp, self.wl
+        decode = wl.max_q_len * (sp.n_heads // sp.n_kv_heads) <= 16 and sp.dtype == "bf16"
+        if decode:
+            max_tiles = (wl.max_kv_len + 63) // 64 + 1
+            tps = max(8, (max_tiles + 63) // 64)
+            return 2 + (1 if (max_tiles + tps - 1) // tps > 1 else 0)
+        return 2
+
+
+def time_steps(step: Step, steps: int, warmup: int, world: int):
+    """Per-step device times of the rope call and the attention call (ms)."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        step.rope()
+        step.attention()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        step.rope()
+        ev[i][1].record(stream)
+        step.attention()
+        ev[i][2].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = start.elapsed_time(end)
+    rope_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    return total_ms, rope_ms, attn_ms
+
+
+def time_e2e(step: Step, steps: int, warmup: int, world: int):
+    """Same step through the public API with host inputs: pinned host -> device
+    copies of the step's inputs, the two calls, device -> host copy of the
+    output, all inside the timed region."""
+    wl = step.wl
+    host = {
+        "q": wl.q.pin_memory(), "k_new": wl.k_new.pin_memory(), "v_new": wl.v_new.pin_memory(),
+        "offsets": torch.from_numpy(wl.q_offsets).pin_memory(),
+        "kv_lens": torch.from_numpy(wl.kv_lens).pin_memory(),
+        "cache_lens": torch.from_numpy(wl.cache_lens).pin_memory(),
+        "block_table": torch.from_numpy(wl.block_table).pin_memory(),
+    }
+    if wl.position_ids is not None:
+        host["position_ids"] = torch.from_numpy(wl.position_ids).pin_memory()
+    out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    dst = {"q": step.q, "k_new": step.k_new, "v_new": step.v_new, "offsets": step.offsets,
+           "kv_lens": step.kv_lens, "cache_lens": step.cache.cache_lens,
+           "block_table": step.cache.block_table}
+    if step.position_ids is not None:
+        dst["position_ids"] = step.position_ids
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    stream = torch.cuda.current_stream()
+
+    def one():
+        for k, t in host.items():
+            dst[k].copy_(t, non_blocking=True)
+        step.rope()
+        step.attention()
+        out_host.copy_(step.out, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return a.elapsed_time(b) / steps, h2d, d2h
+
+
+def prefill_measure(device, world, steps=5, warmup=3):
+    wl = W.make("ragged_prefill", seed=0)
+    step = Step(wl, device)
+    total, rope_ms, attn_ms = time_steps(step, steps, warmup, world)
+    sp = wl.spec
+    flops = M.attention_flops(wl.q_lens, wl.kv_lens, sp.window, sp.n_heads, sp.head_dim)
+    attn = max_over_ranks(statistics.mean(attn_ms), world)
+    peaks = load_peaks()
+    tflops = flops / (attn * 1e-3) / 1e12
+    rope_b = M.rope_bytes(wl.total_tokens, sp.n_heads, sp.n_kv_heads, sp.head_dim,
+                          sp.rotary_dim, 2)
+    rope = max_over_ranks(statistics.mean(rope_ms), world)
+    return {
+        "workload": "ragged_prefill", "total_tokens": wl.total_tokens,
+        "attention_tflops": tflops, "tensor_peak_tflops": peaks["bf16_tflops"],
+        "frac": tflops / peaks["bf16_tflops"], "attention_ms": attn,
+        "visible_pair_flops": flops, "rope_ms": rope,
+        "rope_gbs": rope_b / (rope * 1e-3) / 1e9,
+        "tokens_per_s": world * wl.total_tokens / (max_over_ranks(total / steps, world) * 1e-3),
+        "error_word": int(step.error_word.item()),
+    }
+
+
+# -------------------------------------------------------- the oracle on CPU
+
+def oracle_sample_time(wl: W.Workload, max_seconds: float = 20.0):
+    """Time the fp64 oracle (RoPE, cache image, attention) on a bounded sample
+    of the workload's sequences; returns (seconds, kv_bytes, tokens, sample)."""
+    import oracle as O
+    sp = wl.spec
+    table = O.freqs_cis(wl.max_position, sp.rotary_dim, sp.theta)
+    kp, code = O.oracle._raw(wl.k_pages)
+    vp, _ = O.oracle._raw(wl.v_pages)
+    kp, vp = kp.copy(), vp.copy()
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    args = (wl.q_offsets, wl.cache_lens, wl.position_ids, sp.mrope_section, table,
+            sp.interleaved, sp.rotary_dim)
+    q_rot = O.rope(wl.q, *args)
+    k_rot = O.rope(wl.k_new, *args)
+    O.cache_image(k_rot, wl.v_new, wl.q_offsets, wl.cache_lens, wl.block_table, kp, vp,
+                  inplace=True)
+    qr = O.round_to(q_rot, code)
+    t_rope = time.perf_counter() - t0
+    # attention one sequence at a time until the time budget is used
+    done_b, kv_bytes, toks = 0, 0, 0
+    t1 = time.perf_counter()
+    elt = 2 if sp.dtype == "bf16" else 4
+    for b in range(sp.batch):
+        lo, hi = int(wl.q_offsets[b]), int(wl.q_offsets[b + 1])
+        rows = np.array([[t, h] for t in range(lo, hi) for h in range(sp.n_heads)], np.int32)
+        if len(rows):
+            O.attention(qr, wl.q_offsets, wl.kv_lens, kp, vp, wl.block_table, sp.n_kv_heads,
+                        sp.softmax_scale, sp.window, rows=rows, n_threads=threads)
+        done_b += 1
+        kv_bytes += M.attention_kv_bytes(wl.q_lens[b:b + 1], wl.kv_lens[b:b + 1], sp.window,
+                                         sp.n_kv_heads, sp.head_dim, elt)
+        toks += hi - lo
+        if time.perf_counter() - t1 > max_seconds:
+            break
+    t_attn = time.perf_counter() - t1
+    # RoPE ran over the whole batch; charge the sampled sequences their share
+    share = done_b / sp.batch
+    seconds = t_attn + t_rope * share
+    return seconds, kv_bytes, toks, f"{done_b} of {sp.batch} sequences (all rows), " \
+                                    f"RoPE + cache image + attention", threads
+
+
+# --------------------------------------------------------------------- main
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        return reference_arm(args, world, rank)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl = W.make(args.workload, seed=args.seed + 1000 * rank)
+    sp = wl.spec
+    step = Step(wl, device)
+    elt = 2 if sp.dtype == "bf16" else 4
+    kv_bytes = M.attention_kv_bytes(wl.q_lens, wl.kv_lens, sp.window, sp.n_kv_heads,
+                                    sp.head_dim, elt)
+    with ClockSampler(local) as clocks:
+        total_ms, rope_ms, attn_ms = time_steps(step, args.steps, args.warmup, world)
+    clk = clocks.summary()
+    step_ms = max_over_ranks(total_ms / args.steps, world)
+    attn_ms_mean = max_over_ranks(statistics.mean(attn_ms), world)
+    rope_ms_mean = max_over_ranks(statistics.mean(rope_ms), world)
+    err = int(step.error_word.item())
+    peaks = load_peaks()
+    value = world * kv_bytes / (step_ms * 1e-3) / 1e9
+    achieved = kv_bytes / (attn_ms_mean * 1e-3) / 1e9
+    traffic = load_traffic("attn_decode")
+
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = time_e2e(step, max(3, args.steps // 2), 2, world)
+        e2e_ms = max_over_ranks(e2e_ms, world)
+        e2e = {"value": world * kv_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "note": "pinned host inputs copied in, output copied out, inside the timed region"}
+
+    prefill = None if args.no_prefill else prefill_measure(device, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, kvb, toks, sample, threads = oracle_sample_time(wl)
+        cpu = {"value": kvb / secs / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": sample, "seconds": secs}
+
+    line = {
+        "metric": "decode_attention_kv_GBps", "value": value, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": sp.dtype,
+        "data": "synthetic (seeded N(0,1) values, shuffled page tables)",
+        "config": {"workload": sp.name, "description": sp.description,
+                   "batch_per_gpu": sp.batch, "new_tokens_per_step": wl.total_tokens,
+                   "kv_bytes_per_step": kv_bytes,
+                   "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V per step "
+                         f"vs {L2_BYTES / 2**20:.0f} MiB L2",
+                   "parallelism": f"replicas x{world} (independent sequences, no exchange)"},
+        "tokens_per_s": world * wl.total_tokens / (step_ms * 1e-3),
+        "breakdown_ms": {"rope_qk_paged_ragged": rope_ms_mean,
+                         "ragged_paged_attention": attn_ms_mean},
+        "roofline": {"bound": "hbm", "kernel": "ragged_paged_attention (split-KV decode + combine)",
+                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": None if traffic is None else traffic["bytes_per_launch"],
+                     "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)"
+                     if peaks["source"] == "measured" else "fallback 6.65 TB/s",
+                     "algorithmic_bytes_per_launch": kv_bytes},
+        "clocks": clk,
+        "e2e": e2e,
+        "gpu_launches": step.launches_per_step() * args.steps,
+        "error_word": err,
+        "prefill": prefill,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def reference_arm(args, world, rank):
+    """The fp64 oracle timed on the host cores, as the reference arm."""
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    wl = W.make(args.workload, seed=args.seed)
+    sp = wl.spec
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_sample_time(wl, max_seconds=2.0)
+    times, vals = [], []
+    budget = max(2.0, 120.0 / max(1, args.steps))
+    for _ in range(args.steps):
+        secs, kvb, toks, sample, threads = oracle_sample_time(wl, max_seconds=budget)
+        times.append(secs)
+        vals.append(kvb / secs / 1e9)
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": "decode_attention_kv_GBps", "value": value, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) values, shuffled page tables)",
+        "config": {"workload": sp.name, "description": sp.description},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

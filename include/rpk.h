@@ -1,0 +1,204 @@
+/*
+ * rpk.h -- C ABI of librpk.so: fused QK RoPE into a paged KV cache and ragged
+ * causal grouped-query attention over that cache, on one NVIDIA B200 (sm_100a).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.   Every tensor argument is DEVICE memory owned by the caller; the
+ *           library allocates nothing (scratch space is the caller-given
+ *           workspace). Host-side arguments are marked "host" below. Tensors
+ *           are dense, row-major, with the shapes given; 16-byte alignment of
+ *           every tensor base is required.
+ * Streams.  `stream` is a cudaStream_t (NULL: the legacy default stream). A
+ *           call validates its arguments on the host, queues its kernels on
+ *           that stream and returns before they finish (NumKong "NumKong for
+ *           Python", GPU Tensors through DLPack: a GPU call queues its launch
+ *           on the given stream and returns).
+ * Errors.   Host-side problems (a NULL pointer, a shape, a dtype, an
+ *           unsupported size) return a non-zero rpk_status before anything is
+ *           launched. Problems that only the data shows (a page id outside the
+ *           pool, a position outside the table, kv_len < q_len) are reported
+ *           by OR-ing RPK_DEVERR_* bits into page_table->error_word when it is
+ *           non-NULL; the offending row or slot is skipped and nothing traps.
+ *           A launch failure returns RPK_ERR_CUDA. There is no CPU fallback
+ *           and no silent change of path (aria_kernel crate index,
+ *           resolve_compute: CUDA never falls back to the CPU).
+ * Dtypes.   RPK_BF16 or RPK_F32 for q, k, v, out and the cache; all arithmetic
+ *           is fp32 with one round-to-nearest-even narrowing at the end.
+ */
+#ifndef RPK_H
+#define RPK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RPK_OK = 0,
+  RPK_ERR_NULL = 1,         /* a required pointer is NULL                          */
+  RPK_ERR_SHAPE = 2,        /* inconsistent or out-of-range sizes                   */
+  RPK_ERR_DTYPE = 3,        /* dtype not supported or not equal where it must be    */
+  RPK_ERR_UNSUPPORTED = 4,  /* valid request outside the sizes the kernels support  */
+  RPK_ERR_CUDA = 5,         /* a CUDA runtime / driver call failed                  */
+  RPK_ERR_WORKSPACE = 6     /* workspace missing, too small or misaligned           */
+} rpk_status;
+
+typedef enum { RPK_F32 = 0, RPK_BF16 = 1 } rpk_dtype;
+
+/* Bits OR-ed into *error_word by the kernels. */
+#define RPK_DEVERR_PAGE 0x1u     /* page id outside [0, num_pages) or slot beyond the block table */
+#define RPK_DEVERR_POSITION 0x2u /* position outside [0, max_position)                          */
+#define RPK_DEVERR_LENGTH 0x4u   /* kv_len < q_len, decreasing offsets, or a length above the
+                                    max_q_len / max_kv_len the call was given                 */
+#define RPK_DEVERR_TIMEOUT 0x8u  /* a bounded wait inside a kernel gave up (kernel returned)    */
+
+/*
+ * The paged KV cache ("kv_collection" of Mojo's fused QK RoPE kernel, a
+ * PagedKVCacheCollection whose keys are read and updated in place).
+ * The struct itself is host memory; the pointers in it are device memory.
+ *
+ *   k_pages, v_pages   [num_pages, page_size, n_kv_heads, head_dim] cache_dtype.
+ *                      Slot s of sequence b is page block_table[b][s / page_size],
+ *                      row s % page_size.
+ *   block_table        int32 [batch, max_pages_per_seq]: page ids into the pool.
+ *                      Entries past a sequence's last page are never read.
+ *   cache_lens         int32 [batch]: tokens already cached for each sequence
+ *                      BEFORE the rope_qk_paged_ragged call that appends to it.
+ *                      Read only by rope_qk_paged_ragged.
+ *   error_word         optional int32 (device): RPK_DEVERR_* bits are OR-ed in.
+ */
+typedef struct {
+  void* k_pages;
+  void* v_pages;
+  int32_t num_pages;
+  int32_t page_size;        /* 16, 32, 64 or 128 */
+  int32_t n_kv_heads;
+  int32_t head_dim;         /* 64, 128 or 256 */
+  rpk_dtype cache_dtype;
+  const int32_t* block_table;
+  int32_t max_pages_per_seq;
+  int32_t batch;
+  const int32_t* cache_lens;
+  int32_t* error_word;
+} rpk_paged_kv;
+
+/*
+ * rope_qk_paged_ragged -- rotate Q into out_q, rotate the new keys and write
+ * them, with the new values, into the paged cache.
+ *
+ * Follows Mojo's generic_fused_qk_rope_bshd_paged_ragged_kernel_api (Args and
+ * Parameters: q_proj, input_row_offsets, kv_collection, freqs_cis,
+ * position_ids, interleaved, mrope_section, output), with the new K and V
+ * passed explicitly (k_new, v_new) and written into the next free slots; the
+ * pairings follow aria_kernel's rope (interleaved), rope_half and
+ * rope_half_partial.
+ *
+ *   q_proj             [total_tokens, n_heads, head_dim] dtype
+ *   input_row_offsets  int32 [batch + 1]: rows off[b] .. off[b+1]-1 belong to
+ *                      sequence b; off[0] = 0, non-decreasing, off[batch] =
+ *                      total_tokens
+ *   k_new, v_new       [total_tokens, n_kv_heads, head_dim] dtype
+ *   page_table         the cache (host struct, see rpk_paged_kv); token i of
+ *                      sequence b goes to slot cache_lens[b] + i
+ *   freqs_cis          fp32 [max_position, rotary_dim]: for pair j at position
+ *                      p, (cos, sin) = (freqs_cis[p][2j], freqs_cis[p][2j+1])
+ *                      (rope_freqs_cis below builds it)
+ *   position_ids       NULL: position of token i of sequence b is
+ *                      cache_lens[b] + i. Otherwise int32 [total_tokens], or
+ *                      [3, total_tokens] when mrope_section is given.
+ *   interleaved        nonzero: pair j is channels (2j, 2j+1); zero: (j, j+R/2)
+ *   rotary_dim (R)     even, 0 < R <= head_dim; channels >= R are copied
+ *   out_q              [total_tokens, n_heads, head_dim] dtype; may alias q_proj
+ *   total_tokens, n_heads, dtype, max_position: sizes (host)
+ *   mrope_section      host int32[3] or NULL: numbers of rotary pairs in the
+ *                      three M-RoPE sections (summing to R/2); pair j takes the
+ *                      position of its section's row of position_ids
+ *
+ * Each pair (a, b) becomes (a cos - b sin, b cos + a sin), computed in fp32
+ * and rounded once to the output dtype. Requirements: dtype == cache dtype,
+ * n_heads % n_kv_heads == 0, (R/2) a multiple of 8 (bf16) or 4 (f32).
+ */
+rpk_status rope_qk_paged_ragged(const void* q_proj, const int32_t* input_row_offsets,
+                                const void* k_new, const void* v_new,
+                                const rpk_paged_kv* page_table, const float* freqs_cis,
+                                const int32_t* position_ids, int32_t interleaved,
+                                int32_t rotary_dim, void* out_q, int32_t total_tokens,
+                                int32_t n_heads, rpk_dtype dtype, int32_t max_position,
+                                const int32_t* mrope_section, void* stream);
+
+/*
+ * rope_freqs_cis -- fill freqs_cis (fp32 [max_position, rotary_dim], device)
+ * with cos and sin of p * theta^(-2j / rotary_dim), evaluated in fp64 and
+ * rounded once to fp32 (algenta "Attention variant kernels",
+ * rope_rotation_angle: theta = position * base^(-2i/d)).
+ */
+rpk_status rope_freqs_cis(float* freqs_cis, int32_t max_position, int32_t rotary_dim,
+                          double theta, void* stream);
+
+/*
+ * ragged_paged_attention_workspace_size -- bytes of device workspace that
+ * ragged_paged_attention needs for these sizes (0 when none). The result
+ * depends only on the arguments, so it may be computed once and reused for
+ * every call with the same sizes.
+ */
+size_t ragged_paged_attention_workspace_size(int32_t total_q_tokens, int32_t n_heads,
+                                             int32_t head_dim, int32_t batch,
+                                             int32_t max_kv_len, int32_t page_size);
+
+/*
+ * ragged_paged_attention -- ragged causal scaled-dot-product attention with
+ * grouped-query heads and an optional sliding window, over the paged cache.
+ *
+ * Follows NumKong's attention_packed ("Attention with a Pre-Packed
+ * KV-Cache"): query row r of a sequence with q_len rows and k_len keys sits at
+ * position p = r + k_len - q_len and sees keys [p - (window - 1), p]
+ * (window <= 0: [0, p]); rows that see no key are zeros. Scores are
+ * scale * q.k (algenta scaled_dot_product_attention), normalised by the
+ * flash online-softmax running state (algenta flash_attention module). Query
+ * head h reads KV head h / (n_heads / n_kv_heads) (grouped-query attention).
+ *
+ *   q               [total_q_tokens, n_heads, head_dim] dtype (already rotated)
+ *   q_row_offsets   int32 [batch + 1], as input_row_offsets above
+ *   kv_lens         int32 [batch]: keys of each sequence, including its q_len
+ *                   newest ones; kv_lens[b] >= q_len[b]
+ *   page_table      the cache (host struct); cache_lens is not read
+ *   scale           finite > 0 (1/sqrt(head_dim) for plain SDPA)
+ *   window          <= 0: unbounded; w > 0: w keys including the row's own
+ *   out             [total_q_tokens, n_heads, head_dim] dtype
+ *   batch, total_q_tokens, max_q_len, max_kv_len: sizes (host); max_q_len and
+ *                   max_kv_len bound q_len[b] and kv_lens[b] (device data) and
+ *                   size the launch; a larger device value sets
+ *                   RPK_DEVERR_LENGTH and that sequence is skipped
+ *   workspace       device scratch of at least
+ *                   ragged_paged_attention_workspace_size(...) bytes, 256-byte
+ *                   aligned; may be NULL when that size is 0. Its contents on
+ *                   entry do not matter; calls sharing one workspace must not
+ *                   overlap in time.
+ *
+ * Paths (chosen from the host sizes, never from device data):
+ *   dtype f32                      -> fp32 CUDA-core kernel
+ *   bf16, max_q_len * group <= 16  -> split-KV decode kernel + combine kernel
+ *   bf16, otherwise                -> tcgen05 prefill kernel (head_dim 64/128)
+ */
+rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
+                                  const int32_t* kv_lens, const rpk_paged_kv* page_table,
+                                  int32_t n_heads, int32_t n_kv_heads, int32_t head_dim,
+                                  float scale, int32_t window, void* out, int32_t batch,
+                                  int32_t total_q_tokens, int32_t max_q_len,
+                                  int32_t max_kv_len, rpk_dtype dtype, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* Static text for a status code. */
+const char* rpk_status_string(rpk_status status);
+
+/* Text of the last CUDA error seen by this thread's calls ("" if none). */
+const char* rpk_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RPK_H */

@@ -141,17 +141,20 @@ def rope(x, row_offsets, cache_lens, position_ids, mrope_section, table, interle
 
 
 def cache_image(k_rot: np.ndarray, v_new, row_offsets, cache_lens, block_table, k_pages,
-                v_pages):
+                v_pages, inplace: bool = False):
     """Return (k_pages', v_pages') raw arrays with the new tokens written in.
 
     k_rot is fp64 [T, n_kv_heads, d]; v_new, k_pages and v_pages are tensors or
-    raw arrays of the cache dtype. The inputs are not modified.
+    raw arrays of the cache dtype. The inputs are copied first unless inplace
+    is set, in which case k_pages / v_pages must be raw numpy arrays and are
+    written directly.
     """
     vraw, code = _raw(v_new)
     kp, kcode = _raw(k_pages)
     vp, vcode = _raw(v_pages)
     assert code == kcode == vcode
-    kp, vp = kp.copy(), vp.copy()
+    if not inplace:
+        kp, vp = kp.copy(), vp.copy()
     k_rot = np.ascontiguousarray(k_rot, dtype=np.float64)
     T, hk, d = k_rot.shape
     offs = _i32arr(row_offsets)

@@ -14,6 +14,7 @@ without a CUDA device raises.
 """
 
 from .binding import (  # noqa: F401
+    PagedKVCache,
     RpkError,
     freqs_cis,
     lib,

@@ -1,46 +1,250 @@
 """ctypes binding of librpk.so (declared in include/rpk.h).
 
-Argument marshalling only: every step of the path runs in the library's CUDA
-kernels. Loading fails loudly when the library has not been built.
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, turned into raw pointers and sizes, and handed to the C ABI, whose
+CUDA kernels do every step of the path. There is no CPU fallback: a missing
+library, a CPU tensor or a non-zero status raises.
+
+Entry points keep the C names:
+
+* ``rope_qk_paged_ragged``  fused RoPE on Q and new K, K/V written into the cache
+* ``ragged_paged_attention`` ragged causal GQA attention over the paged cache
+* ``ragged_paged_attention_workspace_size``
+* ``freqs_cis``             builds the fp32 (cos, sin) table with ``rope_freqs_cis``
 """
 
 from __future__ import annotations
 
 import ctypes as C
 import os
+import re
+from dataclasses import dataclass
+
+import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "librpk.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "rpk.h")
+
+RPK_F32, RPK_BF16 = 0, 1
+STATUS = {0: "RPK_OK", 1: "RPK_ERR_NULL", 2: "RPK_ERR_SHAPE", 3: "RPK_ERR_DTYPE",
+          4: "RPK_ERR_UNSUPPORTED", 5: "RPK_ERR_CUDA", 6: "RPK_ERR_WORKSPACE"}
+DEVERR_PAGE, DEVERR_POSITION, DEVERR_LENGTH, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 
 
 class RpkError(RuntimeError):
-    """A non-zero status from the C ABI."""
+    """A non-zero status from the C ABI (``.status`` holds the code)."""
+
+    def __init__(self, msg: str, status: int | None = None):
+        super().__init__(msg)
+        self.status = status
+
+
+class PagedKV(C.Structure):
+    """Mirror of rpk_paged_kv."""
+
+    _fields_ = [
+        ("k_pages", C.c_void_p), ("v_pages", C.c_void_p),
+        ("num_pages", C.c_int32), ("page_size", C.c_int32),
+        ("n_kv_heads", C.c_int32), ("head_dim", C.c_int32),
+        ("cache_dtype", C.c_int),
+        ("block_table", C.c_void_p), ("max_pages_per_seq", C.c_int32), ("batch", C.c_int32),
+        ("cache_lens", C.c_void_p), ("error_word", C.c_void_p),
+    ]
 
 
 _lib = None
 
 
 def lib():
+    """The loaded librpk.so (raises if it has not been built)."""
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
             raise RpkError(f"librpk.so is not built ({LIB_PATH}); run "
                            "python -m ragged_paged_kv_rope_b200.build")
-        _lib = C.CDLL(LIB_PATH)
+        L = C.CDLL(LIB_PATH)
+        _p, _i32 = C.c_void_p, C.c_int32
+        L.rope_qk_paged_ragged.argtypes = [_p, _p, _p, _p, C.POINTER(PagedKV), _p, _p, _i32, _i32,
+                                           _p, _i32, _i32, C.c_int, _i32, _p, _p]
+        L.rope_qk_paged_ragged.restype = C.c_int
+        L.rope_freqs_cis.argtypes = [_p, _i32, _i32, C.c_double, _p]
+        L.rope_freqs_cis.restype = C.c_int
+        L.ragged_paged_attention_workspace_size.argtypes = [_i32] * 6
+        L.ragged_paged_attention_workspace_size.restype = C.c_size_t
+        L.ragged_paged_attention.argtypes = [_p, _p, _p, C.POINTER(PagedKV), _i32, _i32, _i32,
+                                             C.c_float, _i32, _p, _i32, _i32, _i32, _i32, C.c_int,
+                                             _p, C.c_size_t, _p]
+        L.ragged_paged_attention.restype = C.c_int
+        L.rpk_status_string.argtypes = [C.c_int]
+        L.rpk_status_string.restype = C.c_char_p
+        L.rpk_last_cuda_error.argtypes = []
+        L.rpk_last_cuda_error.restype = C.c_char_p
+        _lib = L
     return _lib
 
 
-def rope_qk_paged_ragged(*args, **kwargs):  # pragma: no cover - filled in with the ABI
-    raise RpkError("not built")
+def header_symbols() -> list[str]:
+    """Names of the functions include/rpk.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:rpk_status|size_t|const char\*)\s+(\w+)\s*\(", text, flags=re.M)
 
 
-def ragged_paged_attention(*args, **kwargs):  # pragma: no cover
-    raise RpkError("not built")
+def _check(status: int):
+    if status != 0:
+        L = lib()
+        msg = L.rpk_status_string(status).decode()
+        if status == 5:
+            msg += f" ({L.rpk_last_cuda_error().decode()})"
+        raise RpkError(f"{STATUS.get(status, status)}: {msg}", status)
 
 
-def ragged_paged_attention_workspace_size(*args, **kwargs):  # pragma: no cover
-    raise RpkError("not built")
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return RPK_BF16
+    if t == torch.float32:
+        return RPK_F32
+    raise RpkError(f"unsupported dtype {t}")
 
 
-def freqs_cis(*args, **kwargs):  # pragma: no cover
-    raise RpkError("not built")
+def _dev(t: torch.Tensor, name: str, dtype=None, ndim=None) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise RpkError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise RpkError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if dtype is not None and t.dtype != dtype:
+        raise RpkError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise RpkError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise RpkError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+@dataclass
+class PagedKVCache:
+    """The paged cache: pools, block table, cached lengths, optional error word."""
+
+    k_pages: torch.Tensor          # [num_pages, page_size, n_kv_heads, head_dim]
+    v_pages: torch.Tensor
+    block_table: torch.Tensor      # int32 [batch, max_pages_per_seq]
+    cache_lens: torch.Tensor | None = None   # int32 [batch]
+    error_word: torch.Tensor | None = None   # int32 [1]
+
+    def struct(self) -> PagedKV:
+        kp, vp = self.k_pages, self.v_pages
+        _dev(kp, "k_pages", ndim=4)
+        _dev(vp, "v_pages", dtype=kp.dtype, ndim=4)
+        if vp.shape != kp.shape:
+            raise RpkError("k_pages and v_pages differ in shape")
+        _dev(self.block_table, "block_table", torch.int32, 2)
+        s = PagedKV()
+        s.k_pages, s.v_pages = kp.data_ptr(), vp.data_ptr()
+        s.num_pages, s.page_size, s.n_kv_heads, s.head_dim = (int(x) for x in kp.shape)
+        s.cache_dtype = _dtype_code(kp.dtype)
+        s.block_table = self.block_table.data_ptr()
+        s.batch, s.max_pages_per_seq = (int(x) for x in self.block_table.shape)
+        s.cache_lens = (_dev(self.cache_lens, "cache_lens", torch.int32, 1)
+                        if self.cache_lens is not None else None)
+        s.error_word = (_dev(self.error_word, "error_word", torch.int32)
+                        if self.error_word is not None else None)
+        return s
+
+
+def rope_qk_paged_ragged(q_proj, input_row_offsets, k_new, v_new, page_table: PagedKVCache,
+                         freqs_cis, position_ids, interleaved: bool, rotary_dim: int, out_q, *,
+                         mrope_section=None, stream=None) -> None:
+    """Rotate q_proj into out_q and k_new into the cache; copy v_new into the cache."""
+    pk = page_table.struct()
+    T, H, d = (int(x) for x in q_proj.shape) if q_proj.dim() == 3 else (None,) * 3
+    if T is None:
+        raise RpkError("q_proj must be [tokens, n_heads, head_dim]")
+    qp = _dev(q_proj, "q_proj")
+    kn = _dev(k_new, "k_new", q_proj.dtype, 3)
+    vn = _dev(v_new, "v_new", q_proj.dtype, 3)
+    oq = _dev(out_q, "out_q", q_proj.dtype, 3)
+    if tuple(out_q.shape) != tuple(q_proj.shape):
+        raise RpkError("out_q must have q_proj's shape")
+    if k_new.shape[0] != T or v_new.shape != k_new.shape:
+        raise RpkError("k_new / v_new must be [tokens, n_kv_heads, head_dim]")
+    off = _dev(input_row_offsets, "input_row_offsets", torch.int32, 1)
+    fc = _dev(freqs_cis, "freqs_cis", torch.float32, 2)
+    if int(freqs_cis.shape[1]) != int(rotary_dim):
+        raise RpkError("freqs_cis must be [max_position, rotary_dim]")
+    pid = None
+    if position_ids is not None:
+        pid = _dev(position_ids, "position_ids", torch.int32)
+        want = (3, T) if mrope_section is not None else (T,)
+        if tuple(position_ids.shape) != want:
+            raise RpkError(f"position_ids must be {want}, got {tuple(position_ids.shape)}")
+    ms = None
+    if mrope_section is not None:
+        ms_arr = (C.c_int32 * 3)(*[int(x) for x in mrope_section])
+        ms = C.cast(ms_arr, C.c_void_p)
+    _check(lib().rope_qk_paged_ragged(
+        qp, off, kn, vn, C.byref(pk), fc, pid, int(bool(interleaved)), int(rotary_dim), oq, T, H,
+        _dtype_code(q_proj.dtype), int(freqs_cis.shape[0]), ms, _stream(stream)))
+
+
+def freqs_cis(max_position: int, rotary_dim: int, theta: float, device=None,
+              stream=None) -> torch.Tensor:
+    """fp32 [max_position, rotary_dim] table of (cos, sin) of p * theta^(-2j/R)."""
+    device = device if device is not None else torch.device("cuda")
+    out = torch.empty((int(max_position), int(rotary_dim)), dtype=torch.float32, device=device)
+    _check(lib().rope_freqs_cis(out.data_ptr(), int(max_position), int(rotary_dim), float(theta),
+                                _stream(stream)))
+    return out
+
+
+def ragged_paged_attention_workspace_size(total_q_tokens: int, n_heads: int, head_dim: int,
+                                          batch: int, max_kv_len: int, page_size: int) -> int:
+    return int(lib().ragged_paged_attention_workspace_size(
+        int(total_q_tokens), int(n_heads), int(head_dim), int(batch), int(max_kv_len),
+        int(page_size)))
+
+
+def ragged_paged_attention(q, q_row_offsets, kv_lens, page_table: PagedKVCache, n_heads: int,
+                           n_kv_heads: int, head_dim: int, scale: float | None, window: int,
+                           out, *, max_q_len: int, max_kv_len: int, workspace=None,
+                           stream=None) -> None:
+    """Ragged causal (windowed) GQA attention of q over the paged cache into out.
+
+    max_q_len / max_kv_len are host-side bounds of the device lengths (they
+    size the launch). workspace: a uint8 CUDA tensor of at least
+    ragged_paged_attention_workspace_size(...) bytes, or None to have one
+    allocated here with torch.
+    """
+    pk = page_table.struct()
+    if q.dim() != 3:
+        raise RpkError("q must be [tokens, n_heads, head_dim]")
+    T = int(q.shape[0])
+    qp = _dev(q, "q")
+    op = _dev(out, "out", q.dtype, 3)
+    if tuple(out.shape) != tuple(q.shape):
+        raise RpkError("out must have q's shape")
+    off = _dev(q_row_offsets, "q_row_offsets", torch.int32, 1)
+    kvl = _dev(kv_lens, "kv_lens", torch.int32, 1)
+    batch = int(kv_lens.shape[0])
+    if scale is None:
+        scale = float(head_dim) ** -0.5
+    need = ragged_paged_attention_workspace_size(T, n_heads, head_dim, batch, max_kv_len,
+                                                 pk.page_size)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws, ws_bytes = None, 0
+    if workspace is not None:
+        ws = _dev(workspace, "workspace", torch.uint8)
+        ws_bytes = workspace.numel()
+    _check(lib().ragged_paged_attention(
+        qp, off, kvl, C.byref(pk), int(n_heads), int(n_kv_heads), int(head_dim), float(scale),
+        int(window), op, batch, T, int(max_q_len), int(max_kv_len), _dtype_code(q.dtype), ws,
+        ws_bytes, _stream(stream)))

@@ -1,0 +1,509 @@
+// attn_decode.cu -- split-KV decode attention over the paged cache (bf16).
+//
+// For sequences with few new rows (q_len * group <= 16) attention is bound by
+// reading K and V from HBM (about 4 FLOP per byte). The kernel streams each
+// sequence's visible keys once per KV head:
+//
+//  * grid (split, kv_head, sequence). A split is a run of whole 64-key tiles
+//    of the band [lo, k_len) (lo = start of the first row's window, or 0);
+//    splits cut long contexts so that every SM streams a few hundred KB.
+//  * warp 4 is the TMA producer: for each tile it loads the K and V rows of
+//    this KV head from the pages named by the block table (3-D tensor map over
+//    the pool [pages * page_size, n_kv_heads, head_dim], box of one head,
+//    128-byte swizzle, no multicast) into a ring of shared-memory stages.
+//  * warps 0-3 each own 16 keys of every tile and keep a private flash
+//    online-softmax state (running max m, running sum l, unnormalised output
+//    O; algenta "Attention variant kernels", flash_attention) for the <= 16
+//    rows (token, query head of the group). Scores S = Q K^T and the update
+//    O += P V use mma.sync m16n8k16 (bf16 in, fp32 accumulate): the contraction
+//    is tiny next to the bytes, so the 16-row tile's idle rows cost nothing
+//    that matters.
+//  * at the end the four warps merge their states (the same rescale rule) and
+//    the CTA writes either the final rows (one split) or an fp32 partial
+//    (m, l, O) that attn_combine_kernel merges across splits.
+//
+// Masking follows NumKong "Attention with a Pre-Packed KV-Cache": row r sits
+// at p = r + k_len - q_len and sees [p - (window - 1), p]; masked keys are left
+// out (score -inf, weight 0) and value rows past k_len are zeroed in shared
+// memory before use so that stale or sentinel bytes never reach P V.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace rpk {
+
+DecodePlan decode_plan(int32_t max_kv_len) {
+  // Tiles of the longest band (one extra for a window start inside a tile).
+  const int32_t max_tiles = (max_kv_len + kDecodeTile - 1) / kDecodeTile + 1;
+  int32_t tps = 8;  // 512 keys per split
+  if ((max_tiles + tps - 1) / tps > kDecodeMaxSplits)
+    tps = (max_tiles + kDecodeMaxSplits - 1) / kDecodeMaxSplits;
+  DecodePlan plan;
+  plan.tiles_per_split = tps;
+  plan.max_splits = (max_tiles + tps - 1) / tps;
+  return plan;
+}
+
+size_t decode_workspace_bytes(int32_t total_q_tokens, int32_t n_heads, int32_t head_dim,
+                              int32_t max_kv_len) {
+  const DecodePlan plan = decode_plan(max_kv_len);
+  const size_t rows = (size_t)plan.max_splits * total_q_tokens * n_heads;
+  const size_t o_bytes = (rows * head_dim * sizeof(float) + 255) & ~size_t(255);
+  const size_t ml_bytes = (rows * sizeof(float2) + 255) & ~size_t(255);
+  return o_bytes + ml_bytes;
+}
+
+namespace {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+
+// Band of keys any row of the sequence sees, in whole tiles, and its splits.
+struct SeqSplit {
+  int tile0;     // first tile
+  int n_tiles;
+  int n_splits;  // >= 1
+};
+
+__device__ __forceinline__ SeqSplit seq_split(int q_len, int k_len, int window, int tps) {
+  SeqSplit s;
+  const int p0 = k_len - q_len;  // position of the first row
+  const int lo = window > 0 ? max(0, p0 - window + 1) : 0;
+  if (k_len <= 0 || lo >= k_len) {
+    s.tile0 = 0; s.n_tiles = 0; s.n_splits = 1;
+    return s;
+  }
+  s.tile0 = lo / kDecodeTile;
+  s.n_tiles = (k_len - 1) / kDecodeTile + 1 - s.tile0;
+  s.n_splits = max(1, (s.n_tiles + tps - 1) / tps);
+  return s;
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D += A(16x16 bf16, row) * B(16x8 bf16, col), fp32 accumulators.
+__device__ __forceinline__ void mma_bf16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int D>
+struct DecodeCfg {
+  static constexpr int kBoxes = D / 64;                      // 128-byte column boxes per row
+  static constexpr int kTileBytes = kDecodeTile * D * 2;     // one of K or V
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kStages = D == 256 ? 2 : (D == 128 ? 3 : 6);
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;  // + alignment slack
+  static_assert(kConsumerWarps * 16 * D * 4 <= kStages * kStageBytes, "merge buffer");
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_decode_kernel(const AttnParams p, const __grid_constant__ CUtensorMap k_map,
+                       const __grid_constant__ CUtensorMap v_map, const DecodePlan plan,
+                       const DecodeWorkspace ws) {
+  using Cfg = DecodeCfg<D>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t full_bar[S], empty_bar[S];
+  __shared__ float m_part[kConsumerWarps][kDecodeMaxRows];
+  __shared__ float l_part[kConsumerWarps][kDecodeMaxRows];
+
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q0 = __ldg(p.offsets + b);
+  const int q_len = __ldg(p.offsets + b + 1) - q0;
+  const int k_len = __ldg(p.kv_lens + b);
+  if (q_len <= 0) return;
+  if (q_len > p.max_q_len || q_len * p.G > kDecodeMaxRows || k_len < 0 || k_len > p.max_kv_len) {
+    if (threadIdx.x == 0 && split == 0 && kvh == 0) raise_error(p.error_word, RPK_DEVERR_LENGTH);
+    return;
+  }
+  const SeqSplit ss = seq_split(q_len, k_len, p.window, plan.tiles_per_split);
+  if (split >= ss.n_splits) return;
+  const int tile_begin = ss.tile0 + split * plan.tiles_per_split;
+  const int n_tiles = max(0, min(plan.tiles_per_split, ss.tile0 + ss.n_tiles - tile_begin));
+  const int rows = q_len * p.G;
+
+  // 1024-byte aligned stage ring (128-byte swizzle atoms are 8 rows x 128 bytes).
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  auto k_stage = [&](int s) { return smem + s * Cfg::kStageBytes; };
+  auto v_stage = [&](int s) { return smem + s * Cfg::kStageBytes + Cfg::kTileBytes; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kConsumerWarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&k_map);
+      prefetch_tensormap(&v_map);
+      const int box_rows = p.P < kDecodeTile ? p.P : kDecodeTile;
+      const uint32_t box_bytes = box_rows * 128u;
+      int issued = 0;
+      bool ok = true;
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        const int s = i % S;
+        if (!mbar_wait(&empty_bar[s], ((i / S) & 1) ^ 1)) { ok = false; break; }
+        const int key0 = (tile_begin + i) * kDecodeTile;
+        // Count the boxes to load (pages wholly past k_len or invalid are skipped).
+        uint32_t bytes = 0;
+        for (int r = 0; r < kDecodeTile; r += box_rows) {
+          const int key = key0 + r;
+          if (key >= k_len) break;
+          const int pi = key / p.P;
+          const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
+          if (page >= 0 && page < p.num_pages) bytes += 2u * Cfg::kBoxes * box_bytes;
+        }
+        mbar_arrive_expect_tx(&full_bar[s], bytes);
+        for (int r = 0; r < kDecodeTile; r += box_rows) {
+          const int key = key0 + r;
+          if (key >= k_len) break;
+          const int pi = key / p.P;
+          const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
+          if (page < 0 || page >= p.num_pages) {
+            raise_error(p.error_word, RPK_DEVERR_PAGE);
+            continue;
+          }
+          const int grow = page * p.P + (key - pi * p.P);
+#pragma unroll
+          for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+            tma_load_3d(k_stage(s) + bx * (kDecodeTile * 128) + r * 128, &k_map, bx * 64, kvh,
+                        grow, &full_bar[s]);
+            tma_load_3d(v_stage(s) + bx * (kDecodeTile * 128) + r * 128, &v_map, bx * 64, kvh,
+                        grow, &full_bar[s]);
+          }
+        }
+        ++issued;
+      }
+      if (!ok) raise_error(p.error_word, RPK_DEVERR_TIMEOUT);
+      // Never leave with copies in flight: wait for the last stages issued.
+      for (int i = max(0, issued - S); i < issued; ++i)
+        mbar_wait(&full_bar[i % S], (i / S) & 1);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------- consumers
+  const int g = lane >> 2, c = lane & 3;
+  // Row ids of this lane's two accumulator rows and their visible key ranges.
+  int row_lo[2], row_hi[2];
+  bool row_ok[2];
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    const int rr = g + hr * 8;
+    row_ok[hr] = rr < rows;
+    const int tok = rr / p.G;                 // token index in the sequence
+    const int pos = tok + k_len - q_len;      // its position
+    row_hi[hr] = pos;
+    row_lo[hr] = p.window > 0 ? pos - p.window + 1 : 0;
+  }
+
+  // Q as the A operand (16 rows x D), rows past `rows` are zero.
+  uint32_t qa[D / 16][4];
+  {
+    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.q);
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int rr = g + hr * 8;
+      const __nv_bfloat16* qrow = nullptr;
+      if (rr < rows) {
+        const int t = q0 + rr / p.G;
+        const int h = kvh * p.G + rr % p.G;
+        qrow = qb + ((size_t)t * p.H + h) * D;
+      }
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t lo = 0, hi = 0;
+        if (qrow) {
+          lo = *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * c);
+          hi = *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * c);
+        }
+        qa[ks][hr] = lo;       // a0 (row g) / a1 (row g+8)
+        qa[ks][2 + hr] = hi;   // a2 / a3
+      }
+    }
+  }
+
+  float o[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m_run[2] = {-INFINITY, -INFINITY};
+  float l_run[2] = {0.f, 0.f};
+  bool ok = true;
+
+  for (int i = 0; i < n_tiles; ++i) {
+    const int s = i % S;
+    if (!mbar_wait(&full_bar[s], (i / S) & 1)) { ok = false; break; }
+    const int key0 = (tile_begin + i) * kDecodeTile + warp * 16;  // this warp's 16 keys
+    const uint32_t kbase = smem_u32(k_stage(s));
+    const uint32_t vbase = smem_u32(v_stage(s));
+    const int wrow0 = warp * 16;  // row of this warp's first key inside the tile
+
+    // Zero value rows at or past k_len (stale or never written bytes).
+    const bool tail = key0 + 15 >= k_len;
+    if (tail) {
+      for (int idx = lane; idx < 16 * (D / 8); idx += 32) {
+        const int kr = idx / (D / 8);
+        if (key0 + kr < k_len) continue;
+        const int ch = idx % (D / 8);
+        uint8_t* dst = v_stage(s) + (ch >> 3) * (kDecodeTile * 128) + swz128(wrow0 + kr, ch & 7);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      }
+      __syncwarp();
+    }
+
+    // S = Q K^T for 16 keys: two n-tiles of 8 keys.
+    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      // matrices: (keys 0-7, d lo), (keys 0-7, d hi), (keys 8-15, d lo), (keys 8-15, d hi)
+      const int mi = lane >> 3;
+      const int krow = wrow0 + (mi >> 1) * 8 + (lane & 7);
+      const int chunk = ks * 2 + (mi & 1);
+      const uint32_t addr = kbase + (chunk >> 3) * (kDecodeTile * 128) + swz128(krow, chunk & 7);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(addr, b0, b1, b2, b3);
+      mma_bf16(sc[0], qa[ks], b0, b1);
+      mma_bf16(sc[1], qa[ks], b2, b3);
+    }
+
+    // Mask, scale to log2 units, online-softmax update of both rows.
+    float tmax[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int hr = e >> 1;
+        const int key = key0 + nt * 8 + 2 * c + (e & 1);
+        const bool vis = row_ok[hr] && key >= row_lo[hr] && key <= row_hi[hr];
+        const float v = vis ? sc[nt][e] * p.scale_log2 : -INFINITY;
+        sc[nt][e] = v;
+        tmax[hr] = fmaxf(tmax[hr], v);
+      }
+    float alpha[2], m_use[2];
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      tmax[hr] = fmaxf(tmax[hr], __shfl_xor_sync(0xffffffffu, tmax[hr], 1));
+      tmax[hr] = fmaxf(tmax[hr], __shfl_xor_sync(0xffffffffu, tmax[hr], 2));
+      const float m_new = fmaxf(m_run[hr], tmax[hr]);
+      m_use[hr] = m_new == -INFINITY ? 0.f : m_new;
+      alpha[hr] = fast_exp2(m_run[hr] - m_use[hr]);
+      m_run[hr] = m_new;
+    }
+    float rsum[2] = {0.f, 0.f};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int hr = e >> 1;
+        const float w = fast_exp2(sc[nt][e] - m_use[hr]);
+        sc[nt][e] = w;
+        rsum[hr] += w;
+      }
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) l_run[hr] = l_run[hr] * alpha[hr] + rsum[hr];
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      o[n][0] *= alpha[0]; o[n][1] *= alpha[0];
+      o[n][2] *= alpha[1]; o[n][3] *= alpha[1];
+    }
+
+    // O += P V: P (16 rows x 16 keys) as the A operand straight from registers.
+    uint32_t pa[4];
+    pa[0] = pack_bf16x2(sc[0][0], sc[0][1]);
+    pa[1] = pack_bf16x2(sc[0][2], sc[0][3]);
+    pa[2] = pack_bf16x2(sc[1][0], sc[1][1]);
+    pa[3] = pack_bf16x2(sc[1][2], sc[1][3]);
+#pragma unroll
+    for (int dn = 0; dn < D / 16; ++dn) {
+      // matrices (transposed): (keys 0-7, d n0), (keys 8-15, d n0), (keys 0-7, d n0+8),
+      // (keys 8-15, d n0+8)
+      const int mi = lane >> 3;
+      const int vrow = wrow0 + (mi & 1) * 8 + (lane & 7);
+      const int chunk = dn * 2 + (mi >> 1);
+      const uint32_t addr = vbase + (chunk >> 3) * (kDecodeTile * 128) + swz128(vrow, chunk & 7);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(addr, b0, b1, b2, b3);
+      mma_bf16(o[2 * dn], pa, b0, b1);
+      mma_bf16(o[2 * dn + 1], pa, b2, b3);
+    }
+
+    __syncwarp();
+    if (tail) fence_proxy_async_smem();  // generic zero-writes before the next TMA into s
+    if (lane == 0) mbar_arrive(&empty_bar[s]);
+  }
+  if (!ok) raise_error(p.error_word, RPK_DEVERR_TIMEOUT);
+
+  // ----------------------------------------------- merge the four warps' states
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    l_run[hr] += __shfl_xor_sync(0xffffffffu, l_run[hr], 1);
+    l_run[hr] += __shfl_xor_sync(0xffffffffu, l_run[hr], 2);
+  }
+  if (c == 0) {
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      m_part[warp][g + hr * 8] = m_run[hr];
+      l_part[warp][g + hr * 8] = l_run[hr];
+    }
+  }
+  // All consumers are past the tile loop, so every stage's TMA has landed and
+  // the ring can be reused as the merge buffer.
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+  float* obuf = reinterpret_cast<float*>(smem);  // [warp][16][D]
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    const int rr = g + hr * 8;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) mx = fmaxf(mx, m_part[w][rr]);
+    const float f = m_run[hr] == -INFINITY ? 0.f : fast_exp2(m_run[hr] - mx);
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      float2 v = make_float2(o[n][2 * hr] * f, o[n][2 * hr + 1] * f);
+      *reinterpret_cast<float2*>(obuf + ((size_t)warp * 16 + rr) * D + n * 8 + 2 * c) = v;
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+
+  const bool single = ss.n_splits == 1;
+  for (int idx = threadIdx.x; idx < rows * (D / 4); idx += kConsumerWarps * 32) {
+    const int rr = idx / (D / 4);
+    const int e4 = (idx - rr * (D / 4)) * 4;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) mx = fmaxf(mx, m_part[w][rr]);
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float mw = m_part[w][rr];
+      const float f = mw == -INFINITY ? 0.f : fast_exp2(mw - mx);
+      L += l_part[w][rr] * f;
+      const float4 v = *reinterpret_cast<const float4*>(obuf + ((size_t)w * 16 + rr) * D + e4);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    const int t = q0 + rr / p.G;
+    const int h = kvh * p.G + rr % p.G;
+    const size_t orow = (size_t)t * p.H + h;
+    if (single) {
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + orow * D + e4;
+      uint2 pk;
+      pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+      pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2*>(out) = pk;
+    } else {
+      const size_t prow = (size_t)split * p.T * p.H + orow;
+      *reinterpret_cast<float4*>(ws.o + prow * D + e4) = acc;
+      if (e4 == 0) ws.ml[prow] = make_float2(mx, L);
+    }
+  }
+}
+
+// Merge the split partials of each (token, head) row: m* = max m_s,
+// out = sum_s 2^(m_s - m*) O_s / sum_s 2^(m_s - m*) l_s (zero when empty).
+template <int D>
+__global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p,
+                                                           const DecodePlan plan,
+                                                           const DecodeWorkspace ws) {
+  constexpr int E = D / 32;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= (long long)p.T * p.H) return;
+  const int t = (int)(row / p.H);
+  const int b = find_sequence(p.offsets, p.batch, t);
+  const int q_len = __ldg(p.offsets + b + 1) - __ldg(p.offsets + b);
+  const int k_len = __ldg(p.kv_lens + b);
+  if (q_len > p.max_q_len || q_len * p.G > kDecodeMaxRows || k_len < 0 || k_len > p.max_kv_len)
+    return;
+  const SeqSplit ss = seq_split(q_len, k_len, p.window, plan.tiles_per_split);
+  if (ss.n_splits <= 1) return;  // the decode kernel wrote this row itself
+  const size_t stride = (size_t)p.T * p.H;
+  float mx = -INFINITY;
+  for (int s = 0; s < ss.n_splits; ++s) mx = fmaxf(mx, ws.ml[s * stride + row].x);
+  float L = 0.f, acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  for (int s = 0; s < ss.n_splits; ++s) {
+    const float2 ml = ws.ml[s * stride + row];
+    const float f = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - mx);
+    L += ml.y * f;
+    const float* src = ws.o + (s * stride + row) * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; e += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(src + e);
+      acc[e] += f * v.x; acc[e + 1] += f * v.y; acc[e + 2] += f * v.z; acc[e + 3] += f * v.w;
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * D + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t*>(out + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+}
+
+template <int D>
+cudaError_t launch_d(const AttnParams& p, const CUtensorMap& k_map, const CUtensorMap& v_map,
+                     const DecodePlan& plan, const DecodeWorkspace& ws, cudaStream_t stream) {
+  using Cfg = DecodeCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(plan.max_splits, p.Hk, p.batch);
+  attn_decode_kernel<D><<<grid, kThreads, Cfg::kSmemBytes, stream>>>(p, k_map, v_map, plan, ws);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (plan.max_splits > 1) {
+    const long long rows = (long long)p.T * p.H;
+    attn_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p, plan, ws);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+}  // namespace
+
+cudaError_t launch_attn_decode(const AttnParams& p, const CUtensorMap& k_map,
+                               const CUtensorMap& v_map, const DecodePlan& plan,
+                               const DecodeWorkspace& ws, cudaStream_t stream) {
+  if ((long long)p.T * p.H == 0 || p.batch == 0) return cudaSuccess;
+  switch (p.d) {
+    case 64: return launch_d<64>(p, k_map, v_map, plan, ws, stream);
+    case 128: return launch_d<128>(p, k_map, v_map, plan, ws, stream);
+    case 256: return launch_d<256>(p, k_map, v_map, plan, ws, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace rpk

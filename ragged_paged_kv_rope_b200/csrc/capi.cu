@@ -1,0 +1,233 @@
+// capi.cu -- the extern "C" entry points of librpk.so (declared in include/rpk.h):
+// host-side validation, tensor-map encoding and kernel dispatch. No entry
+// point allocates device memory or synchronises the stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/rpk.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+rpk_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return RPK_OK;
+  snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: %s", cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return RPK_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_head_dim(int32_t d) { return d == 64 || d == 128 || d == 256; }
+bool supported_page(int32_t P) { return P == 16 || P == 32 || P == 64 || P == 128; }
+
+rpk_status check_cache(const rpk_paged_kv* c) {
+  if (!c) return RPK_ERR_NULL;
+  if (!c->k_pages || !c->v_pages || !c->block_table) return RPK_ERR_NULL;
+  if (c->cache_dtype != RPK_BF16 && c->cache_dtype != RPK_F32) return RPK_ERR_DTYPE;
+  if (c->num_pages <= 0 || c->n_kv_heads <= 0 || c->max_pages_per_seq <= 0 || c->batch <= 0)
+    return RPK_ERR_SHAPE;
+  if (!supported_page(c->page_size) || !supported_head_dim(c->head_dim))
+    return RPK_ERR_UNSUPPORTED;
+  if (!aligned16(c->k_pages) || !aligned16(c->v_pages)) return RPK_ERR_SHAPE;
+  if ((long long)c->num_pages * c->page_size > INT32_MAX) return RPK_ERR_UNSUPPORTED;
+  return RPK_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 map over rows of [rows, heads, d]: dims (d, heads, rows), box
+// (64, 1, box_rows), 128-byte swizzle. Used for the KV pools and for Q.
+rpk_status encode_rows_map(CUtensorMap* map, const void* base, int32_t d, int32_t heads,
+                           int64_t rows, int32_t box_heads, int32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) {
+    snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled unavailable");
+    return RPK_ERR_CUDA;
+  }
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
+  cuuint32_t box[3] = {64u, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled failed (%d)",
+             (int)r);
+    return RPK_ERR_CUDA;
+  }
+  return RPK_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rpk_status_string(rpk_status s) {
+  switch (s) {
+    case RPK_OK: return "ok";
+    case RPK_ERR_NULL: return "a required pointer is NULL";
+    case RPK_ERR_SHAPE: return "inconsistent or out-of-range sizes";
+    case RPK_ERR_DTYPE: return "unsupported or mismatched dtype";
+    case RPK_ERR_UNSUPPORTED: return "sizes outside what the kernels support";
+    case RPK_ERR_CUDA: return "CUDA call failed";
+    case RPK_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+  }
+  return "unknown status";
+}
+
+const char* rpk_last_cuda_error(void) { return g_last_cuda_error; }
+
+rpk_status rope_qk_paged_ragged(const void* q_proj, const int32_t* input_row_offsets,
+                                const void* k_new, const void* v_new,
+                                const rpk_paged_kv* page_table, const float* freqs_cis,
+                                const int32_t* position_ids, int32_t interleaved,
+                                int32_t rotary_dim, void* out_q, int32_t total_tokens,
+                                int32_t n_heads, rpk_dtype dtype, int32_t max_position,
+                                const int32_t* mrope_section, void* stream) {
+  if (!q_proj || !input_row_offsets || !k_new || !v_new || !freqs_cis || !out_q)
+    return RPK_ERR_NULL;
+  rpk_status st = check_cache(page_table);
+  if (st != RPK_OK) return st;
+  if (!page_table->cache_lens) return RPK_ERR_NULL;
+  if (dtype != RPK_BF16 && dtype != RPK_F32) return RPK_ERR_DTYPE;
+  if (dtype != page_table->cache_dtype) return RPK_ERR_DTYPE;
+  const int32_t d = page_table->head_dim, Hk = page_table->n_kv_heads;
+  if (total_tokens < 0 || n_heads <= 0 || max_position <= 0) return RPK_ERR_SHAPE;
+  if (n_heads % Hk != 0) return RPK_ERR_SHAPE;
+  if (rotary_dim <= 0 || (rotary_dim & 1) || rotary_dim > d) return RPK_ERR_SHAPE;
+  const int vec = dtype == RPK_BF16 ? 8 : 4;
+  if ((rotary_dim / 2) % vec != 0) return RPK_ERR_UNSUPPORTED;
+  if (mrope_section) {
+    if (!position_ids) return RPK_ERR_NULL;
+    if (mrope_section[0] < 0 || mrope_section[1] < 0 || mrope_section[2] < 0 ||
+        mrope_section[0] + mrope_section[1] + mrope_section[2] != rotary_dim / 2)
+      return RPK_ERR_SHAPE;
+  }
+  if (!aligned16(q_proj) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out_q) ||
+      !aligned16(freqs_cis))
+    return RPK_ERR_SHAPE;
+  if ((long long)total_tokens * n_heads * d > INT32_MAX * 8LL) return RPK_ERR_UNSUPPORTED;
+  if (total_tokens == 0) return RPK_OK;
+
+  rpk::RopeParams p;
+  p.q = q_proj; p.k_new = k_new; p.v_new = v_new; p.out_q = out_q;
+  p.k_pages = page_table->k_pages; p.v_pages = page_table->v_pages;
+  p.offsets = input_row_offsets; p.cache_lens = page_table->cache_lens;
+  p.block_table = page_table->block_table; p.position_ids = position_ids;
+  p.freqs = freqs_cis; p.error_word = page_table->error_word;
+  p.T = total_tokens; p.batch = page_table->batch; p.H = n_heads; p.Hk = Hk; p.d = d;
+  p.R = rotary_dim; p.P = page_table->page_size; p.num_pages = page_table->num_pages;
+  p.max_pages = page_table->max_pages_per_seq; p.max_position = max_position;
+  p.has_mrope = mrope_section != nullptr;
+  p.sec_end0 = mrope_section ? mrope_section[0] : rotary_dim;
+  p.sec_end1 = mrope_section ? mrope_section[0] + mrope_section[1] : rotary_dim;
+  return cuda_status(rpk::launch_rope(p, dtype, interleaved != 0,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+rpk_status rope_freqs_cis(float* freqs_cis, int32_t max_position, int32_t rotary_dim,
+                          double theta, void* stream) {
+  if (!freqs_cis) return RPK_ERR_NULL;
+  if (max_position < 0 || rotary_dim <= 0 || (rotary_dim & 1)) return RPK_ERR_SHAPE;
+  if (!(theta > 0.0) || !std::isfinite(theta)) return RPK_ERR_SHAPE;
+  return cuda_status(rpk::launch_freqs_cis(freqs_cis, max_position, rotary_dim, theta,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+size_t ragged_paged_attention_workspace_size(int32_t total_q_tokens, int32_t n_heads,
+                                             int32_t head_dim, int32_t batch,
+                                             int32_t max_kv_len, int32_t page_size) {
+  (void)batch;
+  (void)page_size;
+  if (total_q_tokens <= 0 || n_heads <= 0 || head_dim <= 0 || max_kv_len < 0) return 0;
+  return rpk::decode_workspace_bytes(total_q_tokens, n_heads, head_dim, max_kv_len);
+}
+
+rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
+                                  const int32_t* kv_lens, const rpk_paged_kv* page_table,
+                                  int32_t n_heads, int32_t n_kv_heads, int32_t head_dim,
+                                  float scale, int32_t window, void* out, int32_t batch,
+                                  int32_t total_q_tokens, int32_t max_q_len,
+                                  int32_t max_kv_len, rpk_dtype dtype, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (!q || !q_row_offsets || !kv_lens || !out) return RPK_ERR_NULL;
+  rpk_status st = check_cache(page_table);
+  if (st != RPK_OK) return st;
+  if (dtype != RPK_BF16 && dtype != RPK_F32) return RPK_ERR_DTYPE;
+  if (dtype != page_table->cache_dtype) return RPK_ERR_DTYPE;
+  if (n_kv_heads != page_table->n_kv_heads || head_dim != page_table->head_dim)
+    return RPK_ERR_SHAPE;
+  if (n_heads <= 0 || n_heads % n_kv_heads != 0) return RPK_ERR_SHAPE;
+  if (batch <= 0 || batch != page_table->batch || batch > 65535) return RPK_ERR_SHAPE;
+  if (total_q_tokens < 0 || max_q_len < 0 || max_kv_len < 0) return RPK_ERR_SHAPE;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return RPK_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(out)) return RPK_ERR_SHAPE;
+  if ((long long)max_kv_len > (long long)page_table->max_pages_per_seq * page_table->page_size)
+    return RPK_ERR_SHAPE;
+  if (total_q_tokens == 0) return RPK_OK;
+
+  rpk::AttnParams p;
+  p.q = q; p.out = out; p.k_pages = page_table->k_pages; p.v_pages = page_table->v_pages;
+  p.offsets = q_row_offsets; p.kv_lens = kv_lens; p.block_table = page_table->block_table;
+  p.error_word = page_table->error_word;
+  p.T = total_q_tokens; p.batch = batch; p.H = n_heads; p.Hk = n_kv_heads;
+  p.G = n_heads / n_kv_heads; p.d = head_dim; p.P = page_table->page_size;
+  p.num_pages = page_table->num_pages; p.max_pages = page_table->max_pages_per_seq;
+  p.window = window > 0 ? window : 0; p.max_q_len = max_q_len; p.max_kv_len = max_kv_len;
+  p.scale = scale;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  if (dtype == RPK_F32) return cuda_status(rpk::launch_attn_simt(p, dtype, s));
+
+  if ((long long)max_q_len * p.G <= rpk::kDecodeMaxRows) {
+    const size_t need = rpk::decode_workspace_bytes(total_q_tokens, n_heads, head_dim, max_kv_len);
+    const rpk::DecodePlan plan = rpk::decode_plan(max_kv_len);
+    if (plan.max_splits > 1) {
+      if (!workspace || workspace_bytes < need) return RPK_ERR_WORKSPACE;
+      if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return RPK_ERR_WORKSPACE;
+    }
+    rpk::DecodeWorkspace ws;
+    const size_t rows = (size_t)plan.max_splits * total_q_tokens * n_heads;
+    const size_t o_bytes = (rows * head_dim * sizeof(float) + 255) & ~size_t(255);
+    ws.o = static_cast<float*>(workspace);
+    ws.ml = workspace ? reinterpret_cast<float2*>(static_cast<char*>(workspace) + o_bytes)
+                      : nullptr;
+    CUtensorMap k_map, v_map;
+    const int32_t box_rows = p.P < rpk::kDecodeTile ? p.P : rpk::kDecodeTile;
+    const int64_t pool_rows = (int64_t)p.num_pages * p.P;
+    st = encode_rows_map(&k_map, p.k_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
+    if (st != RPK_OK) return st;
+    st = encode_rows_map(&v_map, p.v_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
+    if (st != RPK_OK) return st;
+    return cuda_status(rpk::launch_attn_decode(p, k_map, v_map, plan, ws, s));
+  }
+
+  // Prefill shapes: CUDA-core kernel until the tensor-core kernel takes them.
+  return cuda_status(rpk::launch_attn_simt(p, dtype, s));
+}
+
+}  // extern "C"

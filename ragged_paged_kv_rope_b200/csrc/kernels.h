@@ -1,0 +1,81 @@
+// kernels.h -- launch parameters and launchers of the librpk kernels
+// (internal to the library; the public ABI is include/rpk.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/rpk.h"
+
+namespace rpk {
+
+struct RopeParams {
+  const void* q;
+  const void* k_new;
+  const void* v_new;
+  void* out_q;
+  void* k_pages;
+  void* v_pages;
+  const int32_t* offsets;       // [batch + 1]
+  const int32_t* cache_lens;    // [batch]
+  const int32_t* block_table;   // [batch, max_pages]
+  const int32_t* position_ids;  // NULL, [T] or [3, T]
+  const float* freqs;           // [max_position, R]
+  int32_t* error_word;
+  int32_t T, batch, H, Hk, d, R, P, num_pages, max_pages, max_position;
+  int32_t sec_end0, sec_end1;   // M-RoPE: pair j < sec_end0 -> section 0, < sec_end1 -> 1, else 2
+  int32_t has_mrope;
+};
+
+cudaError_t launch_rope(const RopeParams& p, rpk_dtype dtype, bool interleaved,
+                        cudaStream_t stream);
+cudaError_t launch_freqs_cis(float* out, int32_t max_position, int32_t rotary_dim, double theta,
+                             cudaStream_t stream);
+
+struct AttnParams {
+  const void* q;
+  void* out;
+  const void* k_pages;
+  const void* v_pages;
+  const int32_t* offsets;      // [batch + 1]
+  const int32_t* kv_lens;      // [batch]
+  const int32_t* block_table;  // [batch, max_pages]
+  int32_t* error_word;
+  int32_t T, batch, H, Hk, G, d, P, num_pages, max_pages, window, max_q_len, max_kv_len;
+  float scale;
+  float scale_log2;            // scale * log2(e)
+};
+
+// fp32 / bf16 CUDA-core attention: one warp per (token, head) row.
+cudaError_t launch_attn_simt(const AttnParams& p, rpk_dtype dtype, cudaStream_t stream);
+
+// Split-KV decode (bf16): key tiles of this many keys, splits of whole tiles.
+constexpr int kDecodeTile = 64;
+constexpr int kDecodeMaxRows = 16;   // max_q_len * group must fit one m16 tile
+constexpr int kDecodeMaxSplits = 64;
+
+struct DecodePlan {
+  int32_t tiles_per_split;
+  int32_t max_splits;
+};
+DecodePlan decode_plan(int32_t max_kv_len);
+size_t decode_workspace_bytes(int32_t total_q_tokens, int32_t n_heads, int32_t head_dim,
+                              int32_t max_kv_len);
+
+struct DecodeWorkspace {
+  float* o;       // [max_splits, T, H, d]
+  float2* ml;     // [max_splits, T, H]: (running max in log2 units, running sum)
+};
+
+cudaError_t launch_attn_decode(const AttnParams& p, const CUtensorMap& k_map,
+                               const CUtensorMap& v_map, const DecodePlan& plan,
+                               const DecodeWorkspace& ws, cudaStream_t stream);
+
+// tcgen05 prefill (bf16, head_dim 64 or 128).
+cudaError_t launch_attn_prefill(const AttnParams& p, const CUtensorMap& q_map,
+                                const CUtensorMap& k_map, const CUtensorMap& v_map,
+                                cudaStream_t stream);
+int prefill_rows_per_tile(int group);
+
+}  // namespace rpk

@@ -1,0 +1,204 @@
+// rope.cu -- fused RoPE on Q and K with K/V scattered into the paged cache.
+//
+// Semantics: Mojo "generic_fused_qk_rope_bshd_paged_ragged_kernel_api" (ragged
+// rows by input_row_offsets, rotation of Q into the output and of K into the
+// paged cache, interleaved vs half pairing, per-token position_ids, M-RoPE
+// sections) and aria_kernel's rope / rope_half / rope_half_partial (pairings
+// and partial rotary_dim). Pair (a, b) at angle theta becomes
+// (a cos - b sin, b cos + a sin), with (cos, sin) read from freqs_cis[pos].
+//
+// Design: pure bandwidth. One CTA per token; its threads walk 16-byte units of
+// the token's q, k and v head rows. A rotation unit of the half layout holds
+// kVec pairs (kVec channels from each half), one of the interleaved layout a
+// 16-byte chunk of kVec/2 adjacent pairs, whose (cos, sin) entries are the
+// same 16-byte-aligned run of the table row. Channels >= rotary_dim and V rows
+// are 16-byte copies. Every global access is a 16-byte vector.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace rpk {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <typename T, bool kInterleaved>
+__global__ void __launch_bounds__(kThreads) rope_scatter_kernel(const RopeParams p) {
+  constexpr int V = Elt<T>::kVec;
+  const int t = blockIdx.x;
+  if (t >= p.T) return;
+
+  // Sequence, index in it, cache slot and page of this token.
+  const int b = find_sequence(p.offsets, p.batch, t);
+  const int i = t - __ldg(p.offsets + b);
+  const int slot = __ldg(p.cache_lens + b) + i;
+  int page = -1;
+  if (slot >= 0) {
+    const int pi = slot / p.P;
+    if (pi < p.max_pages) page = __ldg(p.block_table + (size_t)b * p.max_pages + pi);
+  }
+  const bool page_ok = page >= 0 && page < p.num_pages;
+  const int row_in_page = slot >= 0 ? slot % p.P : 0;
+
+  // Position of each M-RoPE section (all equal without M-RoPE).
+  int pos[3];
+  if (p.position_ids == nullptr) {
+    pos[0] = pos[1] = pos[2] = slot;
+  } else if (p.has_mrope) {
+#pragma unroll
+    for (int s = 0; s < 3; ++s) pos[s] = __ldg(p.position_ids + (size_t)s * p.T + t);
+  } else {
+    pos[0] = pos[1] = pos[2] = __ldg(p.position_ids + t);
+  }
+  bool pos_ok = true;
+#pragma unroll
+  for (int s = 0; s < 3; ++s) pos_ok &= (pos[s] >= 0 && pos[s] < p.max_position);
+  if (threadIdx.x == 0) {
+    if (!page_ok) raise_error(p.error_word, RPK_DEVERR_PAGE);
+    if (!pos_ok) raise_error(p.error_word, RPK_DEVERR_POSITION);
+  }
+
+  const int half = p.R >> 1;
+  // Units per head row: rotation units, then pass-through units.
+  const int rot_units = kInterleaved ? p.R / V : half / V;
+  const int pass_units = (p.d - p.R) / V;
+  const int units_row = rot_units + pass_units;
+  const int q_units = p.H * units_row;
+  const int k_units = p.Hk * units_row;
+  const int v_units = p.Hk * (p.d / V);
+  const int total = q_units + k_units + v_units;
+
+  const T* __restrict__ q = static_cast<const T*>(p.q);
+  const T* __restrict__ kn = static_cast<const T*>(p.k_new);
+  const T* __restrict__ vn = static_cast<const T*>(p.v_new);
+  T* out_q = static_cast<T*>(p.out_q);
+  T* kp = static_cast<T*>(p.k_pages);
+  T* vp = static_cast<T*>(p.v_pages);
+
+  for (int u = threadIdx.x; u < total; u += kThreads) {
+    const T* src;
+    T* dst;
+    int unit;
+    if (u < q_units + k_units) {
+      int row;
+      if (u < q_units) {
+        row = u / units_row;
+        unit = u - row * units_row;
+        src = q + ((size_t)t * p.H + row) * p.d;
+        dst = out_q + ((size_t)t * p.H + row) * p.d;
+      } else {
+        if (!page_ok) continue;
+        const int uk = u - q_units;
+        row = uk / units_row;
+        unit = uk - row * units_row;
+        src = kn + ((size_t)t * p.Hk + row) * p.d;
+        dst = kp + (((size_t)page * p.P + row_in_page) * p.Hk + row) * p.d;
+      }
+      if (unit >= rot_units) {  // channels >= rotary_dim: copy
+        const int off = p.R + (unit - rot_units) * V;
+        *reinterpret_cast<uint4*>(dst + off) = *reinterpret_cast<const uint4*>(src + off);
+        continue;
+      }
+      if (!pos_ok) continue;
+      // Pairs covered by this unit and the channels of their two members.
+      const int j0 = kInterleaved ? unit * (V / 2) : unit * V;
+      constexpr int NP = kInterleaved ? V / 2 : V;
+      const int s0 = p.has_mrope ? (j0 < p.sec_end0 ? 0 : (j0 < p.sec_end1 ? 1 : 2)) : 0;
+      const int jl = j0 + NP - 1;
+      const int s1 = p.has_mrope ? (jl < p.sec_end0 ? 0 : (jl < p.sec_end1 ? 1 : 2)) : 0;
+      float cs[2 * NP];  // (cos, sin) of each pair
+      if (s0 == s1) {
+        const float* tab = p.freqs + (size_t)pos[s0] * p.R + 2 * j0;
+#pragma unroll
+        for (int k = 0; k < 2 * NP; k += 4) {
+          const float4 c4 = __ldg(reinterpret_cast<const float4*>(tab + k));
+          cs[k] = c4.x; cs[k + 1] = c4.y; cs[k + 2] = c4.z; cs[k + 3] = c4.w;
+        }
+      } else {  // the unit straddles an M-RoPE section boundary
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+          const int j = j0 + k;
+          const int s = j < p.sec_end0 ? 0 : (j < p.sec_end1 ? 1 : 2);
+          const float* tab = p.freqs + (size_t)pos[s] * p.R + 2 * j;
+          cs[2 * k] = __ldg(tab);
+          cs[2 * k + 1] = __ldg(tab + 1);
+        }
+      }
+      if (kInterleaved) {
+        float x[V];
+        load16(src + 2 * j0, x);
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+          const float a = x[2 * k], bb = x[2 * k + 1], c = cs[2 * k], s = cs[2 * k + 1];
+          x[2 * k] = fmaf(a, c, -bb * s);
+          x[2 * k + 1] = fmaf(bb, c, a * s);
+        }
+        store16(dst + 2 * j0, x);
+      } else {
+        float x1[V], x2[V];
+        load16(src + j0, x1);
+        load16(src + half + j0, x2);
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+          const float a = x1[k], bb = x2[k], c = cs[2 * k], s = cs[2 * k + 1];
+          x1[k] = fmaf(a, c, -bb * s);
+          x2[k] = fmaf(bb, c, a * s);
+        }
+        store16(dst + j0, x1);
+        store16(dst + half + j0, x2);
+      }
+    } else {  // V rows: copy into the cache slot
+      if (!page_ok) continue;
+      const int uv = u - q_units - k_units;
+      const int row = uv / (p.d / V);
+      const int off = (uv - row * (p.d / V)) * V;
+      src = vn + ((size_t)t * p.Hk + row) * p.d + off;
+      dst = vp + (((size_t)page * p.P + row_in_page) * p.Hk + row) * p.d + off;
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+    }
+  }
+}
+
+// freqs_cis[p][2j] = cos(p * theta^(-2j/R)), [2j+1] = sin(...), in fp64, rounded once.
+__global__ void freqs_cis_kernel(float* __restrict__ out, int32_t max_position, int32_t R,
+                                 double theta) {
+  const int half = R >> 1;
+  const long long n = (long long)max_position * half;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int pos = (int)(idx / half);
+    const int j = (int)(idx - (long long)pos * half);
+    const double omega = pow(theta, -2.0 * (double)j / (double)R);
+    double s, c;
+    sincos((double)pos * omega, &s, &c);
+    out[(size_t)pos * R + 2 * j] = __double2float_rn(c);
+    out[(size_t)pos * R + 2 * j + 1] = __double2float_rn(s);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_rope(const RopeParams& p, rpk_dtype dtype, bool interleaved,
+                        cudaStream_t stream) {
+  if (p.T == 0) return cudaSuccess;
+  dim3 grid(p.T), block(kThreads);
+  if (dtype == RPK_BF16) {
+    if (interleaved) rope_scatter_kernel<__nv_bfloat16, true><<<grid, block, 0, stream>>>(p);
+    else rope_scatter_kernel<__nv_bfloat16, false><<<grid, block, 0, stream>>>(p);
+  } else {
+    if (interleaved) rope_scatter_kernel<float, true><<<grid, block, 0, stream>>>(p);
+    else rope_scatter_kernel<float, false><<<grid, block, 0, stream>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_freqs_cis(float* out, int32_t max_position, int32_t rotary_dim, double theta,
+                             cudaStream_t stream) {
+  const long long n = (long long)max_position * (rotary_dim / 2);
+  if (n == 0) return cudaSuccess;
+  long long blocks = (n + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  freqs_cis_kernel<<<(unsigned)blocks, 256, 0, stream>>>(out, max_position, rotary_dim, theta);
+  return cudaGetLastError();
+}
+
+}  // namespace rpk
