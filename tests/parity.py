@@ -5,9 +5,10 @@ tolerances.
 Tolerances (written here once, used by every test):
 
 * RoPE, bf16: an output passes if |got - ref| <= 2 bf16 ulp of |ref|, or
-  |got - ref| <= 2^-22 (|a| + |b|) for its pair (a, b) -- the fp32 evaluation
-  bound of a*c - b*s when the result cancels. fp32 mode: 1e-5 relative, with
-  the same cancellation floor (2^-10 (|a| + |b|)).
+  |got - ref| <= 2^-22 (|a| + |b|) for its pair (a, b) -- twice the fp32
+  evaluation bound 2^-23 (|a| + |b|) of a*c - b*s, which governs when the
+  result cancels. fp32 mode: 1e-5 relative, with the same cancellation floor
+  2^-22 (|a| + |b|).
 * Attention: bf16 max-abs 2e-2 and mean-abs 2e-3; fp32 max-abs 1e-4, against
   the oracle's fp64 rows before rounding.
 * Cache placement, V bytes, untouched slots, channels >= rotary_dim and rows
@@ -116,7 +117,7 @@ def check_rope(got: torch.Tensor, ref: np.ndarray, x_in, rotary_dim: int, interl
     if dtype == "bf16":
         ok = (diff <= 2 * bf16_ulp(ref)) | (diff <= 2.0 ** -22 * ps)
     else:
-        ok = diff <= 1e-5 * np.maximum(np.abs(ref), 2.0 ** -10 * ps)
+        ok = diff <= np.maximum(1e-5 * np.abs(ref), 2.0 ** -22 * ps)
     assert np.all(np.isfinite(g)), f"{what}: non-finite output"
     bad = np.argwhere(~ok)
     assert bad.size == 0, (f"{what}: {len(bad)} outputs outside the RoPE tolerance, first at "
