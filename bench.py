@@ -46,8 +46,8 @@ L2_BYTES = 126 * 1024 * 1024
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="rpk", choices=["rpk", "reference"])
     ap.add_argument("--workload", default="llama3_8b_decode", choices=sorted(W.SPECS))
     ap.add_argument("--seed", type=int, default=0)
@@ -115,56 +115,92 @@ def load_traffic(kernel: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples during the timed region."""
+    """nvidia-smi clock / throttle samples taken while the timed region runs.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    The sampler is started (and seen to produce samples) before the warm-up;
+    samples carry nvidia-smi's timestamp and those inside the timed window
+    (widened by one sampling period on each side) are summarised. When the
+    timed region is shorter than the sampling period, the nearest samples are
+    used and the summary says so.
+    """
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 20
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.file = None
+        self.path = None
+        self.window = None
 
     def __enter__(self):
         try:
-            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            self.out = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=self.file, stderr=subprocess.DEVNULL)
+                 "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+            t0 = time.time()
+            while time.time() - t0 < 5.0 and os.path.getsize(self.path) == 0:
+                time.sleep(0.05)
         except OSError:
             self.proc = None
         return self
 
+    def mark(self, t_begin: float, t_end: float):
+        self.window = (t_begin, t_end)
+
     def __exit__(self, *exc):
         if self.proc is not None:
+            time.sleep(2 * self.PERIOD_MS / 1000.0)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+            self.out.close()
 
-    def summary(self):
-        if self.proc is None or self.file is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.file.flush()
+    def _rows(self):
+        import datetime
         rows = []
-        with open(self.file.name) as f:
+        with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.file.name)
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+                except ValueError:
+                    continue
+        return rows
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = self._rows()
+        os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        note = "samples inside the timed region"
+        sel = rows
+        if self.window is not None:
+            pad = self.PERIOD_MS / 1000.0
+            a, b = self.window
+            sel = [r for r in rows if a - pad <= r[0] <= b + pad]
+            if not sel:
+                mid = 0.5 * (a + b)
+                sel = sorted(rows, key=lambda r: abs(r[0] - mid))[:3]
+                note = (f"timed region ({1e3 * (b - a):.1f} ms) shorter than the sampling "
+                        f"period; nearest {len(sel)} samples")
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+        reasons = sorted({n for r in sel for n, v in zip(names, r[3]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[1] for r in sel),
+                "sm_max_mhz": max(r[2] for r in sel), "reasons": reasons,
+                "samples": len(sel), "note": note}
 
 
 # ------------------------------------------------------------- the GPU path
@@ -218,7 +254,7 @@ class Step:
         return 2
 
 
-def time_steps(step: Step, steps: int, warmup: int, world: int):
+def time_steps(step: Step, steps: int, warmup: int, world: int, clocks=None):
     """Per-step device times of the rope call and the attention call (ms)."""
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
@@ -230,6 +266,7 @@ def time_steps(step: Step, steps: int, warmup: int, world: int):
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    t_begin = time.time()
     start.record(stream)
     for i in range(steps):
         ev[i][0].record(stream)
@@ -239,6 +276,8 @@ def time_steps(step: Step, steps: int, warmup: int, world: int):
         ev[i][2].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.mark(t_begin, time.time())
     barrier(world)
     total_ms = start.elapsed_time(end)
     rope_ms = [e[0].elapsed_time(e[1]) for e in ev]
@@ -375,7 +414,7 @@ def main():
     kv_bytes = M.attention_kv_bytes(wl.q_lens, wl.kv_lens, sp.window, sp.n_kv_heads,
                                     sp.head_dim, elt)
     with ClockSampler(local) as clocks:
-        total_ms, rope_ms, attn_ms = time_steps(step, args.steps, args.warmup, world)
+        total_ms, rope_ms, attn_ms = time_steps(step, args.steps, args.warmup, world, clocks)
     clk = clocks.summary()
     step_ms = max_over_ranks(total_ms / args.steps, world)
     attn_ms_mean = max_over_ranks(statistics.mean(attn_ms), world)
@@ -398,9 +437,15 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        secs, kvb, toks, sample, threads = oracle_sample_time(wl)
-        cpu = {"value": kvb / secs / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-               "sample": sample, "seconds": secs}
+        # whole passes of the oracle over (a bounded sample of) the batch, ~10-30 s in all
+        total_s, total_b, passes, t_all = 0.0, 0, 0, time.perf_counter()
+        while passes < 1 or (time.perf_counter() - t_all < 10.0 and passes < 50):
+            secs, kvb, toks, sample, threads = oracle_sample_time(wl)
+            total_s += secs
+            total_b += kvb
+            passes += 1
+        cpu = {"value": total_b / total_s / 1e9, "unit": "GB/s", "cores": threads,
+               "kind": "oracle", "sample": f"{sample}; {passes} passes", "seconds": total_s}
 
     line = {
         "metric": "decode_attention_kv_GBps", "value": value, "unit": "GB/s",
