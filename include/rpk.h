@@ -191,6 +191,47 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
                                   int32_t max_kv_len, rpk_dtype dtype, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
+/*
+ * ragged_paged_attention_noalloc -- ragged_paged_attention for callers that
+ * cannot allocate device memory at call time. The pages have no counterpart
+ * for it; it is a convenience of this library.
+ *
+ * Who needs it: a serving engine that reserved all free HBM for its KV cache
+ * at start-up and refuses later allocations; a plugin inside a host
+ * framework that owns every allocator; a decode loop that cannot pay the
+ * implicit synchronisation of cudaMalloc. They cannot supply the workspace
+ * that ragged_paged_attention takes.
+ *
+ * Arguments and results are those of ragged_paged_attention, without the
+ * workspace. It runs the same split-KV decode kernels, so it takes only the
+ * decode shapes: dtype RPK_BF16 and max_q_len * (n_heads / n_kv_heads) <= 16.
+ * Other shapes return RPK_ERR_UNSUPPORTED.
+ *
+ * Scratch: the kernels' fp32 partials go to one array inside the library,
+ * RPK_NOALLOC_SCRATCH_BYTES (32 MiB) per GPU, held from the moment the
+ * library is loaded on that GPU until the process exits. Sizes whose
+ * partials would not fit (ragged_paged_attention_workspace_size(...) >
+ * RPK_NOALLOC_SCRATCH_BYTES) return RPK_ERR_WORKSPACE before anything is
+ * launched. The call itself never allocates (no cudaMalloc, no cudaFree).
+ *
+ * The first call on each device looks up the array's device address and
+ * caches it; make that first call before any stream capture on that device.
+ *
+ * All calls on a device share the one array, and it keeps whatever the last
+ * call left in it. Nothing in it needs to start at zero. Calls whose kernels
+ * overlap on the GPU (different streams, no ordering between them) race on
+ * the array and give wrong results: order them on one stream, or use
+ * ragged_paged_attention with separate workspaces.
+ */
+#define RPK_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+rpk_status ragged_paged_attention_noalloc(const void* q, const int32_t* q_row_offsets,
+                                          const int32_t* kv_lens,
+                                          const rpk_paged_kv* page_table, int32_t n_heads,
+                                          int32_t n_kv_heads, int32_t head_dim, float scale,
+                                          int32_t window, void* out, int32_t batch,
+                                          int32_t total_q_tokens, int32_t max_q_len,
+                                          int32_t max_kv_len, rpk_dtype dtype, void* stream);
+
 /* Static text for a status code. */
 const char* rpk_status_string(rpk_status status);
 

@@ -248,3 +248,40 @@ def ragged_paged_attention(q, q_row_offsets, kv_lens, page_table: PagedKVCache, 
         qp, off, kvl, C.byref(pk), int(n_heads), int(n_kv_heads), int(head_dim), float(scale),
         int(window), op, batch, T, int(max_q_len), int(max_kv_len), _dtype_code(q.dtype), ws,
         ws_bytes, _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def ragged_paged_attention_noalloc(q, q_row_offsets, kv_lens, page_table: PagedKVCache,
+                                   n_heads: int, n_kv_heads: int, head_dim: int,
+                                   scale: float | None, window: int, out, *, max_q_len: int,
+                                   max_kv_len: int, stream=None) -> None:
+    """ragged_paged_attention for callers that cannot allocate device memory.
+
+    Runs the split-KV decode path (bf16, max_q_len * group <= 16) with its
+    scratch in a fixed 32 MiB array inside the library instead of a
+    workspace; neither this function nor the C call allocates. Calls on one
+    device share that array, so do not let two of them overlap on the GPU.
+    """
+    L = lib()
+    fn = L.ragged_paged_attention_noalloc
+    if fn.argtypes is None:
+        _p, _i32 = C.c_void_p, C.c_int32
+        fn.argtypes = [_p, _p, _p, C.POINTER(PagedKV), _i32, _i32, _i32, C.c_float, _i32, _p,
+                       _i32, _i32, _i32, _i32, C.c_int, _p]
+        fn.restype = C.c_int
+    pk = page_table.struct()
+    if q.dim() != 3:
+        raise RpkError("q must be [tokens, n_heads, head_dim]")
+    qp = _dev(q, "q")
+    op = _dev(out, "out", q.dtype, 3)
+    if tuple(out.shape) != tuple(q.shape):
+        raise RpkError("out must have q's shape")
+    off = _dev(q_row_offsets, "q_row_offsets", torch.int32, 1)
+    kvl = _dev(kv_lens, "kv_lens", torch.int32, 1)
+    if scale is None:
+        scale = float(head_dim) ** -0.5
+    _check(fn(qp, off, kvl, C.byref(pk), int(n_heads), int(n_kv_heads), int(head_dim),
+              float(scale), int(window), op, int(kv_lens.shape[0]), int(q.shape[0]),
+              int(max_q_len), int(max_kv_len), _dtype_code(q.dtype), _stream(stream)))
