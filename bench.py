@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--impl", default="rpk", choices=["rpk", "reference"])
     ap.add_argument("--workload", default="llama3_8b_decode", choices=sorted(W.SPECS))
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -407,7 +409,8 @@ def main():
         return reference_arm(args, world, rank)
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    wl = W.make(args.workload, seed=args.seed + 1000 * rank)
+    over = {} if args.batch is None else {"batch": args.batch}
+    wl = W.make(args.workload, seed=args.seed + 1000 * rank, **over)
     sp = wl.spec
     step = Step(wl, device)
     elt = 2 if sp.dtype == "bf16" else 4
