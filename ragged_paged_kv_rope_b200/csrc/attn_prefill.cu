@@ -1,0 +1,484 @@
+// attn_prefill.cu -- ragged causal GQA attention over the paged cache on the
+// 5th-generation tensor cores (tcgen05), bf16 in, fp32 accumulate.
+//
+// Semantics: NumKong "Attention with a Pre-Packed KV-Cache" (row r of a
+// sequence with q_len rows and k_len keys sits at p = r + k_len - q_len and
+// sees keys [p - (window - 1), p]; rows that see no key are zeros), scores
+// scale * q.k (algenta scaled_dot_product_attention) and the flash
+// online-softmax running state (algenta flash_attention: running max,
+// running sum and output rescaled by e^(m_old - m_new), final divide).
+//
+// Tile: 128 rows x 128 keys. The 128 rows are the (token, query head) pairs
+// of one KV head's group, token-major, so the G query heads that share a KV
+// head share every K/V tile (tokens_per_tile = 128 / G). One CTA per
+// (query tile, KV head, sequence), heaviest tiles first.
+//
+// Warp roles (192 threads):
+//   warp 0     TMA producer: Q tile once, then K and V tiles of 128 keys into
+//              a 2-stage ring, one box per page segment (3-D map over the pool
+//              [pages * page_size, kv_heads, d], 128-byte swizzle, no multicast)
+//   warp 1     allocates TMEM (512 columns: S double buffer 2 x 128, O) and
+//              issues the MMAs from one thread: S_j = Q K_j^T into S[j % 2],
+//              then O += P_j V_j, with tcgen05.commit into mbarriers
+//   warps 2-5  softmax: thread r owns row r (TMEM lane r); loads S_j from
+//              TMEM, masks the band, keeps (m, l), writes P_j (bf16) into
+//              128-byte-swizzled shared memory as the A operand of P V, and
+//              rescales O in TMEM only when the running max grew by more than
+//              2^8 (the final O / l uses the same max, so this is exact);
+//              then normalises O and stores the rows.
+// Value rows at or past k_len are zeroed in shared memory before P V, so the
+// NaN sentinels of unused slots never meet a zero weight. Every mbarrier wait
+// is bounded; on a timeout the CTA raises RPK_DEVERR_TIMEOUT, drains its copies
+// and MMAs, frees TMEM and returns.
+#include "common.cuh"
+#include "kernels.h"
+#include "tcgen05.cuh"
+
+namespace rpk {
+
+int prefill_rows_per_tile(int group) { return group >= 1 && group <= 128 ? (128 / group) : 0; }
+
+namespace {
+
+constexpr int kBM = 128;   // rows per tile (MMA M)
+constexpr int kBN = 128;   // keys per tile
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows > 2^8
+
+template <int D>
+struct Cfg {
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kQBytes = kBM * D * 2;
+  static constexpr int kKVBytes = kBN * D * 2;
+  static constexpr int kPBytes = kBM * kBN * 2;
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + kQBytes;
+  static constexpr int kVOff = kKOff + 2 * kKVBytes;
+  static constexpr int kPOff = kVOff + 2 * kKVBytes;
+  // At least half the SM's shared memory, so that one CTA holds the SM's TMEM.
+  static constexpr int kSmemBytes =
+      (kPOff + kPBytes + 1024) > 118 * 1024 ? (kPOff + kPBytes + 1024) : 118 * 1024;
+  static constexpr uint32_t kOCol = 2 * kBN;
+  static_assert(kOCol + D <= kTmemCols, "TMEM budget");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t k_full[2];
+  uint64_t v_full[2];
+  uint64_t kv_empty[2];
+  uint64_t s_full[2];
+  uint64_t p_full;
+  uint64_t o_done;
+  uint64_t drain;
+};
+
+// A CTA that gives up on a wait publishes RPK_DEVERR_TIMEOUT in the error
+// word; every other CTA of the launch (and of later launches, until the caller
+// clears the word) sees it and stops early instead of waiting out its own
+// bound, so a broken launch ends in about one bound, not one per CTA.
+__device__ __forceinline__ bool timed_out_elsewhere(const int32_t* error_word) {
+  return error_word &&
+         (*reinterpret_cast<const volatile int32_t*>(error_word) & (int32_t)RPK_DEVERR_TIMEOUT);
+}
+
+// Bounded wait by one thread; false on timeout or abort.
+__device__ __forceinline__ bool thread_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                            const int32_t* error_word) {
+  const uint32_t a = smem_u32(bar);
+  const unsigned long long t0 = global_timer_ns();
+#pragma unroll 1
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(a, parity)) return true;
+    if ((it & 63u) == 63u) {
+      if (*abort || timed_out_elsewhere(error_word)) return false;
+      if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
+    }
+  }
+}
+
+// Bounded wait shared by the whole warp: every lane polls (so each lane has
+// acquired the phase) and the lanes agree on the outcome.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          const int32_t* error_word) {
+  const bool ok = thread_wait(bar, parity, abort, error_word);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void do_abort(volatile int* abort, int32_t* error_word) {
+  if (!*abort) {
+    *abort = 1;
+    raise_error(error_word, RPK_DEVERR_TIMEOUT);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_prefill_kernel(const AttnParams p, const __grid_constant__ CUtensorMap q_map,
+                        const __grid_constant__ CUtensorMap k_map,
+                        const __grid_constant__ CUtensorMap v_map, const int tpt,
+                        const int n_qtiles) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ Bars bars;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  volatile int* abort = &abort_sh;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = n_qtiles - 1 - (int)blockIdx.x;  // heaviest (latest) tiles first
+  const int kvh = blockIdx.y, b = blockIdx.z;
+  const int q0 = __ldg(p.offsets + b);
+  const int q_len = __ldg(p.offsets + b + 1) - q0;
+  const int k_len = __ldg(p.kv_lens + b);
+  if (q_len > p.max_q_len || k_len < 0 || k_len > p.max_kv_len) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0) raise_error(p.error_word, RPK_DEVERR_LENGTH);
+    return;
+  }
+  const int t_begin = qt * tpt;
+  if (t_begin >= q_len) return;
+  if (timed_out_elsewhere(p.error_word)) return;
+  const int t_end = min(q_len, t_begin + tpt);
+  const int G = p.G;
+  const int rows_used = tpt * G;
+
+  // Keys any row of this tile sees, in whole key tiles.
+  const int p_first = t_begin + k_len - q_len;
+  const int p_last = (t_end - 1) + k_len - q_len;
+  const int lo_first = p.window > 0 ? max(0, p_first - p.window + 1) : 0;
+  const int hi_all = min(p_last, k_len - 1);
+  int j_begin = 0, n_tiles = 0;
+  if (hi_all >= lo_first) {
+    j_begin = lo_first / kBN;
+    n_tiles = hi_all / kBN + 1 - j_begin;
+  }
+
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t q_s = sbase + C::kQOff;
+  auto k_s = [&](int s) { return sbase + C::kKOff + s * C::kKVBytes; };
+  auto v_s = [&](int s) { return sbase + C::kVOff + s * C::kKVBytes; };
+  const uint32_t p_s = sbase + C::kPOff;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars.q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars.k_full[s], 1);
+      mbar_init(&bars.v_full[s], 1);
+      mbar_init(&bars.kv_empty[s], 1);
+      mbar_init(&bars.s_full[s], 1);
+    }
+    mbar_init(&bars.p_full, 128);
+    mbar_init(&bars.o_done, 1);
+    mbar_init(&bars.drain, 1);
+    abort_sh = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = tmem_base_sh;
+  const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&q_map);
+      prefetch_tensormap(&k_map);
+      prefetch_tensormap(&v_map);
+      const uint32_t q_box_bytes = 128u * (uint32_t)rows_used;
+      mbar_arrive_expect_tx(&bars.q_full, C::kBoxes * q_box_bytes);
+#pragma unroll
+      for (int bx = 0; bx < C::kBoxes; ++bx)
+        tma_load_3d(smem + C::kQOff + bx * (kBM * 128), &q_map, bx * 64, kvh * G, q0 + t_begin,
+                    &bars.q_full);
+      const int box_rows = p.P < kBN ? p.P : kBN;
+      const uint32_t seg_bytes = (uint32_t)box_rows * 128u * C::kBoxes;
+      int issued = 0;
+      for (int i = 0; i < n_tiles; ++i) {
+        const int s = i & 1;
+        if (i >= 2) {
+          // bounded single-thread wait (the rest of warp 0 is idle)
+          if (!thread_wait(&bars.kv_empty[s], ((i >> 1) & 1) ^ 1, abort, p.error_word)) {
+            do_abort(abort, p.error_word);
+            break;
+          }
+        }
+        const int key0 = (j_begin + i) * kBN;
+        uint32_t bytes = 0;
+        for (int r = 0; r < kBN; r += box_rows) {
+          const int key = key0 + r;
+          if (key >= k_len) break;
+          const int pi = key / p.P;
+          const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
+          if (page >= 0 && page < p.num_pages) bytes += seg_bytes;
+        }
+        mbar_arrive_expect_tx(&bars.k_full[s], bytes);
+        mbar_arrive_expect_tx(&bars.v_full[s], bytes);
+        for (int r = 0; r < kBN; r += box_rows) {
+          const int key = key0 + r;
+          if (key >= k_len) break;
+          const int pi = key / p.P;
+          const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
+          if (page < 0 || page >= p.num_pages) {
+            raise_error(p.error_word, RPK_DEVERR_PAGE);
+            continue;
+          }
+          const int grow = page * p.P + (key - pi * p.P);
+#pragma unroll
+          for (int bx = 0; bx < C::kBoxes; ++bx) {
+            tma_load_3d(smem + C::kKOff + s * C::kKVBytes + bx * (kBN * 128) + r * 128, &k_map,
+                        bx * 64, kvh, grow, &bars.k_full[s]);
+            tma_load_3d(smem + C::kVOff + s * C::kKVBytes + bx * (kBN * 128) + r * 128, &v_map,
+                        bx * 64, kvh, grow, &bars.v_full[s]);
+          }
+        }
+        ++issued;
+      }
+      // Never leave with copies in flight.
+      mbar_wait(&bars.q_full, 0);
+      for (int i = max(0, issued - 2); i < issued; ++i) {
+        mbar_wait(&bars.k_full[i & 1], (i >> 1) & 1);
+        mbar_wait(&bars.v_full[i & 1], (i >> 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(kBM, kBN, 0);
+    constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(kBM, D, 1);
+    bool ok = warp_wait(&bars.q_full, 0, abort, p.error_word);
+    tc::fence_after_sync();
+    auto issue_s = [&](int i) -> bool {
+      const int s = i & 1;
+      if (!warp_wait(&bars.k_full[s], (i >> 1) & 1, abort, p.error_word)) return false;
+      tc::fence_after_sync();
+      if (lane == 0) {
+        const uint32_t d_tmem = tmem + (uint32_t)(s * kBN);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
+          const uint32_t koff = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
+          tc::mma_ss(d_tmem, tc::smem_desc_sw128(q_s + off, 16, 1024),
+                     tc::smem_desc_sw128(k_s(s) + koff, 16, 1024), idesc_qk, kk > 0);
+        }
+        tc::commit(smem_u32(&bars.s_full[s]));
+      }
+      __syncwarp();
+      return true;
+    };
+    if (ok && n_tiles > 0) ok = issue_s(0);
+    for (int i = 0; ok && i < n_tiles; ++i) {
+      const int s = i & 1;
+      if (i + 1 < n_tiles && !issue_s(i + 1)) { ok = false; break; }
+      if (!warp_wait(&bars.p_full, i & 1, abort, p.error_word)) { ok = false; break; }
+      if (!warp_wait(&bars.v_full[s], (i >> 1) & 1, abort, p.error_word)) { ok = false; break; }
+      tc::fence_after_sync();
+      const int key0 = (j_begin + i) * kBN;
+      if (key0 + kBN > k_len) {
+        // zero value rows at or past k_len
+        const int r0 = max(0, k_len - key0);
+        const int chunks = (kBN - r0) * C::kBoxes * 8;
+        for (int idx = lane; idx < chunks; idx += 32) {
+          const int ch = idx & 7;
+          const int rb = idx >> 3;
+          const int bx = rb % C::kBoxes;
+          const int r = r0 + rb / C::kBoxes;
+          uint8_t* dst = smem + C::kVOff + s * C::kKVBytes + bx * (kBN * 128) + r * 128 + ch * 16;
+          *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      if (lane == 0) {
+        const uint32_t d_tmem = tmem + C::kOCol;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint32_t poff = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
+          tc::mma_ss(d_tmem, tc::smem_desc_sw128(p_s + poff, 16, 1024),
+                     tc::smem_desc_sw128(v_s(s) + kk * (16 * 128), kBN * 128, 1024), idesc_pv,
+                     (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::commit(smem_u32(&bars.o_done));
+        tc::commit(smem_u32(&bars.kv_empty[s]));
+      }
+      __syncwarp();
+    }
+    if (!ok) do_abort(abort, p.error_word);
+    // Drain: every MMA issued above has completed before TMEM is freed.
+    if (lane == 0) tc::commit(smem_u32(&bars.drain));
+    __syncwarp();
+    if (!warp_wait(&bars.drain, 0, abort, p.error_word)) mbar_wait(&bars.drain, 0);
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int qw = warp & 3;             // TMEM lane quarter of this warp
+    const int r = qw * 32 + lane;        // row of this thread
+    const int t_local = r / G;
+    const int tok = t_begin + t_local;
+    const bool row_ok = r < rows_used && tok < q_len;
+    const int pos = tok + k_len - q_len;
+    const int lo = p.window > 0 ? pos - p.window + 1 : 0;
+    const int hi = pos;
+    const uint32_t lane_base = (uint32_t)(qw * 32) << 16;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    float v[kBN];
+    for (int i = 0; i < n_tiles; ++i) {
+      const int buf = i & 1;
+      if (!warp_wait(&bars.s_full[buf], (i >> 1) & 1, abort, p.error_word)) { ok = false; break; }
+      tc::fence_after_sync();
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c)
+        tc::tmem_ld32(tmem + lane_base + (uint32_t)(buf * kBN + c * 32), v + c * 32);
+      tc::tmem_wait_ld();
+      const int key0 = (j_begin + i) * kBN;
+      const bool full = row_ok && key0 >= lo && key0 + kBN - 1 <= hi;
+      float mx = -INFINITY;
+      if (full) {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) {
+          v[c] *= p.scale_log2;
+          mx = fmaxf(mx, v[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) {
+          const int key = key0 + c;
+          const bool vis = row_ok && key >= lo && key <= hi;
+          v[c] = vis ? v[c] * p.scale_log2 : -INFINITY;
+          mx = fmaxf(mx, v[c]);
+        }
+      }
+      // Running max: taken at once while empty, else only when it grows by
+      // more than the threshold (then O and l are rescaled).
+      float alpha = 1.f;
+      bool rescale = false;
+      if (m == -INFINITY) {
+        m = mx;
+      } else if (mx > m + kRescaleThreshold) {
+        alpha = fast_exp2(m - mx);
+        m = mx;
+        rescale = true;
+      }
+      // P buffer and O are free once P_{i-1} V_{i-1} has completed.
+      if (i > 0) {
+        if (!warp_wait(&bars.o_done, (i - 1) & 1, abort, p.error_word)) { ok = false; break; }
+        tc::fence_after_sync();
+        if (__any_sync(0xffffffffu, rescale)) {
+          float o[32];
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            const uint32_t ta = tmem + lane_base + C::kOCol + c * 32;
+            tc::tmem_ld32(ta, o);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tc::tmem_st32(ta, o);
+          }
+          tc::tmem_wait_st();
+        }
+      }
+      l *= alpha;
+      float rs = 0.f;
+      const bool live = m != -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kBN; ++c) {
+        const float w = live ? fast_exp2(v[c] - m) : 0.f;
+        v[c] = w;
+        rs += w;
+      }
+      l += rs;
+      // P row r as bf16, 128-byte swizzled K-major (two 64-key boxes).
+#pragma unroll
+      for (int c8 = 0; c8 < kBN / 8; ++c8) {
+        uint4 pk;
+        pk.x = pack_bf16x2(v[c8 * 8 + 0], v[c8 * 8 + 1]);
+        pk.y = pack_bf16x2(v[c8 * 8 + 2], v[c8 * 8 + 3]);
+        pk.z = pack_bf16x2(v[c8 * 8 + 4], v[c8 * 8 + 5]);
+        pk.w = pack_bf16x2(v[c8 * 8 + 6], v[c8 * 8 + 7]);
+        uint8_t* dst = smem + C::kPOff + (c8 >> 3) * (kBM * 128) + swz128(r, c8 & 7);
+        *reinterpret_cast<uint4*>(dst) = pk;
+      }
+      fence_proxy_async_smem();
+      tc::fence_before_sync();
+      mbar_arrive(&bars.p_full);
+    }
+    if (!ok) do_abort(abort, p.error_word);
+    // ------------------------------------------------------------ epilogue
+    bool have_o = n_tiles > 0;
+    if (have_o) {
+      have_o = warp_wait(&bars.o_done, (n_tiles - 1) & 1, abort, p.error_word);
+      tc::fence_after_sync();
+    }
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+    const size_t orow = ((size_t)(q0 + tok) * p.H + (size_t)kvh * G + (r % G)) * D;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      float o[32];
+      if (have_o) {
+        tc::tmem_ld32(tmem + lane_base + C::kOCol + c * 32, o);
+        tc::tmem_wait_ld();
+      }
+      if (row_ok) {
+#pragma unroll
+        for (int e8 = 0; e8 < 4; ++e8) {
+          uint4 pk;
+          if (have_o && l > 0.f) {
+            pk.x = pack_bf16x2(o[e8 * 8 + 0] * inv, o[e8 * 8 + 1] * inv);
+            pk.y = pack_bf16x2(o[e8 * 8 + 2] * inv, o[e8 * 8 + 3] * inv);
+            pk.z = pack_bf16x2(o[e8 * 8 + 4] * inv, o[e8 * 8 + 5] * inv);
+            pk.w = pack_bf16x2(o[e8 * 8 + 6] * inv, o[e8 * 8 + 7] * inv);
+          } else {
+            pk = make_uint4(0, 0, 0, 0);
+          }
+          *reinterpret_cast<uint4*>(out + orow + c * 32 + e8 * 8) = pk;
+        }
+      }
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch_d(const AttnParams& p, const CUtensorMap& q_map, const CUtensorMap& k_map,
+                     const CUtensorMap& v_map, cudaStream_t stream) {
+  using C = Cfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int tpt = prefill_rows_per_tile(p.G);
+  const int n_qtiles = (p.max_q_len + tpt - 1) / tpt;
+  if (n_qtiles == 0) return cudaSuccess;
+  dim3 grid(n_qtiles, p.Hk, p.batch);
+  attn_prefill_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(p, q_map, k_map, v_map, tpt,
+                                                                     n_qtiles);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_prefill(const AttnParams& p, const CUtensorMap& q_map,
+                                const CUtensorMap& k_map, const CUtensorMap& v_map,
+                                cudaStream_t stream) {
+  if ((long long)p.T * p.H == 0 || p.batch == 0) return cudaSuccess;
+  switch (p.d) {
+    case 64: return launch_d<64>(p, q_map, k_map, v_map, stream);
+    case 128: return launch_d<128>(p, q_map, k_map, v_map, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace rpk

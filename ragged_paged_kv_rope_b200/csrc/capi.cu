@@ -226,7 +226,21 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
     return cuda_status(rpk::launch_attn_decode(p, k_map, v_map, plan, ws, s));
   }
 
-  // Prefill shapes: CUDA-core kernel until the tensor-core kernel takes them.
+  // Prefill shapes: tcgen05 kernel for head_dim 64 / 128 and groups up to 128.
+  const int tpt = rpk::prefill_rows_per_tile(p.G);
+  if ((head_dim == 64 || head_dim == 128) && tpt > 0) {
+    CUtensorMap q_map, k_map, v_map;
+    const int32_t box_rows = p.P < 128 ? p.P : 128;
+    const int64_t pool_rows = (int64_t)p.num_pages * p.P;
+    st = encode_rows_map(&q_map, q, head_dim, n_heads, total_q_tokens, p.G, tpt);
+    if (st != RPK_OK) return st;
+    st = encode_rows_map(&k_map, p.k_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
+    if (st != RPK_OK) return st;
+    st = encode_rows_map(&v_map, p.v_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
+    if (st != RPK_OK) return st;
+    return cuda_status(rpk::launch_attn_prefill(p, q_map, k_map, v_map, s));
+  }
+  // head_dim 256 (or groups above 128): CUDA-core kernel.
   return cuda_status(rpk::launch_attn_simt(p, dtype, s));
 }
 

@@ -68,6 +68,13 @@ __device__ __forceinline__ void store16(T* p, const float* in) {
   *reinterpret_cast<uint4*>(p) = raw;
 }
 
+// 2^x by the MUFU approximation (relative error ~2^-22; 2^-inf = +0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
