@@ -15,17 +15,20 @@
 //
 // Warp roles (192 threads):
 //   warp 0     TMA producer: Q tile once, then K and V tiles of 128 keys into
-//              a 2-stage ring, one box per page segment (3-D map over the pool
-//              [pages * page_size, kv_heads, d], 128-byte swizzle, no multicast)
-//   warp 1     allocates TMEM (512 columns: S double buffer 2 x 128, O) and
-//              issues the MMAs from one thread: S_j = Q K_j^T into S[j % 2],
-//              then O += P_j V_j, with tcgen05.commit into mbarriers
-//   warps 2-5  softmax: thread r owns row r (TMEM lane r); loads S_j from
-//              TMEM, masks the band, keeps (m, l), writes P_j (bf16) into
-//              128-byte-swizzled shared memory as the A operand of P V, and
-//              rescales O in TMEM only when the running max grew by more than
-//              2^8 (the final O / l uses the same max, so this is exact);
-//              then normalises O and stores the rows.
+//              a ring of shared-memory stages, one box per page segment (3-D
+//              map over the pool [pages * page_size, kv_heads, d], 128-byte
+//              swizzle, no multicast)
+//   warp 1     allocates TMEM (512 columns: S0, S1, O, P0, P1) and issues the
+//              MMAs from one thread: S_j = Q K_j^T into S[j % 2] (both operands
+//              from shared memory), then O += P_j V_j with P_j read from TMEM
+//              (P[j % 2]) and V_j from shared memory as an MN-major operand
+//   warps 2-5  softmax: thread r owns row r (TMEM lane r); loads S_j, frees the
+//              S buffer, masks the band, keeps (m, l) in log2 units, writes P_j
+//              as packed bf16 pairs into P[j % 2] with tcgen05.st. O is
+//              rescaled in TMEM only when the running max grew by more than
+//              2^8 (the final O / l uses the same max, so this is exact), and
+//              only then does the softmax wait for the previous P V. Finally it
+//              normalises O and stores the rows.
 // Value rows at or past k_len are zeroed in shared memory before P V, so the
 // NaN sentinels of unused slots never meet a zero weight. Every mbarrier wait
 // is bounded; on a timeout the CTA raises RPK_DEVERR_TIMEOUT, drains its copies
@@ -49,29 +52,32 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max
 template <int D>
 struct Cfg {
   static constexpr int kBoxes = D / 64;
+  static constexpr int kStages = D == 128 ? 3 : 4;   // K/V ring depth
   static constexpr int kQBytes = kBM * D * 2;
   static constexpr int kKVBytes = kBN * D * 2;
-  static constexpr int kPBytes = kBM * kBN * 2;
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kQBytes;
-  static constexpr int kVOff = kKOff + 2 * kKVBytes;
-  static constexpr int kPOff = kVOff + 2 * kKVBytes;
+  static constexpr int kVOff = kKOff + kStages * kKVBytes;
+  static constexpr int kEnd = kVOff + kStages * kKVBytes + 1024;
   // At least half the SM's shared memory, so that one CTA holds the SM's TMEM.
-  static constexpr int kSmemBytes =
-      (kPOff + kPBytes + 1024) > 118 * 1024 ? (kPOff + kPBytes + 1024) : 118 * 1024;
+  static constexpr int kSmemBytes = kEnd > 118 * 1024 ? kEnd : 118 * 1024;
+  // TMEM columns: S0, S1 (fp32, 128 each), O (fp32, D), P0, P1 (bf16 pairs, 64 each)
+  static constexpr uint32_t kSCol = 0;
   static constexpr uint32_t kOCol = 2 * kBN;
-  static_assert(kOCol + D <= kTmemCols, "TMEM budget");
+  static constexpr uint32_t kPCol = kOCol + D;
+  static_assert(kPCol + 2 * (kBN / 2) <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
 struct Bars {
   uint64_t q_full;
-  uint64_t k_full[2];
-  uint64_t v_full[2];
-  uint64_t kv_empty[2];
+  uint64_t k_full[4];
+  uint64_t v_full[4];
+  uint64_t kv_empty[4];
   uint64_t s_full[2];
-  uint64_t p_full;
-  uint64_t o_done;
+  uint64_t s_free[2];
+  uint64_t p_full[2];
+  uint64_t pv_done[2];
   uint64_t drain;
 };
 
@@ -128,13 +134,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort = &abort_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = n_qtiles - 1 - (int)blockIdx.x;  // heaviest (latest) tiles first
-  const int kvh = blockIdx.y, b = blockIdx.z;
+  // The q-tile index is the slowest grid dimension, reversed: the first waves
+  // hold the last (heaviest) tile of every (sequence, KV head), so the long
+  // tiles start first and the short ones fill the tail.
+  const int qt = n_qtiles - 1 - (int)blockIdx.z;
+  const int kvh = blockIdx.x, b = blockIdx.y;
   const int q0 = __ldg(p.offsets + b);
   const int q_len = __ldg(p.offsets + b + 1) - q0;
   const int k_len = __ldg(p.kv_lens + b);
   if (q_len > p.max_q_len || k_len < 0 || k_len > p.max_kv_len) {
-    if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0) raise_error(p.error_word, RPK_DEVERR_LENGTH);
+    if (threadIdx.x == 0 && blockIdx.z == 0 && kvh == 0) raise_error(p.error_word, RPK_DEVERR_LENGTH);
     return;
   }
   const int t_begin = qt * tpt;
@@ -155,24 +164,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     n_tiles = hi_all / kBN + 1 - j_begin;
   }
 
+  constexpr int S = C::kStages;
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t q_s = sbase + C::kQOff;
-  auto k_s = [&](int s) { return sbase + C::kKOff + s * C::kKVBytes; };
-  auto v_s = [&](int s) { return sbase + C::kVOff + s * C::kKVBytes; };
-  const uint32_t p_s = sbase + C::kPOff;
+  auto k_s = [&](int st) { return sbase + C::kKOff + st * C::kKVBytes; };
+  auto v_s = [&](int st) { return sbase + C::kVOff + st * C::kKVBytes; };
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars.k_full[s], 1);
-      mbar_init(&bars.v_full[s], 1);
-      mbar_init(&bars.kv_empty[s], 1);
-      mbar_init(&bars.s_full[s], 1);
+    for (int st = 0; st < S; ++st) {
+      mbar_init(&bars.k_full[st], 1);
+      mbar_init(&bars.v_full[st], 1);
+      mbar_init(&bars.kv_empty[st], 1);
     }
-    mbar_init(&bars.p_full, 128);
-    mbar_init(&bars.o_done, 1);
+    for (int bb = 0; bb < 2; ++bb) {
+      mbar_init(&bars.s_full[bb], 1);
+      mbar_init(&bars.s_free[bb], 128);
+      mbar_init(&bars.p_full[bb], 128);
+      mbar_init(&bars.pv_done[bb], 1);
+    }
     mbar_init(&bars.drain, 1);
     abort_sh = 0;
     fence_barrier_init();
@@ -203,13 +215,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t seg_bytes = (uint32_t)box_rows * 128u * C::kBoxes;
       int issued = 0;
       for (int i = 0; i < n_tiles; ++i) {
-        const int s = i & 1;
-        if (i >= 2) {
-          // bounded single-thread wait (the rest of warp 0 is idle)
-          if (!thread_wait(&bars.kv_empty[s], ((i >> 1) & 1) ^ 1, abort, p.error_word)) {
-            do_abort(abort, p.error_word);
-            break;
-          }
+        const int st = i % S;
+        if (i >= S &&
+            !thread_wait(&bars.kv_empty[st], ((i / S) & 1) ^ 1, abort, p.error_word)) {
+          do_abort(abort, p.error_word);
+          break;
         }
         const int key0 = (j_begin + i) * kBN;
         uint32_t bytes = 0;
@@ -220,8 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
           if (page >= 0 && page < p.num_pages) bytes += seg_bytes;
         }
-        mbar_arrive_expect_tx(&bars.k_full[s], bytes);
-        mbar_arrive_expect_tx(&bars.v_full[s], bytes);
+        mbar_arrive_expect_tx(&bars.k_full[st], bytes);
+        mbar_arrive_expect_tx(&bars.v_full[st], bytes);
         for (int r = 0; r < kBN; r += box_rows) {
           const int key = key0 + r;
           if (key >= k_len) break;
@@ -234,19 +244,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int grow = page * p.P + (key - pi * p.P);
 #pragma unroll
           for (int bx = 0; bx < C::kBoxes; ++bx) {
-            tma_load_3d(smem + C::kKOff + s * C::kKVBytes + bx * (kBN * 128) + r * 128, &k_map,
-                        bx * 64, kvh, grow, &bars.k_full[s]);
-            tma_load_3d(smem + C::kVOff + s * C::kKVBytes + bx * (kBN * 128) + r * 128, &v_map,
-                        bx * 64, kvh, grow, &bars.v_full[s]);
+            tma_load_3d(smem + C::kKOff + st * C::kKVBytes + bx * (kBN * 128) + r * 128, &k_map,
+                        bx * 64, kvh, grow, &bars.k_full[st]);
+            tma_load_3d(smem + C::kVOff + st * C::kKVBytes + bx * (kBN * 128) + r * 128, &v_map,
+                        bx * 64, kvh, grow, &bars.v_full[st]);
           }
         }
         ++issued;
       }
       // Never leave with copies in flight.
       mbar_wait(&bars.q_full, 0);
-      for (int i = max(0, issued - 2); i < issued; ++i) {
-        mbar_wait(&bars.k_full[i & 1], (i >> 1) & 1);
-        mbar_wait(&bars.v_full[i & 1], (i >> 1) & 1);
+      for (int i = max(0, issued - S); i < issued; ++i) {
+        mbar_wait(&bars.k_full[i % S], (i / S) & 1);
+        mbar_wait(&bars.v_full[i % S], (i / S) & 1);
       }
     }
   } else if (warp == 1) {
@@ -256,29 +266,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = warp_wait(&bars.q_full, 0, abort, p.error_word);
     tc::fence_after_sync();
     auto issue_s = [&](int i) -> bool {
-      const int s = i & 1;
-      if (!warp_wait(&bars.k_full[s], (i >> 1) & 1, abort, p.error_word)) return false;
+      const int st = i % S;
+      if (!warp_wait(&bars.k_full[st], (i / S) & 1, abort, p.error_word)) return false;
       tc::fence_after_sync();
       if (lane == 0) {
-        const uint32_t d_tmem = tmem + (uint32_t)(s * kBN);
+        const uint32_t d_tmem = tmem + C::kSCol + (uint32_t)((i & 1) * kBN);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
+          const uint32_t qoff = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
           const uint32_t koff = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-          tc::mma_ss(d_tmem, tc::smem_desc_sw128(q_s + off, 16, 1024),
-                     tc::smem_desc_sw128(k_s(s) + koff, 16, 1024), idesc_qk, kk > 0);
+          tc::mma_ss(d_tmem, tc::smem_desc_sw128(q_s + qoff, 16, 1024),
+                     tc::smem_desc_sw128(k_s(st) + koff, 16, 1024), idesc_qk, kk > 0);
         }
-        tc::commit(smem_u32(&bars.s_full[s]));
+        tc::commit(smem_u32(&bars.s_full[i & 1]));
       }
       __syncwarp();
       return true;
     };
     if (ok && n_tiles > 0) ok = issue_s(0);
     for (int i = 0; ok && i < n_tiles; ++i) {
-      const int s = i & 1;
-      if (i + 1 < n_tiles && !issue_s(i + 1)) { ok = false; break; }
-      if (!warp_wait(&bars.p_full, i & 1, abort, p.error_word)) { ok = false; break; }
-      if (!warp_wait(&bars.v_full[s], (i >> 1) & 1, abort, p.error_word)) { ok = false; break; }
+      const int st = i % S, pb = i & 1;
+      if (i + 1 < n_tiles) {
+        // S buffer (i+1)%2 is free once the softmax has read S_{i-1} from it.
+        if (i >= 1 && !warp_wait(&bars.s_free[(i + 1) & 1], ((i - 1) >> 1) & 1, abort,
+                                 p.error_word)) { ok = false; break; }
+        if (!issue_s(i + 1)) { ok = false; break; }
+      }
+      if (!warp_wait(&bars.p_full[pb], (i >> 1) & 1, abort, p.error_word)) { ok = false; break; }
+      if (!warp_wait(&bars.v_full[st], (i / S) & 1, abort, p.error_word)) { ok = false; break; }
       tc::fence_after_sync();
       const int key0 = (j_begin + i) * kBN;
       if (key0 + kBN > k_len) {
@@ -290,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int rb = idx >> 3;
           const int bx = rb % C::kBoxes;
           const int r = r0 + rb / C::kBoxes;
-          uint8_t* dst = smem + C::kVOff + s * C::kKVBytes + bx * (kBN * 128) + r * 128 + ch * 16;
+          uint8_t* dst = smem + C::kVOff + st * C::kKVBytes + bx * (kBN * 128) + r * 128 + ch * 16;
           *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
@@ -298,15 +313,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (lane == 0) {
         const uint32_t d_tmem = tmem + C::kOCol;
+        const uint32_t a_tmem = tmem + C::kPCol + (uint32_t)(pb * (kBN / 2));
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint32_t poff = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-          tc::mma_ss(d_tmem, tc::smem_desc_sw128(p_s + poff, 16, 1024),
-                     tc::smem_desc_sw128(v_s(s) + kk * (16 * 128), kBN * 128, 1024), idesc_pv,
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          tc::mma_ts(d_tmem, a_tmem + kk * 8,
+                     tc::smem_desc_sw128(v_s(st) + kk * (16 * 128), kBN * 128, 1024), idesc_pv,
                      (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc::commit(smem_u32(&bars.o_done));
-        tc::commit(smem_u32(&bars.kv_empty[s]));
+        tc::commit(smem_u32(&bars.pv_done[pb]));
+        tc::commit(smem_u32(&bars.kv_empty[st]));
       }
       __syncwarp();
     }
@@ -326,35 +340,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lo = p.window > 0 ? pos - p.window + 1 : 0;
     const int hi = pos;
     const uint32_t lane_base = (uint32_t)(qw * 32) << 16;
-    float m = -INFINITY, l = 0.f;
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY, l = 0.f;        // running max (log2 units) and sum
     bool ok = true;
     float v[kBN];
     for (int i = 0; i < n_tiles; ++i) {
-      const int buf = i & 1;
-      if (!warp_wait(&bars.s_full[buf], (i >> 1) & 1, abort, p.error_word)) { ok = false; break; }
+      const int pb = i & 1;
+      if (!warp_wait(&bars.s_full[pb], (i >> 1) & 1, abort, p.error_word)) { ok = false; break; }
       tc::fence_after_sync();
 #pragma unroll
       for (int c = 0; c < kBN / 32; ++c)
-        tc::tmem_ld32(tmem + lane_base + (uint32_t)(buf * kBN + c * 32), v + c * 32);
+        tc::tmem_ld32(tmem + lane_base + C::kSCol + (uint32_t)(pb * kBN + c * 32), v + c * 32);
       tc::tmem_wait_ld();
+      tc::fence_before_sync();
+      mbar_arrive(&bars.s_free[pb]);
       const int key0 = (j_begin + i) * kBN;
-      const bool full = row_ok && key0 >= lo && key0 + kBN - 1 <= hi;
-      float mx = -INFINITY;
-      if (full) {
-#pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          v[c] *= p.scale_log2;
-          mx = fmaxf(mx, v[c]);
-        }
-      } else {
+      if (!(row_ok && key0 >= lo && key0 + kBN - 1 <= hi)) {
 #pragma unroll
         for (int c = 0; c < kBN; ++c) {
           const int key = key0 + c;
-          const bool vis = row_ok && key >= lo && key <= hi;
-          v[c] = vis ? v[c] * p.scale_log2 : -INFINITY;
-          mx = fmaxf(mx, v[c]);
+          if (!(row_ok && key >= lo && key <= hi)) v[c] = -INFINITY;
         }
       }
+      float mx = v[0];
+#pragma unroll
+      for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, v[c]);
+      mx *= sl2;  // scale > 0: max of the scaled scores
       // Running max: taken at once while empty, else only when it grows by
       // more than the threshold (then O and l are rescaled).
       float alpha = 1.f;
@@ -366,54 +377,58 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = mx;
         rescale = true;
       }
-      // P buffer and O are free once P_{i-1} V_{i-1} has completed.
-      if (i > 0) {
-        if (!warp_wait(&bars.o_done, (i - 1) & 1, abort, p.error_word)) { ok = false; break; }
-        tc::fence_after_sync();
-        if (__any_sync(0xffffffffu, rescale)) {
-          float o[32];
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            const uint32_t ta = tmem + lane_base + C::kOCol + c * 32;
-            tc::tmem_ld32(ta, o);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tc::tmem_st32(ta, o);
-          }
-          tc::tmem_wait_st();
+      if (i > 0 && __any_sync(0xffffffffu, rescale)) {
+        // O holds P_{i-1} V_{i-1} once that MMA has completed.
+        if (!warp_wait(&bars.pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, abort, p.error_word)) {
+          ok = false;
+          break;
         }
+        tc::fence_after_sync();
+        float o[32];
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          const uint32_t ta = tmem + lane_base + C::kOCol + c * 32;
+          tc::tmem_ld32(ta, o);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] *= alpha;
+          tc::tmem_st32(ta, o);
+        }
+        tc::tmem_wait_st();
       }
       l *= alpha;
+      const float neg_m = m == -INFINITY ? 0.f : -m;  // an empty row keeps P = 0
       float rs = 0.f;
-      const bool live = m != -INFINITY;
+      uint32_t pk[kBN / 2];
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        const float w = live ? fast_exp2(v[c] - m) : 0.f;
-        v[c] = w;
-        rs += w;
+      for (int c = 0; c < kBN; c += 2) {
+        const float w0 = fast_exp2(fmaf(v[c], sl2, neg_m));
+        const float w1 = fast_exp2(fmaf(v[c + 1], sl2, neg_m));
+        rs += w0 + w1;
+        pk[c >> 1] = pack_bf16x2(w0, w1);
       }
       l += rs;
-      // P row r as bf16, 128-byte swizzled K-major (two 64-key boxes).
-#pragma unroll
-      for (int c8 = 0; c8 < kBN / 8; ++c8) {
-        uint4 pk;
-        pk.x = pack_bf16x2(v[c8 * 8 + 0], v[c8 * 8 + 1]);
-        pk.y = pack_bf16x2(v[c8 * 8 + 2], v[c8 * 8 + 3]);
-        pk.z = pack_bf16x2(v[c8 * 8 + 4], v[c8 * 8 + 5]);
-        pk.w = pack_bf16x2(v[c8 * 8 + 6], v[c8 * 8 + 7]);
-        uint8_t* dst = smem + C::kPOff + (c8 >> 3) * (kBM * 128) + swz128(r, c8 & 7);
-        *reinterpret_cast<uint4*>(dst) = pk;
+      // P buffer pb is free once P_{i-2} V_{i-2} has completed.
+      if (i >= 2) {
+        if (!warp_wait(&bars.pv_done[pb], ((i - 2) >> 1) & 1, abort, p.error_word)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
       }
-      fence_proxy_async_smem();
+      const uint32_t pa = tmem + lane_base + C::kPCol + (uint32_t)(pb * (kBN / 2));
+      tc::tmem_st32(pa, reinterpret_cast<const float*>(pk));
+      tc::tmem_st32(pa + 32, reinterpret_cast<const float*>(pk + 32));
+      tc::tmem_wait_st();
       tc::fence_before_sync();
-      mbar_arrive(&bars.p_full);
+      mbar_arrive(&bars.p_full[pb]);
     }
     if (!ok) do_abort(abort, p.error_word);
     // ------------------------------------------------------------ epilogue
     bool have_o = n_tiles > 0;
     if (have_o) {
-      have_o = warp_wait(&bars.o_done, (n_tiles - 1) & 1, abort, p.error_word);
+      have_o = warp_wait(&bars.pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort,
+                         p.error_word);
       tc::fence_after_sync();
     }
     const float inv = (l > 0.f) ? 1.f / l : 0.f;
@@ -429,16 +444,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (row_ok) {
 #pragma unroll
         for (int e8 = 0; e8 < 4; ++e8) {
-          uint4 pk;
+          uint4 q4;
           if (have_o && l > 0.f) {
-            pk.x = pack_bf16x2(o[e8 * 8 + 0] * inv, o[e8 * 8 + 1] * inv);
-            pk.y = pack_bf16x2(o[e8 * 8 + 2] * inv, o[e8 * 8 + 3] * inv);
-            pk.z = pack_bf16x2(o[e8 * 8 + 4] * inv, o[e8 * 8 + 5] * inv);
-            pk.w = pack_bf16x2(o[e8 * 8 + 6] * inv, o[e8 * 8 + 7] * inv);
+            q4.x = pack_bf16x2(o[e8 * 8 + 0] * inv, o[e8 * 8 + 1] * inv);
+            q4.y = pack_bf16x2(o[e8 * 8 + 2] * inv, o[e8 * 8 + 3] * inv);
+            q4.z = pack_bf16x2(o[e8 * 8 + 4] * inv, o[e8 * 8 + 5] * inv);
+            q4.w = pack_bf16x2(o[e8 * 8 + 6] * inv, o[e8 * 8 + 7] * inv);
           } else {
-            pk = make_uint4(0, 0, 0, 0);
+            q4 = make_uint4(0, 0, 0, 0);
           }
-          *reinterpret_cast<uint4*>(out + orow + c * 32 + e8 * 8) = pk;
+          *reinterpret_cast<uint4*>(out + orow + c * 32 + e8 * 8) = q4;
         }
       }
     }
@@ -462,7 +477,8 @@ cudaError_t launch_d(const AttnParams& p, const CUtensorMap& q_map, const CUtens
   const int tpt = prefill_rows_per_tile(p.G);
   const int n_qtiles = (p.max_q_len + tpt - 1) / tpt;
   if (n_qtiles == 0) return cudaSuccess;
-  dim3 grid(n_qtiles, p.Hk, p.batch);
+  if (n_qtiles > 65535) return cudaErrorInvalidValue;
+  dim3 grid(p.Hk, p.batch, n_qtiles);
   attn_prefill_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(p, q_map, k_map, v_map, tpt,
                                                                      n_qtiles);
   return cudaGetLastError();

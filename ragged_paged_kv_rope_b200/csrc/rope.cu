@@ -7,8 +7,10 @@
 // and partial rotary_dim). Pair (a, b) at angle theta becomes
 // (a cos - b sin, b cos + a sin), with (cos, sin) read from freqs_cis[pos].
 //
-// Design: pure bandwidth. One CTA per token; its threads walk 16-byte units of
-// the token's q, k and v head rows. A rotation unit of the half layout holds
+// Design: pure bandwidth. One CTA per kTokens tokens; the per-token metadata
+// (sequence, cache slot, page, positions) is computed once per token by one
+// thread each and shared, then the CTA's threads walk 16-byte units of the
+// tokens' q, k and v head rows. A rotation unit of the half layout holds
 // kVec pairs (kVec channels from each half), one of the interleaved layout a
 // 16-byte chunk of kVec/2 adjacent pairs, whose (cos, sin) entries are the
 // same 16-byte-aligned run of the table row. Channels >= rotary_dim and V rows
@@ -20,42 +22,54 @@ namespace rpk {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kTokens = 4;  // tokens per CTA
+
+struct TokenInfo {
+  int page;         // -1 when the slot has no valid page
+  int row_in_page;
+  int pos[3];       // position of each M-RoPE section (all equal without M-RoPE)
+  int pos_ok;
+};
 
 template <typename T, bool kInterleaved>
 __global__ void __launch_bounds__(kThreads) rope_scatter_kernel(const RopeParams p) {
   constexpr int V = Elt<T>::kVec;
-  const int t = blockIdx.x;
-  if (t >= p.T) return;
+  __shared__ TokenInfo info[kTokens];
+  const int t0 = blockIdx.x * kTokens;
+  const int ntok = min(kTokens, p.T - t0);
+  if (ntok <= 0) return;
 
-  // Sequence, index in it, cache slot and page of this token.
-  const int b = find_sequence(p.offsets, p.batch, t);
-  const int i = t - __ldg(p.offsets + b);
-  const int slot = __ldg(p.cache_lens + b) + i;
-  int page = -1;
-  if (slot >= 0) {
-    const int pi = slot / p.P;
-    if (pi < p.max_pages) page = __ldg(p.block_table + (size_t)b * p.max_pages + pi);
-  }
-  const bool page_ok = page >= 0 && page < p.num_pages;
-  const int row_in_page = slot >= 0 ? slot % p.P : 0;
-
-  // Position of each M-RoPE section (all equal without M-RoPE).
-  int pos[3];
-  if (p.position_ids == nullptr) {
-    pos[0] = pos[1] = pos[2] = slot;
-  } else if (p.has_mrope) {
+  if (threadIdx.x < ntok) {
+    // Sequence, index in it, cache slot and page of this token.
+    const int t = t0 + threadIdx.x;
+    const int b = find_sequence(p.offsets, p.batch, t);
+    const int i = t - __ldg(p.offsets + b);
+    const int slot = __ldg(p.cache_lens + b) + i;
+    int page = -1;
+    if (slot >= 0) {
+      const int pi = slot / p.P;
+      if (pi < p.max_pages) page = __ldg(p.block_table + (size_t)b * p.max_pages + pi);
+    }
+    TokenInfo ti;
+    ti.page = (page >= 0 && page < p.num_pages) ? page : -1;
+    ti.row_in_page = slot >= 0 ? slot % p.P : 0;
+    if (p.position_ids == nullptr) {
+      ti.pos[0] = ti.pos[1] = ti.pos[2] = slot;
+    } else if (p.has_mrope) {
 #pragma unroll
-    for (int s = 0; s < 3; ++s) pos[s] = __ldg(p.position_ids + (size_t)s * p.T + t);
-  } else {
-    pos[0] = pos[1] = pos[2] = __ldg(p.position_ids + t);
-  }
-  bool pos_ok = true;
+      for (int s = 0; s < 3; ++s) ti.pos[s] = __ldg(p.position_ids + (size_t)s * p.T + t);
+    } else {
+      ti.pos[0] = ti.pos[1] = ti.pos[2] = __ldg(p.position_ids + t);
+    }
+    bool ok = true;
 #pragma unroll
-  for (int s = 0; s < 3; ++s) pos_ok &= (pos[s] >= 0 && pos[s] < p.max_position);
-  if (threadIdx.x == 0) {
-    if (!page_ok) raise_error(p.error_word, RPK_DEVERR_PAGE);
-    if (!pos_ok) raise_error(p.error_word, RPK_DEVERR_POSITION);
+    for (int s = 0; s < 3; ++s) ok &= (ti.pos[s] >= 0 && ti.pos[s] < p.max_position);
+    ti.pos_ok = ok;
+    info[threadIdx.x] = ti;
+    if (ti.page < 0) raise_error(p.error_word, RPK_DEVERR_PAGE);
+    if (!ok) raise_error(p.error_word, RPK_DEVERR_POSITION);
   }
+  __syncthreads();
 
   const int half = p.R >> 1;
   // Units per head row: rotation units, then pass-through units.
@@ -65,7 +79,8 @@ __global__ void __launch_bounds__(kThreads) rope_scatter_kernel(const RopeParams
   const int q_units = p.H * units_row;
   const int k_units = p.Hk * units_row;
   const int v_units = p.Hk * (p.d / V);
-  const int total = q_units + k_units + v_units;
+  const int per_token = q_units + k_units + v_units;
+  const int total = per_token * ntok;
 
   const T* __restrict__ q = static_cast<const T*>(p.q);
   const T* __restrict__ kn = static_cast<const T*>(p.k_new);
@@ -74,7 +89,16 @@ __global__ void __launch_bounds__(kThreads) rope_scatter_kernel(const RopeParams
   T* kp = static_cast<T*>(p.k_pages);
   T* vp = static_cast<T*>(p.v_pages);
 
-  for (int u = threadIdx.x; u < total; u += kThreads) {
+  for (int uu = threadIdx.x; uu < total; uu += kThreads) {
+    const int tk = uu / per_token;
+    const int u = uu - tk * per_token;
+    const int t = t0 + tk;
+    const TokenInfo& ti = info[tk];
+    const int page = ti.page;
+    const bool page_ok = page >= 0;
+    const int row_in_page = ti.row_in_page;
+    const bool pos_ok = ti.pos_ok != 0;
+    const int* pos = ti.pos;
     const T* src;
     T* dst;
     int unit;
@@ -180,7 +204,7 @@ __global__ void freqs_cis_kernel(float* __restrict__ out, int32_t max_position, 
 cudaError_t launch_rope(const RopeParams& p, rpk_dtype dtype, bool interleaved,
                         cudaStream_t stream) {
   if (p.T == 0) return cudaSuccess;
-  dim3 grid(p.T), block(kThreads);
+  dim3 grid((p.T + kTokens - 1) / kTokens), block(kThreads);
   if (dtype == RPK_BF16) {
     if (interleaved) rope_scatter_kernel<__nv_bfloat16, true><<<grid, block, 0, stream>>>(p);
     else rope_scatter_kernel<__nv_bfloat16, false><<<grid, block, 0, stream>>>(p);
