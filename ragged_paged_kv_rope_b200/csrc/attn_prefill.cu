@@ -8,27 +8,33 @@
 // online-softmax running state (algenta flash_attention: running max,
 // running sum and output rescaled by e^(m_old - m_new), final divide).
 //
-// Tile: 128 rows x 128 keys. The 128 rows are the (token, query head) pairs
-// of one KV head's group, token-major, so the G query heads that share a KV
-// head share every K/V tile (tokens_per_tile = 128 / G). One CTA per
-// (query tile, KV head, sequence), heaviest tiles first.
+// Work unit: two query tiles A and B of 128 rows each against 128-key tiles.
+// The 128 rows of a tile are the (token, query head) pairs of one KV head's
+// group, token-major (tokens_per_tile = 128 / G), so the G query heads that
+// share a KV head share every K/V tile; tile B holds the next tokens_per_tile
+// tokens after tile A. One CTA per (pair of query tiles, KV head, sequence),
+// heaviest pairs first.
 //
-// Warp roles (192 threads):
-//   warp 0     TMA producer: Q tile once, then K and V tiles of 128 keys into
-//              a ring of shared-memory stages, one box per page segment (3-D
-//              map over the pool [pages * page_size, kv_heads, d], 128-byte
-//              swizzle, no multicast)
-//   warp 1     allocates TMEM (512 columns: S0, S1, O, P0, P1) and issues the
-//              MMAs from one thread: S_j = Q K_j^T into S[j % 2] (both operands
-//              from shared memory), then O += P_j V_j with P_j read from TMEM
-//              (P[j % 2]) and V_j from shared memory as an MN-major operand
-//   warps 2-5  softmax: thread r owns row r (TMEM lane r); loads S_j, frees the
-//              S buffer, masks the band, keeps (m, l) in log2 units, writes P_j
-//              as packed bf16 pairs into P[j % 2] with tcgen05.st. O is
-//              rescaled in TMEM only when the running max grew by more than
-//              2^8 (the final O / l uses the same max, so this is exact), and
-//              only then does the softmax wait for the previous P V. Finally it
-//              normalises O and stores the rows.
+// Warp roles (320 threads):
+//   warp 0     TMA producer: both Q tiles once, then K and V tiles of 128 keys
+//              into a 2-stage ring, one box per page segment (3-D map over the
+//              pool [pages * page_size, kv_heads, d], 128-byte swizzle, no
+//              multicast)
+//   warp 1     allocates TMEM (512 columns: S_A, S_B, O_A, O_B) and issues the
+//              MMAs from one thread, alternating the tiles: S_t = Q_t K_j^T
+//              (operands in shared memory), then O_t += P_t V_j with P_t read
+//              from TMEM (written over the first 64 columns of S_t) and V_j an
+//              MN-major operand in shared memory. While one softmax warpgroup
+//              works on its tile, the tensor core runs the other tile's MMAs.
+//   warps 2-5  softmax of tile A, warps 6-9 softmax of tile B: thread r owns
+//              row r (TMEM lane r); loads S_t, masks the band, keeps (m, l) in
+//              log2 units, writes P_t as packed bf16 pairs, and rescales O_t in
+//              TMEM only when the running max grew by more than 2^8 (the final
+//              O / l uses the same max, so this is exact); then normalises O_t
+//              and stores the rows.
+// MMAs issued by one thread run in issue order, so P_t(j) V_j completes before
+// S_t(j+1) overwrites the columns P_t(j) lives in, and the completion of
+// S_t(j+1) also tells the softmax that O_t holds P_t(j) V_j.
 // Value rows at or past k_len are zeroed in shared memory before P V, so the
 // NaN sentinels of unused slots never meet a zero weight. Every mbarrier wait
 // is bounded; on a timeout the CTA raises RPK_DEVERR_TIMEOUT, drains its copies
@@ -45,27 +51,26 @@ namespace {
 
 constexpr int kBM = 128;   // rows per tile (MMA M)
 constexpr int kBN = 128;   // keys per tile
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows > 2^8
 
 template <int D>
 struct Cfg {
   static constexpr int kBoxes = D / 64;
-  static constexpr int kStages = D == 128 ? 3 : 4;   // K/V ring depth
-  static constexpr int kQBytes = kBM * D * 2;
+  static constexpr int kStages = D == 128 ? 2 : 4;   // K/V ring depth
+  static constexpr int kQBytes = kBM * D * 2;         // one query tile
   static constexpr int kKVBytes = kBN * D * 2;
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kQBytes;
+  static constexpr int kKOff = kQOff + 2 * kQBytes;
   static constexpr int kVOff = kKOff + kStages * kKVBytes;
   static constexpr int kEnd = kVOff + kStages * kKVBytes + 1024;
   // At least half the SM's shared memory, so that one CTA holds the SM's TMEM.
   static constexpr int kSmemBytes = kEnd > 118 * 1024 ? kEnd : 118 * 1024;
-  // TMEM columns: S0, S1 (fp32, 128 each), O (fp32, D), P0, P1 (bf16 pairs, 64 each)
+  // TMEM columns: S_A, S_B (fp32, 128 each; P_t over the first 64 of S_t), O_A, O_B
   static constexpr uint32_t kSCol = 0;
   static constexpr uint32_t kOCol = 2 * kBN;
-  static constexpr uint32_t kPCol = kOCol + D;
-  static_assert(kPCol + 2 * (kBN / 2) <= kTmemCols, "TMEM budget");
+  static_assert(kOCol + 2 * D <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -73,11 +78,11 @@ struct Bars {
   uint64_t q_full;
   uint64_t k_full[4];
   uint64_t v_full[4];
-  uint64_t kv_empty[4];
-  uint64_t s_full[2];
-  uint64_t s_free[2];
-  uint64_t p_full[2];
-  uint64_t pv_done[2];
+  uint64_t k_empty[4];
+  uint64_t v_empty[4];
+  uint64_t s_full[2];   // per query tile
+  uint64_t p_full[2];   // per query tile
+  uint64_t o_final[2];  // per query tile: its last P V has completed
   uint64_t drain;
 };
 
@@ -146,14 +151,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0 && blockIdx.z == 0 && kvh == 0) raise_error(p.error_word, RPK_DEVERR_LENGTH);
     return;
   }
-  const int t_begin = qt * tpt;
+  const int t_begin = qt * 2 * tpt;           // first token of tile A
   if (t_begin >= q_len) return;
   if (timed_out_elsewhere(p.error_word)) return;
-  const int t_end = min(q_len, t_begin + tpt);
+  const bool has_b = t_begin + tpt < q_len;    // tile B holds at least one token
+  const int t_end = min(q_len, t_begin + 2 * tpt);
   const int G = p.G;
   const int rows_used = tpt * G;
 
-  // Keys any row of this tile sees, in whole key tiles.
+  // Keys any row of the two tiles sees, in whole key tiles.
   const int p_first = t_begin + k_len - q_len;
   const int p_last = (t_end - 1) + k_len - q_len;
   const int lo_first = p.window > 0 ? max(0, p_first - p.window + 1) : 0;
@@ -168,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t q_s = sbase + C::kQOff;
+  auto q_s = [&](int t) { return sbase + C::kQOff + t * C::kQBytes; };
   auto k_s = [&](int st) { return sbase + C::kKOff + st * C::kKVBytes; };
   auto v_s = [&](int st) { return sbase + C::kVOff + st * C::kKVBytes; };
 
@@ -177,13 +183,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int st = 0; st < S; ++st) {
       mbar_init(&bars.k_full[st], 1);
       mbar_init(&bars.v_full[st], 1);
-      mbar_init(&bars.kv_empty[st], 1);
+      mbar_init(&bars.k_empty[st], 1);
+      mbar_init(&bars.v_empty[st], 1);
     }
-    for (int bb = 0; bb < 2; ++bb) {
-      mbar_init(&bars.s_full[bb], 1);
-      mbar_init(&bars.s_free[bb], 128);
-      mbar_init(&bars.p_full[bb], 128);
-      mbar_init(&bars.pv_done[bb], 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars.s_full[t], 1);
+      mbar_init(&bars.p_full[t], 128);
+      mbar_init(&bars.o_final[t], 1);
     }
     mbar_init(&bars.drain, 1);
     abort_sh = 0;
@@ -205,22 +211,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&q_map);
       prefetch_tensormap(&k_map);
       prefetch_tensormap(&v_map);
+      const int n_q = has_b ? 2 : 1;
       const uint32_t q_box_bytes = 128u * (uint32_t)rows_used;
-      mbar_arrive_expect_tx(&bars.q_full, C::kBoxes * q_box_bytes);
+      mbar_arrive_expect_tx(&bars.q_full, n_q * C::kBoxes * q_box_bytes);
+      for (int t = 0; t < n_q; ++t)
 #pragma unroll
-      for (int bx = 0; bx < C::kBoxes; ++bx)
-        tma_load_3d(smem + C::kQOff + bx * (kBM * 128), &q_map, bx * 64, kvh * G, q0 + t_begin,
-                    &bars.q_full);
+        for (int bx = 0; bx < C::kBoxes; ++bx)
+          tma_load_3d(smem + C::kQOff + t * C::kQBytes + bx * (kBM * 128), &q_map, bx * 64,
+                      kvh * G, q0 + t_begin + t * tpt, &bars.q_full);
       const int box_rows = p.P < kBN ? p.P : kBN;
       const uint32_t seg_bytes = (uint32_t)box_rows * 128u * C::kBoxes;
       int issued = 0;
-      for (int i = 0; i < n_tiles; ++i) {
+      // K_i and V_i go to stage i % S; K of a stage frees after the last S
+      // MMA that reads it, V after the last P V, so K runs ahead of V.
+      auto load = [&](int i, bool is_v) -> bool {
         const int st = i % S;
-        if (i >= S &&
-            !thread_wait(&bars.kv_empty[st], ((i / S) & 1) ^ 1, abort, p.error_word)) {
-          do_abort(abort, p.error_word);
-          break;
-        }
+        uint64_t* empty = is_v ? &bars.v_empty[st] : &bars.k_empty[st];
+        uint64_t* full = is_v ? &bars.v_full[st] : &bars.k_full[st];
+        if (i >= S && !thread_wait(empty, ((i / S) & 1) ^ 1, abort, p.error_word)) return false;
         const int key0 = (j_begin + i) * kBN;
         uint32_t bytes = 0;
         for (int r = 0; r < kBN; r += box_rows) {
@@ -230,25 +238,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
           if (page >= 0 && page < p.num_pages) bytes += seg_bytes;
         }
-        mbar_arrive_expect_tx(&bars.k_full[st], bytes);
-        mbar_arrive_expect_tx(&bars.v_full[st], bytes);
+        mbar_arrive_expect_tx(full, bytes);
         for (int r = 0; r < kBN; r += box_rows) {
           const int key = key0 + r;
           if (key >= k_len) break;
           const int pi = key / p.P;
           const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
           if (page < 0 || page >= p.num_pages) {
-            raise_error(p.error_word, RPK_DEVERR_PAGE);
+            if (!is_v) raise_error(p.error_word, RPK_DEVERR_PAGE);
             continue;
           }
           const int grow = page * p.P + (key - pi * p.P);
+          uint8_t* base = smem + (is_v ? C::kVOff : C::kKOff) + st * C::kKVBytes + r * 128;
 #pragma unroll
-          for (int bx = 0; bx < C::kBoxes; ++bx) {
-            tma_load_3d(smem + C::kKOff + st * C::kKVBytes + bx * (kBN * 128) + r * 128, &k_map,
-                        bx * 64, kvh, grow, &bars.k_full[st]);
-            tma_load_3d(smem + C::kVOff + st * C::kKVBytes + bx * (kBN * 128) + r * 128, &v_map,
-                        bx * 64, kvh, grow, &bars.v_full[st]);
-          }
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            tma_load_3d(base + bx * (kBN * 128), is_v ? &v_map : &k_map, bx * 64, kvh, grow, full);
+        }
+        return true;
+      };
+      for (int i = 0; i < n_tiles; ++i) {
+        if (!load(i, false) || !load(i, true)) {
+          do_abort(abort, p.error_word);
+          break;
         }
         ++issued;
       }
@@ -265,34 +276,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(kBM, D, 1);
     bool ok = warp_wait(&bars.q_full, 0, abort, p.error_word);
     tc::fence_after_sync();
-    auto issue_s = [&](int i) -> bool {
-      const int st = i % S;
-      if (!warp_wait(&bars.k_full[st], (i / S) & 1, abort, p.error_word)) return false;
-      tc::fence_after_sync();
+    // S_t = Q_t K_i^T into S_t's columns.
+    auto issue_s = [&](int t, int i) {
       if (lane == 0) {
-        const uint32_t d_tmem = tmem + C::kSCol + (uint32_t)((i & 1) * kBN);
+        const int st = i % S;
+        const uint32_t d_tmem = tmem + C::kSCol + (uint32_t)(t * kBN);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t qoff = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
           const uint32_t koff = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-          tc::mma_ss(d_tmem, tc::smem_desc_sw128(q_s + qoff, 16, 1024),
+          tc::mma_ss(d_tmem, tc::smem_desc_sw128(q_s(t) + qoff, 16, 1024),
                      tc::smem_desc_sw128(k_s(st) + koff, 16, 1024), idesc_qk, kk > 0);
         }
-        tc::commit(smem_u32(&bars.s_full[i & 1]));
+        tc::commit(smem_u32(&bars.s_full[t]));
       }
       __syncwarp();
-      return true;
     };
-    if (ok && n_tiles > 0) ok = issue_s(0);
-    for (int i = 0; ok && i < n_tiles; ++i) {
-      const int st = i % S, pb = i & 1;
-      if (i + 1 < n_tiles) {
-        // S buffer (i+1)%2 is free once the softmax has read S_{i-1} from it.
-        if (i >= 1 && !warp_wait(&bars.s_free[(i + 1) & 1], ((i - 1) >> 1) & 1, abort,
-                                 p.error_word)) { ok = false; break; }
-        if (!issue_s(i + 1)) { ok = false; break; }
+    // O_t += P_t V_i, P_t in the first 64 columns of S_t.
+    auto issue_pv = [&](int t, int i) {
+      if (lane == 0) {
+        const int st = i % S;
+        const uint32_t d_tmem = tmem + C::kOCol + (uint32_t)(t * D);
+        const uint32_t a_tmem = tmem + C::kSCol + (uint32_t)(t * kBN);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          tc::mma_ts(d_tmem, a_tmem + kk * 8,
+                     tc::smem_desc_sw128(v_s(st) + kk * (16 * 128), kBN * 128, 1024), idesc_pv,
+                     (i > 0 || kk > 0) ? 1u : 0u);
       }
-      if (!warp_wait(&bars.p_full[pb], (i >> 1) & 1, abort, p.error_word)) { ok = false; break; }
+      __syncwarp();
+    };
+    if (ok && n_tiles > 0) {
+      ok = warp_wait(&bars.k_full[0], 0, abort, p.error_word);
+      tc::fence_after_sync();
+      if (ok) {
+        issue_s(0, 0);
+        if (has_b) issue_s(1, 0);
+        if (lane == 0) tc::commit(smem_u32(&bars.k_empty[0]));
+        __syncwarp();
+      }
+    }
+    for (int i = 0; ok && i < n_tiles; ++i) {
+      const int st = i % S;
+      const bool last = i + 1 == n_tiles;
+      // tile A: P_A(i) V_i, then S_A(i+1)
+      if (!warp_wait(&bars.p_full[0], i & 1, abort, p.error_word)) { ok = false; break; }
       if (!warp_wait(&bars.v_full[st], (i / S) & 1, abort, p.error_word)) { ok = false; break; }
       tc::fence_after_sync();
       const int key0 = (j_begin + i) * kBN;
@@ -311,17 +339,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
       }
-      if (lane == 0) {
-        const uint32_t d_tmem = tmem + C::kOCol;
-        const uint32_t a_tmem = tmem + C::kPCol + (uint32_t)(pb * (kBN / 2));
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          tc::mma_ts(d_tmem, a_tmem + kk * 8,
-                     tc::smem_desc_sw128(v_s(st) + kk * (16 * 128), kBN * 128, 1024), idesc_pv,
-                     (i > 0 || kk > 0) ? 1u : 0u);
-        tc::commit(smem_u32(&bars.pv_done[pb]));
-        tc::commit(smem_u32(&bars.kv_empty[st]));
+      issue_pv(0, i);
+      if (last && lane == 0) tc::commit(smem_u32(&bars.o_final[0]));
+      if (!last) {
+        if (!warp_wait(&bars.k_full[(i + 1) % S], ((i + 1) / S) & 1, abort, p.error_word)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        issue_s(0, i + 1);
       }
+      // tile B: P_B(i) V_i, then S_B(i+1)
+      if (has_b) {
+        if (!warp_wait(&bars.p_full[1], i & 1, abort, p.error_word)) { ok = false; break; }
+        tc::fence_after_sync();
+        issue_pv(1, i);
+        if (last && lane == 0) tc::commit(smem_u32(&bars.o_final[1]));
+      }
+      if (lane == 0) tc::commit(smem_u32(&bars.v_empty[st]));
+      __syncwarp();
+      if (has_b && !last) issue_s(1, i + 1);
+      // K_{i+1} has now been read by every S MMA that needs it.
+      if (!last && lane == 0) tc::commit(smem_u32(&bars.k_empty[(i + 1) % S]));
       __syncwarp();
     }
     if (!ok) do_abort(abort, p.error_word);
@@ -331,29 +370,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!warp_wait(&bars.drain, 0, abort, p.error_word)) mbar_wait(&bars.drain, 0);
   } else {
     // ------------------------------------------------------------- softmax
+    const int t = (warp - 2) >> 2;       // query tile: warps 2-5 -> A, 6-9 -> B
     const int qw = warp & 3;             // TMEM lane quarter of this warp
     const int r = qw * 32 + lane;        // row of this thread
-    const int t_local = r / G;
-    const int tok = t_begin + t_local;
+    const int tok = t_begin + t * tpt + r / G;
     const bool row_ok = r < rows_used && tok < q_len;
     const int pos = tok + k_len - q_len;
     const int lo = p.window > 0 ? pos - p.window + 1 : 0;
     const int hi = pos;
     const uint32_t lane_base = (uint32_t)(qw * 32) << 16;
+    const uint32_t s_col = tmem + lane_base + C::kSCol + (uint32_t)(t * kBN);
+    const uint32_t o_col = tmem + lane_base + C::kOCol + (uint32_t)(t * D);
     const float sl2 = p.scale_log2;
+    const int my_tiles = (t == 0 || has_b) ? n_tiles : 0;
     float m = -INFINITY, l = 0.f;        // running max (log2 units) and sum
     bool ok = true;
     float v[kBN];
-    for (int i = 0; i < n_tiles; ++i) {
-      const int pb = i & 1;
-      if (!warp_wait(&bars.s_full[pb], (i >> 1) & 1, abort, p.error_word)) { ok = false; break; }
+    for (int i = 0; i < my_tiles; ++i) {
+      if (!warp_wait(&bars.s_full[t], i & 1, abort, p.error_word)) { ok = false; break; }
       tc::fence_after_sync();
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c)
-        tc::tmem_ld32(tmem + lane_base + C::kSCol + (uint32_t)(pb * kBN + c * 32), v + c * 32);
+      for (int c = 0; c < kBN / 32; ++c) tc::tmem_ld32(s_col + c * 32, v + c * 32);
       tc::tmem_wait_ld();
-      tc::fence_before_sync();
-      mbar_arrive(&bars.s_free[pb]);
       const int key0 = (j_begin + i) * kBN;
       if (!(row_ok && key0 >= lo && key0 + kBN - 1 <= hi)) {
 #pragma unroll
@@ -367,7 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, v[c]);
       mx *= sl2;  // scale > 0: max of the scaled scores
       // Running max: taken at once while empty, else only when it grows by
-      // more than the threshold (then O and l are rescaled).
+      // more than the threshold (then O and l are rescaled). O_t holds
+      // P_t(i-1) V_{i-1} here: S_t(i) was issued after it and has completed.
       float alpha = 1.f;
       bool rescale = false;
       if (m == -INFINITY) {
@@ -377,58 +416,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = mx;
         rescale = true;
       }
-      if (i > 0 && __any_sync(0xffffffffu, rescale)) {
-        // O holds P_{i-1} V_{i-1} once that MMA has completed.
-        if (!warp_wait(&bars.pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, abort, p.error_word)) {
-          ok = false;
-          break;
+      l *= alpha;
+      const float neg_m = m == -INFINITY ? 0.f : -m;  // an empty row keeps P = 0
+      float rs0 = 0.f, rs1 = 0.f;
+      // P in two halves of 64 keys (32 packed columns each) to bound registers.
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float w0 = fast_exp2(fmaf(v[h * 64 + c], sl2, neg_m));
+          const float w1 = fast_exp2(fmaf(v[h * 64 + c + 1], sl2, neg_m));
+          rs0 += w0;
+          rs1 += w1;
+          pk[c >> 1] = pack_bf16x2(w0, w1);
         }
-        tc::fence_after_sync();
+        tc::tmem_st32(s_col + h * 32, reinterpret_cast<const float*>(pk));
+      }
+      l += rs0 + rs1;
+      // Rescale O_t (after P, so that the scores are dead): it must finish
+      // before P_t(i) V_i is issued, i.e. before p_full.
+      if (i > 0 && __any_sync(0xffffffffu, rescale)) {
         float o[32];
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
-          const uint32_t ta = tmem + lane_base + C::kOCol + c * 32;
-          tc::tmem_ld32(ta, o);
+          tc::tmem_ld32(o_col + c * 32, o);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tc::tmem_st32(ta, o);
+          tc::tmem_st32(o_col + c * 32, o);
         }
-        tc::tmem_wait_st();
       }
-      l *= alpha;
-      const float neg_m = m == -INFINITY ? 0.f : -m;  // an empty row keeps P = 0
-      float rs = 0.f;
-      uint32_t pk[kBN / 2];
-#pragma unroll
-      for (int c = 0; c < kBN; c += 2) {
-        const float w0 = fast_exp2(fmaf(v[c], sl2, neg_m));
-        const float w1 = fast_exp2(fmaf(v[c + 1], sl2, neg_m));
-        rs += w0 + w1;
-        pk[c >> 1] = pack_bf16x2(w0, w1);
-      }
-      l += rs;
-      // P buffer pb is free once P_{i-2} V_{i-2} has completed.
-      if (i >= 2) {
-        if (!warp_wait(&bars.pv_done[pb], ((i - 2) >> 1) & 1, abort, p.error_word)) {
-          ok = false;
-          break;
-        }
-        tc::fence_after_sync();
-      }
-      const uint32_t pa = tmem + lane_base + C::kPCol + (uint32_t)(pb * (kBN / 2));
-      tc::tmem_st32(pa, reinterpret_cast<const float*>(pk));
-      tc::tmem_st32(pa + 32, reinterpret_cast<const float*>(pk + 32));
       tc::tmem_wait_st();
       tc::fence_before_sync();
-      mbar_arrive(&bars.p_full[pb]);
+      mbar_arrive(&bars.p_full[t]);
     }
     if (!ok) do_abort(abort, p.error_word);
     // ------------------------------------------------------------ epilogue
-    bool have_o = n_tiles > 0;
+    bool have_o = my_tiles > 0;
     if (have_o) {
-      have_o = warp_wait(&bars.pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort,
-                         p.error_word);
+      have_o = warp_wait(&bars.o_final[t], 0, abort, p.error_word);
       tc::fence_after_sync();
     }
     const float inv = (l > 0.f) ? 1.f / l : 0.f;
@@ -438,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = 0; c < D / 32; ++c) {
       float o[32];
       if (have_o) {
-        tc::tmem_ld32(tmem + lane_base + C::kOCol + c * 32, o);
+        tc::tmem_ld32(o_col + c * 32, o);
         tc::tmem_wait_ld();
       }
       if (row_ok) {
@@ -475,7 +502,7 @@ cudaError_t launch_d(const AttnParams& p, const CUtensorMap& q_map, const CUtens
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int tpt = prefill_rows_per_tile(p.G);
-  const int n_qtiles = (p.max_q_len + tpt - 1) / tpt;
+  const int n_qtiles = (p.max_q_len + 2 * tpt - 1) / (2 * tpt);  // pairs of query tiles
   if (n_qtiles == 0) return cudaSuccess;
   if (n_qtiles > 65535) return cudaErrorInvalidValue;
   dim3 grid(p.Hk, p.batch, n_qtiles);
