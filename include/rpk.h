@@ -140,9 +140,10 @@ rpk_status rope_freqs_cis(float* freqs_cis, int32_t max_position, int32_t rotary
 
 /*
  * ragged_paged_attention_workspace_size -- bytes of device workspace that
- * ragged_paged_attention needs for these sizes (0 when none). The result
- * depends only on the arguments, so it may be computed once and reused for
- * every call with the same sizes.
+ * ragged_paged_attention needs for these sizes (the split-KV partials of the
+ * decode path; 0 when there are no query tokens). The result depends only on
+ * the arguments, so it may be computed once and reused for every call with
+ * the same sizes.
  */
 size_t ragged_paged_attention_workspace_size(int32_t total_q_tokens, int32_t n_heads,
                                              int32_t head_dim, int32_t batch,
@@ -174,14 +175,16 @@ size_t ragged_paged_attention_workspace_size(int32_t total_q_tokens, int32_t n_h
  *                   RPK_DEVERR_LENGTH and that sequence is skipped
  *   workspace       device scratch of at least
  *                   ragged_paged_attention_workspace_size(...) bytes, 256-byte
- *                   aligned; may be NULL when that size is 0. Its contents on
- *                   entry do not matter; calls sharing one workspace must not
- *                   overlap in time.
+ *                   aligned (only the decode path with several splits reads it;
+ *                   the other paths accept NULL). Its contents on entry do not matter;
+ *                   calls sharing one workspace must not overlap in time.
  *
  * Paths (chosen from the host sizes, never from device data):
  *   dtype f32                      -> fp32 CUDA-core kernel
  *   bf16, max_q_len * group <= 16  -> split-KV decode kernel + combine kernel
- *   bf16, otherwise                -> tcgen05 prefill kernel (head_dim 64/128)
+ *   bf16, otherwise                -> tcgen05 prefill kernel (head_dim 64/128,
+ *                                     group <= 128; other shapes run on the
+ *                                     CUDA-core kernel)
  */
 rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
                                   const int32_t* kv_lens, const rpk_paged_kv* page_table,

@@ -15,7 +15,7 @@
 // tokens after tile A. One CTA per (pair of query tiles, KV head, sequence),
 // heaviest pairs first.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warp 0     TMA producer: both Q tiles once, then K and V tiles of 128 keys
 //              into a 2-stage ring, one box per page segment (3-D map over the
 //              pool [pages * page_size, kv_heads, d], 128-byte swizzle, no
@@ -26,12 +26,17 @@
 //              from TMEM (written over the first 64 columns of S_t) and V_j an
 //              MN-major operand in shared memory. While one softmax warpgroup
 //              works on its tile, the tensor core runs the other tile's MMAs.
-//   warps 2-5  softmax of tile A, warps 6-9 softmax of tile B: thread r owns
+//   warps 2-3  idle (they complete the first warpgroup)
+//   warps 4-7  softmax of tile A, warps 8-11 softmax of tile B: thread r owns
 //              row r (TMEM lane r); loads S_t, masks the band, keeps (m, l) in
 //              log2 units, writes P_t as packed bf16 pairs, and rescales O_t in
 //              TMEM only when the running max grew by more than 2^8 (the final
 //              O / l uses the same max, so this is exact); then normalises O_t
 //              and stores the rows.
+// Registers: the first warpgroup gives registers back (setmaxnreg 64) and the
+// two softmax warpgroups take them (setmaxnreg 208), so that a softmax thread
+// holds a whole 128-score row without spilling; 4*32*64 + 8*32*208 = 61440
+// registers, within the 384 * 168 the CTA is launched with.
 // MMAs issued by one thread run in issue order, so P_t(j) V_j completes before
 // S_t(j+1) overwrites the columns P_t(j) lives in, and the completion of
 // S_t(j+1) also tells the softmax that O_t holds P_t(j) V_j.
@@ -51,9 +56,41 @@ namespace {
 
 constexpr int kBM = 128;   // rows per tile (MMA M)
 constexpr int kBN = 128;   // keys per tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr int kRegsControl = 64;    // warpgroup 0: producer, MMA issuer, 2 idle warps
+constexpr int kRegsSoftmax = 208;   // warpgroups 1 and 2: softmax
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows > 2^8
+
+// Packed and three-input fp32 instructions of sm_100: the softmax is bound by
+// instruction issue (one softmax warp per SM sub-partition), so two scores per
+// instruction where the hardware allows it.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// (d0, d1) = (a0, a1) * b + c
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %4};\n\t"
+      "mov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+// (s0, s1) += (a0, a1)
+__device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(s0), "=f"(s1)
+      : "f"(a0), "f"(a1), "f"(s0), "f"(s1));
+}
 
 template <int D>
 struct Cfg {
@@ -95,18 +132,23 @@ __device__ __forceinline__ bool timed_out_elsewhere(const int32_t* error_word) {
          (*reinterpret_cast<const volatile int32_t*>(error_word) & (int32_t)RPK_DEVERR_TIMEOUT);
 }
 
-// Bounded wait by one thread; false on timeout or abort.
+// Bounded wait by one thread; false on timeout or abort. The thread sleeps in
+// try_wait (woken when the phase completes, at most 0.2 ms per try), so
+// waiting warps leave the issue slots to the warps that compute; between
+// tries it looks at the abort flag, the timer and, once the wait has lasted
+// longer than any healthy one (50 us), the global error word.
 __device__ __forceinline__ bool thread_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                             const int32_t* error_word) {
   const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
 #pragma unroll 1
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(a, parity)) return true;
-    if ((it & 63u) == 63u) {
-      if (*abort || timed_out_elsewhere(error_word)) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
-    }
+  while (true) {
+    if (mbar_try_wait_suspend(a, parity, 200000u)) return true;
+    if (*abort) return false;
+    const unsigned long long dt = global_timer_ns() - t0;
+    if (dt > kWaitTimeoutNs) return false;
+    if (dt > 50000ull && timed_out_elsewhere(error_word)) return false;
   }
 }
 
@@ -207,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
     if (lane == 0) {
       prefetch_tensormap(&q_map);
       prefetch_tensormap(&k_map);
@@ -272,6 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
     constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(kBM, kBN, 0);
     constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(kBM, D, 1);
     bool ok = warp_wait(&bars.q_full, 0, abort, p.error_word);
@@ -368,9 +412,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) tc::commit(smem_u32(&bars.drain));
     __syncwarp();
     if (!warp_wait(&bars.drain, 0, abort, p.error_word)) mbar_wait(&bars.drain, 0);
+  } else if (warp < 4) {
+    // idle warps of the first warpgroup
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   } else {
     // ------------------------------------------------------------- softmax
-    const int t = (warp - 2) >> 2;       // query tile: warps 2-5 -> A, 6-9 -> B
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    const int t = (warp - 4) >> 2;       // query tile: warps 4-7 -> A, 8-11 -> B
     const int qw = warp & 3;             // TMEM lane quarter of this warp
     const int r = qw * 32 + lane;        // row of this thread
     const int tok = t_begin + t * tpt + r / G;
@@ -394,15 +442,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tmem_wait_ld();
       const int key0 = (j_begin + i) * kBN;
       if (!(row_ok && key0 >= lo && key0 + kBN - 1 <= hi)) {
+        // visible columns [c_lo, c_hi] of this tile (empty for an invalid row)
+        const int c_lo = row_ok ? lo - key0 : kBN;
+        const int c_hi = row_ok ? hi - key0 : -1;
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          const int key = key0 + c;
-          if (!(row_ok && key >= lo && key <= hi)) v[c] = -INFINITY;
-        }
+        for (int c = 0; c < kBN; ++c)
+          if (c < c_lo || c > c_hi) v[c] = -INFINITY;
       }
-      float mx = v[0];
+      // Row max: 8 independent chains of three-input max.
+      float m8[8];
 #pragma unroll
-      for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, v[c]);
+      for (int k = 0; k < 8; ++k) m8[k] = fmaxf(v[k], v[8 + k]);
+#pragma unroll
+      for (int c = 16; c < kBN; c += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m8[k] = max3(m8[k], v[c + k], v[c + 8 + k]);
+      float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
       mx *= sl2;  // scale > 0: max of the scaled scores
       // Running max: taken at once while empty, else only when it grows by
       // more than the threshold (then O and l are rescaled). O_t holds
@@ -418,22 +473,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       l *= alpha;
       const float neg_m = m == -INFINITY ? 0.f : -m;  // an empty row keeps P = 0
-      float rs0 = 0.f, rs1 = 0.f;
+      float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 4 packed partial sums
       // P in two halves of 64 keys (32 packed columns each) to bound registers.
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
-          const float w0 = fast_exp2(fmaf(v[h * 64 + c], sl2, neg_m));
-          const float w1 = fast_exp2(fmaf(v[h * 64 + c + 1], sl2, neg_m));
-          rs0 += w0;
-          rs1 += w1;
+          float x0, x1;
+          fma2(x0, x1, v[h * 64 + c], v[h * 64 + c + 1], sl2, neg_m);
+          const float w0 = fast_exp2(x0);
+          const float w1 = fast_exp2(x1);
+          const int k = (c >> 1) & 3;
+          add2(rs[2 * k], rs[2 * k + 1], w0, w1);
           pk[c >> 1] = pack_bf16x2(w0, w1);
         }
         tc::tmem_st32(s_col + h * 32, reinterpret_cast<const float*>(pk));
       }
-      l += rs0 + rs1;
+      l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
       // Rescale O_t (after P, so that the scores are dead): it must finish
       // before P_t(i) V_i is issued, i.e. before p_full.
       if (i > 0 && __any_sync(0xffffffffu, rescale)) {

@@ -52,6 +52,7 @@ def test_attention_decode_full_size():
     _attn_case(sp, q_lens, kv_lens)
 
 
+@pytest.mark.slow
 def test_attention_swa_decode_full_size():
     sp = W.SPECS["gemma_swa_decode"]
     _attn_case(sp, [1] * sp.batch, [32769] * sp.batch)
