@@ -61,15 +61,26 @@ def parse():
 
 # ----------------------------------------------------------------- plumbing
 
-def dist_setup():
+def dist_setup(backend: str | None = None):
+    """(world, rank, local_rank) from the torchrun environment; joins the
+    process group when world > 1 (NCCL on GPUs, gloo where there is none)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        if backend is None:
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
+
+
+def _reduce_device():
+    if torch.distributed.is_initialized() and torch.distributed.get_backend() == "nccl":
+        return torch.device("cuda", torch.cuda.current_device())
+    return torch.device("cpu")
 
 
 def barrier(world):
@@ -78,11 +89,32 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest value over all ranks (device times are max-reduced)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_reduce_device())
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    """The sum over all ranks (units every rank processed)."""
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=_reduce_device())
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own batch: sequences are independent, so the path
+    shards across ranks with no exchange (weak scaling)."""
+    return seed + 1000 * rank
+
+
+def whole_job_throughput(units_this_rank: float, seconds_this_rank: float, world: int) -> float:
+    """Units all ranks processed divided by the slowest rank's time."""
+    return sum_over_ranks(units_this_rank, world) / max_over_ranks(seconds_this_rank, world)
 
 
 def load_peaks():
@@ -350,7 +382,7 @@ def prefill_measure(device, world, steps=5, warmup=3):
         "frac": tflops / peaks["bf16_tflops"], "attention_ms": attn,
         "visible_pair_flops": flops, "rope_ms": rope,
         "rope_gbs": rope_b / (rope * 1e-3) / 1e9,
-        "tokens_per_s": world * wl.total_tokens / (max_over_ranks(total / steps, world) * 1e-3),
+        "tokens_per_s": whole_job_throughput(wl.total_tokens, total / steps * 1e-3, world),
         "error_word": int(step.error_word.item()),
     }
 
@@ -410,7 +442,7 @@ def main():
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     over = {} if args.batch is None else {"batch": args.batch}
-    wl = W.make(args.workload, seed=args.seed + 1000 * rank, **over)
+    wl = W.make(args.workload, seed=rank_seed(args.seed, rank), **over)
     sp = wl.spec
     step = Step(wl, device)
     elt = 2 if sp.dtype == "bf16" else 4
@@ -420,11 +452,13 @@ def main():
         total_ms, rope_ms, attn_ms = time_steps(step, args.steps, args.warmup, world, clocks)
     clk = clocks.summary()
     step_ms = max_over_ranks(total_ms / args.steps, world)
+    job_kv_bytes = sum_over_ranks(kv_bytes, world)
+    job_tokens = sum_over_ranks(wl.total_tokens, world)
     attn_ms_mean = max_over_ranks(statistics.mean(attn_ms), world)
     rope_ms_mean = max_over_ranks(statistics.mean(rope_ms), world)
     err = int(step.error_word.item())
     peaks = load_peaks()
-    value = world * kv_bytes / (step_ms * 1e-3) / 1e9
+    value = job_kv_bytes / (step_ms * 1e-3) / 1e9
     achieved = kv_bytes / (attn_ms_mean * 1e-3) / 1e9
     traffic = load_traffic("attn_decode")
 
@@ -432,7 +466,7 @@ def main():
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_e2e(step, max(3, args.steps // 2), 2, world)
         e2e_ms = max_over_ranks(e2e_ms, world)
-        e2e = {"value": world * kv_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e = {"value": job_kv_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "note": "pinned host inputs copied in, output copied out, inside the timed region"}
 
@@ -461,7 +495,7 @@ def main():
                    "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V per step "
                          f"vs {L2_BYTES / 2**20:.0f} MiB L2",
                    "parallelism": f"replicas x{world} (independent sequences, no exchange)"},
-        "tokens_per_s": world * wl.total_tokens / (step_ms * 1e-3),
+        "tokens_per_s": job_tokens / (step_ms * 1e-3),
         "breakdown_ms": {"rope_qk_paged_ragged": rope_ms_mean,
                          "ragged_paged_attention": attn_ms_mean},
         "roofline": {"bound": "hbm", "kernel": "ragged_paged_attention (split-KV decode + combine)",

@@ -144,6 +144,7 @@ rpk_status rope_qk_paged_ragged(const void* q_proj, const int32_t* input_row_off
   p.has_mrope = mrope_section != nullptr;
   p.sec_end0 = mrope_section ? mrope_section[0] : rotary_dim;
   p.sec_end1 = mrope_section ? mrope_section[0] + mrope_section[1] : rotary_dim;
+  p.tokens_per_cta = 1;
   return cuda_status(rpk::launch_rope(p, dtype, interleaved != 0,
                                       static_cast<cudaStream_t>(stream)));
 }

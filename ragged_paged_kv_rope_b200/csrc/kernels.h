@@ -26,6 +26,7 @@ struct RopeParams {
   int32_t T, batch, H, Hk, d, R, P, num_pages, max_pages, max_position;
   int32_t sec_end0, sec_end1;   // M-RoPE: pair j < sec_end0 -> section 0, < sec_end1 -> 1, else 2
   int32_t has_mrope;
+  int32_t tokens_per_cta;       // 1..4, chosen by the launcher
 };
 
 cudaError_t launch_rope(const RopeParams& p, rpk_dtype dtype, bool interleaved,

@@ -7,7 +7,9 @@
 // and partial rotary_dim). Pair (a, b) at angle theta becomes
 // (a cos - b sin, b cos + a sin), with (cos, sin) read from freqs_cis[pos].
 //
-// Design: pure bandwidth. One CTA per kTokens tokens; the per-token metadata
+// Design: pure bandwidth. One CTA per 1-4 tokens (4 when there are enough
+// tokens to fill the GPU several times over, 1 for small decode batches so
+// that they still spread over many SMs); the per-token metadata
 // (sequence, cache slot, page, positions) is computed once per token by one
 // thread each and shared, then the CTA's threads walk 16-byte units of the
 // tokens' q, k and v head rows. A rotation unit of the half layout holds
@@ -22,7 +24,7 @@ namespace rpk {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kTokens = 4;  // tokens per CTA
+constexpr int kTokens = 4;  // most tokens per CTA
 
 struct TokenInfo {
   int page;         // -1 when the slot has no valid page
@@ -35,8 +37,8 @@ template <typename T, bool kInterleaved>
 __global__ void __launch_bounds__(kThreads) rope_scatter_kernel(const RopeParams p) {
   constexpr int V = Elt<T>::kVec;
   __shared__ TokenInfo info[kTokens];
-  const int t0 = blockIdx.x * kTokens;
-  const int ntok = min(kTokens, p.T - t0);
+  const int t0 = blockIdx.x * p.tokens_per_cta;
+  const int ntok = min(p.tokens_per_cta, p.T - t0);
   if (ntok <= 0) return;
 
   if (threadIdx.x < ntok) {
@@ -204,13 +206,15 @@ __global__ void freqs_cis_kernel(float* __restrict__ out, int32_t max_position, 
 cudaError_t launch_rope(const RopeParams& p, rpk_dtype dtype, bool interleaved,
                         cudaStream_t stream) {
   if (p.T == 0) return cudaSuccess;
-  dim3 grid((p.T + kTokens - 1) / kTokens), block(kThreads);
+  RopeParams q = p;
+  q.tokens_per_cta = p.T >= 8 * 148 * kTokens ? kTokens : 1;
+  dim3 grid((p.T + q.tokens_per_cta - 1) / q.tokens_per_cta), block(kThreads);
   if (dtype == RPK_BF16) {
-    if (interleaved) rope_scatter_kernel<__nv_bfloat16, true><<<grid, block, 0, stream>>>(p);
-    else rope_scatter_kernel<__nv_bfloat16, false><<<grid, block, 0, stream>>>(p);
+    if (interleaved) rope_scatter_kernel<__nv_bfloat16, true><<<grid, block, 0, stream>>>(q);
+    else rope_scatter_kernel<__nv_bfloat16, false><<<grid, block, 0, stream>>>(q);
   } else {
-    if (interleaved) rope_scatter_kernel<float, true><<<grid, block, 0, stream>>>(p);
-    else rope_scatter_kernel<float, false><<<grid, block, 0, stream>>>(p);
+    if (interleaved) rope_scatter_kernel<float, true><<<grid, block, 0, stream>>>(q);
+    else rope_scatter_kernel<float, false><<<grid, block, 0, stream>>>(q);
   }
   return cudaGetLastError();
 }
