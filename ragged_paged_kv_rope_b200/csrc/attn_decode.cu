@@ -20,7 +20,9 @@
 //    that matters.
 //  * at the end the four warps merge their states (the same rescale rule) and
 //    the CTA writes either the final rows (one split) or an fp32 partial
-//    (m, l, O) that attn_combine_kernel merges across splits.
+//    (m, l, O) that attn_combine_kernel merges across splits. The combine
+//    kernel is a programmatic dependent launch: it starts while the last
+//    decode CTAs finish and waits (griddepcontrol.wait) before reading.
 //
 // Masking follows NumKong "Attention with a Pre-Packed KV-Cache": row r sits
 // at p = r + k_len - q_len and sees [p - (window - 1), p]; masked keys are left
@@ -357,6 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) mbar_arrive(&empty_bar[s]);
   }
   if (!ok) raise_error(p.error_word, RPK_DEVERR_TIMEOUT);
+  // Let the combine kernel launch now (it waits for this grid's completion
+  // before reading any partial, so this only moves its launch earlier).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ----------------------------------------------- merge the four warps' states
 #pragma unroll
@@ -432,6 +437,9 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p,
                                                            const DecodePlan plan,
                                                            const DecodeWorkspace ws) {
   constexpr int E = D / 32;
+  // Launched as a programmatic dependent of the decode kernel: wait until that
+  // grid has completed and its partials are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= (long long)p.T * p.H) return;
@@ -480,8 +488,17 @@ cudaError_t launch_d(const AttnParams& p, const CUtensorMap& k_map, const CUtens
   if (e != cudaSuccess) return e;
   if (plan.max_splits > 1) {
     const long long rows = (long long)p.T * p.H;
-    attn_combine_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p, plan, ws);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((rows + 7) / 8));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, attn_combine_kernel<D>, p, plan, ws);
   }
   return e;
 }
