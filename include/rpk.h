@@ -140,10 +140,11 @@ rpk_status rope_freqs_cis(float* freqs_cis, int32_t max_position, int32_t rotary
 
 /*
  * ragged_paged_attention_workspace_size -- bytes of device workspace that
- * ragged_paged_attention needs for these sizes (the split-KV partials of the
- * decode path; 0 when there are no query tokens). The result depends only on
- * the arguments, so it may be computed once and reused for every call with
- * the same sizes.
+ * ragged_paged_attention needs for these sizes (the larger of the split-KV
+ * partials of the decode path and the 256-byte work counter of the prefill
+ * path; 0 when there are no query tokens). The result depends only on the
+ * arguments, so it may be computed once and reused for every call with the
+ * same sizes.
  */
 size_t ragged_paged_attention_workspace_size(int32_t total_q_tokens, int32_t n_heads,
                                              int32_t head_dim, int32_t batch,
@@ -175,9 +176,12 @@ size_t ragged_paged_attention_workspace_size(int32_t total_q_tokens, int32_t n_h
  *                   RPK_DEVERR_LENGTH and that sequence is skipped
  *   workspace       device scratch of at least
  *                   ragged_paged_attention_workspace_size(...) bytes, 256-byte
- *                   aligned (only the decode path with several splits reads it;
- *                   the other paths accept NULL). Its contents on entry do not matter;
- *                   calls sharing one workspace must not overlap in time.
+ *                   aligned. The decode path with several splits keeps its
+ *                   partial results there and the tcgen05 prefill path its work
+ *                   counter (first 4 bytes); the fp32 path and single-split
+ *                   decode accept NULL. Missing, small or misaligned where it
+ *                   is needed: RPK_ERR_WORKSPACE. Its contents on entry do not
+ *                   matter; calls sharing one workspace must not overlap in time.
  *
  * Paths (chosen from the host sizes, never from device data):
  *   dtype f32                      -> fp32 CUDA-core kernel

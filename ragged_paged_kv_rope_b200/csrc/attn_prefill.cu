@@ -8,24 +8,32 @@
 // online-softmax running state (algenta flash_attention: running max,
 // running sum and output rescaled by e^(m_old - m_new), final divide).
 //
-// Work unit: two query tiles A and B of 128 rows each against 128-key tiles.
-// The 128 rows of a tile are the (token, query head) pairs of one KV head's
-// group, token-major (tokens_per_tile = 128 / G), so the G query heads that
-// share a KV head share every K/V tile; tile B holds the next tokens_per_tile
-// tokens after tile A. One CTA per (pair of query tiles, KV head, sequence),
-// heaviest pairs first.
+// Work unit (item): two query tiles A and B of 128 rows each of one
+// (sequence, KV head), against 128-key tiles. The 128 rows of a tile are the
+// (token, query head) pairs of one KV head's group, token-major
+// (tokens_per_tile = 128 / G), so the G query heads that share a KV head share
+// every K/V tile; tile B holds the next tokens_per_tile tokens after tile A.
+//
+// Persistent launch: one CTA per SM claims items from a counter in the
+// caller's workspace (zeroed by the launch). Items run sequence by sequence,
+// the last (longest) query pair of a sequence first: the CTAs that work on one
+// sequence at the same time read the same K/V tiles in the same order, so a
+// tile read from HBM for one of them is an L2 hit for the others.
 //
 // Warp roles (384 threads, three warpgroups):
-//   warp 0     TMA producer: both Q tiles once, then K and V tiles of 128 keys
-//              into a 2-stage ring, one box per page segment (3-D map over the
-//              pool [pages * page_size, kv_heads, d], 128-byte swizzle, no
-//              multicast)
+//   warp 0     TMA producer: claims the next item, hands its index to the
+//              other roles through a two-slot ring in shared memory, loads the
+//              item's Q tiles, then its K and V tiles of 128 keys into a ring
+//              of stages (3-D map over the pool [pages * page_size, kv_heads,
+//              d], one box per page segment, 128-byte swizzle, no multicast)
 //   warp 1     allocates TMEM (512 columns: S_A, S_B, O_A, O_B) and issues the
 //              MMAs from one thread, alternating the tiles: S_t = Q_t K_j^T
 //              (operands in shared memory), then O_t += P_t V_j with P_t read
 //              from TMEM (written over the first 64 columns of S_t) and V_j an
 //              MN-major operand in shared memory. While one softmax warpgroup
-//              works on its tile, the tensor core runs the other tile's MMAs.
+//              works on its tile, the tensor core runs the other tile's MMAs;
+//              the next item's first S MMAs run while the softmax warps
+//              store the current item's rows.
 //   warps 2-3  idle (they complete the first warpgroup)
 //   warps 4-7  softmax of tile A, warps 8-11 softmax of tile B: thread r owns
 //              row r (TMEM lane r); loads S_t, masks the band, keeps (m, l) in
@@ -33,10 +41,12 @@
 //              TMEM only when the running max grew by more than 2^8 (the final
 //              O / l uses the same max, so this is exact); then normalises O_t
 //              and stores the rows.
-// Registers: the first warpgroup gives registers back (setmaxnreg 64) and the
-// two softmax warpgroups take them (setmaxnreg 208), so that a softmax thread
-// holds a whole 128-score row without spilling; 4*32*64 + 8*32*208 = 61440
-// registers, within the 384 * 168 the CTA is launched with.
+// Registers: the first warpgroup gives registers back (setmaxnreg 56) and the
+// two softmax warpgroups take them (setmaxnreg 224), so that a softmax thread
+// holds a whole 128-score row and its item state in registers (ptxas spills 24
+// bytes at this split; at 232 the softmax spills none but the control warps,
+// left with 40, spill instead);
+// 4*32*56 + 8*32*224 = 64512 registers, the 384 * 168 the CTA is launched with.
 // MMAs issued by one thread run in issue order, so P_t(j) V_j completes before
 // S_t(j+1) overwrites the columns P_t(j) lives in, and the completion of
 // S_t(j+1) also tells the softmax that O_t holds P_t(j) V_j.
@@ -44,6 +54,8 @@
 // NaN sentinels of unused slots never meet a zero weight. Every mbarrier wait
 // is bounded; on a timeout the CTA raises RPK_DEVERR_TIMEOUT, drains its copies
 // and MMAs, frees TMEM and returns.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tcgen05.cuh"
@@ -57,8 +69,8 @@ namespace {
 constexpr int kBM = 128;   // rows per tile (MMA M)
 constexpr int kBN = 128;   // keys per tile
 constexpr int kThreads = 384;
-constexpr int kRegsControl = 64;    // warpgroup 0: producer, MMA issuer, 2 idle warps
-constexpr int kRegsSoftmax = 208;   // warpgroups 1 and 2: softmax
+constexpr int kRegsControl = 56;    // warpgroup 0: producer, MMA issuer, 2 idle warps
+constexpr int kRegsSoftmax = 224;   // warpgroups 1 and 2: softmax
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows > 2^8
 
@@ -112,7 +124,8 @@ struct Cfg {
 };
 
 struct Bars {
-  uint64_t q_full;
+  uint64_t q_full[2];   // per query tile
+  uint64_t q_empty[2];  // per query tile: the item's last S MMA reading it has completed
   uint64_t k_full[4];
   uint64_t v_full[4];
   uint64_t k_empty[4];
@@ -120,6 +133,9 @@ struct Bars {
   uint64_t s_full[2];   // per query tile
   uint64_t p_full[2];   // per query tile
   uint64_t o_final[2];  // per query tile: its last P V has completed
+  uint64_t o_empty[2];  // per query tile: the epilogue has read O
+  uint64_t item_full[2];   // work-item ring: index written by the producer
+  uint64_t item_empty[2];  // work-item ring: index read by the MMA and softmax warps
   uint64_t drain;
 };
 
@@ -167,52 +183,71 @@ __device__ __forceinline__ void do_abort(volatile int* abort, int32_t* error_wor
   }
 }
 
+// One work item: a pair of query tiles of one (sequence, KV head).
+struct Item {
+  int b, kvh, q0, q_len, k_len;
+  int t_begin;      // first token of tile A
+  bool has_b;       // tile B holds at least one token
+  int j_begin;      // first key tile
+  int n_tiles;      // key tiles (0: every row sees no key)
+};
+
+// Decode work item w (items ordered by sequence, then query-pair index
+// descending, then KV head). False when the item is empty or the sequence's
+// lengths are out of bounds (then RPK_DEVERR_LENGTH is raised once).
+__device__ __forceinline__ bool decode_item(const AttnParams& p, int w, int n_qpairs, int tpt,
+                                            bool report, Item& it) {
+  const int per_seq = n_qpairs * p.Hk;
+  it.b = w / per_seq;
+  const int rem = w - it.b * per_seq;
+  const int qt = n_qpairs - 1 - rem / p.Hk;
+  it.kvh = rem - (rem / p.Hk) * p.Hk;
+  it.q0 = __ldg(p.offsets + it.b);
+  it.q_len = __ldg(p.offsets + it.b + 1) - it.q0;
+  it.k_len = __ldg(p.kv_lens + it.b);
+  if (it.q_len > p.max_q_len || it.k_len < 0 || it.k_len > p.max_kv_len) {
+    if (report && rem == 0) raise_error(p.error_word, RPK_DEVERR_LENGTH);
+    return false;
+  }
+  it.t_begin = qt * 2 * tpt;
+  if (it.t_begin >= it.q_len) return false;
+  it.has_b = it.t_begin + tpt < it.q_len;
+  const int t_end = min(it.q_len, it.t_begin + 2 * tpt);
+  const int p_first = it.t_begin + it.k_len - it.q_len;
+  const int p_last = (t_end - 1) + it.k_len - it.q_len;
+  const int lo_first = p.window > 0 ? max(0, p_first - p.window + 1) : 0;
+  const int hi_all = min(p_last, it.k_len - 1);
+  it.j_begin = 0;
+  it.n_tiles = 0;
+  if (hi_all >= lo_first) {
+    it.j_begin = lo_first / kBN;
+    it.n_tiles = hi_all / kBN + 1 - it.j_begin;
+  }
+  return true;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_prefill_kernel(const AttnParams p, const __grid_constant__ CUtensorMap q_map,
                         const __grid_constant__ CUtensorMap k_map,
                         const __grid_constant__ CUtensorMap v_map, const int tpt,
-                        const int n_qtiles) {
+                        const int n_qpairs, int* __restrict__ work_counter) {
   using C = Cfg<D>;
+  constexpr int S = C::kStages;
+  constexpr int kItemReaders = 9;  // MMA warp + 8 softmax warps
   extern __shared__ uint8_t smem_raw[];
   __shared__ Bars bars;
+  __shared__ int item_slot[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
+  __shared__ int skip_sh;
   volatile int* abort = &abort_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // The q-tile index is the slowest grid dimension, reversed: the first waves
-  // hold the last (heaviest) tile of every (sequence, KV head), so the long
-  // tiles start first and the short ones fill the tail.
-  const int qt = n_qtiles - 1 - (int)blockIdx.z;
-  const int kvh = blockIdx.x, b = blockIdx.y;
-  const int q0 = __ldg(p.offsets + b);
-  const int q_len = __ldg(p.offsets + b + 1) - q0;
-  const int k_len = __ldg(p.kv_lens + b);
-  if (q_len > p.max_q_len || k_len < 0 || k_len > p.max_kv_len) {
-    if (threadIdx.x == 0 && blockIdx.z == 0 && kvh == 0) raise_error(p.error_word, RPK_DEVERR_LENGTH);
-    return;
-  }
-  const int t_begin = qt * 2 * tpt;           // first token of tile A
-  if (t_begin >= q_len) return;
-  if (timed_out_elsewhere(p.error_word)) return;
-  const bool has_b = t_begin + tpt < q_len;    // tile B holds at least one token
-  const int t_end = min(q_len, t_begin + 2 * tpt);
+  const int n_items = n_qpairs * p.batch * p.Hk;
   const int G = p.G;
   const int rows_used = tpt * G;
 
-  // Keys any row of the two tiles sees, in whole key tiles.
-  const int p_first = t_begin + k_len - q_len;
-  const int p_last = (t_end - 1) + k_len - q_len;
-  const int lo_first = p.window > 0 ? max(0, p_first - p.window + 1) : 0;
-  const int hi_all = min(p_last, k_len - 1);
-  int j_begin = 0, n_tiles = 0;
-  if (hi_all >= lo_first) {
-    j_begin = lo_first / kBN;
-    n_tiles = hi_all / kBN + 1 - j_begin;
-  }
-
-  constexpr int S = C::kStages;
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const uint32_t sbase = smem_u32(smem);
@@ -221,7 +256,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto v_s = [&](int st) { return sbase + C::kVOff + st * C::kKVBytes; };
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars.q_full, 1);
     for (int st = 0; st < S; ++st) {
       mbar_init(&bars.k_full[st], 1);
       mbar_init(&bars.v_full[st], 1);
@@ -229,12 +263,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.v_empty[st], 1);
     }
     for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars.q_full[t], 1);
+      mbar_init(&bars.q_empty[t], 1);
       mbar_init(&bars.s_full[t], 1);
       mbar_init(&bars.p_full[t], 128);
       mbar_init(&bars.o_final[t], 1);
+      mbar_init(&bars.o_empty[t], 128);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&bars.item_full[k], 1);
+      mbar_init(&bars.item_empty[k], kItemReaders);
     }
     mbar_init(&bars.drain, 1);
     abort_sh = 0;
+    // Read once and shared, so that every thread takes the same branch below.
+    skip_sh = timed_out_elsewhere(p.error_word) ? 1 : 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -245,85 +288,142 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = tmem_base_sh;
-  const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
 
-  if (warp == 0) {
+  if (skip_sh) {
+    // An earlier CTA timed out: free TMEM below and leave.
+  } else if (warp == 0) {
     // ------------------------------------------------------------ producer
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
     if (lane == 0) {
       prefetch_tensormap(&q_map);
       prefetch_tensormap(&k_map);
       prefetch_tensormap(&v_map);
-      const int n_q = has_b ? 2 : 1;
       const uint32_t q_box_bytes = 128u * (uint32_t)rows_used;
-      mbar_arrive_expect_tx(&bars.q_full, n_q * C::kBoxes * q_box_bytes);
-      for (int t = 0; t < n_q; ++t)
-#pragma unroll
-        for (int bx = 0; bx < C::kBoxes; ++bx)
-          tma_load_3d(smem + C::kQOff + t * C::kQBytes + bx * (kBM * 128), &q_map, bx * 64,
-                      kvh * G, q0 + t_begin + t * tpt, &bars.q_full);
       const int box_rows = p.P < kBN ? p.P : kBN;
       const uint32_t seg_bytes = (uint32_t)box_rows * 128u * C::kBoxes;
-      int issued = 0;
-      // K_i and V_i go to stage i % S; K of a stage frees after the last S
-      // MMA that reads it, V after the last P V, so K runs ahead of V.
-      auto load = [&](int i, bool is_v) -> bool {
-        const int st = i % S;
-        uint64_t* empty = is_v ? &bars.v_empty[st] : &bars.k_empty[st];
-        uint64_t* full = is_v ? &bars.v_full[st] : &bars.k_full[st];
-        if (i >= S && !thread_wait(empty, ((i / S) & 1) ^ 1, abort, p.error_word)) return false;
-        const int key0 = (j_begin + i) * kBN;
-        uint32_t bytes = 0;
-        for (int r = 0; r < kBN; r += box_rows) {
-          const int key = key0 + r;
-          if (key >= k_len) break;
-          const int pi = key / p.P;
-          const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
-          if (page >= 0 && page < p.num_pages) bytes += seg_bytes;
-        }
-        mbar_arrive_expect_tx(full, bytes);
-        for (int r = 0; r < kBN; r += box_rows) {
-          const int key = key0 + r;
-          if (key >= k_len) break;
-          const int pi = key / p.P;
-          const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
-          if (page < 0 || page >= p.num_pages) {
-            if (!is_v) raise_error(p.error_word, RPK_DEVERR_PAGE);
-            continue;
-          }
-          const int grow = page * p.P + (key - pi * p.P);
-          uint8_t* base = smem + (is_v ? C::kVOff : C::kKOff) + st * C::kKVBytes + r * 128;
+      int g = 0;                // first global key tile of the current item
+      int k_issued = 0, v_issued = 0;  // K / V tile loads issued over all items
+      int q_loads[2] = {0, 0};  // Q loads per tile over all items
+      bool ok = true;
+      // Claim a non-empty work item and hand its index to the MMA and softmax warps through the ring. The next
+      // item is claimed after the current one's Q and first K/V stages are in
+      // flight, so the claim's latency hides behind real work.
+      auto claim = [&](Item& it) -> int {
+        int w;
+        do {
+          w = atomicAdd(work_counter, 1);
+        } while (w < n_items && !decode_item(p, w, n_qpairs, tpt, true, it));
+        return w < n_items ? w : -1;
+      };
+      auto publish = [&](int seq, int w) -> bool {
+        const int slot = seq & 1;
+        if (seq >= 2 &&
+            !thread_wait(&bars.item_empty[slot], ((seq >> 1) & 1) ^ 1, abort, p.error_word))
+          return false;
+        *reinterpret_cast<volatile int*>(&item_slot[slot]) = w;
+        mbar_arrive(&bars.item_full[slot]);
+        return true;
+      };
+      // Q tiles of an item: each buffer is refilled once the previous item's
+      // S MMAs that read it have completed.
+      auto load_q = [&](const Item& it) -> bool {
+        for (int t = 0; t < (it.has_b ? 2 : 1); ++t) {
+          if (q_loads[t] > 0 &&
+              !thread_wait(&bars.q_empty[t], (q_loads[t] - 1) & 1, abort, p.error_word))
+            return false;
+          mbar_arrive_expect_tx(&bars.q_full[t], C::kBoxes * q_box_bytes);
 #pragma unroll
           for (int bx = 0; bx < C::kBoxes; ++bx)
-            tma_load_3d(base + bx * (kBN * 128), is_v ? &v_map : &k_map, bx * 64, kvh, grow, full);
+            tma_load_3d(smem + C::kQOff + t * C::kQBytes + bx * (kBM * 128), &q_map, bx * 64,
+                        it.kvh * G, it.q0 + it.t_begin + t * tpt, &bars.q_full[t]);
+          ++q_loads[t];
         }
         return true;
       };
-      for (int i = 0; i < n_tiles; ++i) {
-        if (!load(i, false) || !load(i, true)) {
-          do_abort(abort, p.error_word);
-          break;
+      // K and V of key tile i of an item (global tile index g + i); K of a
+      // stage frees after the last S MMA that reads it, V after the last P V.
+      auto load_kv = [&](const Item& it, int i) -> bool {
+        const int32_t* bt = p.block_table + (size_t)it.b * p.max_pages;
+        const int gi = g + i;
+        const int st = gi % S;
+        const int key0 = (it.j_begin + i) * kBN;
+        for (int is_v = 0; is_v < 2; ++is_v) {
+          uint64_t* empty = is_v ? &bars.v_empty[st] : &bars.k_empty[st];
+          uint64_t* full = is_v ? &bars.v_full[st] : &bars.k_full[st];
+          if (gi >= S && !thread_wait(empty, ((gi / S) & 1) ^ 1, abort, p.error_word))
+            return false;
+          uint32_t bytes = 0;
+          for (int r = 0; r < kBN; r += box_rows) {
+            const int key = key0 + r;
+            if (key >= it.k_len) break;
+            const int pi = key / p.P;
+            const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
+            if (page >= 0 && page < p.num_pages) bytes += seg_bytes;
+          }
+          mbar_arrive_expect_tx(full, bytes);
+          for (int r = 0; r < kBN; r += box_rows) {
+            const int key = key0 + r;
+            if (key >= it.k_len) break;
+            const int pi = key / p.P;
+            const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
+            if (page < 0 || page >= p.num_pages) {
+              if (!is_v) raise_error(p.error_word, RPK_DEVERR_PAGE);
+              continue;
+            }
+            const int grow = page * p.P + (key - pi * p.P);
+            uint8_t* base = smem + (is_v ? C::kVOff : C::kKOff) + st * C::kKVBytes + r * 128;
+#pragma unroll
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+              tma_load_3d(base + bx * (kBN * 128), is_v ? &v_map : &k_map, bx * 64, it.kvh,
+                          grow, full);
+          }
+          if (is_v) ++v_issued; else ++k_issued;
         }
-        ++issued;
+        return true;
+      };
+      Item cur;
+      int cur_w = claim(cur);
+      ok = publish(0, cur_w);
+      for (int seq = 0; ok && cur_w >= 0; ++seq) {
+        const int n = cur.n_tiles;
+        const int first = n < S ? n : S;
+        if (n > 0) {
+          ok = load_q(cur);
+          for (int i = 0; ok && i < first; ++i) ok = load_kv(cur, i);
+        }
+        if (!ok) break;
+        Item next;
+        const int next_w = claim(next);
+        if (!publish(seq + 1, next_w)) { ok = false; break; }
+        for (int i = first; ok && i < n; ++i) ok = load_kv(cur, i);
+        if (!ok) break;
+        g += n;
+        cur = next;
+        cur_w = next_w;
       }
+      if (!ok) do_abort(abort, p.error_word);
       // Never leave with copies in flight.
-      mbar_wait(&bars.q_full, 0);
-      for (int i = max(0, issued - S); i < issued; ++i) {
-        mbar_wait(&bars.k_full[i % S], (i / S) & 1);
-        mbar_wait(&bars.v_full[i % S], (i / S) & 1);
-      }
+      for (int t = 0; t < 2; ++t)
+        if (q_loads[t] > 0) mbar_wait(&bars.q_full[t], (q_loads[t] - 1) & 1);
+      for (int gi = max(0, k_issued - S); gi < k_issued; ++gi)
+        mbar_wait(&bars.k_full[gi % S], (gi / S) & 1);
+      for (int gi = max(0, v_issued - S); gi < v_issued; ++gi)
+        mbar_wait(&bars.v_full[gi % S], (gi / S) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
     constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(kBM, kBN, 0);
     constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(kBM, D, 1);
-    bool ok = warp_wait(&bars.q_full, 0, abort, p.error_word);
-    tc::fence_after_sync();
-    // S_t = Q_t K_i^T into S_t's columns.
-    auto issue_s = [&](int t, int i) {
+    int g = 0;                          // key tiles consumed over all items
+    int q_seen[2] = {0, 0};             // Q loads consumed per tile
+    int s_issued[2] = {0, 0};           // S MMAs (= s_full commits) per tile
+    int p_seen[2] = {0, 0};             // p_full phases consumed per tile
+    int o_commits[2] = {0, 0};          // o_final commits per tile
+    bool ok = true;
+    auto issue_s = [&](int t, int gi) {
       if (lane == 0) {
-        const int st = i % S;
+        const int st = gi % S;
         const uint32_t d_tmem = tmem + C::kSCol + (uint32_t)(t * kBN);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -335,82 +435,113 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::commit(smem_u32(&bars.s_full[t]));
       }
       __syncwarp();
+      ++s_issued[t];
     };
-    // O_t += P_t V_i, P_t in the first 64 columns of S_t.
-    auto issue_pv = [&](int t, int i) {
+    auto issue_pv = [&](int t, int gi, bool first) {
       if (lane == 0) {
-        const int st = i % S;
+        const int st = gi % S;
         const uint32_t d_tmem = tmem + C::kOCol + (uint32_t)(t * D);
         const uint32_t a_tmem = tmem + C::kSCol + (uint32_t)(t * kBN);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
           tc::mma_ts(d_tmem, a_tmem + kk * 8,
                      tc::smem_desc_sw128(v_s(st) + kk * (16 * 128), kBN * 128, 1024), idesc_pv,
-                     (i > 0 || kk > 0) ? 1u : 0u);
+                     (!first || kk > 0) ? 1u : 0u);
       }
       __syncwarp();
     };
-    if (ok && n_tiles > 0) {
-      ok = warp_wait(&bars.k_full[0], 0, abort, p.error_word);
-      tc::fence_after_sync();
-      if (ok) {
-        issue_s(0, 0);
-        if (has_b) issue_s(1, 0);
-        if (lane == 0) tc::commit(smem_u32(&bars.k_empty[0]));
-        __syncwarp();
-      }
-    }
-    for (int i = 0; ok && i < n_tiles; ++i) {
-      const int st = i % S;
-      const bool last = i + 1 == n_tiles;
-      // tile A: P_A(i) V_i, then S_A(i+1)
-      if (!warp_wait(&bars.p_full[0], i & 1, abort, p.error_word)) { ok = false; break; }
-      if (!warp_wait(&bars.v_full[st], (i / S) & 1, abort, p.error_word)) { ok = false; break; }
-      tc::fence_after_sync();
-      const int key0 = (j_begin + i) * kBN;
-      if (key0 + kBN > k_len) {
-        // zero value rows at or past k_len
-        const int r0 = max(0, k_len - key0);
-        const int chunks = (kBN - r0) * C::kBoxes * 8;
-        for (int idx = lane; idx < chunks; idx += 32) {
-          const int ch = idx & 7;
-          const int rb = idx >> 3;
-          const int bx = rb % C::kBoxes;
-          const int r = r0 + rb / C::kBoxes;
-          uint8_t* dst = smem + C::kVOff + st * C::kKVBytes + bx * (kBN * 128) + r * 128 + ch * 16;
-          *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-      }
-      issue_pv(0, i);
-      if (last && lane == 0) tc::commit(smem_u32(&bars.o_final[0]));
-      if (!last) {
-        if (!warp_wait(&bars.k_full[(i + 1) % S], ((i + 1) / S) & 1, abort, p.error_word)) {
-          ok = false;
-          break;
-        }
-        tc::fence_after_sync();
-        issue_s(0, i + 1);
-      }
-      // tile B: P_B(i) V_i, then S_B(i+1)
-      if (has_b) {
-        if (!warp_wait(&bars.p_full[1], i & 1, abort, p.error_word)) { ok = false; break; }
-        tc::fence_after_sync();
-        issue_pv(1, i);
-        if (last && lane == 0) tc::commit(smem_u32(&bars.o_final[1]));
-      }
-      if (lane == 0) tc::commit(smem_u32(&bars.v_empty[st]));
+    auto commit_to = [&](uint64_t* bar) {
+      if (lane == 0) tc::commit(smem_u32(bar));
       __syncwarp();
-      if (has_b && !last) issue_s(1, i + 1);
-      // K_{i+1} has now been read by every S MMA that needs it.
-      if (!last && lane == 0) tc::commit(smem_u32(&bars.k_empty[(i + 1) % S]));
+    };
+    for (int seq = 0; ok; ++seq) {
+      const int slot = seq & 1;
+      if (!warp_wait(&bars.item_full[slot], (seq >> 1) & 1, abort, p.error_word)) {
+        ok = false;
+        break;
+      }
+      const int w = *reinterpret_cast<volatile int*>(&item_slot[slot]);
       __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.item_empty[slot]);
+      if (w < 0) break;
+      Item it;
+      if (!decode_item(p, w, n_qpairs, tpt, false, it) || it.n_tiles == 0) continue;
+      const int nq = it.has_b ? 2 : 1;
+      const int n = it.n_tiles;
+      for (int t = 0; t < nq && ok; ++t) {
+        ok = warp_wait(&bars.q_full[t], q_seen[t] & 1, abort, p.error_word);
+        ++q_seen[t];
+      }
+      if (ok) ok = warp_wait(&bars.k_full[g % S], (g / S) & 1, abort, p.error_word);
+      if (!ok) break;
+      tc::fence_after_sync();
+      for (int t = 0; t < nq; ++t) issue_s(t, g);
+      commit_to(&bars.k_empty[g % S]);
+      if (n == 1)
+        for (int t = 0; t < nq; ++t) commit_to(&bars.q_empty[t]);
+      for (int i = 0; ok && i < n; ++i) {
+        const int gi = g + i;
+        const int st = gi % S;
+        const bool last = i + 1 == n;
+        for (int t = 0; t < nq; ++t) {
+          // P_t(i) V_i
+          if (!warp_wait(&bars.p_full[t], p_seen[t] & 1, abort, p.error_word)) { ok = false; break; }
+          ++p_seen[t];
+          if (t == 0) {
+            if (!warp_wait(&bars.v_full[st], (gi / S) & 1, abort, p.error_word)) { ok = false; break; }
+            tc::fence_after_sync();
+            const int key0 = (it.j_begin + i) * kBN;
+            if (key0 + kBN > it.k_len) {
+              // zero value rows at or past k_len
+              const int r0 = max(0, it.k_len - key0);
+              const int chunks = (kBN - r0) * C::kBoxes * 8;
+              for (int idx = lane; idx < chunks; idx += 32) {
+                const int ch = idx & 7;
+                const int rb = idx >> 3;
+                const int bx = rb % C::kBoxes;
+                const int r = r0 + rb / C::kBoxes;
+                uint8_t* dst =
+                    smem + C::kVOff + st * C::kKVBytes + bx * (kBN * 128) + r * 128 + ch * 16;
+                *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+            }
+          }
+          tc::fence_after_sync();
+          if (i == 0 && o_commits[t] > 0) {
+            // O_t of the previous item has been read by its epilogue.
+            if (!warp_wait(&bars.o_empty[t], (o_commits[t] - 1) & 1, abort, p.error_word)) {
+              ok = false;
+              break;
+            }
+            tc::fence_after_sync();
+          }
+          issue_pv(t, gi, i == 0);
+          if (last) {
+            commit_to(&bars.o_final[t]);
+            ++o_commits[t];
+          } else {
+            // S_t(i+1) overwrites the columns P_t(i) lives in; the MMAs run in
+            // issue order, so P_t(i) V_i has read them by then.
+            if (t == 0) {
+              if (!warp_wait(&bars.k_full[(gi + 1) % S], ((gi + 1) / S) & 1, abort,
+                             p.error_word)) { ok = false; break; }
+              tc::fence_after_sync();
+            }
+            issue_s(t, gi + 1);
+            if (i + 2 == n) commit_to(&bars.q_empty[t]);  // last S_t of this item
+          }
+        }
+        if (!ok) break;
+        commit_to(&bars.v_empty[st]);
+        if (!last) commit_to(&bars.k_empty[(gi + 1) % S]);
+      }
+      if (ok) g += n;
     }
     if (!ok) do_abort(abort, p.error_word);
     // Drain: every MMA issued above has completed before TMEM is freed.
-    if (lane == 0) tc::commit(smem_u32(&bars.drain));
-    __syncwarp();
+    commit_to(&bars.drain);
     if (!warp_wait(&bars.drain, 0, abort, p.error_word)) mbar_wait(&bars.drain, 0);
   } else if (warp < 4) {
     // idle warps of the first warpgroup
@@ -421,126 +552,149 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = (warp - 4) >> 2;       // query tile: warps 4-7 -> A, 8-11 -> B
     const int qw = warp & 3;             // TMEM lane quarter of this warp
     const int r = qw * 32 + lane;        // row of this thread
-    const int tok = t_begin + t * tpt + r / G;
-    const bool row_ok = r < rows_used && tok < q_len;
-    const int pos = tok + k_len - q_len;
-    const int lo = p.window > 0 ? pos - p.window + 1 : 0;
-    const int hi = pos;
     const uint32_t lane_base = (uint32_t)(qw * 32) << 16;
     const uint32_t s_col = tmem + lane_base + C::kSCol + (uint32_t)(t * kBN);
     const uint32_t o_col = tmem + lane_base + C::kOCol + (uint32_t)(t * D);
     const float sl2 = p.scale_log2;
-    const int my_tiles = (t == 0 || has_b) ? n_tiles : 0;
-    float m = -INFINITY, l = 0.f;        // running max (log2 units) and sum
+    int s_seen = 0, o_seen = 0;
     bool ok = true;
-    float v[kBN];
-    for (int i = 0; i < my_tiles; ++i) {
-      if (!warp_wait(&bars.s_full[t], i & 1, abort, p.error_word)) { ok = false; break; }
-      tc::fence_after_sync();
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) tc::tmem_ld32(s_col + c * 32, v + c * 32);
-      tc::tmem_wait_ld();
-      const int key0 = (j_begin + i) * kBN;
-      if (!(row_ok && key0 >= lo && key0 + kBN - 1 <= hi)) {
-        // visible columns [c_lo, c_hi] of this tile (empty for an invalid row)
-        const int c_lo = row_ok ? lo - key0 : kBN;
-        const int c_hi = row_ok ? hi - key0 : -1;
-#pragma unroll
-        for (int c = 0; c < kBN; ++c)
-          if (c < c_lo || c > c_hi) v[c] = -INFINITY;
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+    for (int seq = 0; ok; ++seq) {
+      const int slot = seq & 1;
+      if (!warp_wait(&bars.item_full[slot], (seq >> 1) & 1, abort, p.error_word)) {
+        ok = false;
+        break;
       }
-      // Row max: 8 independent chains of three-input max.
-      float m8[8];
+      const int w = *reinterpret_cast<volatile int*>(&item_slot[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.item_empty[slot]);
+      if (w < 0) break;
+      Item it;
+      if (!decode_item(p, w, n_qpairs, tpt, false, it)) continue;
+      if (t == 1 && !it.has_b) continue;
+      const int tok = it.t_begin + t * tpt + r / G;
+      const bool row_ok = r < rows_used && tok < it.q_len;
+      const int pos = tok + it.k_len - it.q_len;
+      const int lo = p.window > 0 ? pos - p.window + 1 : 0;
+      const int hi = pos;
+      const int n = it.n_tiles;
+      float m = -INFINITY, l = 0.f;      // running max (log2 units) and sum
+      float v[kBN];
+      for (int i = 0; i < n; ++i) {
+        if (!warp_wait(&bars.s_full[t], s_seen & 1, abort, p.error_word)) { ok = false; break; }
+        ++s_seen;
+        tc::fence_after_sync();
 #pragma unroll
-      for (int k = 0; k < 8; ++k) m8[k] = fmaxf(v[k], v[8 + k]);
+        for (int c = 0; c < kBN / 32; ++c) tc::tmem_ld32(s_col + c * 32, v + c * 32);
+        tc::tmem_wait_ld();
+        const int key0 = (it.j_begin + i) * kBN;
+        if (!(row_ok && key0 >= lo && key0 + kBN - 1 <= hi)) {
+          // visible columns [c_lo, c_hi] of this tile (empty for an invalid row)
+          const int c_lo = row_ok ? lo - key0 : kBN;
+          const int c_hi = row_ok ? hi - key0 : -1;
 #pragma unroll
-      for (int c = 16; c < kBN; c += 16)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) m8[k] = max3(m8[k], v[c + k], v[c + 8 + k]);
-      float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-      mx *= sl2;  // scale > 0: max of the scaled scores
-      // Running max: taken at once while empty, else only when it grows by
-      // more than the threshold (then O and l are rescaled). O_t holds
-      // P_t(i-1) V_{i-1} here: S_t(i) was issued after it and has completed.
-      float alpha = 1.f;
-      bool rescale = false;
-      if (m == -INFINITY) {
-        m = mx;
-      } else if (mx > m + kRescaleThreshold) {
-        alpha = fast_exp2(m - mx);
-        m = mx;
-        rescale = true;
-      }
-      l *= alpha;
-      const float neg_m = m == -INFINITY ? 0.f : -m;  // an empty row keeps P = 0
-      float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 4 packed partial sums
-      // P in two halves of 64 keys (32 packed columns each) to bound registers.
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          float x0, x1;
-          fma2(x0, x1, v[h * 64 + c], v[h * 64 + c + 1], sl2, neg_m);
-          const float w0 = fast_exp2(x0);
-          const float w1 = fast_exp2(x1);
-          const int k = (c >> 1) & 3;
-          add2(rs[2 * k], rs[2 * k + 1], w0, w1);
-          pk[c >> 1] = pack_bf16x2(w0, w1);
+          for (int c = 0; c < kBN; ++c)
+            if (c < c_lo || c > c_hi) v[c] = -INFINITY;
         }
-        tc::tmem_st32(s_col + h * 32, reinterpret_cast<const float*>(pk));
-      }
-      l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
-      // Rescale O_t (after P, so that the scores are dead): it must finish
-      // before P_t(i) V_i is issued, i.e. before p_full.
-      if (i > 0 && __any_sync(0xffffffffu, rescale)) {
-        float o[32];
+        // Row max: 8 independent chains of three-input max.
+        float m8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m8[k] = fmaxf(v[k], v[8 + k]);
+#pragma unroll
+        for (int c = 16; c < kBN; c += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) m8[k] = max3(m8[k], v[c + k], v[c + 8 + k]);
+        float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+        mx *= sl2;  // scale > 0: max of the scaled scores
+        // Running max: taken at once while empty, else only when it grows by
+        // more than the threshold (then O and l are rescaled). O_t holds
+        // P_t(i-1) V_{i-1} here: S_t(i) was issued after it and has completed.
+        float alpha = 1.f;
+        bool rescale = false;
+        if (m == -INFINITY) {
+          m = mx;
+        } else if (mx > m + kRescaleThreshold) {
+          alpha = fast_exp2(m - mx);
+          m = mx;
+          rescale = true;
+        }
+        l *= alpha;
+        const float neg_m = m == -INFINITY ? 0.f : -m;  // an empty row keeps P = 0
+        float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
+        // P in two halves of 64 keys (32 packed columns each) to bound registers.
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            float x0, x1;
+            fma2(x0, x1, v[h * 64 + c], v[h * 64 + c + 1], sl2, neg_m);
+            const float w0 = fast_exp2(x0);
+            const float w1 = fast_exp2(x1);
+            const int k = (c >> 1) & 3;
+            add2(rs[2 * k], rs[2 * k + 1], w0, w1);
+            pk[c >> 1] = pack_bf16x2(w0, w1);
+          }
+          tc::tmem_st32(s_col + h * 32, reinterpret_cast<const float*>(pk));
+        }
+        l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+        // Rescale O_t (after P, so that the scores are dead): it must finish
+        // before P_t(i) V_i is issued, i.e. before p_full.
+        if (i > 0 && __any_sync(0xffffffffu, rescale)) {
+          float o[32];
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
+            tc::tmem_ld32(o_col + c * 32, o);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tc::tmem_st32(o_col + c * 32, o);
+          }
+        }
+        tc::tmem_wait_st();
+        tc::fence_before_sync();
+        mbar_arrive(&bars.p_full[t]);
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      const bool have_o = n > 0;
+      if (have_o) {
+        if (!warp_wait(&bars.o_final[t], o_seen & 1, abort, p.error_word)) { ok = false; break; }
+        ++o_seen;
+        tc::fence_after_sync();
+      }
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      const size_t orow = ((size_t)(it.q0 + tok) * p.H + (size_t)it.kvh * G + (r % G)) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        if (have_o) {
           tc::tmem_ld32(o_col + c * 32, o);
           tc::tmem_wait_ld();
+          if (c + 1 == D / 32) {
+            // O_t may now be overwritten by the next item's first P V.
+            tc::fence_before_sync();
+            mbar_arrive(&bars.o_empty[t]);
+          }
+        }
+        if (row_ok) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tc::tmem_st32(o_col + c * 32, o);
+          for (int e8 = 0; e8 < 4; ++e8) {
+            uint4 q4;
+            if (have_o && l > 0.f) {
+              q4.x = pack_bf16x2(o[e8 * 8 + 0] * inv, o[e8 * 8 + 1] * inv);
+              q4.y = pack_bf16x2(o[e8 * 8 + 2] * inv, o[e8 * 8 + 3] * inv);
+              q4.z = pack_bf16x2(o[e8 * 8 + 4] * inv, o[e8 * 8 + 5] * inv);
+              q4.w = pack_bf16x2(o[e8 * 8 + 6] * inv, o[e8 * 8 + 7] * inv);
+            } else {
+              q4 = make_uint4(0, 0, 0, 0);
+            }
+            *reinterpret_cast<uint4*>(out + orow + c * 32 + e8 * 8) = q4;
+          }
         }
       }
-      tc::tmem_wait_st();
-      tc::fence_before_sync();
-      mbar_arrive(&bars.p_full[t]);
     }
     if (!ok) do_abort(abort, p.error_word);
-    // ------------------------------------------------------------ epilogue
-    bool have_o = my_tiles > 0;
-    if (have_o) {
-      have_o = warp_wait(&bars.o_final[t], 0, abort, p.error_word);
-      tc::fence_after_sync();
-    }
-    const float inv = (l > 0.f) ? 1.f / l : 0.f;
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-    const size_t orow = ((size_t)(q0 + tok) * p.H + (size_t)kvh * G + (r % G)) * D;
-#pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
-      float o[32];
-      if (have_o) {
-        tc::tmem_ld32(o_col + c * 32, o);
-        tc::tmem_wait_ld();
-      }
-      if (row_ok) {
-#pragma unroll
-        for (int e8 = 0; e8 < 4; ++e8) {
-          uint4 q4;
-          if (have_o && l > 0.f) {
-            q4.x = pack_bf16x2(o[e8 * 8 + 0] * inv, o[e8 * 8 + 1] * inv);
-            q4.y = pack_bf16x2(o[e8 * 8 + 2] * inv, o[e8 * 8 + 3] * inv);
-            q4.z = pack_bf16x2(o[e8 * 8 + 4] * inv, o[e8 * 8 + 5] * inv);
-            q4.w = pack_bf16x2(o[e8 * 8 + 6] * inv, o[e8 * 8 + 7] * inv);
-          } else {
-            q4 = make_uint4(0, 0, 0, 0);
-          }
-          *reinterpret_cast<uint4*>(out + orow + c * 32 + e8 * 8) = q4;
-        }
-      }
-    }
   }
 
   tc::fence_before_sync();
@@ -551,20 +705,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+int sm_count() {
+  static int n[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (n[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    n[dev] = v;
+  }
+  return n[dev];
+}
+
 template <int D>
 cudaError_t launch_d(const AttnParams& p, const CUtensorMap& q_map, const CUtensorMap& k_map,
-                     const CUtensorMap& v_map, cudaStream_t stream) {
+                     const CUtensorMap& v_map, int* work_counter, cudaStream_t stream) {
   using C = Cfg<D>;
   cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int tpt = prefill_rows_per_tile(p.G);
-  const int n_qtiles = (p.max_q_len + 2 * tpt - 1) / (2 * tpt);  // pairs of query tiles
-  if (n_qtiles == 0) return cudaSuccess;
-  if (n_qtiles > 65535) return cudaErrorInvalidValue;
-  dim3 grid(p.Hk, p.batch, n_qtiles);
+  const int n_qpairs = (p.max_q_len + 2 * tpt - 1) / (2 * tpt);  // pairs of query tiles
+  const long long n_items = (long long)n_qpairs * p.batch * p.Hk;
+  if (n_items == 0) return cudaSuccess;
+  // Every CTA claims once past the last item, so the counter reaches n_items + grid.
+  if (n_items > INT32_MAX - 65536) return cudaErrorInvalidValue;
+  // Persistent: one CTA per SM; CTAs claim items from a counter the call zeroes.
+  e = cudaMemsetAsync(work_counter, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return e;
+  const int grid = (int)std::min<long long>(n_items, sm_count());
   attn_prefill_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(p, q_map, k_map, v_map, tpt,
-                                                                     n_qtiles);
+                                                                     n_qpairs, work_counter);
   return cudaGetLastError();
 }
 
@@ -572,11 +744,12 @@ cudaError_t launch_d(const AttnParams& p, const CUtensorMap& q_map, const CUtens
 
 cudaError_t launch_attn_prefill(const AttnParams& p, const CUtensorMap& q_map,
                                 const CUtensorMap& k_map, const CUtensorMap& v_map,
-                                cudaStream_t stream) {
+                                int* work_counter, cudaStream_t stream) {
   if ((long long)p.T * p.H == 0 || p.batch == 0) return cudaSuccess;
+  if (work_counter == nullptr) return cudaErrorInvalidValue;
   switch (p.d) {
-    case 64: return launch_d<64>(p, q_map, k_map, v_map, stream);
-    case 128: return launch_d<128>(p, q_map, k_map, v_map, stream);
+    case 64: return launch_d<64>(p, q_map, k_map, v_map, work_counter, stream);
+    case 128: return launch_d<128>(p, q_map, k_map, v_map, work_counter, stream);
     default: return cudaErrorInvalidValue;
   }
 }

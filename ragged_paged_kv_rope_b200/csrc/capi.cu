@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -164,7 +165,9 @@ size_t ragged_paged_attention_workspace_size(int32_t total_q_tokens, int32_t n_h
   (void)batch;
   (void)page_size;
   if (total_q_tokens <= 0 || n_heads <= 0 || head_dim <= 0 || max_kv_len < 0) return 0;
-  return rpk::decode_workspace_bytes(total_q_tokens, n_heads, head_dim, max_kv_len);
+  // The larger of the decode partials and the prefill work counter.
+  return std::max(rpk::decode_workspace_bytes(total_q_tokens, n_heads, head_dim, max_kv_len),
+                  rpk::kPrefillWorkspaceBytes);
 }
 
 rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
@@ -230,6 +233,8 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
   // Prefill shapes: tcgen05 kernel for head_dim 64 / 128 and groups up to 128.
   const int tpt = rpk::prefill_rows_per_tile(p.G);
   if ((head_dim == 64 || head_dim == 128) && tpt > 0) {
+    if (!workspace || workspace_bytes < rpk::kPrefillWorkspaceBytes) return RPK_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return RPK_ERR_WORKSPACE;
     CUtensorMap q_map, k_map, v_map;
     const int32_t box_rows = p.P < 128 ? p.P : 128;
     const int64_t pool_rows = (int64_t)p.num_pages * p.P;
@@ -239,7 +244,8 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
     if (st != RPK_OK) return st;
     st = encode_rows_map(&v_map, p.v_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
     if (st != RPK_OK) return st;
-    return cuda_status(rpk::launch_attn_prefill(p, q_map, k_map, v_map, s));
+    return cuda_status(
+        rpk::launch_attn_prefill(p, q_map, k_map, v_map, static_cast<int*>(workspace), s));
   }
   // head_dim 256 (or groups above 128): CUDA-core kernel.
   return cuda_status(rpk::launch_attn_simt(p, dtype, s));

@@ -73,10 +73,13 @@ cudaError_t launch_attn_decode(const AttnParams& p, const CUtensorMap& k_map,
                                const CUtensorMap& v_map, const DecodePlan& plan,
                                const DecodeWorkspace& ws, cudaStream_t stream);
 
-// tcgen05 prefill (bf16, head_dim 64 or 128).
+// tcgen05 prefill (bf16, head_dim 64 or 128), persistent: its CTAs claim work
+// items from `work_counter` (device int, zeroed by the launch; one per
+// concurrently running launch).
+constexpr size_t kPrefillWorkspaceBytes = 256;
 cudaError_t launch_attn_prefill(const AttnParams& p, const CUtensorMap& q_map,
                                 const CUtensorMap& k_map, const CUtensorMap& v_map,
-                                cudaStream_t stream);
+                                int* work_counter, cudaStream_t stream);
 int prefill_rows_per_tile(int group);
 
 }  // namespace rpk

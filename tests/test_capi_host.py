@@ -111,6 +111,10 @@ def test_rope_rejects_cache(L, ckw, status):
     ({"mq": 1, "mk": 1000, "ws": None, "wsb": 0}, 6),
     ({"mq": 1, "mk": 1000, "ws": FAKE + 16, "wsb": 1 << 30}, 6),  # misaligned
     ({"mq": 1, "mk": 1000, "ws": FAKE, "wsb": 64}, 6),            # too small
+    # the tcgen05 prefill path keeps its work counter in the workspace
+    ({"mq": 5, "ws": None, "wsb": 0}, 6),
+    ({"mq": 5, "ws": FAKE + 16, "wsb": 1 << 20}, 6),               # misaligned
+    ({"mq": 5, "ws": FAKE, "wsb": 128}, 6),                        # too small
 ])
 def test_attention_rejects(L, kw, status):
     assert attn(L, cache(max_pages_per_seq=16), **kw) == status
@@ -119,6 +123,8 @@ def test_attention_rejects(L, kw, status):
 def test_workspace_size(L):
     f = R.ragged_paged_attention_workspace_size
     assert f(0, 32, 128, 64, 8193, 64) == 0
+    # never below the prefill work counter's 256 bytes
+    assert f(1, 1, 64, 1, 1, 16) >= 256
     a = f(64, 32, 128, 64, 8193, 64)
     b = f(64, 32, 128, 64, 16000, 64)
     assert 0 < a <= b
