@@ -46,7 +46,7 @@ L2_BYTES = 126 * 1024 * 1024
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="rpk", choices=["rpk", "reference"])
     ap.add_argument("--workload", default="llama3_8b_decode", choices=sorted(W.SPECS))
@@ -387,11 +387,35 @@ def prefill_measure(device, world, steps=5, warmup=3):
     }
 
 
+# ------------------------------------------------------------ the metric
+
+def is_decode(wl: W.Workload) -> bool:
+    """True when the attention call takes the split-KV decode path (bf16, at
+    most 16 (token, query head) rows per KV head and sequence)."""
+    sp = wl.spec
+    return sp.dtype == "bf16" and int(wl.q_lens.max()) * (sp.n_heads // sp.n_kv_heads) <= 16
+
+
+def metric_of(wl: W.Workload):
+    """(metric, unit, amount per step, scale to the unit) of a workload: K/V
+    bytes read for decode (GB/s, HBM-bound), visible-pair FLOPs for prefill
+    (TFLOP/s, tensor-bound)."""
+    sp = wl.spec
+    if is_decode(wl):
+        elt = 2
+        return ("decode_attention_kv_GBps", "GB/s",
+                M.attention_kv_bytes(wl.q_lens, wl.kv_lens, sp.window, sp.n_kv_heads,
+                                     sp.head_dim, elt), 1e9)
+    return ("prefill_attention_TFLOPs", "TFLOP/s",
+            M.attention_flops(wl.q_lens, wl.kv_lens, sp.window, sp.n_heads, sp.head_dim), 1e12)
+
+
 # -------------------------------------------------------- the oracle on CPU
 
 def oracle_sample_time(wl: W.Workload, max_seconds: float = 20.0):
     """Time the fp64 oracle (RoPE, cache image, attention) on a bounded sample
-    of the workload's sequences; returns (seconds, kv_bytes, tokens, sample)."""
+    of the workload's sequences; returns (seconds, amount, tokens, sample,
+    threads), amount in the workload's unit (K/V bytes or visible-pair FLOPs)."""
     import oracle as O
     sp = wl.spec
     table = O.freqs_cis(wl.max_position, sp.rotary_dim, sp.theta)
@@ -409,7 +433,7 @@ def oracle_sample_time(wl: W.Workload, max_seconds: float = 20.0):
     qr = O.round_to(q_rot, code)
     t_rope = time.perf_counter() - t0
     # attention one sequence at a time until the time budget is used
-    done_b, kv_bytes, toks = 0, 0, 0
+    done_b, kv_bytes, flops, toks = 0, 0, 0, 0
     t1 = time.perf_counter()
     elt = 2 if sp.dtype == "bf16" else 4
     for b in range(sp.batch):
@@ -421,6 +445,8 @@ def oracle_sample_time(wl: W.Workload, max_seconds: float = 20.0):
         done_b += 1
         kv_bytes += M.attention_kv_bytes(wl.q_lens[b:b + 1], wl.kv_lens[b:b + 1], sp.window,
                                          sp.n_kv_heads, sp.head_dim, elt)
+        flops += M.attention_flops(wl.q_lens[b:b + 1], wl.kv_lens[b:b + 1], sp.window,
+                                   sp.n_heads, sp.head_dim)
         toks += hi - lo
         if time.perf_counter() - t1 > max_seconds:
             break
@@ -428,8 +454,9 @@ def oracle_sample_time(wl: W.Workload, max_seconds: float = 20.0):
     # RoPE ran over the whole batch; charge the sampled sequences their share
     share = done_b / sp.batch
     seconds = t_attn + t_rope * share
-    return seconds, kv_bytes, toks, f"{done_b} of {sp.batch} sequences (all rows), " \
-                                    f"RoPE + cache image + attention", threads
+    amount = kv_bytes if is_decode(wl) else flops
+    return seconds, amount, toks, f"{done_b} of {sp.batch} sequences (all rows), " \
+                                  f"RoPE + cache image + attention", threads
 
 
 # --------------------------------------------------------------------- main
@@ -448,25 +475,45 @@ def main():
     elt = 2 if sp.dtype == "bf16" else 4
     kv_bytes = M.attention_kv_bytes(wl.q_lens, wl.kv_lens, sp.window, sp.n_kv_heads,
                                     sp.head_dim, elt)
+    metric, unit, amount, scale = metric_of(wl)
+    decode = is_decode(wl)
     with ClockSampler(local) as clocks:
         total_ms, rope_ms, attn_ms = time_steps(step, args.steps, args.warmup, world, clocks)
     clk = clocks.summary()
     step_ms = max_over_ranks(total_ms / args.steps, world)
-    job_kv_bytes = sum_over_ranks(kv_bytes, world)
+    job_amount = sum_over_ranks(amount, world)
     job_tokens = sum_over_ranks(wl.total_tokens, world)
     attn_ms_mean = max_over_ranks(statistics.mean(attn_ms), world)
     rope_ms_mean = max_over_ranks(statistics.mean(rope_ms), world)
     err = int(step.error_word.item())
     peaks = load_peaks()
-    value = job_kv_bytes / (step_ms * 1e-3) / 1e9
-    achieved = kv_bytes / (attn_ms_mean * 1e-3) / 1e9
-    traffic = load_traffic("attn_decode")
+    value = job_amount / (step_ms * 1e-3) / scale
+    achieved = amount / (attn_ms_mean * 1e-3) / scale
+    traffic = load_traffic("attn_decode") if decode else None
+    if decode:
+        roofline = {"bound": "hbm", "kernel": "ragged_paged_attention (split-KV decode + combine)",
+                    "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": unit,
+                    "frac": achieved / peaks["hbm_gbs"],
+                    "traffic": None if traffic is None else traffic["bytes_per_launch"],
+                    "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"
+                    if peaks["source"] == "measured" else "fallback 6.65 TB/s",
+                    "algorithmic_bytes_per_launch": kv_bytes}
+    else:
+        kernel = ("ragged_paged_attention (tcgen05 prefill)"
+                  if sp.dtype == "bf16" and sp.head_dim in (64, 128)
+                  else "ragged_paged_attention (CUDA-core kernel)")
+        roofline = {"bound": "tensor", "kernel": kernel, "achieved": achieved,
+                    "peak": peaks["bf16_tflops"], "unit": unit,
+                    "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                    "peak_source": "measured (MEASURED_PEAKS.json bf16_tflops)"
+                    if peaks["source"] == "measured" else "fallback 1.59 PFLOP/s",
+                    "algorithmic_flops_per_launch": amount}
 
     e2e = None
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_e2e(step, max(3, args.steps // 2), 2, world)
         e2e_ms = max_over_ranks(e2e_ms, world)
-        e2e = {"value": job_kv_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e = {"value": job_amount / (e2e_ms * 1e-3) / scale, "unit": unit,
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "note": "pinned host inputs copied in, output copied out, inside the timed region"}
 
@@ -481,11 +528,11 @@ def main():
             total_s += secs
             total_b += kvb
             passes += 1
-        cpu = {"value": total_b / total_s / 1e9, "unit": "GB/s", "cores": threads,
+        cpu = {"value": total_b / total_s / scale, "unit": unit, "cores": threads,
                "kind": "oracle", "sample": f"{sample}; {passes} passes", "seconds": total_s}
 
     line = {
-        "metric": "decode_attention_kv_GBps", "value": value, "unit": "GB/s",
+        "metric": metric, "value": value, "unit": unit,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": sp.dtype,
         "data": "synthetic (seeded N(0,1) values, shuffled page tables)",
@@ -498,13 +545,7 @@ def main():
         "tokens_per_s": job_tokens / (step_ms * 1e-3),
         "breakdown_ms": {"rope_qk_paged_ragged": rope_ms_mean,
                          "ragged_paged_attention": attn_ms_mean},
-        "roofline": {"bound": "hbm", "kernel": "ragged_paged_attention (split-KV decode + combine)",
-                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": None if traffic is None else traffic["bytes_per_launch"],
-                     "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)"
-                     if peaks["source"] == "measured" else "fallback 6.65 TB/s",
-                     "algorithmic_bytes_per_launch": kv_bytes},
+        "roofline": roofline,
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": step.launches_per_step() * args.steps,
@@ -524,8 +565,10 @@ def reference_arm(args, world, rank):
         if world > 1:
             torch.distributed.destroy_process_group()
         return
-    wl = W.make(args.workload, seed=args.seed)
+    over = {} if args.batch is None else {"batch": args.batch}
+    wl = W.make(args.workload, seed=args.seed, **over)
     sp = wl.spec
+    metric, unit, _, scale = metric_of(wl)
     for _ in range(max(0, min(args.warmup, 1))):
         oracle_sample_time(wl, max_seconds=2.0)
     times, vals = [], []
@@ -533,18 +576,18 @@ def reference_arm(args, world, rank):
     for _ in range(args.steps):
         secs, kvb, toks, sample, threads = oracle_sample_time(wl, max_seconds=budget)
         times.append(secs)
-        vals.append(kvb / secs / 1e9)
+        vals.append(kvb / secs / scale)
     value = statistics.mean(vals)
     line = {
-        "impl": "reference", "metric": "decode_attention_kv_GBps", "value": value, "unit": "GB/s",
+        "impl": "reference", "metric": metric, "value": value, "unit": unit,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) values, shuffled page tables)",
         "config": {"workload": sp.name, "description": sp.description},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
                          "sample": sample},
-        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
     if world > 1:
