@@ -54,7 +54,8 @@ def _declare(L):
     L.rpko_band.argtypes = [_i32, _i32, _i32, _i32, C.POINTER(_i32), C.POINTER(_i32)]
     L.rpko_band.restype = None
     L.rpko_attention.argtypes = [_p, C.c_int, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p,
-                                 _i32, _i32, _p, _i32, C.c_double, _i32, _p, _i64, _p, C.c_int]
+                                 _i32, _i32, _p, _i32, C.c_double, _i32, _p, _i64, _p, _p,
+                                 C.c_int]
     L.rpko_attention.restype = C.c_int
     L.rpko_flash_step.argtypes = [C.POINTER(C.c_double)] * 3 + [C.c_double, C.c_double]
     L.rpko_flash_step.restype = None
@@ -174,11 +175,13 @@ def band(r: int, q_len: int, k_len: int, window: int) -> tuple[int, int]:
 
 
 def attention(q, q_offsets, kv_lens, k_pages, v_pages, block_table, n_kv_heads, scale,
-              window, rows=None, n_threads: int | None = None) -> np.ndarray:
+              window, rows=None, n_threads: int | None = None, with_lse: bool = False):
     """fp64 attention rows.
 
     rows=None: all rows, shape [T, n_heads, head_dim]. Otherwise rows is an
     int array [n, 2] of (token, head) pairs and the result is [n, head_dim].
+    with_lse: return (out, lse), lse the natural log-sum-exp of each row's
+    scores ([T, n_heads] or [n]; -inf for a row that sees no key).
     """
     qraw, code = _raw(q)
     kp, kcode = _raw(k_pages)
@@ -192,18 +195,20 @@ def attention(q, q_offsets, kv_lens, k_pages, v_pages, block_table, n_kv_heads, 
         n_threads = os.cpu_count() or 1
     if rows is None:
         out = np.empty((T, H, d), dtype=np.float64)
+        lse = np.empty((T, H), dtype=np.float64) if with_lse else None
         rptr, n = None, T * H
     else:
         rows = _i32arr(rows).reshape(-1, 2)
         out = np.empty((rows.shape[0], d), dtype=np.float64)
+        lse = np.empty(rows.shape[0], dtype=np.float64) if with_lse else None
         rptr, n = _ptr(rows), rows.shape[0]
     rc = lib().rpko_attention(_ptr(qraw), code, _ptr(offs), _ptr(kvl), len(offs) - 1, T, H,
                               int(n_kv_heads), d, _ptr(kp), _ptr(vp), kp.shape[1], kp.shape[0],
                               _ptr(bt), bt.shape[1], float(scale), int(window), rptr, n,
-                              _ptr(out), int(n_threads))
+                              _ptr(out), None if lse is None else _ptr(lse), int(n_threads))
     if rc:
         raise ValueError(f"rpko_attention failed ({rc})")
-    return out
+    return (out, lse) if with_lse else out
 
 
 def flash_step(m: float, l: float, o: float, s: float, v: float) -> tuple[float, float, float]:

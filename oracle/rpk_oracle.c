@@ -272,6 +272,7 @@ typedef struct {
   const int32_t* rows; /* pairs (t, h), or NULL for all */
   int64_t n_rows;
   double* out;         /* [n_rows, head_dim] */
+  double* lse;         /* [n_rows] or NULL */
   int status;
 } attn_job;
 
@@ -281,10 +282,15 @@ typedef struct {
   int status;
 } attn_slice;
 
-/* One output row: two passes over the visible keys (max, then weights). */
-static int attention_row(const attn_job* J, int32_t t, int32_t h, double* o, double* w) {
+/* One output row: two passes over the visible keys (max, then weights).
+ * With lse != NULL also its natural log-sum-exp of the scores, ln sum_j e^{s_j}
+ * = m + ln sum_j e^{s_j - m} (NumKong attention_packed's log_sum_exp output);
+ * -inf for a row that sees no key (an empty sum). */
+static int attention_row(const attn_job* J, int32_t t, int32_t h, double* o, double* w,
+                         double* lse) {
   int d = J->head_dim;
   for (int c = 0; c < d; ++c) o[c] = 0.0;
+  if (lse) *lse = -INFINITY;
   int b = owner_of(J->q_offsets, J->batch, t);
   if (b < 0 || h < 0 || h >= J->n_heads) return RPKO_ERR_ARG;
   int32_t q_len = J->q_offsets[b + 1] - J->q_offsets[b];
@@ -317,6 +323,7 @@ static int attention_row(const attn_job* J, int32_t t, int32_t h, double* o, dou
     w[j - lo] = exp(w[j - lo] - m);
     den += w[j - lo];
   }
+  if (lse) *lse = m + log(den);
   for (int32_t j = lo; j <= hi; ++j) {
     double wj = w[j - lo] / den;
     int32_t page = J->block_table[(size_t)b * J->max_pages_per_seq + j / J->page_size];
@@ -343,7 +350,8 @@ static void* attention_worker(void* arg) {
     int32_t t, h;
     if (J->rows) { t = J->rows[2 * i]; h = J->rows[2 * i + 1]; }
     else { t = (int32_t)(i / J->n_heads); h = (int32_t)(i % J->n_heads); }
-    S->status = attention_row(J, t, h, J->out + (size_t)i * J->head_dim, w);
+    S->status = attention_row(J, t, h, J->out + (size_t)i * J->head_dim, w,
+                              J->lse ? J->lse + i : NULL);
   }
   free(w);
   return NULL;
@@ -354,7 +362,8 @@ static void* attention_worker(void* arg) {
  * pools. Query head h reads KV head h / (n_heads / n_kv_heads). Row r of
  * sequence b (q_len rows, kv_lens[b] keys) sees keys [lo, p], p = r + kv_len -
  * q_len (rpko_band). Output fp64, one row of head_dim per requested (t, h),
- * in the order given (rows == NULL: all T * n_heads rows, t-major).
+ * in the order given (rows == NULL: all T * n_heads rows, t-major), and, when
+ * lse != NULL, each row's natural log-sum-exp of its scores (-inf when empty).
  * n_threads > 1 splits the rows over POSIX threads.
  */
 int rpko_attention(const void* q, int dtype, const int32_t* q_offsets, const int32_t* kv_lens,
@@ -362,14 +371,15 @@ int rpko_attention(const void* q, int dtype, const int32_t* q_offsets, const int
                    int32_t head_dim, const void* k_pages, const void* v_pages,
                    int32_t page_size, int32_t num_pages, const int32_t* block_table,
                    int32_t max_pages_per_seq, double scale, int32_t window,
-                   const int32_t* rows, int64_t n_rows, double* out, int n_threads) {
+                   const int32_t* rows, int64_t n_rows, double* out, double* lse,
+                   int n_threads) {
   if (!q || !q_offsets || !kv_lens || !k_pages || !v_pages || !block_table || !out)
     return RPKO_ERR_ARG;
   if (n_kv_heads <= 0 || n_heads % n_kv_heads != 0 || head_dim <= 0 || page_size <= 0)
     return RPKO_ERR_ARG;
   attn_job J = {q, dtype, q_offsets, kv_lens, batch, T, n_heads, n_kv_heads, head_dim,
                 k_pages, v_pages, page_size, num_pages, max_pages_per_seq, block_table,
-                scale, window, rows, rows ? n_rows : (int64_t)T * n_heads, out, RPKO_OK};
+                scale, window, rows, rows ? n_rows : (int64_t)T * n_heads, out, lse, RPKO_OK};
   if (n_threads < 1) n_threads = 1;
   if (n_threads > 256) n_threads = 256;
   if ((int64_t)n_threads > J.n_rows) n_threads = J.n_rows > 0 ? (int)J.n_rows : 1;

@@ -20,6 +20,7 @@ def dense_reference(q, k_dense, v_dense, q_lens, scale, window):
     Hk = k_dense[0].shape[1]
     G = H // Hk
     out = np.zeros(q.shape, dtype=np.float64)
+    lse = np.full(q.shape[:2], -np.inf)
     t0 = 0
     for b, ql in enumerate(q_lens):
         kl = k_dense[b].shape[0]
@@ -41,8 +42,11 @@ def dense_reference(q, k_dense, v_dense, q_lens, scale, window):
             w[has] = np.exp(s[has] - m[has])
             w[has] /= w[has].sum(axis=1, keepdims=True)
             out[t0:t0 + ql, h] = w @ vv if kl else 0.0
+            # log-sum-exp straight from its definition (the scores are small)
+            with np.errstate(divide="ignore"):
+                lse[t0:t0 + ql, h] = np.log(np.where(mask, np.exp(s), 0.0).sum(axis=1))
         t0 += ql
-    return out
+    return out, lse
 
 
 CASES = [
@@ -68,6 +72,10 @@ def test_oracle_matches_dense_bruteforce(idx):
     kp, vp, bt = paged(k, v, page_size=P, seed=len(q_lens))
     offs = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
     scale = 1.0 / np.sqrt(d)
-    got = O.attention(q, offs, kv_lens, kp, vp, bt, Hk, scale, w, n_threads=2)
-    want = dense_reference(q, k, v, q_lens, scale, w)
+    got, got_lse = O.attention(q, offs, kv_lens, kp, vp, bt, Hk, scale, w, n_threads=2,
+                               with_lse=True)
+    want, want_lse = dense_reference(q, k, v, q_lens, scale, w)
     assert np.max(np.abs(got - want)) < 1e-12
+    assert np.array_equal(np.isinf(got_lse), np.isinf(want_lse))
+    fin = np.isfinite(want_lse)
+    assert np.max(np.abs(got_lse[fin] - want_lse[fin]), initial=0.0) < 1e-12

@@ -33,6 +33,8 @@ MUTATIONS = {
     "running_sum_not_rescaled": ("*l = *l * alpha + p;", "*l = *l + p;"),
     "slot_row": ("int32_t row = slot % page_size;", "int32_t row = (slot + 1) % page_size;"),
     "value_weight_unnormalised": ("double wj = w[j - lo] / den;", "double wj = w[j - lo];"),
+    "lse_log_base": ("if (lse) *lse = m + log(den);", "if (lse) *lse = m + log2(den);"),
+    "lse_max_dropped": ("if (lse) *lse = m + log(den);", "if (lse) *lse = log(den);"),
 }
 
 

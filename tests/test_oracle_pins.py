@@ -256,6 +256,68 @@ def test_rows_without_keys_are_zero():
     assert not np.all(out[3] == 0.0)
 
 
+# ------------------------------------------------------ log-sum-exp output
+# NumKong attention_packed fills a (tokens, heads) log-sum-exp for training:
+# the natural log of the row's sum of e^score over its visible keys.
+
+
+def one_row_lse(q_vec, keys, scale, window=0):
+    q = np.asarray(q_vec, dtype=np.float32)[None, None, :]
+    k = np.asarray(keys, dtype=np.float32)[:, None, :]
+    kp, vp, bt = paged([k], [k], page_size=2)
+    _, lse = O.attention(q, [0, 1], [k.shape[0]], kp, vp, bt, 1, scale, window, with_lse=True)
+    return lse[0, 0]
+
+
+def test_lse_worked_example_score(golden):
+    # q.k = 8 with d = 64 scores exactly 1.0: alone, its log-sum-exp is 1.0;
+    # beside a key scoring 0 it is ln(e + 1).
+    g = golden["scaled_score"]
+    d = g["d_k"]
+    s = g["score"]
+    assert one_row_lse(e(0, d, g["dot"]), [e(0, d)], 1 / math.sqrt(d)) == s
+    lse2 = one_row_lse(e(0, d, g["dot"]), [e(0, d), np.zeros(d, np.float32)], 1 / math.sqrt(d))
+    assert lse2 == pytest.approx(math.log(math.exp(s) + 1.0), rel=1e-15)
+
+
+@pytest.mark.parametrize("n,score", [(2, 0.0), (3, 1.5), (8, -2.0), (5, 40.0)])
+def test_lse_of_equal_scores(n, score):
+    # n keys of one score s: ln(n e^s) = s + ln n.
+    d = 4
+    lse = one_row_lse(e(0, d, score), [e(0, d)] * n, 1.0)
+    assert lse == pytest.approx(score + math.log(n), rel=1e-14, abs=1e-14)
+
+
+def test_lse_of_rows_without_keys_is_minus_infinity():
+    rng = np.random.default_rng(7)
+    d = 8
+    q = rng.normal(size=(4, 1, d)).astype(np.float32)
+    k = rng.normal(size=(2, 1, d)).astype(np.float32)
+    kp, vp, bt = paged([k], [k], page_size=4)
+    _, lse = O.attention(q, [0, 4], [2], kp, vp, bt, 1, 0.5, 0, with_lse=True)
+    assert lse[0, 0] == -math.inf and lse[1, 0] == -math.inf
+    assert np.isfinite(lse[2, 0]) and np.isfinite(lse[3, 0])
+
+
+def test_lse_normalises_the_output():
+    # e^(s_j - lse) are the softmax weights: they sum to one and weight V into
+    # the output. Scores are recomputed here from the dense inputs.
+    rng = np.random.default_rng(11)
+    d, L, scale = 16, 13, 0.3
+    q = rng.normal(size=(L, 2, d)).astype(np.float32)
+    k = rng.normal(size=(L, 1, d)).astype(np.float32)
+    v = rng.normal(size=(L, 1, d)).astype(np.float32)
+    kp, vp, bt = paged([k], [v], page_size=4)
+    out, lse = O.attention(q, [0, L], [L], kp, vp, bt, 1, scale, 0, with_lse=True)
+    for r in range(L):
+        for h in range(2):
+            sc = scale * (k[:r + 1, 0].astype(np.float64) @ q[r, h].astype(np.float64))
+            w = np.exp(sc - lse[r, h])
+            assert w.sum() == pytest.approx(1.0, abs=1e-13)
+            np.testing.assert_allclose(out[r, h], w @ v[:r + 1, 0].astype(np.float64),
+                                       rtol=1e-12, atol=1e-13)
+
+
 def test_decode_equals_last_prefill_row():
     rng = np.random.default_rng(8)
     d, L, H, Hk = 16, 13, 4, 2
