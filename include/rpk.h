@@ -182,6 +182,12 @@ size_t ragged_paged_attention_workspace_size(int32_t total_q_tokens, int32_t n_h
  *                   decode accept NULL. Missing, small or misaligned where it
  *                   is needed: RPK_ERR_WORKSPACE. Its contents on entry do not
  *                   matter; calls sharing one workspace must not overlap in time.
+ *   log_sum_exp     NULL, or float32 [total_q_tokens, n_heads] (4-byte aligned):
+ *                   each row's natural log-sum-exp ln sum_j e^(scale q.k_j) over
+ *                   its visible keys, -inf for a row that sees no key (the
+ *                   output NumKong's attention_packed fills for training,
+ *                   "Attention with a Pre-Packed KV-Cache"). Rows of a sequence
+ *                   with a length error are left unwritten, as in out.
  *
  * Paths (chosen from the host sizes, never from device data):
  *   dtype f32                      -> fp32 CUDA-core kernel
@@ -196,7 +202,7 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
                                   float scale, int32_t window, void* out, int32_t batch,
                                   int32_t total_q_tokens, int32_t max_q_len,
                                   int32_t max_kv_len, rpk_dtype dtype, void* workspace,
-                                  size_t workspace_bytes, void* stream);
+                                  size_t workspace_bytes, float* log_sum_exp, void* stream);
 
 /*
  * ragged_paged_attention_noalloc -- ragged_paged_attention for callers that

@@ -422,6 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
       pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
       *reinterpret_cast<uint2*>(out) = pk;
+      if (p.lse != nullptr && e4 == 0) p.lse[orow] = lse_from_log2_state(mx, L);
     } else {
       const size_t prow = (size_t)split * p.T * p.H + orow;
       *reinterpret_cast<float4*>(ws.o + prow * D + e4) = acc;
@@ -431,7 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the split partials of each (token, head) row: m* = max m_s,
-// out = sum_s 2^(m_s - m*) O_s / sum_s 2^(m_s - m*) l_s (zero when empty).
+// out = sum_s 2^(m_s - m*) O_s / sum_s 2^(m_s - m*) l_s (zero when empty), and
+// the row's log-sum-exp from (m*, sum_s 2^(m_s - m*) l_s) when asked for.
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p,
                                                            const DecodePlan plan,
@@ -469,6 +471,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p,
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
+  if (p.lse != nullptr && lane == 0) p.lse[row] = lse_from_log2_state(mx, L);
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * D + lane * E;
 #pragma unroll
   for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t*>(out + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);

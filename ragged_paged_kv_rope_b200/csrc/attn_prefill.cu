@@ -664,7 +664,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_after_sync();
       }
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      const size_t orow = ((size_t)(it.q0 + tok) * p.H + (size_t)it.kvh * G + (r % G)) * D;
+      const size_t hrow = (size_t)(it.q0 + tok) * p.H + (size_t)it.kvh * G + (r % G);
+      const size_t orow = hrow * D;
+      // l is relative to the (possibly stale) running max m, so m + log2 l is exact.
+      if (p.lse != nullptr && row_ok) p.lse[hrow] = lse_from_log2_state(m, l);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         float o[32];

@@ -36,6 +36,7 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const AttnParams
 #pragma unroll
   for (int e = 0; e < E; ++e) o[e] = 0.f;
   float l = 0.f;
+  float m = -INFINITY;
 
   const bool len_ok = k_len >= 0 && k_len <= p.max_kv_len && q_len <= p.max_q_len;
   if (!len_ok) {
@@ -52,7 +53,6 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const AttnParams
     const T* __restrict__ kp = static_cast<const T*>(p.k_pages);
     const T* __restrict__ vp = static_cast<const T*>(p.v_pages);
     const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
-    float m = -INFINITY;
     for (int j = lo; j <= hi; ++j) {
       const int pi = j / p.P;
       const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const AttnParams
   const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
   for (int e = 0; e < E; ++e) orow[e] = Elt<T>::from_f32(o[e] * inv);
+  if (p.lse != nullptr && lane == 0) p.lse[row] = lse_from_log2_state(m, l);
 }
 
 template <typename T>

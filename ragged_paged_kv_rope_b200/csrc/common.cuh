@@ -69,6 +69,13 @@ __device__ __forceinline__ void store16(T* p, const float* in) {
 }
 
 // 2^x by the MUFU approximation (relative error ~2^-22; 2^-inf = +0).
+// Natural log-sum-exp of a row from its running state in log2 units: the
+// scores' maximum m (times log2 e) and the sum l of 2^(score - m); -inf for a
+// row with no key (l = 0).
+__device__ __forceinline__ float lse_from_log2_state(float m, float l) {
+  return l > 0.f ? (m + log2f(l)) * 0.693147180559945309f : -INFINITY;
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

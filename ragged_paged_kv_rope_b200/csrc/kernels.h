@@ -46,6 +46,7 @@ struct AttnParams {
   int32_t T, batch, H, Hk, G, d, P, num_pages, max_pages, window, max_q_len, max_kv_len;
   float scale;
   float scale_log2;            // scale * log2(e)
+  float* lse = nullptr;        // [T, H] natural log-sum-exp of each row's scores, or null
 };
 
 // fp32 / bf16 CUDA-core attention: one warp per (token, head) row.

@@ -11,6 +11,13 @@ Tolerances (written here once, used by every test):
   2^-22 (|a| + |b|).
 * Attention: bf16 max-abs 2e-2 and mean-abs 2e-3; fp32 max-abs 1e-4, against
   the oracle's fp64 rows before rounding.
+* Log-sum-exp: |got - ref| <= 2e-3 + 1e-4 |ref|, and -inf exactly where the
+  row sees no key. It is a smooth maximum of the scores, so its error is at
+  most the largest score error plus the relative error of the sum: an fp32
+  dot product of d <= 256 terms errs by at most d 2^-24 sum|q_i k_i| (under
+  2.5e-3 at scale 1 for the N(0,1)-scale inputs here, far less at
+  1/sqrt(d)), and the sum of n fp32 terms with ex2.approx by about
+  (n + 2) 2^-23 relative, i.e. 1e-4 |lse| covers it with margin.
 * Cache placement, V bytes, untouched slots, channels >= rotary_dim and rows
   at position 0: bit-exact.
 """
@@ -28,6 +35,7 @@ import ragged_paged_kv_rope_b200 as R
 from ragged_paged_kv_rope_b200 import workloads as W
 
 ATTN_TOL = {"bf16": (2e-2, 2e-3), "f32": (1e-4, 1e-4)}
+LSE_TOL = (2e-3, 1e-4)  # absolute, relative
 
 
 @dataclass
@@ -77,12 +85,13 @@ def oracle_rope(wl: W.Workload, table: np.ndarray):
     return O.rope(wl.q, *args), O.rope(wl.k_new, *args)
 
 
-def gpu_attention(wl: W.Workload, dev: Dev, q: torch.Tensor, window=None) -> torch.Tensor:
+def gpu_attention(wl: W.Workload, dev: Dev, q: torch.Tensor, window=None, lse=None):
     sp = wl.spec
     out = torch.empty_like(q)
     R.ragged_paged_attention(q, dev.offsets, dev.kv_lens, dev.cache, sp.n_heads, sp.n_kv_heads,
                              sp.head_dim, sp.softmax_scale, sp.window if window is None else window,
-                             out, max_q_len=wl.max_q_len, max_kv_len=wl.max_kv_len)
+                             out, max_q_len=wl.max_q_len, max_kv_len=wl.max_kv_len,
+                             log_sum_exp=lse)
     return out
 
 
@@ -135,6 +144,19 @@ def check_attention(got: torch.Tensor | np.ndarray, ref: np.ndarray, dtype: str,
     assert mx <= max_tol, f"{what}: max abs error {mx:.3g} > {max_tol}"
     assert mean <= mean_tol, f"{what}: mean abs error {mean:.3g} > {mean_tol}"
     return mx, mean
+
+
+def check_lse(got: torch.Tensor | np.ndarray, ref: np.ndarray, what: str):
+    g = got.detach().cpu().numpy().astype(np.float64) if isinstance(got, torch.Tensor) else got
+    empty = np.isneginf(ref)
+    assert np.array_equal(np.isneginf(g), empty), f"{what}: -inf rows differ"
+    assert np.all(np.isfinite(g[~empty])), f"{what}: non-finite log-sum-exp"
+    diff = np.abs(g[~empty] - ref[~empty])
+    tol = LSE_TOL[0] + LSE_TOL[1] * np.abs(ref[~empty])
+    bad = np.argwhere(diff > tol)
+    assert bad.size == 0, (f"{what}: {len(bad)} log-sum-exp values outside tolerance, worst "
+                           f"{float((diff - tol).max()):.3g} over")
+    return float(diff.max()) if diff.size else 0.0
 
 
 def gather_logical(pool: torch.Tensor, wl: W.Workload, slots_of) -> torch.Tensor:

@@ -13,7 +13,7 @@ import torch
 import oracle as O
 import ragged_paged_kv_rope_b200 as R
 from ragged_paged_kv_rope_b200 import workloads as W
-from parity import REDUCED, check_attention, gpu_attention, sample_rows, to_device
+from parity import REDUCED, check_attention, check_lse, gpu_attention, sample_rows, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -22,15 +22,21 @@ def _attn_case(sp: W.Spec, q_lens, kv_lens, seed=0, rows=None, window=None):
     wl = W.attention_only(sp, seed, q_lens, kv_lens)
     dev = to_device(wl)
     w = sp.window if window is None else window
-    out = gpu_attention(wl, dev, dev.q, window=w)
+    # every case also checks the log-sum-exp output against the oracle's
+    lse = torch.full((wl.total_tokens, sp.n_heads), float("nan"), device="cuda")
+    out = gpu_attention(wl, dev, dev.q, window=w, lse=lse)
     torch.cuda.synchronize()
     assert int(dev.error_word.item()) == 0
-    ref = O.attention(wl.q, wl.q_offsets, wl.kv_lens, wl.k_pages, wl.v_pages, wl.block_table,
-                      sp.n_kv_heads, sp.softmax_scale, w, rows=rows)
-    got = out.cpu()
+    ref, ref_lse = O.attention(wl.q, wl.q_offsets, wl.kv_lens, wl.k_pages, wl.v_pages,
+                               wl.block_table, sp.n_kv_heads, sp.softmax_scale, w, rows=rows,
+                               with_lse=True)
+    got, got_lse = out.cpu(), lse.cpu()
     if rows is not None:
-        got = got[torch.from_numpy(rows[:, 0]).long(), torch.from_numpy(rows[:, 1]).long()]
-    return check_attention(got, ref, sp.dtype, f"{sp.name} q={list(q_lens)[:4]}")
+        ti, hi = torch.from_numpy(rows[:, 0]).long(), torch.from_numpy(rows[:, 1]).long()
+        got, got_lse = got[ti, hi], got_lse[ti, hi]
+    what = f"{sp.name} q={list(q_lens)[:4]}"
+    check_lse(got_lse, ref_lse, what)
+    return check_attention(got, ref, sp.dtype, what)
 
 
 def _lens_from(wl_spec, seed):
