@@ -51,6 +51,8 @@ def _declare(L):
     L.rpko_cache_image.argtypes = [_p, _p, C.c_int, _i32, _i32, _i32, _p, _i32, _p, _p, _i32,
                                    _i32, _i32, _p, _p]
     L.rpko_cache_image.restype = C.c_int
+    L.rpko_freqs_cis_proportional.argtypes = [_i32, _i32, _i32, C.c_double, _p]
+    L.rpko_freqs_cis_proportional.restype = C.c_int
     L.rpko_band.argtypes = [_i32, _i32, _i32, _i32, C.POINTER(_i32), C.POINTER(_i32)]
     L.rpko_band.restype = None
     L.rpko_attention.argtypes = [_p, C.c_int, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p,
@@ -119,6 +121,19 @@ def freqs_cis(max_position: int, rotary_dim: int, base: float) -> np.ndarray:
     rc = lib().rpko_freqs_cis(int(max_position), int(rotary_dim), float(base), _ptr(out))
     if rc:
         raise ValueError(f"rpko_freqs_cis failed ({rc})")
+    return out
+
+
+def freqs_cis_proportional(max_position: int, head_dim: int, rotated_pairs: int,
+                           base: float) -> np.ndarray:
+    """fp32 [max_position, head_dim] p-RoPE table: (cos, sin) of p * base^(-2j/head_dim)
+    for pairs j < rotated_pairs, (1, 0) for the rest (read with rotary_dim = head_dim,
+    half layout)."""
+    out = np.empty((max_position, head_dim), dtype=np.float32)
+    rc = lib().rpko_freqs_cis_proportional(int(max_position), int(head_dim), int(rotated_pairs),
+                                           float(base), _ptr(out))
+    if rc:
+        raise ValueError(f"rpko_freqs_cis_proportional failed ({rc})")
     return out
 
 

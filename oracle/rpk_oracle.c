@@ -134,6 +134,34 @@ int rpko_freqs_cis(int32_t max_position, int32_t rotary_dim, double base, float*
   return RPKO_OK;
 }
 
+/* p-RoPE table (algenta "Attention variant kernels", rope_half_proportional:
+ * the first factor * head_dim / 2 pairs of the rotate-half layout turn, the
+ * other pairs are left as they are, and the frequencies take the full
+ * head_dim as denominator). Width head_dim, read with rotary_dim = head_dim
+ * in the half layout, so pair j is (x[j], x[j + head_dim/2]):
+ *   j <  rotated_pairs: (cos, sin)(p * base^(-2j/head_dim)), fp64 rounded once;
+ *   j >= rotated_pairs: (1, 0), the identity. */
+int rpko_freqs_cis_proportional(int32_t max_position, int32_t head_dim, int32_t rotated_pairs,
+                                double base, float* out) {
+  if (max_position < 0 || head_dim <= 0 || (head_dim & 1) || !(base > 0.0) || !out)
+    return RPKO_ERR_ARG;
+  int half = head_dim / 2;
+  if (rotated_pairs < 0 || rotated_pairs > half) return RPKO_ERR_ARG;
+  for (int32_t p = 0; p < max_position; ++p) {
+    for (int j = 0; j < half; ++j) {
+      double c = 1.0, s = 0.0;
+      if (j < rotated_pairs) {
+        double omega = pow(base, -2.0 * (double)j / (double)head_dim);
+        c = cos((double)p * omega);
+        s = sin((double)p * omega);
+      }
+      out[(size_t)p * head_dim + 2 * j] = f64_to_f32(c);
+      out[(size_t)p * head_dim + 2 * j + 1] = f64_to_f32(s);
+    }
+  }
+  return RPKO_OK;
+}
+
 /* ---------------------------------------------------------------- RoPE */
 
 /* Sequence that owns row t: the b with off[b] <= t < off[b+1]. */

@@ -33,6 +33,9 @@ MUTATIONS = {
     "running_sum_not_rescaled": ("*l = *l * alpha + p;", "*l = *l + p;"),
     "slot_row": ("int32_t row = slot % page_size;", "int32_t row = (slot + 1) % page_size;"),
     "value_weight_unnormalised": ("double wj = w[j - lo] / den;", "double wj = w[j - lo];"),
+    "p_rope_denominator": ("double omega = pow(base, -2.0 * (double)j / (double)head_dim);",
+                           "double omega = pow(base, -2.0 * (double)j / (2.0 * rotated_pairs));"),
+    "p_rope_tail_rotated": ("      if (j < rotated_pairs) {", "      if (j <= rotated_pairs) {"),
     "lse_log_base": ("if (lse) *lse = m + log(den);", "if (lse) *lse = m + log2(den);"),
     "lse_max_dropped": ("if (lse) *lse = m + log(den);", "if (lse) *lse = log(den);"),
 }

@@ -419,6 +419,55 @@ def _rope(x, offs, cache_lens, table, interleaved, R, pos=None, mrope=None):
     return O.rope(x, offs, cache_lens, pos, mrope, table, interleaved, R)
 
 
+# ------------------------------------------------- p-RoPE (proportional)
+# algenta rope_half_proportional: the first factor * head_dim / 2 pairs of
+# the rotate-half layout turn with frequencies over the full head_dim, the
+# remaining pairs stay as they are.
+
+
+def test_p_rope_table_uses_full_head_dim_denominator():
+    # head_dim 128, 32 rotated pairs: pair 16 has frequency 10000^(-32/128) = 0.1,
+    # so position 10 turns it by exactly 1 radian (a rotated-subset denominator,
+    # 64, would give 0.01).
+    t = O.freqs_cis_proportional(11, 128, 32, 10000.0)
+    assert abs(float(t[10, 32]) - math.cos(1.0)) <= 2 * 2**-24
+    assert abs(float(t[10, 33]) - math.sin(1.0)) <= 2 * 2**-24
+    assert np.all(t[0, 0:64:2] == 1.0) and np.all(t[0, 1:64:2] == 0.0)
+
+
+def test_p_rope_table_tail_pairs_are_identity():
+    t = O.freqs_cis_proportional(50, 256, 32, 10000.0)
+    assert np.all(t[:, 64::2] == 1.0) and np.all(t[:, 65::2] == 0.0)
+    assert np.any(t[1:, 62] != 1.0)  # the last rotated pair does turn
+
+
+def test_p_rope_table_factor_one_is_the_full_table():
+    for d in (64, 128):
+        assert np.array_equal(O.freqs_cis_proportional(300, d, d // 2, 500000.0),
+                              O.freqs_cis(300, d, 500000.0))
+
+
+def test_p_rope_rotation_pairs_and_identity_tail():
+    # Pair j = (x[j], x[j + d/2]) turns by pos * 10000^(-2j/d) for j < 16; the
+    # others (and so channels 16..63 and 80..127) come back bit for bit.
+    rng = np.random.default_rng(21)
+    d, rot = 128, 16
+    x = rng.normal(size=(6, 2, d)).astype(np.float32)
+    pos = np.array([0, 1, 7, 100, 2047, 5], np.int32)
+    tab = O.freqs_cis_proportional(2048, d, rot, 10000.0)
+    out = _rope(x, [0, 6], [0], tab, False, d, pos=pos)
+    keep = np.r_[rot:d // 2, d // 2 + rot:d]
+    assert np.array_equal(out[..., keep], x[..., keep].astype(np.float64))
+    for t, p in enumerate(pos):
+        for j in range(rot):
+            ang = float(p) * 10000.0 ** (-2.0 * j / d)
+            a, b = x[t, :, j].astype(np.float64), x[t, :, j + d // 2].astype(np.float64)
+            np.testing.assert_allclose(out[t, :, j], a * math.cos(ang) - b * math.sin(ang),
+                                       atol=4e-7 * (1 + np.abs(a) + np.abs(b)).max())
+            np.testing.assert_allclose(out[t, :, j + d // 2], b * math.cos(ang) + a * math.sin(ang),
+                                       atol=4e-7 * (1 + np.abs(a) + np.abs(b)).max())
+
+
 def test_rope_position0_is_identity():
     rng = np.random.default_rng(11)
     x = torch.from_numpy(rng.normal(size=(5, 3, 64)).astype(np.float32)).to(torch.bfloat16)
