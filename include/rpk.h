@@ -69,6 +69,14 @@ typedef enum { RPK_F32 = 0, RPK_BF16 = 1 } rpk_dtype;
  *                      BEFORE the rope_qk_paged_ragged call that appends to it.
  *                      Read only by rope_qk_paged_ragged.
  *   error_word         optional int32 (device): RPK_DEVERR_* bits are OR-ed in.
+ *   num_layers,        a multi-layer collection (Mojo's layer_idx argument, "index
+ *   layer_idx          of the layer whose keys are updated in the cache"): the
+ *                      pools hold num_layers layer-major copies of the layout
+ *                      above, [num_layers, num_pages, page_size, n_kv_heads,
+ *                      head_dim], and a call reads / writes layer layer_idx
+ *                      only, sharing block_table and cache_lens with the other
+ *                      layers. num_layers 0 (a zero-initialised struct) means 1.
+ *                      layer_idx outside [0, num_layers): RPK_ERR_SHAPE.
  */
 typedef struct {
   void* k_pages;
@@ -83,6 +91,8 @@ typedef struct {
   int32_t batch;
   const int32_t* cache_lens;
   int32_t* error_word;
+  int32_t num_layers;
+  int32_t layer_idx;
 } rpk_paged_kv;
 
 /*
@@ -137,6 +147,27 @@ rpk_status rope_qk_paged_ragged(const void* q_proj, const int32_t* input_row_off
  */
 rpk_status rope_freqs_cis(float* freqs_cis, int32_t max_position, int32_t rotary_dim,
                           double theta, void* stream);
+
+/*
+ * rope_freqs_cis_proportional -- the table of p-RoPE, algenta "Attention
+ * variant kernels", rope_half_proportional (Gemma-4 global layers): of the
+ * head_dim/2 pairs of the rotate-half layout only the first rotated_pairs
+ * (= factor * head_dim / 2) turn, with frequencies over the full head_dim;
+ * the other pairs are the identity.
+ *
+ *   freqs_cis      [max_position, head_dim] fp32 (device, caller-owned):
+ *                  pair j < rotated_pairs holds (cos, sin)(p * theta^(-2j/head_dim)),
+ *                  computed in fp64 and rounded once; pair j >= rotated_pairs
+ *                  holds (1, 0).
+ *   rotated_pairs  0 .. head_dim/2 (host)
+ *
+ * Use it with rope_qk_paged_ragged(..., interleaved = 0, rotary_dim = head_dim,
+ * ...): pair j is then (x[j], x[j + head_dim/2]), and the identity pairs come
+ * back bit for bit (a*1 - b*0 = a, b*1 + a*0 = b in fp32). Errors as
+ * rope_freqs_cis; RPK_ERR_SHAPE for rotated_pairs outside 0 .. head_dim/2.
+ */
+rpk_status rope_freqs_cis_proportional(float* freqs_cis, int32_t max_position, int32_t head_dim,
+                                       int32_t rotated_pairs, double theta, void* stream);
 
 /*
  * ragged_paged_attention_workspace_size -- bytes of device workspace that

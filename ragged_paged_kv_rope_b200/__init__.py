@@ -17,6 +17,7 @@ from .binding import (  # noqa: F401
     PagedKVCache,
     RpkError,
     freqs_cis,
+    freqs_cis_proportional,
     lib,
     ragged_paged_attention,
     ragged_paged_attention_workspace_size,

@@ -11,11 +11,13 @@ Entry points keep the C names:
 * ``ragged_paged_attention`` ragged causal GQA attention over the paged cache
 * ``ragged_paged_attention_workspace_size``
 * ``freqs_cis``             builds the fp32 (cos, sin) table with ``rope_freqs_cis``
+* ``freqs_cis_proportional`` builds the p-RoPE table with ``rope_freqs_cis_proportional``
 """
 
 from __future__ import annotations
 
 import ctypes as C
+import math
 import os
 import re
 from dataclasses import dataclass
@@ -50,6 +52,7 @@ class PagedKV(C.Structure):
         ("cache_dtype", C.c_int),
         ("block_table", C.c_void_p), ("max_pages_per_seq", C.c_int32), ("batch", C.c_int32),
         ("cache_lens", C.c_void_p), ("error_word", C.c_void_p),
+        ("num_layers", C.c_int32), ("layer_idx", C.c_int32),
     ]
 
 
@@ -76,6 +79,8 @@ def lib():
                                              C.c_float, _i32, _p, _i32, _i32, _i32, _i32, C.c_int,
                                              _p, C.c_size_t, _p, _p]
         L.ragged_paged_attention.restype = C.c_int
+        L.rope_freqs_cis_proportional.argtypes = [_p, _i32, _i32, _i32, C.c_double, _p]
+        L.rope_freqs_cis_proportional.restype = C.c_int
         L.rpk_status_string.argtypes = [C.c_int]
         L.rpk_status_string.restype = C.c_char_p
         L.rpk_last_cuda_error.argtypes = []
@@ -132,24 +137,35 @@ def _stream(stream) -> int:
 
 @dataclass
 class PagedKVCache:
-    """The paged cache: pools, block table, cached lengths, optional error word."""
+    """The paged cache: pools, block table, cached lengths, optional error word.
 
-    k_pages: torch.Tensor          # [num_pages, page_size, n_kv_heads, head_dim]
+    The pools are [num_pages, page_size, n_kv_heads, head_dim], or, for a
+    multi-layer collection, [num_layers, num_pages, page_size, n_kv_heads,
+    head_dim] with layer_idx choosing the layer the calls read and write.
+    """
+
+    k_pages: torch.Tensor
     v_pages: torch.Tensor
     block_table: torch.Tensor      # int32 [batch, max_pages_per_seq]
     cache_lens: torch.Tensor | None = None   # int32 [batch]
     error_word: torch.Tensor | None = None   # int32 [1]
+    layer_idx: int = 0
 
     def struct(self) -> PagedKV:
         kp, vp = self.k_pages, self.v_pages
-        _dev(kp, "k_pages", ndim=4)
-        _dev(vp, "v_pages", dtype=kp.dtype, ndim=4)
+        if kp.dim() not in (4, 5):
+            raise RpkError("k_pages must be [(num_layers,) num_pages, page_size, kv_heads, d]")
+        _dev(kp, "k_pages", ndim=kp.dim())
+        _dev(vp, "v_pages", dtype=kp.dtype, ndim=kp.dim())
         if vp.shape != kp.shape:
             raise RpkError("k_pages and v_pages differ in shape")
         _dev(self.block_table, "block_table", torch.int32, 2)
         s = PagedKV()
         s.k_pages, s.v_pages = kp.data_ptr(), vp.data_ptr()
-        s.num_pages, s.page_size, s.n_kv_heads, s.head_dim = (int(x) for x in kp.shape)
+        shape = tuple(int(x) for x in kp.shape)
+        s.num_layers = shape[0] if len(shape) == 5 else 1
+        s.layer_idx = int(self.layer_idx)
+        s.num_pages, s.page_size, s.n_kv_heads, s.head_dim = shape[-4:]
         s.cache_dtype = _dtype_code(kp.dtype)
         s.block_table = self.block_table.data_ptr()
         s.batch, s.max_pages_per_seq = (int(x) for x in self.block_table.shape)
@@ -202,6 +218,19 @@ def freqs_cis(max_position: int, rotary_dim: int, theta: float, device=None,
     out = torch.empty((int(max_position), int(rotary_dim)), dtype=torch.float32, device=device)
     _check(lib().rope_freqs_cis(out.data_ptr(), int(max_position), int(rotary_dim), float(theta),
                                 _stream(stream)))
+    return out
+
+
+def freqs_cis_proportional(max_position: int, head_dim: int, factor: float, theta: float,
+                           device=None, stream=None) -> torch.Tensor:
+    """fp32 [max_position, head_dim] p-RoPE table (rope_half_proportional): the first
+    floor(factor * head_dim / 2) rotate-half pairs turn by p * theta^(-2j/head_dim),
+    the others are the identity. Use with rotary_dim = head_dim, interleaved False."""
+    rotated = int(math.floor(float(factor) * int(head_dim) / 2))
+    device = device if device is not None else torch.device("cuda")
+    out = torch.empty((int(max_position), int(head_dim)), dtype=torch.float32, device=device)
+    _check(lib().rope_freqs_cis_proportional(out.data_ptr(), int(max_position), int(head_dim),
+                                             rotated, float(theta), _stream(stream)))
     return out
 
 

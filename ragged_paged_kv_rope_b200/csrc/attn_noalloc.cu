@@ -107,6 +107,8 @@ extern "C" rpk_status ragged_paged_attention_noalloc(
   if (!aligned16(q) || !aligned16(out) || !aligned16(c->k_pages) || !aligned16(c->v_pages))
     return RPK_ERR_SHAPE;
   if ((long long)c->num_pages * c->page_size > INT32_MAX) return RPK_ERR_UNSUPPORTED;
+  void *k_layer, *v_layer;
+  if (!rpk::layer_pools(c, &k_layer, &v_layer)) return RPK_ERR_SHAPE;
   if ((long long)max_kv_len > (long long)c->max_pages_per_seq * c->page_size)
     return RPK_ERR_SHAPE;
   const int32_t group = n_heads / n_kv_heads;
@@ -123,7 +125,7 @@ extern "C" rpk_status ragged_paged_attention_noalloc(
   if (st != RPK_OK) return st;
 
   rpk::AttnParams p;
-  p.q = q; p.out = out; p.k_pages = c->k_pages; p.v_pages = c->v_pages;
+  p.q = q; p.out = out; p.k_pages = k_layer; p.v_pages = v_layer;
   p.offsets = q_row_offsets; p.kv_lens = kv_lens; p.block_table = c->block_table;
   p.error_word = c->error_word;
   p.T = total_q_tokens; p.batch = batch; p.H = n_heads; p.Hk = n_kv_heads; p.G = group;

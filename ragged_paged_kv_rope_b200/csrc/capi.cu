@@ -40,6 +40,8 @@ rpk_status check_cache(const rpk_paged_kv* c) {
     return RPK_ERR_UNSUPPORTED;
   if (!aligned16(c->k_pages) || !aligned16(c->v_pages)) return RPK_ERR_SHAPE;
   if ((long long)c->num_pages * c->page_size > INT32_MAX) return RPK_ERR_UNSUPPORTED;
+  void *k, *v;
+  if (!rpk::layer_pools(c, &k, &v)) return RPK_ERR_SHAPE;
   return RPK_OK;
 }
 
@@ -135,7 +137,7 @@ rpk_status rope_qk_paged_ragged(const void* q_proj, const int32_t* input_row_off
 
   rpk::RopeParams p;
   p.q = q_proj; p.k_new = k_new; p.v_new = v_new; p.out_q = out_q;
-  p.k_pages = page_table->k_pages; p.v_pages = page_table->v_pages;
+  rpk::layer_pools(page_table, &p.k_pages, &p.v_pages);
   p.offsets = input_row_offsets; p.cache_lens = page_table->cache_lens;
   p.block_table = page_table->block_table; p.position_ids = position_ids;
   p.freqs = freqs_cis; p.error_word = page_table->error_word;
@@ -155,7 +157,19 @@ rpk_status rope_freqs_cis(float* freqs_cis, int32_t max_position, int32_t rotary
   if (!freqs_cis) return RPK_ERR_NULL;
   if (max_position < 0 || rotary_dim <= 0 || (rotary_dim & 1)) return RPK_ERR_SHAPE;
   if (!(theta > 0.0) || !std::isfinite(theta)) return RPK_ERR_SHAPE;
-  return cuda_status(rpk::launch_freqs_cis(freqs_cis, max_position, rotary_dim, theta,
+  return cuda_status(rpk::launch_freqs_cis(freqs_cis, max_position, rotary_dim, rotary_dim,
+                                           rotary_dim / 2, theta,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+rpk_status rope_freqs_cis_proportional(float* freqs_cis, int32_t max_position, int32_t head_dim,
+                                       int32_t rotated_pairs, double theta, void* stream) {
+  if (!freqs_cis) return RPK_ERR_NULL;
+  if (max_position < 0 || head_dim <= 0 || (head_dim & 1)) return RPK_ERR_SHAPE;
+  if (rotated_pairs < 0 || rotated_pairs > head_dim / 2) return RPK_ERR_SHAPE;
+  if (!(theta > 0.0) || !std::isfinite(theta)) return RPK_ERR_SHAPE;
+  return cuda_status(rpk::launch_freqs_cis(freqs_cis, max_position, head_dim, head_dim,
+                                           rotated_pairs, theta,
                                            static_cast<cudaStream_t>(stream)));
 }
 
@@ -196,7 +210,12 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
 
   rpk::AttnParams p;
   p.lse = log_sum_exp;
-  p.q = q; p.out = out; p.k_pages = page_table->k_pages; p.v_pages = page_table->v_pages;
+  p.q = q; p.out = out;
+  {
+    void *k, *v;
+    rpk::layer_pools(page_table, &k, &v);
+    p.k_pages = k; p.v_pages = v;
+  }
   p.offsets = q_row_offsets; p.kv_lens = kv_lens; p.block_table = page_table->block_table;
   p.error_word = page_table->error_word;
   p.T = total_q_tokens; p.batch = batch; p.H = n_heads; p.Hk = n_kv_heads;

@@ -10,6 +10,20 @@
 
 namespace rpk {
 
+// The pools of the layer a call uses: layer layer_idx of num_layers (0 means
+// one) layer-major copies of [num_pages, page_size, n_kv_heads, head_dim].
+// False when layer_idx is out of range.
+inline bool layer_pools(const rpk_paged_kv* c, void** k, void** v) {
+  const int32_t layers = c->num_layers > 0 ? c->num_layers : 1;
+  if (c->num_layers < 0 || c->layer_idx < 0 || c->layer_idx >= layers) return false;
+  const size_t elt = c->cache_dtype == RPK_F32 ? 4 : 2;
+  const size_t per_layer =
+      (size_t)c->num_pages * c->page_size * c->n_kv_heads * c->head_dim * elt;
+  *k = static_cast<char*>(c->k_pages) + (size_t)c->layer_idx * per_layer;
+  *v = static_cast<char*>(c->v_pages) + (size_t)c->layer_idx * per_layer;
+  return true;
+}
+
 struct RopeParams {
   const void* q;
   const void* k_new;
@@ -31,8 +45,8 @@ struct RopeParams {
 
 cudaError_t launch_rope(const RopeParams& p, rpk_dtype dtype, bool interleaved,
                         cudaStream_t stream);
-cudaError_t launch_freqs_cis(float* out, int32_t max_position, int32_t rotary_dim, double theta,
-                             cudaStream_t stream);
+cudaError_t launch_freqs_cis(float* out, int32_t max_position, int32_t width, int32_t denom,
+                             int32_t rotated_pairs, double theta, cudaStream_t stream);
 
 struct AttnParams {
   const void* q;

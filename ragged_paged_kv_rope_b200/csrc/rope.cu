@@ -184,20 +184,25 @@ __global__ void __launch_bounds__(kThreads) rope_scatter_kernel(const RopeParams
   }
 }
 
-// freqs_cis[p][2j] = cos(p * theta^(-2j/R)), [2j+1] = sin(...), in fp64, rounded once.
-__global__ void freqs_cis_kernel(float* __restrict__ out, int32_t max_position, int32_t R,
-                                 double theta) {
-  const int half = R >> 1;
+// Table of width W (W/2 pairs): freqs_cis[p][2j] = cos(p * theta^(-2j/denom)),
+// [2j+1] = sin(...), in fp64 and rounded once, for pairs j < n_rot; (1, 0) for
+// the others. Plain RoPE: W = denom = rotary_dim, n_rot = W/2. p-RoPE (algenta
+// rope_half_proportional): W = denom = head_dim, n_rot = the rotated pairs.
+__global__ void freqs_cis_kernel(float* __restrict__ out, int32_t max_position, int32_t W,
+                                 int32_t denom, int32_t n_rot, double theta) {
+  const int half = W >> 1;
   const long long n = (long long)max_position * half;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
        idx += (long long)gridDim.x * blockDim.x) {
     const int pos = (int)(idx / half);
     const int j = (int)(idx - (long long)pos * half);
-    const double omega = pow(theta, -2.0 * (double)j / (double)R);
-    double s, c;
-    sincos((double)pos * omega, &s, &c);
-    out[(size_t)pos * R + 2 * j] = __double2float_rn(c);
-    out[(size_t)pos * R + 2 * j + 1] = __double2float_rn(s);
+    double s = 0.0, c = 1.0;
+    if (j < n_rot) {
+      const double omega = pow(theta, -2.0 * (double)j / (double)denom);
+      sincos((double)pos * omega, &s, &c);
+    }
+    out[(size_t)pos * W + 2 * j] = __double2float_rn(c);
+    out[(size_t)pos * W + 2 * j + 1] = __double2float_rn(s);
   }
 }
 
@@ -219,13 +224,14 @@ cudaError_t launch_rope(const RopeParams& p, rpk_dtype dtype, bool interleaved,
   return cudaGetLastError();
 }
 
-cudaError_t launch_freqs_cis(float* out, int32_t max_position, int32_t rotary_dim, double theta,
-                             cudaStream_t stream) {
-  const long long n = (long long)max_position * (rotary_dim / 2);
+cudaError_t launch_freqs_cis(float* out, int32_t max_position, int32_t width, int32_t denom,
+                             int32_t rotated_pairs, double theta, cudaStream_t stream) {
+  const long long n = (long long)max_position * (width / 2);
   if (n == 0) return cudaSuccess;
   long long blocks = (n + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  freqs_cis_kernel<<<(unsigned)blocks, 256, 0, stream>>>(out, max_position, rotary_dim, theta);
+  freqs_cis_kernel<<<(unsigned)blocks, 256, 0, stream>>>(out, max_position, width, denom,
+                                                         rotated_pairs, theta);
   return cudaGetLastError();
 }
 

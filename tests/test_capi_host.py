@@ -56,6 +56,8 @@ def cache(**kw):
     s.batch = kw.get("batch", 2)
     s.cache_lens = kw.get("cache_lens", FAKE)
     s.error_word = None
+    s.num_layers = kw.get("num_layers", 0)
+    s.layer_idx = kw.get("layer_idx", 0)
     return s
 
 
@@ -97,6 +99,8 @@ def test_rope_rejects(L, kw, status):
     ({"k_pages": None}, 1), ({"block_table": None}, 1), ({"cache_lens": None}, 1),
     ({"page_size": 48}, 4), ({"head_dim": 96}, 4), ({"num_pages": 0}, 2),
     ({"cache_dtype": 9}, 3),
+    ({"layer_idx": 1}, 2), ({"num_layers": 3, "layer_idx": 3}, 2),
+    ({"num_layers": 3, "layer_idx": -1}, 2), ({"num_layers": -2}, 2),
 ])
 def test_rope_rejects_cache(L, ckw, status):
     assert rope(L, cache(**ckw)) == status
@@ -122,6 +126,15 @@ def test_attention_rejects(L, kw, status):
     assert attn(L, cache(max_pages_per_seq=16), **kw) == status
 
 
+@host_only
+def test_attention_rejects_layer_out_of_range(L):
+    assert attn(L, cache(max_pages_per_seq=16, num_layers=2, layer_idx=2)) == 2
+    assert L.ragged_paged_attention_noalloc(
+        C.c_void_p(FAKE), C.c_void_p(FAKE), C.c_void_p(FAKE),
+        C.byref(cache(max_pages_per_seq=16, layer_idx=1)), 32, 8, 128, C.c_float(0.1), 0,
+        C.c_void_p(FAKE), 2, 2, 1, 200, B.RPK_BF16, None) == 2
+
+
 def test_workspace_size(L):
     f = R.ragged_paged_attention_workspace_size
     assert f(0, 32, 128, 64, 8193, 64) == 0
@@ -140,6 +153,11 @@ def test_freqs_rejects(L):
     assert L.rope_freqs_cis(None, 10, 8, 1e4, None) == 1
     assert L.rope_freqs_cis(FAKE, 10, 7, 1e4, None) == 2
     assert L.rope_freqs_cis(FAKE, 10, 8, -1.0, None) == 2
+    assert L.rope_freqs_cis_proportional(None, 10, 128, 16, 1e4, None) == 1
+    assert L.rope_freqs_cis_proportional(FAKE, 10, 127, 16, 1e4, None) == 2
+    assert L.rope_freqs_cis_proportional(FAKE, 10, 128, 65, 1e4, None) == 2
+    assert L.rope_freqs_cis_proportional(FAKE, 10, 128, -1, 1e4, None) == 2
+    assert L.rope_freqs_cis_proportional(FAKE, 10, 128, 16, 0.0, None) == 2
 
 
 def test_binding_refuses_cpu_tensors():

@@ -18,10 +18,10 @@ from parity import (REDUCED, check_rope, gather_logical, gpu_rope, new_token_slo
 pytestmark = pytest.mark.gpu
 
 
-def _run_and_check(wl: W.Workload, in_place: bool = False):
+def _run_and_check(wl: W.Workload, in_place: bool = False, tab_np=None):
     sp = wl.spec
     dev = to_device(wl)
-    tab_np = oracle_table(wl)
+    tab_np = oracle_table(wl) if tab_np is None else tab_np
     tab = torch.from_numpy(tab_np).cuda()
     out = gpu_rope(wl, dev, tab, out_q=dev.q if in_place else None)
     torch.cuda.synchronize()
@@ -105,6 +105,32 @@ def test_freqs_table_matches_oracle():
         gi, wi = got.view(np.int32).astype(np.int64), want.view(np.int32).astype(np.int64)
         assert np.max(np.abs(gi - wi)) <= 1
         assert np.mean(gi != wi) < 1e-3
+
+
+@pytest.mark.parametrize("maxp,d,rot,theta", [(40000, 256, 32, 1e6), (3000, 128, 64, 1e4),
+                                              (100, 64, 0, 1e4), (100, 64, 32, 1e4)])
+def test_p_rope_table_matches_oracle(maxp, d, rot, theta):
+    got = R.freqs_cis_proportional(maxp, d, rot * 2 / d, theta).cpu().numpy()
+    want = O.freqs_cis_proportional(maxp, d, rot, theta)
+    gi, wi = got.view(np.int32).astype(np.int64), want.view(np.int32).astype(np.int64)
+    assert np.max(np.abs(gi - wi)) <= 1
+    assert np.array_equal(got[:, 2 * rot:], want[:, 2 * rot:])  # identity pairs exact
+
+
+@pytest.mark.parametrize("d,rot", [(256, 32), (128, 16)])
+def test_p_rope_rotation(d, rot):
+    # p-RoPE through the same kernel: half layout, rotary_dim = head_dim and the
+    # proportional table; the identity pairs come back bit for bit.
+    sp = W.spec("ragged_prefill", batch=3, new_tokens=("uniform", 1, 60),
+                cache_tokens=("uniform", 0, 500), head_dim=d, rotary_dim=d, interleaved=False,
+                n_heads=8, n_kv_heads=4, page_size=32, theta=1e6)
+    wl = W.make(sp, seed=9)
+    tab = O.freqs_cis_proportional(wl.max_position, d, rot, sp.theta)
+    _run_and_check(wl, tab_np=tab)
+    dev = to_device(wl)
+    out = gpu_rope(wl, dev, torch.from_numpy(tab).cuda())
+    keep = np.r_[rot:d // 2, d // 2 + rot:d]
+    assert np.array_equal(raw_bits(out)[..., keep], raw_bits(wl.q)[..., keep])
 
 
 def test_rope_bad_page_sets_error_bit():
