@@ -53,11 +53,13 @@ def _declare(L):
     L.rpko_cache_image.restype = C.c_int
     L.rpko_freqs_cis_proportional.argtypes = [_i32, _i32, _i32, C.c_double, _p]
     L.rpko_freqs_cis_proportional.restype = C.c_int
+    L.rpko_visible.argtypes = [_i32] * 6
+    L.rpko_visible.restype = C.c_int
     L.rpko_band.argtypes = [_i32, _i32, _i32, _i32, C.POINTER(_i32), C.POINTER(_i32)]
     L.rpko_band.restype = None
     L.rpko_attention.argtypes = [_p, C.c_int, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p,
-                                 _i32, _i32, _p, _i32, C.c_double, _i32, _p, _i64, _p, _p,
-                                 C.c_int]
+                                 _i32, _i32, _p, _i32, C.c_double, _i32, _i32, _p, _i64, _p,
+                                 _p, C.c_int]
     L.rpko_attention.restype = C.c_int
     L.rpko_flash_step.argtypes = [C.POINTER(C.c_double)] * 3 + [C.c_double, C.c_double]
     L.rpko_flash_step.restype = None
@@ -183,6 +185,12 @@ def cache_image(k_rot: np.ndarray, v_new, row_offsets, cache_lens, block_table, 
     return kp, vp
 
 
+def visible(r: int, q_len: int, k_len: int, window: int, sinks: int, j: int) -> bool:
+    """Key j is visible to row r (window and attention sinks)."""
+    return bool(lib().rpko_visible(int(r), int(q_len), int(k_len), int(window), int(sinks),
+                                   int(j)))
+
+
 def band(r: int, q_len: int, k_len: int, window: int) -> tuple[int, int]:
     lo, hi = C.c_int32(), C.c_int32()
     lib().rpko_band(int(r), int(q_len), int(k_len), int(window), C.byref(lo), C.byref(hi))
@@ -190,13 +198,15 @@ def band(r: int, q_len: int, k_len: int, window: int) -> tuple[int, int]:
 
 
 def attention(q, q_offsets, kv_lens, k_pages, v_pages, block_table, n_kv_heads, scale,
-              window, rows=None, n_threads: int | None = None, with_lse: bool = False):
+              window, rows=None, n_threads: int | None = None, with_lse: bool = False,
+              sinks: int = 0):
     """fp64 attention rows.
 
     rows=None: all rows, shape [T, n_heads, head_dim]. Otherwise rows is an
     int array [n, 2] of (token, head) pairs and the result is [n, head_dim].
     with_lse: return (out, lse), lse the natural log-sum-exp of each row's
     scores ([T, n_heads] or [n]; -inf for a row that sees no key).
+    sinks: under a window, the first `sinks` keys stay visible (StreamingLLM).
     """
     qraw, code = _raw(q)
     kp, kcode = _raw(k_pages)
@@ -219,7 +229,8 @@ def attention(q, q_offsets, kv_lens, k_pages, v_pages, block_table, n_kv_heads, 
         rptr, n = _ptr(rows), rows.shape[0]
     rc = lib().rpko_attention(_ptr(qraw), code, _ptr(offs), _ptr(kvl), len(offs) - 1, T, H,
                               int(n_kv_heads), d, _ptr(kp), _ptr(vp), kp.shape[1], kp.shape[0],
-                              _ptr(bt), bt.shape[1], float(scale), int(window), rptr, n,
+                              _ptr(bt), bt.shape[1], float(scale), int(window), int(sinks),
+                              rptr, n,
                               _ptr(out), None if lse is None else _ptr(lse), int(n_threads))
     if rc:
         raise ValueError(f"rpko_attention failed ({rc})")

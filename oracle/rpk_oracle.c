@@ -285,6 +285,19 @@ void rpko_band(int32_t r, int32_t q_len, int32_t k_len, int32_t window, int32_t*
   *hi = (int32_t)h;
 }
 
+/* Key j is visible to row r (StreamingLLM attention sinks with a window,
+ * algenta "Attention variant kernels", sparse_attention
+ * streaming_llm_sink_score: the first `sinks` keys plus the recent window):
+ * j <= p, and, under a window w > 0, either j >= p - (w - 1) or j < sinks.
+ * sinks = 0 is the plain band of rpko_band. */
+int rpko_visible(int32_t r, int32_t q_len, int32_t k_len, int32_t window, int32_t sinks,
+                 int32_t j) {
+  int64_t pos = (int64_t)r + k_len - q_len;
+  if (j < 0 || j >= k_len || j > pos) return 0;
+  if (window <= 0) return 1;
+  return j >= pos - (window - 1) || j < sinks;
+}
+
 typedef struct {
   const void* q;
   int dtype;
@@ -297,6 +310,7 @@ typedef struct {
   const int32_t* block_table;
   double scale;
   int32_t window;
+  int32_t sinks;
   const int32_t* rows; /* pairs (t, h), or NULL for all */
   int64_t n_rows;
   double* out;         /* [n_rows, head_dim] */
@@ -326,13 +340,16 @@ static int attention_row(const attn_job* J, int32_t t, int32_t h, double* o, dou
   int32_t r = t - J->q_offsets[b];
   int32_t lo, hi;
   rpko_band(r, q_len, k_len, J->window, &lo, &hi);
-  if (hi < lo) return RPKO_OK; /* no visible key: zeros */
+  (void)lo; /* the sinks may reach below the window's first key */
+  if (hi < 0) return RPKO_OK; /* no visible key: zeros */
   int group = J->n_heads / J->n_kv_heads;
   int kvh = h / group;
   size_t qbase = ((size_t)t * J->n_heads + h) * d;
-  /* scores s_j = scale * sum_c q_c k_jc */
+  /* scores s_j = scale * sum_c q_c k_jc of the visible keys, in key order */
   double m = -INFINITY;
-  for (int32_t j = lo; j <= hi; ++j) {
+  int64_t n = 0;
+  for (int32_t j = 0; j <= hi; ++j) {
+    if (!rpko_visible(r, q_len, k_len, J->window, J->sinks, j)) continue;
     int32_t pi = j / J->page_size;
     if (pi >= J->max_pages_per_seq) return RPKO_ERR_PAGE;
     int32_t page = J->block_table[(size_t)b * J->max_pages_per_seq + pi];
@@ -342,18 +359,21 @@ static int attention_row(const attn_job* J, int32_t t, int32_t h, double* o, dou
     for (int c = 0; c < d; ++c)
       acc += load_elt(J->q, J->dtype, qbase + c) * load_elt(J->k_pages, J->dtype, kbase + c);
     double s = J->scale * acc;
-    w[j - lo] = s;
+    w[n++] = s;
     if (s > m) m = s;
   }
+  if (n == 0) return RPKO_OK;
   /* weights e^{s_j - m} / sum e^{s - m}, then out = sum_j w_j v_j */
   double den = 0.0;
-  for (int32_t j = lo; j <= hi; ++j) {
-    w[j - lo] = exp(w[j - lo] - m);
-    den += w[j - lo];
+  for (int64_t i = 0; i < n; ++i) {
+    w[i] = exp(w[i] - m);
+    den += w[i];
   }
   if (lse) *lse = m + log(den);
-  for (int32_t j = lo; j <= hi; ++j) {
-    double wj = w[j - lo] / den;
+  int64_t i = 0;
+  for (int32_t j = 0; j <= hi; ++j) {
+    if (!rpko_visible(r, q_len, k_len, J->window, J->sinks, j)) continue;
+    double wj = w[i++] / den;
     int32_t page = J->block_table[(size_t)b * J->max_pages_per_seq + j / J->page_size];
     size_t vbase = (((size_t)page * J->page_size + j % J->page_size) * J->n_kv_heads + kvh) * d;
     for (int c = 0; c < d; ++c) o[c] += wj * load_elt(J->v_pages, J->dtype, vbase + c);
@@ -386,8 +406,9 @@ static void* attention_worker(void* arg) {
 }
 
 /*
- * Ragged causal (optionally windowed) grouped-query attention over the paged
- * pools. Query head h reads KV head h / (n_heads / n_kv_heads). Row r of
+ * Ragged causal (optionally windowed, optionally with attention sinks)
+ * grouped-query attention over the paged pools; the visible keys of a row are
+ * those of rpko_visible. Query head h reads KV head h / (n_heads / n_kv_heads). Row r of
  * sequence b (q_len rows, kv_lens[b] keys) sees keys [lo, p], p = r + kv_len -
  * q_len (rpko_band). Output fp64, one row of head_dim per requested (t, h),
  * in the order given (rows == NULL: all T * n_heads rows, t-major), and, when
@@ -398,7 +419,7 @@ int rpko_attention(const void* q, int dtype, const int32_t* q_offsets, const int
                    int32_t batch, int32_t T, int32_t n_heads, int32_t n_kv_heads,
                    int32_t head_dim, const void* k_pages, const void* v_pages,
                    int32_t page_size, int32_t num_pages, const int32_t* block_table,
-                   int32_t max_pages_per_seq, double scale, int32_t window,
+                   int32_t max_pages_per_seq, double scale, int32_t window, int32_t sinks,
                    const int32_t* rows, int64_t n_rows, double* out, double* lse,
                    int n_threads) {
   if (!q || !q_offsets || !kv_lens || !k_pages || !v_pages || !block_table || !out)
@@ -407,7 +428,7 @@ int rpko_attention(const void* q, int dtype, const int32_t* q_offsets, const int
     return RPKO_ERR_ARG;
   attn_job J = {q, dtype, q_offsets, kv_lens, batch, T, n_heads, n_kv_heads, head_dim,
                 k_pages, v_pages, page_size, num_pages, max_pages_per_seq, block_table,
-                scale, window, rows, rows ? n_rows : (int64_t)T * n_heads, out, lse, RPKO_OK};
+                scale, window, sinks, rows, rows ? n_rows : (int64_t)T * n_heads, out, lse, RPKO_OK};
   if (n_threads < 1) n_threads = 1;
   if (n_threads > 256) n_threads = 256;
   if ((int64_t)n_threads > J.n_rows) n_threads = J.n_rows > 0 ? (int)J.n_rows : 1;

@@ -32,7 +32,14 @@ MUTATIONS = {
                            "double r = floor(a / ulp + 0.5) * ulp;"),
     "running_sum_not_rescaled": ("*l = *l * alpha + p;", "*l = *l + p;"),
     "slot_row": ("int32_t row = slot % page_size;", "int32_t row = (slot + 1) % page_size;"),
-    "value_weight_unnormalised": ("double wj = w[j - lo] / den;", "double wj = w[j - lo];"),
+    "value_weight_unnormalised": ("double wj = w[i++] / den;", "double wj = w[i++];"),
+    "visible_window_off_by_one": ("return j >= pos - (window - 1) || j < sinks;",
+                                  "return j >= pos - window || j < sinks;"),
+    "visible_alignment": ("int64_t pos = (int64_t)r + k_len - q_len;", "int64_t pos = (int64_t)r;"),
+    "sinks_one_too_many": ("return j >= pos - (window - 1) || j < sinks;",
+                           "return j >= pos - (window - 1) || j <= sinks;"),
+    "sinks_not_causal": ("if (j < 0 || j >= k_len || j > pos) return 0;",
+                         "if (j < 0 || j >= k_len || (j > pos && j >= sinks)) return 0;"),
     "p_rope_denominator": ("double omega = pow(base, -2.0 * (double)j / (double)head_dim);",
                            "double omega = pow(base, -2.0 * (double)j / (2.0 * rotated_pairs));"),
     "p_rope_tail_rotated": ("      if (j < rotated_pairs) {", "      if (j <= rotated_pairs) {"),

@@ -318,6 +318,49 @@ def test_lse_normalises_the_output():
                                        rtol=1e-12, atol=1e-13)
 
 
+# ------------------------------------------------ attention sinks + window
+
+
+def test_sinks_worked_example(golden):
+    # The last of seq_len keys is the query (q_len 1); it sees the 4 sink
+    # tokens and the 20-key recent window, nothing in between.
+    g = golden["streaming_llm_sinks"]
+    n = g["seq_len"]
+    got = [int(O.visible(0, 1, n, g["window_size"], g["n_sink_tokens"], p))
+           for p in g["positions"]]
+    assert got == g["attended"]
+    assert sum(O.visible(0, 1, n, g["window_size"], g["n_sink_tokens"], j) for j in range(n)) \
+        == g["n_sink_tokens"] + g["window_size"]
+
+
+def test_sinks_are_causal_and_need_a_window():
+    # a row at position 2 (8 rows over 10 keys, row 0) with window 1 and 4 sinks
+    # sees keys 0, 1, 2: sink 3 lies after it
+    assert [O.visible(0, 8, 10, 1, 4, j) for j in range(5)] == [True, True, True, False, False]
+    # without a window every earlier key is visible whatever the sinks
+    assert all(O.visible(3, 4, 50, 0, 2, j) for j in range(50))
+    assert not O.visible(3, 4, 50, 0, 2, 50)
+
+
+def test_sinks_attention_equals_explicit_key_subset():
+    # 1 query row over 40 keys, window 6, 3 sinks: the same as plain attention
+    # over the 9 visible keys placed in a sequence of their own.
+    rng = np.random.default_rng(23)
+    d = 8
+    k = rng.normal(size=(40, 1, d)).astype(np.float32)
+    v = rng.normal(size=(40, 1, d)).astype(np.float32)
+    q = rng.normal(size=(1, 1, d)).astype(np.float32)
+    kp, vp, bt = paged([k], [v], page_size=4)
+    got, lse = O.attention(q, [0, 1], [40], kp, vp, bt, 1, 0.4, 6, sinks=3, with_lse=True)
+    keep = [0, 1, 2] + list(range(34, 40))
+    kp2, vp2, bt2 = paged([k[keep]], [v[keep]], page_size=4)
+    want, lse2 = O.attention(q, [0, 1], [len(keep)], kp2, vp2, bt2, 1, 0.4, 0, with_lse=True)
+    np.testing.assert_allclose(got, want, rtol=1e-14, atol=1e-15)
+    assert lse[0, 0] == pytest.approx(lse2[0, 0], rel=1e-14)
+    full = O.attention(q, [0, 1], [40], kp, vp, bt, 1, 0.4, 0, sinks=3)
+    assert np.array_equal(full, O.attention(q, [0, 1], [40], kp, vp, bt, 1, 0.4, 0))
+
+
 def test_decode_equals_last_prefill_row():
     rng = np.random.default_rng(8)
     d, L, H, Hk = 16, 13, 4, 2
