@@ -219,6 +219,12 @@ size_t ragged_paged_attention_workspace_size(int32_t total_q_tokens, int32_t n_h
  *                   output NumKong's attention_packed fills for training,
  *                   "Attention with a Pre-Packed KV-Cache"). Rows of a sequence
  *                   with a length error are left unwritten, as in out.
+ *   sink_tokens     >= 0 (host). Under a window (window > 0), the first
+ *                   sink_tokens keys of every sequence stay visible to each row
+ *                   at or after them, beside its window: StreamingLLM attention
+ *                   sinks (algenta "Attention variant kernels", sparse_attention
+ *                   streaming_llm_sink_score). Ignored when window <= 0 (every
+ *                   earlier key is visible then). Negative: RPK_ERR_SHAPE.
  *
  * Paths (chosen from the host sizes, never from device data):
  *   dtype f32                      -> fp32 CUDA-core kernel
@@ -233,7 +239,8 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
                                   float scale, int32_t window, void* out, int32_t batch,
                                   int32_t total_q_tokens, int32_t max_q_len,
                                   int32_t max_kv_len, rpk_dtype dtype, void* workspace,
-                                  size_t workspace_bytes, float* log_sum_exp, void* stream);
+                                  size_t workspace_bytes, float* log_sum_exp,
+                                  int32_t sink_tokens, void* stream);
 
 /*
  * ragged_paged_attention_noalloc -- ragged_paged_attention for callers that

@@ -77,7 +77,7 @@ def lib():
         L.ragged_paged_attention_workspace_size.restype = C.c_size_t
         L.ragged_paged_attention.argtypes = [_p, _p, _p, C.POINTER(PagedKV), _i32, _i32, _i32,
                                              C.c_float, _i32, _p, _i32, _i32, _i32, _i32, C.c_int,
-                                             _p, C.c_size_t, _p, _p]
+                                             _p, C.c_size_t, _p, _i32, _p]
         L.ragged_paged_attention.restype = C.c_int
         L.rope_freqs_cis_proportional.argtypes = [_p, _i32, _i32, _i32, C.c_double, _p]
         L.rope_freqs_cis_proportional.restype = C.c_int
@@ -244,7 +244,7 @@ def ragged_paged_attention_workspace_size(total_q_tokens: int, n_heads: int, hea
 def ragged_paged_attention(q, q_row_offsets, kv_lens, page_table: PagedKVCache, n_heads: int,
                            n_kv_heads: int, head_dim: int, scale: float | None, window: int,
                            out, *, max_q_len: int, max_kv_len: int, workspace=None,
-                           log_sum_exp=None, stream=None) -> None:
+                           log_sum_exp=None, sink_tokens: int = 0, stream=None) -> None:
     """Ragged causal (windowed) GQA attention of q over the paged cache into out.
 
     max_q_len / max_kv_len are host-side bounds of the device lengths (they
@@ -252,7 +252,8 @@ def ragged_paged_attention(q, q_row_offsets, kv_lens, page_table: PagedKVCache, 
     ragged_paged_attention_workspace_size(...) bytes, or None to have one
     allocated here with torch. log_sum_exp: None, or a float32 CUDA tensor
     [tokens, n_heads] that receives each row's natural log-sum-exp of its
-    scores (-inf for a row that sees no key).
+    scores (-inf for a row that sees no key). sink_tokens: under a window, the
+    first sink_tokens keys of every sequence stay visible (attention sinks).
     """
     pk = page_table.struct()
     if q.dim() != 3:
@@ -283,7 +284,7 @@ def ragged_paged_attention(q, q_row_offsets, kv_lens, page_table: PagedKVCache, 
     _check(lib().ragged_paged_attention(
         qp, off, kvl, C.byref(pk), int(n_heads), int(n_kv_heads), int(head_dim), float(scale),
         int(window), op, batch, T, int(max_q_len), int(max_kv_len), _dtype_code(q.dtype), ws,
-        ws_bytes, lp, _stream(stream)))
+        ws_bytes, lp, int(sink_tokens), _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024

@@ -59,23 +59,31 @@ namespace {
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 
-// Band of keys any row of the sequence sees, in whole tiles, and its splits.
+// Keys any row of the sequence sees, in whole tiles, and its splits: the
+// attention-sink tiles [0, n_sink) (keys below the window's first key that
+// stay visible), then the band's tiles from tile0 on. Tile v of this list is
+// tile_at(v).
 struct SeqSplit {
-  int tile0;     // first tile
-  int n_tiles;
+  int tile0;     // first tile of the band
+  int n_sink;    // sink tiles, all below tile0
+  int n_tiles;   // sink and band tiles
   int n_splits;  // >= 1
+  __device__ __forceinline__ int tile_at(int v) const { return v < n_sink ? v : tile0 + (v - n_sink); }
 };
 
-__device__ __forceinline__ SeqSplit seq_split(int q_len, int k_len, int window, int tps) {
+__device__ __forceinline__ SeqSplit seq_split(int q_len, int k_len, int window, int sinks,
+                                              int tps) {
   SeqSplit s;
   const int p0 = k_len - q_len;  // position of the first row
   const int lo = window > 0 ? max(0, p0 - window + 1) : 0;
   if (k_len <= 0 || lo >= k_len) {
-    s.tile0 = 0; s.n_tiles = 0; s.n_splits = 1;
+    s.tile0 = 0; s.n_sink = 0; s.n_tiles = 0; s.n_splits = 1;
     return s;
   }
   s.tile0 = lo / kDecodeTile;
-  s.n_tiles = (k_len - 1) / kDecodeTile + 1 - s.tile0;
+  const int sink_keys = min(sinks, lo);
+  s.n_sink = min((sink_keys + kDecodeTile - 1) / kDecodeTile, s.tile0);
+  s.n_tiles = s.n_sink + (k_len - 1) / kDecodeTile + 1 - s.tile0;
   s.n_splits = max(1, (s.n_tiles + tps - 1) / tps);
   return s;
 }
@@ -135,10 +143,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0 && split == 0 && kvh == 0) raise_error(p.error_word, RPK_DEVERR_LENGTH);
     return;
   }
-  const SeqSplit ss = seq_split(q_len, k_len, p.window, plan.tiles_per_split);
+  const SeqSplit ss = seq_split(q_len, k_len, p.window, p.sinks, plan.tiles_per_split);
   if (split >= ss.n_splits) return;
-  const int tile_begin = ss.tile0 + split * plan.tiles_per_split;
-  const int n_tiles = max(0, min(plan.tiles_per_split, ss.tile0 + ss.n_tiles - tile_begin));
+  const int v_begin = split * plan.tiles_per_split;  // first entry of this split's tile list
+  const int n_tiles = max(0, min(plan.tiles_per_split, ss.n_tiles - v_begin));
   const int rows = q_len * p.G;
 
   // 1024-byte aligned stage ring (128-byte swizzle atoms are 8 rows x 128 bytes).
@@ -170,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < n_tiles && ok; ++i) {
         const int s = i % S;
         if (!mbar_wait(&empty_bar[s], ((i / S) & 1) ^ 1)) { ok = false; break; }
-        const int key0 = (tile_begin + i) * kDecodeTile;
+        const int key0 = ss.tile_at(v_begin + i) * kDecodeTile;
         // Count the boxes to load (pages wholly past k_len or invalid are skipped).
         uint32_t bytes = 0;
         for (int r = 0; r < kDecodeTile; r += box_rows) {
@@ -260,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = 0; i < n_tiles; ++i) {
     const int s = i % S;
     if (!mbar_wait(&full_bar[s], (i / S) & 1)) { ok = false; break; }
-    const int key0 = (tile_begin + i) * kDecodeTile + warp * 16;  // this warp's 16 keys
+    const int key0 = ss.tile_at(v_begin + i) * kDecodeTile + warp * 16;  // this warp's 16 keys
     const uint32_t kbase = smem_u32(k_stage(s));
     const uint32_t vbase = smem_u32(v_stage(s));
     const int wrow0 = warp * 16;  // row of this warp's first key inside the tile
@@ -301,7 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int e = 0; e < 4; ++e) {
         const int hr = e >> 1;
         const int key = key0 + nt * 8 + 2 * c + (e & 1);
-        const bool vis = row_ok[hr] && key >= row_lo[hr] && key <= row_hi[hr];
+        const bool vis =
+            row_ok[hr] && key <= row_hi[hr] && (key >= row_lo[hr] || key < p.sinks);
         const float v = vis ? sc[nt][e] * p.scale_log2 : -INFINITY;
         sc[nt][e] = v;
         tmax[hr] = fmaxf(tmax[hr], v);
@@ -451,7 +460,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p,
   const int k_len = __ldg(p.kv_lens + b);
   if (q_len > p.max_q_len || q_len * p.G > kDecodeMaxRows || k_len < 0 || k_len > p.max_kv_len)
     return;
-  const SeqSplit ss = seq_split(q_len, k_len, p.window, plan.tiles_per_split);
+  const SeqSplit ss = seq_split(q_len, k_len, p.window, p.sinks, plan.tiles_per_split);
   if (ss.n_splits <= 1) return;  // the decode kernel wrote this row itself
   const size_t stride = (size_t)p.T * p.H;
   float mx = -INFINITY;

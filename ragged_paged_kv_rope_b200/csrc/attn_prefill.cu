@@ -55,6 +55,7 @@
 // is bounded; on a timeout the CTA raises RPK_DEVERR_TIMEOUT, drains its copies
 // and MMAs, frees TMEM and returns.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -131,9 +132,9 @@ struct Bars {
   uint64_t k_empty[4];
   uint64_t v_empty[4];
   uint64_t s_full[2];   // per query tile
-  uint64_t p_full[2];   // per query tile
+  uint64_t p_full[2];   // per query tile: P_t written (one arrival per softmax warp)
   uint64_t o_final[2];  // per query tile: its last P V has completed
-  uint64_t o_empty[2];  // per query tile: the epilogue has read O
+  uint64_t o_empty[2];  // per query tile: the epilogue has read O (one arrival per warp)
   uint64_t item_full[2];   // work-item ring: index written by the producer
   uint64_t item_empty[2];  // work-item ring: index read by the MMA and softmax warps
   uint64_t drain;
@@ -188,9 +189,15 @@ struct Item {
   int b, kvh, q0, q_len, k_len;
   int t_begin;      // first token of tile A
   bool has_b;       // tile B holds at least one token
-  int j_begin;      // first key tile
-  int n_tiles;      // key tiles (0: every row sees no key)
+  int j_begin;      // first key tile of the band
+  int n_sink;       // attention-sink tiles [0, n_sink), all below j_begin
+  int n_tiles;      // sink and band key tiles (0: every row sees no key)
 };
+
+// Key tile of entry i of an item's tile list: the sink tiles, then the band.
+__device__ __forceinline__ int tile_of(const Item& it, int i) {
+  return i < it.n_sink ? i : it.j_begin + (i - it.n_sink);
+}
 
 // Decode work item w (items ordered by sequence, then query-pair index
 // descending, then KV head). False when the item is empty or the sequence's
@@ -218,10 +225,13 @@ __device__ __forceinline__ bool decode_item(const AttnParams& p, int w, int n_qp
   const int lo_first = p.window > 0 ? max(0, p_first - p.window + 1) : 0;
   const int hi_all = min(p_last, it.k_len - 1);
   it.j_begin = 0;
+  it.n_sink = 0;
   it.n_tiles = 0;
   if (hi_all >= lo_first) {
     it.j_begin = lo_first / kBN;
-    it.n_tiles = hi_all / kBN + 1 - it.j_begin;
+    const int sink_keys = min(p.sinks, lo_first);  // keys below the band that stay visible
+    it.n_sink = min((sink_keys + kBN - 1) / kBN, it.j_begin);
+    it.n_tiles = it.n_sink + hi_all / kBN + 1 - it.j_begin;
   }
   return true;
 }
@@ -266,9 +276,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.q_full[t], 1);
       mbar_init(&bars.q_empty[t], 1);
       mbar_init(&bars.s_full[t], 1);
-      mbar_init(&bars.p_full[t], 128);
+      mbar_init(&bars.p_full[t], 4);     // one arrival per softmax warp
       mbar_init(&bars.o_final[t], 1);
-      mbar_init(&bars.o_empty[t], 128);
+      mbar_init(&bars.o_empty[t], 4);
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&bars.item_full[k], 1);
@@ -346,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t* bt = p.block_table + (size_t)it.b * p.max_pages;
         const int gi = g + i;
         const int st = gi % S;
-        const int key0 = (it.j_begin + i) * kBN;
+        const int key0 = tile_of(it, i) * kBN;
         for (int is_v = 0; is_v < 2; ++is_v) {
           uint64_t* empty = is_v ? &bars.v_empty[st] : &bars.k_empty[st];
           uint64_t* full = is_v ? &bars.v_full[st] : &bars.k_full[st];
@@ -490,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (t == 0) {
             if (!warp_wait(&bars.v_full[st], (gi / S) & 1, abort, p.error_word)) { ok = false; break; }
             tc::fence_after_sync();
-            const int key0 = (it.j_begin + i) * kBN;
+            const int key0 = tile_of(it, i) * kBN;
             if (key0 + kBN > it.k_len) {
               // zero value rows at or past k_len
               const int r0 = max(0, it.k_len - key0);
@@ -579,82 +589,109 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int hi = pos;
       const int n = it.n_tiles;
       float m = -INFINITY, l = 0.f;      // running max (log2 units) and sum
-      float v[kBN];
-      for (int i = 0; i < n; ++i) {
-        if (!warp_wait(&bars.s_full[t], s_seen & 1, abort, p.error_word)) { ok = false; break; }
-        ++s_seen;
-        tc::fence_after_sync();
+      // The tile loop, compiled twice: without attention sinks (the common
+      // case keeps the plain single-interval mask) and with them.
+      auto tile_loop = [&](auto with_sinks) {
+        constexpr bool kSinks = decltype(with_sinks)::value;
+        float v[kBN];
+        for (int i = 0; i < n; ++i) {
+          if (!warp_wait(&bars.s_full[t], s_seen & 1, abort, p.error_word)) { ok = false; break; }
+          ++s_seen;
+          tc::fence_after_sync();
 #pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) tc::tmem_ld32(s_col + c * 32, v + c * 32);
-        tc::tmem_wait_ld();
-        const int key0 = (it.j_begin + i) * kBN;
-        if (!(row_ok && key0 >= lo && key0 + kBN - 1 <= hi)) {
-          // visible columns [c_lo, c_hi] of this tile (empty for an invalid row)
-          const int c_lo = row_ok ? lo - key0 : kBN;
-          const int c_hi = row_ok ? hi - key0 : -1;
+          for (int c = 0; c < kBN / 32; ++c) tc::tmem_ld32(s_col + c * 32, v + c * 32);
+          tc::tmem_wait_ld();
+          const int key0 = tile_of(it, i) * kBN;
+          if constexpr (!kSinks) {
+            if (!(row_ok && key0 >= lo && key0 + kBN - 1 <= hi)) {
+              // visible columns [c_lo, c_hi] of this tile (empty for an invalid row)
+              const int c_lo = row_ok ? lo - key0 : kBN;
+              const int c_hi = row_ok ? hi - key0 : -1;
 #pragma unroll
-          for (int c = 0; c < kBN; ++c)
-            if (c < c_lo || c > c_hi) v[c] = -INFINITY;
-        }
-        // Row max: 8 independent chains of three-input max.
-        float m8[8];
+              for (int c = 0; c < kBN; ++c)
+                if (c < c_lo || c > c_hi) v[c] = -INFINITY;
+            }
+          } else {
+            // Visible columns: the window's [c_lo, c_hi] and the sinks below
+            // c_sink (none for an invalid row). The sinks either join the window
+            // (c_sink >= c_lo: one interval from 0) or lie below it.
+            int c_lo = row_ok ? lo - key0 : kBN;
+            const int c_hi = row_ok ? hi - key0 : -1;
+            const int c_sink = p.sinks - key0;
+            if (c_sink >= c_lo) c_lo = 0;
+            if (c_sink > 0 && c_sink < c_lo) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) m8[k] = fmaxf(v[k], v[8 + k]);
+              for (int c = 0; c < kBN; ++c)
+                if (c > c_hi || (c < c_lo && c >= c_sink)) v[c] = -INFINITY;
+            } else if (c_lo > 0 || c_hi < kBN - 1) {
 #pragma unroll
-        for (int c = 16; c < kBN; c += 16)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) m8[k] = max3(m8[k], v[c + k], v[c + 8 + k]);
-        float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-        mx *= sl2;  // scale > 0: max of the scaled scores
-        // Running max: taken at once while empty, else only when it grows by
-        // more than the threshold (then O and l are rescaled). O_t holds
-        // P_t(i-1) V_{i-1} here: S_t(i) was issued after it and has completed.
-        float alpha = 1.f;
-        bool rescale = false;
-        if (m == -INFINITY) {
-          m = mx;
-        } else if (mx > m + kRescaleThreshold) {
-          alpha = fast_exp2(m - mx);
-          m = mx;
-          rescale = true;
-        }
-        l *= alpha;
-        const float neg_m = m == -INFINITY ? 0.f : -m;  // an empty row keeps P = 0
-        float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
-        // P in two halves of 64 keys (32 packed columns each) to bound registers.
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            float x0, x1;
-            fma2(x0, x1, v[h * 64 + c], v[h * 64 + c + 1], sl2, neg_m);
-            const float w0 = fast_exp2(x0);
-            const float w1 = fast_exp2(x1);
-            const int k = (c >> 1) & 3;
-            add2(rs[2 * k], rs[2 * k + 1], w0, w1);
-            pk[c >> 1] = pack_bf16x2(w0, w1);
+              for (int c = 0; c < kBN; ++c)
+                if (c < c_lo || c > c_hi) v[c] = -INFINITY;
+            }
           }
-          tc::tmem_st32(s_col + h * 32, reinterpret_cast<const float*>(pk));
-        }
-        l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
-        // Rescale O_t (after P, so that the scores are dead): it must finish
-        // before P_t(i) V_i is issued, i.e. before p_full.
-        if (i > 0 && __any_sync(0xffffffffu, rescale)) {
-          float o[32];
+          // Row max: 8 independent chains of three-input max.
+          float m8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) m8[k] = fmaxf(v[k], v[8 + k]);
+#pragma unroll
+          for (int c = 16; c < kBN; c += 16)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m8[k] = max3(m8[k], v[c + k], v[c + 8 + k]);
+          float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+          mx *= sl2;  // scale > 0: max of the scaled scores
+          // Running max: taken at once while empty, else only when it grows by
+          // more than the threshold (then O and l are rescaled). O_t holds
+          // P_t(i-1) V_{i-1} here: S_t(i) was issued after it and has completed.
+          float alpha = 1.f;
+          bool rescale = false;
+          if (m == -INFINITY) {
+            m = mx;
+          } else if (mx > m + kRescaleThreshold) {
+            alpha = fast_exp2(m - mx);
+            m = mx;
+            rescale = true;
+          }
+          l *= alpha;
+          const float neg_m = m == -INFINITY ? 0.f : -m;  // an empty row keeps P = 0
+          float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
+          // P in two halves of 64 keys (32 packed columns each) to bound registers.
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+              float x0, x1;
+              fma2(x0, x1, v[h * 64 + c], v[h * 64 + c + 1], sl2, neg_m);
+              const float w0 = fast_exp2(x0);
+              const float w1 = fast_exp2(x1);
+              const int k = (c >> 1) & 3;
+              add2(rs[2 * k], rs[2 * k + 1], w0, w1);
+              pk[c >> 1] = pack_bf16x2(w0, w1);
+            }
+            tc::tmem_st32(s_col + h * 32, reinterpret_cast<const float*>(pk));
+          }
+          l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+          // Rescale O_t (after P, so that the scores are dead): it must finish
+          // before P_t(i) V_i is issued, i.e. before p_full.
+          if (i > 0 && __any_sync(0xffffffffu, rescale)) {
+            float o[32];
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            tc::tmem_ld32(o_col + c * 32, o);
-            tc::tmem_wait_ld();
+            for (int c = 0; c < D / 32; ++c) {
+              tc::tmem_ld32(o_col + c * 32, o);
+              tc::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tc::tmem_st32(o_col + c * 32, o);
+              for (int e = 0; e < 32; ++e) o[e] *= alpha;
+              tc::tmem_st32(o_col + c * 32, o);
+            }
           }
+          tc::tmem_wait_st();
+          tc::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars.p_full[t]);
         }
-        tc::tmem_wait_st();
-        tc::fence_before_sync();
-        mbar_arrive(&bars.p_full[t]);
-      }
+      };
+      if (p.sinks > 0) tile_loop(std::true_type{});
+      else tile_loop(std::false_type{});
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
       const bool have_o = n > 0;
@@ -677,7 +714,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c + 1 == D / 32) {
             // O_t may now be overwritten by the next item's first P V.
             tc::fence_before_sync();
-            mbar_arrive(&bars.o_empty[t]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.o_empty[t]);
           }
         }
         if (row_ok) {

@@ -8,7 +8,8 @@
 // running sum l rescaled by e^(m_old - m_new), running output likewise, final
 // divide). Keys of row r of a sequence with q_len rows and k_len keys are
 // [p - (window - 1), p] with p = r + k_len - q_len (NumKong "Attention with a
-// Pre-Packed KV-Cache"); a row with no visible key is written as zeros.
+// Pre-Packed KV-Cache"), plus, under a window, the first `sinks` keys (algenta
+// streaming_llm_sink_score); a row with no visible key is written as zeros.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -53,7 +54,10 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const AttnParams
     const T* __restrict__ kp = static_cast<const T*>(p.k_pages);
     const T* __restrict__ vp = static_cast<const T*>(p.v_pages);
     const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
-    for (int j = lo; j <= hi; ++j) {
+    // Attention sinks first (keys below the window that stay visible), then the band.
+    const int sink_end = min(p.sinks, lo);
+    for (int jj = 0; jj < sink_end + (hi - lo + 1); ++jj) {
+      const int j = jj < sink_end ? jj : lo + (jj - sink_end);
       const int pi = j / p.P;
       const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
       if (page < 0 || page >= p.num_pages) {

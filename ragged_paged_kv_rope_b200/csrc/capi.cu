@@ -190,7 +190,8 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
                                   float scale, int32_t window, void* out, int32_t batch,
                                   int32_t total_q_tokens, int32_t max_q_len,
                                   int32_t max_kv_len, rpk_dtype dtype, void* workspace,
-                                  size_t workspace_bytes, float* log_sum_exp, void* stream) {
+                                  size_t workspace_bytes, float* log_sum_exp,
+                                  int32_t sink_tokens, void* stream) {
   if (!q || !q_row_offsets || !kv_lens || !out) return RPK_ERR_NULL;
   rpk_status st = check_cache(page_table);
   if (st != RPK_OK) return st;
@@ -204,12 +205,14 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
   if (!(scale > 0.f) || !std::isfinite(scale)) return RPK_ERR_SHAPE;
   if (!aligned16(q) || !aligned16(out)) return RPK_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(log_sum_exp) & 3u) != 0) return RPK_ERR_SHAPE;
+  if (sink_tokens < 0) return RPK_ERR_SHAPE;
   if ((long long)max_kv_len > (long long)page_table->max_pages_per_seq * page_table->page_size)
     return RPK_ERR_SHAPE;
   if (total_q_tokens == 0) return RPK_OK;
 
   rpk::AttnParams p;
   p.lse = log_sum_exp;
+  p.sinks = window > 0 ? sink_tokens : 0;
   p.q = q; p.out = out;
   {
     void *k, *v;

@@ -61,6 +61,7 @@ struct AttnParams {
   float scale;
   float scale_log2;            // scale * log2(e)
   float* lse = nullptr;        // [T, H] natural log-sum-exp of each row's scores, or null
+  int32_t sinks = 0;           // under a window: the first `sinks` keys stay visible
 };
 
 // fp32 / bf16 CUDA-core attention: one warp per (token, head) row.

@@ -85,13 +85,13 @@ def oracle_rope(wl: W.Workload, table: np.ndarray):
     return O.rope(wl.q, *args), O.rope(wl.k_new, *args)
 
 
-def gpu_attention(wl: W.Workload, dev: Dev, q: torch.Tensor, window=None, lse=None):
+def gpu_attention(wl: W.Workload, dev: Dev, q: torch.Tensor, window=None, lse=None, sinks=0):
     sp = wl.spec
     out = torch.empty_like(q)
     R.ragged_paged_attention(q, dev.offsets, dev.kv_lens, dev.cache, sp.n_heads, sp.n_kv_heads,
                              sp.head_dim, sp.softmax_scale, sp.window if window is None else window,
                              out, max_q_len=wl.max_q_len, max_kv_len=wl.max_kv_len,
-                             log_sum_exp=lse)
+                             log_sum_exp=lse, sink_tokens=sinks)
     return out
 
 

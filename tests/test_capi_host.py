@@ -72,12 +72,12 @@ def rope(L, c, **kw):
 
 def attn(L, c, **kw):
     a = dict(q=FAKE, off=FAKE, kvl=FAKE, H=32, Hk=8, d=128, scale=0.1, w=0, out=FAKE, batch=2,
-             T=5, mq=4, mk=200, dtype=B.RPK_BF16, ws=None, wsb=0, lse=None)
+             T=5, mq=4, mk=200, dtype=B.RPK_BF16, ws=None, wsb=0, lse=None, sinks=0)
     a.update(kw)
     return L.ragged_paged_attention(a["q"], a["off"], a["kvl"], C.byref(c), a["H"], a["Hk"],
                                     a["d"], a["scale"], a["w"], a["out"], a["batch"], a["T"],
                                     a["mq"], a["mk"], a["dtype"], a["ws"], a["wsb"], a["lse"],
-                                    None)
+                                    a["sinks"], None)
 
 
 @host_only
@@ -121,6 +121,7 @@ def test_rope_rejects_cache(L, ckw, status):
     ({"mq": 5, "ws": FAKE + 16, "wsb": 1 << 20}, 6),               # misaligned
     ({"mq": 5, "ws": FAKE, "wsb": 128}, 6),                        # too small
     ({"lse": FAKE + 2}, 2),                                        # misaligned log-sum-exp
+    ({"sinks": -1}, 2),
 ])
 def test_attention_rejects(L, kw, status):
     assert attn(L, cache(max_pages_per_seq=16), **kw) == status

@@ -18,18 +18,18 @@ from parity import REDUCED, check_attention, check_lse, gpu_attention, sample_ro
 pytestmark = pytest.mark.gpu
 
 
-def _attn_case(sp: W.Spec, q_lens, kv_lens, seed=0, rows=None, window=None):
+def _attn_case(sp: W.Spec, q_lens, kv_lens, seed=0, rows=None, window=None, sinks=0):
     wl = W.attention_only(sp, seed, q_lens, kv_lens)
     dev = to_device(wl)
     w = sp.window if window is None else window
     # every case also checks the log-sum-exp output against the oracle's
     lse = torch.full((wl.total_tokens, sp.n_heads), float("nan"), device="cuda")
-    out = gpu_attention(wl, dev, dev.q, window=w, lse=lse)
+    out = gpu_attention(wl, dev, dev.q, window=w, lse=lse, sinks=sinks)
     torch.cuda.synchronize()
     assert int(dev.error_word.item()) == 0
     ref, ref_lse = O.attention(wl.q, wl.q_offsets, wl.kv_lens, wl.k_pages, wl.v_pages,
                                wl.block_table, sp.n_kv_heads, sp.softmax_scale, w, rows=rows,
-                               with_lse=True)
+                               with_lse=True, sinks=sinks)
     got, got_lse = out.cpu(), lse.cpu()
     if rows is not None:
         ti, hi = torch.from_numpy(rows[:, 0]).long(), torch.from_numpy(rows[:, 1]).long()
@@ -100,6 +100,49 @@ def test_attention_edge_cases(idx, dtype):
     base.update(over)
     sp = W.spec("ragged_prefill", **base)
     _attn_case(sp, q_lens, kv_lens, seed=idx, window=window)
+
+
+# ------------------------------------------------ attention sinks + window
+
+SINKS = [
+    # (description, spec overrides, q_lens, kv_lens, window, sinks)
+    ("decode, 4 sinks", {}, [1, 1, 1], [5000, 300, 70], 1000, 4),
+    ("decode, sinks over several tiles", {}, [1, 1], [9000, 2000], 700, 150),
+    ("decode, sinks reach the window", {}, [1, 1], [400, 90], 300, 200),
+    ("decode, group 8 two tokens", {"n_heads": 16, "n_kv_heads": 2}, [2, 1], [3000, 129], 64, 3),
+    ("prefill, 4 sinks", {}, [300, 200], [300, 900], 100, 4),
+    ("prefill, sinks over two tiles", {}, [260, 40], [700, 260], 129, 200),
+    ("prefill head_dim 64", {"head_dim": 64, "rotary_dim": 64}, [150, 90], [600, 90], 64, 17),
+    ("head_dim 256", {"head_dim": 256, "rotary_dim": 128}, [1, 40], [3000, 500], 256, 8),
+    ("window 1 with sinks", {}, [50, 1], [50, 1000], 1, 5),
+]
+
+
+@pytest.mark.parametrize("idx", range(len(SINKS)))
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_attention_sinks(idx, dtype):
+    desc, over, q_lens, kv_lens, window, sinks = SINKS[idx]
+    base = dict(n_heads=8, n_kv_heads=2, head_dim=128, page_size=32, dtype=dtype)
+    base.update(over)
+    sp = W.spec("ragged_prefill", **base)
+    _attn_case(sp, q_lens, kv_lens, seed=40 + idx, window=window, sinks=sinks)
+
+
+def test_attention_sinks_ignored_without_window():
+    sp = W.spec("ragged_prefill", n_heads=8, n_kv_heads=2, batch=2)
+    wl = W.attention_only(sp, 50, [70, 1], [70, 500])
+    dev = to_device(wl)
+    a = gpu_attention(wl, dev, dev.q, window=0, sinks=0).cpu()
+    b = gpu_attention(wl, dev, dev.q, window=0, sinks=9).cpu()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+@pytest.mark.slow
+def test_attention_gemma_window_with_sinks_sampled():
+    # the Gemma-like sliding-window decode at full context, with 4 sink tokens
+    sp = W.SPECS["gemma_swa_decode"]
+    rng_rows = np.array([[t, h] for t in range(sp.batch) for h in range(sp.n_heads)], np.int32)
+    _attn_case(sp, [1] * sp.batch, [32769] * sp.batch, seed=51, rows=rng_rows, sinks=4)
 
 
 def test_attention_prefill_shapes_bf16():
