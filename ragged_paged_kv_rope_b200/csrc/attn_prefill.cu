@@ -9,8 +9,8 @@
 // running sum and output rescaled by e^(m_old - m_new), final divide).
 //
 // Work unit (item): two query tiles A and B of 128 rows each of one
-// (sequence, KV head), against 128-key tiles. The 128 rows of a tile are the
-// (token, query head) pairs of one KV head's group, token-major
+// (sequence, KV head), against key tiles of 64 keys. The 128 rows of a tile
+// are the (token, query head) pairs of one KV head's group, token-major
 // (tokens_per_tile = 128 / G), so the G query heads that share a KV head share
 // every K/V tile; tile B holds the next tokens_per_tile tokens after tile A.
 //
@@ -20,36 +20,45 @@
 // sequence at the same time read the same K/V tiles in the same order, so a
 // tile read from HBM for one of them is an L2 hit for the others.
 //
+// Tensor memory (512 columns): two score buffers of 64 columns per query
+// tile (S_t[0], S_t[1]) and one 128-row output accumulator per tile (O_A,
+// O_B). Score tile i of both query tiles lives in buffer i mod 2, and P_t(i)
+// (packed bf16 pairs) is written over the first 32 columns of S_t(i). The MMA
+// issuer computes S(i+2) right after issuing P(i) V_i, so while the softmax
+// warpgroups turn S(i) into P(i), the tensor core has already computed S(i+1):
+// the softmax does not wait for the tensor core in the steady state, and the
+// two softmax warpgroups keep the exponential unit busy together. Every item
+// runs both query tiles (tile B's rows past the sequence are masked and never
+// stored), so the two tiles share every barrier phase.
+//
 // Warp roles (384 threads, three warpgroups):
 //   warp 0     TMA producer: claims the next item, hands its index to the
 //              other roles through a two-slot ring in shared memory, loads the
-//              item's Q tiles, then its K and V tiles of 128 keys into a ring
-//              of stages (3-D map over the pool [pages * page_size, kv_heads,
+//              item's two Q tiles, then each key tile's K and V into one stage
+//              of a ring (3-D map over the pool [pages * page_size, kv_heads,
 //              d], one box per page segment, 128-byte swizzle, no multicast)
-//   warp 1     allocates TMEM (512 columns: S_A, S_B, O_A, O_B) and issues the
-//              MMAs from one thread, alternating the tiles: S_t = Q_t K_j^T
-//              (operands in shared memory), then O_t += P_t V_j with P_t read
-//              from TMEM (written over the first 64 columns of S_t) and V_j an
-//              MN-major operand in shared memory. While one softmax warpgroup
-//              works on its tile, the tensor core runs the other tile's MMAs;
-//              the next item's first S MMAs run while the softmax warps
-//              store the current item's rows.
+//   warp 1     allocates TMEM and issues the MMAs from one thread: per item
+//              S(0), S(1), then per key tile i one burst of O_A += P_A(i) V_i,
+//              O_B += P_B(i) V_i (P from TMEM, V an MN-major operand in shared
+//              memory), S_A(i+2) and S_B(i+2) (Q_t K^T, both operands in shared
+//              memory); the next item's first S MMAs follow the last P V of the
+//              current one
 //   warps 2-3  idle (they complete the first warpgroup)
 //   warps 4-7  softmax of tile A, warps 8-11 softmax of tile B: thread r owns
-//              row r (TMEM lane r); loads S_t, masks the band, keeps (m, l) in
-//              log2 units, writes P_t as packed bf16 pairs, and rescales O_t in
-//              TMEM only when the running max grew by more than 2^8 (the final
-//              O / l uses the same max, so this is exact); then normalises O_t
-//              and stores the rows.
+//              row r (TMEM lane r); loads S_t(i), masks the band, keeps (m, l)
+//              in log2 units, writes P_t(i), and rescales O_t in TMEM only
+//              when the running max grew by more than 2^8 (the final O / l
+//              uses the same max, so this is exact); then normalises O_t and
+//              stores the rows.
+// A rescale of O_t during tile i must fall between P(i-1) V_{i-1} and
+// P(i) V_i. For i < n - 1 the softmax waits for S(i+1), which the issuer
+// placed after P(i-1) V_{i-1}; for the item's last tile it waits for a
+// barrier the issuer commits once per item after P(n-2) V_{n-2}. Either
+// barrier can be at most one phase short of the one waited for (P(i) V_i
+// needs this warp's own P(i)), so the phase parity is unambiguous.
 // Registers: the first warpgroup gives registers back (setmaxnreg 56) and the
-// two softmax warpgroups take them (setmaxnreg 224), so that a softmax thread
-// holds a whole 128-score row and its item state in registers (ptxas spills 24
-// bytes at this split; at 232 the softmax spills none but the control warps,
-// left with 40, spill instead);
+// two softmax warpgroups take them (setmaxnreg 224);
 // 4*32*56 + 8*32*224 = 64512 registers, the 384 * 168 the CTA is launched with.
-// MMAs issued by one thread run in issue order, so P_t(j) V_j completes before
-// S_t(j+1) overwrites the columns P_t(j) lives in, and the completion of
-// S_t(j+1) also tells the softmax that O_t holds P_t(j) V_j.
 // Value rows at or past k_len are zeroed in shared memory before P V, so the
 // NaN sentinels of unused slots never meet a zero weight. Every mbarrier wait
 // is bounded; on a timeout the CTA raises RPK_DEVERR_TIMEOUT, drains its copies
@@ -67,8 +76,8 @@ int prefill_rows_per_tile(int group) { return group >= 1 && group <= 128 ? (128 
 
 namespace {
 
-constexpr int kBM = 128;   // rows per tile (MMA M)
-constexpr int kBN = 128;   // keys per tile
+constexpr int kBM = 128;              // rows per tile (MMA M)
+constexpr int kBN = kPrefillKeyTile;  // keys per tile (64)
 constexpr int kThreads = 384;
 constexpr int kRegsControl = 56;    // warpgroup 0: producer, MMA issuer, 2 idle warps
 constexpr int kRegsSoftmax = 224;   // warpgroups 1 and 2: softmax
@@ -108,33 +117,33 @@ __device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1) {
 template <int D>
 struct Cfg {
   static constexpr int kBoxes = D / 64;
-  static constexpr int kStages = D == 128 ? 2 : 4;   // K/V ring depth
+  static constexpr int kStages = D == 128 ? 5 : 10;  // K/V ring depth (key tiles)
   static constexpr int kQBytes = kBM * D * 2;         // one query tile
-  static constexpr int kKVBytes = kBN * D * 2;
+  static constexpr int kKVBytes = kBN * D * 2;        // one K or V tile
+  static constexpr int kStageBytes = 2 * kKVBytes;    // K then V of one key tile
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + 2 * kQBytes;
-  static constexpr int kVOff = kKOff + kStages * kKVBytes;
-  static constexpr int kEnd = kVOff + kStages * kKVBytes + 1024;
+  static constexpr int kKVOff = kQOff + 2 * kQBytes;
+  static constexpr int kEnd = kKVOff + kStages * kStageBytes + 1024;
   // At least half the SM's shared memory, so that one CTA holds the SM's TMEM.
   static constexpr int kSmemBytes = kEnd > 118 * 1024 ? kEnd : 118 * 1024;
-  // TMEM columns: S_A, S_B (fp32, 128 each; P_t over the first 64 of S_t), O_A, O_B
-  static constexpr uint32_t kSCol = 0;
-  static constexpr uint32_t kOCol = 2 * kBN;
+  // TMEM columns: S_t[b] (fp32, 64 each) at (2t + b) * 64, then O_A, O_B.
+  static constexpr uint32_t kOCol = 4 * kBN;
   static_assert(kOCol + 2 * D <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
+__host__ __device__ constexpr uint32_t s_col(int t, int b) { return (uint32_t)((2 * t + b) * kBN); }
+
 struct Bars {
-  uint64_t q_full[2];   // per query tile
-  uint64_t q_empty[2];  // per query tile: the item's last S MMA reading it has completed
-  uint64_t k_full[4];
-  uint64_t v_full[4];
-  uint64_t k_empty[4];
-  uint64_t v_empty[4];
-  uint64_t s_full[2];   // per query tile
-  uint64_t p_full[2];   // per query tile: P_t written (one arrival per softmax warp)
-  uint64_t o_final[2];  // per query tile: its last P V has completed
-  uint64_t o_empty[2];  // per query tile: the epilogue has read O (one arrival per warp)
+  uint64_t q_full;       // both query tiles loaded
+  uint64_t q_empty;      // the item's last S MMAs reading them have completed
+  uint64_t kv_full[10];  // per stage: K and V of one key tile loaded
+  uint64_t kv_empty[10]; // per stage: its last P V has completed
+  uint64_t s_full[2];    // per score buffer: S_A and S_B computed
+  uint64_t p_full[2];    // per score buffer: P_A and P_B written (one arrival per softmax warp)
+  uint64_t pv_item[1];   // one phase per item with two or more key tiles: P(n-2) V done
+  uint64_t o_final;      // the item's last P V has completed
+  uint64_t o_empty;      // the epilogue has read O (one arrival per softmax warp)
   uint64_t item_full[2];   // work-item ring: index written by the producer
   uint64_t item_empty[2];  // work-item ring: index read by the MMA and softmax warps
   uint64_t drain;
@@ -188,7 +197,6 @@ __device__ __forceinline__ void do_abort(volatile int* abort, int32_t* error_wor
 struct Item {
   int b, kvh, q0, q_len, k_len;
   int t_begin;      // first token of tile A
-  bool has_b;       // tile B holds at least one token
   int j_begin;      // first key tile of the band
   int n_sink;       // attention-sink tiles [0, n_sink), all below j_begin
   int n_tiles;      // sink and band key tiles (0: every row sees no key)
@@ -218,7 +226,6 @@ __device__ __forceinline__ bool decode_item(const AttnParams& p, int w, int n_qp
   }
   it.t_begin = qt * 2 * tpt;
   if (it.t_begin >= it.q_len) return false;
-  it.has_b = it.t_begin + tpt < it.q_len;
   const int t_end = min(it.q_len, it.t_begin + 2 * tpt);
   const int p_first = it.t_begin + it.k_len - it.q_len;
   const int p_last = (t_end - 1) + it.k_len - it.q_len;
@@ -245,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = Cfg<D>;
   constexpr int S = C::kStages;
   constexpr int kItemReaders = 9;  // MMA warp + 8 softmax warps
+  constexpr int kSoftmaxWarps = 8;
   extern __shared__ uint8_t smem_raw[];
   __shared__ Bars bars;
   __shared__ int item_slot[2];
@@ -262,24 +270,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const uint32_t sbase = smem_u32(smem);
   auto q_s = [&](int t) { return sbase + C::kQOff + t * C::kQBytes; };
-  auto k_s = [&](int st) { return sbase + C::kKOff + st * C::kKVBytes; };
-  auto v_s = [&](int st) { return sbase + C::kVOff + st * C::kKVBytes; };
+  auto k_s = [&](int st) { return sbase + C::kKVOff + st * C::kStageBytes; };
+  auto v_s = [&](int st) { return sbase + C::kKVOff + st * C::kStageBytes + C::kKVBytes; };
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < S; ++st) {
-      mbar_init(&bars.k_full[st], 1);
-      mbar_init(&bars.v_full[st], 1);
-      mbar_init(&bars.k_empty[st], 1);
-      mbar_init(&bars.v_empty[st], 1);
+      mbar_init(&bars.kv_full[st], 1);
+      mbar_init(&bars.kv_empty[st], 1);
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&bars.q_full[t], 1);
-      mbar_init(&bars.q_empty[t], 1);
-      mbar_init(&bars.s_full[t], 1);
-      mbar_init(&bars.p_full[t], 4);     // one arrival per softmax warp
-      mbar_init(&bars.o_final[t], 1);
-      mbar_init(&bars.o_empty[t], 4);
+    mbar_init(&bars.q_full, 1);
+    mbar_init(&bars.q_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars.s_full[b], 1);
+      mbar_init(&bars.p_full[b], kSoftmaxWarps);
     }
+    mbar_init(&bars.pv_item[0], 1);
+    mbar_init(&bars.o_final, 1);
+    mbar_init(&bars.o_empty, kSoftmaxWarps);
     for (int k = 0; k < 2; ++k) {
       mbar_init(&bars.item_full[k], 1);
       mbar_init(&bars.item_empty[k], kItemReaders);
@@ -311,13 +318,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_box_bytes = 128u * (uint32_t)rows_used;
       const int box_rows = p.P < kBN ? p.P : kBN;
       const uint32_t seg_bytes = (uint32_t)box_rows * 128u * C::kBoxes;
-      int g = 0;                // first global key tile of the current item
-      int k_issued = 0, v_issued = 0;  // K / V tile loads issued over all items
-      int q_loads[2] = {0, 0};  // Q loads per tile over all items
+      int kv_issued = 0;  // key tiles loaded over all items
+      int q_loads = 0;    // Q loads over all items
       bool ok = true;
-      // Claim a non-empty work item and hand its index to the MMA and softmax warps through the ring. The next
-      // item is claimed after the current one's Q and first K/V stages are in
-      // flight, so the claim's latency hides behind real work.
+      // Claim a non-empty work item and hand its index to the MMA and softmax
+      // warps through the ring. The next item is claimed after the current
+      // one's Q and first key tiles are in flight, so the claim's latency hides
+      // behind real work.
       auto claim = [&](Item& it) -> int {
         int w;
         do {
@@ -334,61 +341,58 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bars.item_full[slot]);
         return true;
       };
-      // Q tiles of an item: each buffer is refilled once the previous item's
-      // S MMAs that read it have completed.
+      // The two Q tiles of an item, once the previous item's S MMAs that read
+      // them have completed. Rows past the last token read the fill value.
       auto load_q = [&](const Item& it) -> bool {
-        for (int t = 0; t < (it.has_b ? 2 : 1); ++t) {
-          if (q_loads[t] > 0 &&
-              !thread_wait(&bars.q_empty[t], (q_loads[t] - 1) & 1, abort, p.error_word))
-            return false;
-          mbar_arrive_expect_tx(&bars.q_full[t], C::kBoxes * q_box_bytes);
+        if (q_loads > 0 && !thread_wait(&bars.q_empty, (q_loads - 1) & 1, abort, p.error_word))
+          return false;
+        mbar_arrive_expect_tx(&bars.q_full, 2 * C::kBoxes * q_box_bytes);
+        for (int t = 0; t < 2; ++t)
 #pragma unroll
           for (int bx = 0; bx < C::kBoxes; ++bx)
             tma_load_3d(smem + C::kQOff + t * C::kQBytes + bx * (kBM * 128), &q_map, bx * 64,
-                        it.kvh * G, it.q0 + it.t_begin + t * tpt, &bars.q_full[t]);
-          ++q_loads[t];
-        }
+                        it.kvh * G, it.q0 + it.t_begin + t * tpt, &bars.q_full);
+        ++q_loads;
         return true;
       };
-      // K and V of key tile i of an item (global tile index g + i); K of a
-      // stage frees after the last S MMA that reads it, V after the last P V.
-      auto load_kv = [&](const Item& it, int i) -> bool {
+      // K and V of key tile i of an item into the next stage of the ring; a
+      // stage frees once the P V MMAs that read its V have completed.
+      auto load_stage = [&](const Item& it, int i) -> bool {
         const int32_t* bt = p.block_table + (size_t)it.b * p.max_pages;
-        const int gi = g + i;
+        const int gi = kv_issued;
         const int st = gi % S;
         const int key0 = tile_of(it, i) * kBN;
-        for (int is_v = 0; is_v < 2; ++is_v) {
-          uint64_t* empty = is_v ? &bars.v_empty[st] : &bars.k_empty[st];
-          uint64_t* full = is_v ? &bars.v_full[st] : &bars.k_full[st];
-          if (gi >= S && !thread_wait(empty, ((gi / S) & 1) ^ 1, abort, p.error_word))
-            return false;
-          uint32_t bytes = 0;
-          for (int r = 0; r < kBN; r += box_rows) {
-            const int key = key0 + r;
-            if (key >= it.k_len) break;
-            const int pi = key / p.P;
-            const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
-            if (page >= 0 && page < p.num_pages) bytes += seg_bytes;
-          }
-          mbar_arrive_expect_tx(full, bytes);
-          for (int r = 0; r < kBN; r += box_rows) {
-            const int key = key0 + r;
-            if (key >= it.k_len) break;
-            const int pi = key / p.P;
-            const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
-            if (page < 0 || page >= p.num_pages) {
-              if (!is_v) raise_error(p.error_word, RPK_DEVERR_PAGE);
-              continue;
-            }
-            const int grow = page * p.P + (key - pi * p.P);
-            uint8_t* base = smem + (is_v ? C::kVOff : C::kKOff) + st * C::kKVBytes + r * 128;
-#pragma unroll
-            for (int bx = 0; bx < C::kBoxes; ++bx)
-              tma_load_3d(base + bx * (kBN * 128), is_v ? &v_map : &k_map, bx * 64, it.kvh,
-                          grow, full);
-          }
-          if (is_v) ++v_issued; else ++k_issued;
+        if (gi >= S &&
+            !thread_wait(&bars.kv_empty[st], ((gi / S) & 1) ^ 1, abort, p.error_word))
+          return false;
+        uint32_t bytes = 0;
+        for (int r = 0; r < kBN; r += box_rows) {
+          const int key = key0 + r;
+          if (key >= it.k_len) break;
+          const int pi = key / p.P;
+          const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
+          if (page >= 0 && page < p.num_pages) bytes += 2 * seg_bytes;
         }
+        mbar_arrive_expect_tx(&bars.kv_full[st], bytes);
+        for (int r = 0; r < kBN; r += box_rows) {
+          const int key = key0 + r;
+          if (key >= it.k_len) break;
+          const int pi = key / p.P;
+          const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
+          if (page < 0 || page >= p.num_pages) {
+            raise_error(p.error_word, RPK_DEVERR_PAGE);
+            continue;
+          }
+          const int grow = page * p.P + (key - pi * p.P);
+          uint8_t* kb = smem + C::kKVOff + st * C::kStageBytes + r * 128;
+#pragma unroll
+          for (int bx = 0; bx < C::kBoxes; ++bx) {
+            tma_load_3d(kb + bx * (kBN * 128), &k_map, bx * 64, it.kvh, grow, &bars.kv_full[st]);
+            tma_load_3d(kb + C::kKVBytes + bx * (kBN * 128), &v_map, bx * 64, it.kvh, grow,
+                        &bars.kv_full[st]);
+          }
+        }
+        ++kv_issued;
         return true;
       };
       Item cur;
@@ -396,73 +400,87 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = publish(0, cur_w);
       for (int seq = 0; ok && cur_w >= 0; ++seq) {
         const int n = cur.n_tiles;
-        const int first = n < S ? n : S;
         if (n > 0) {
           ok = load_q(cur);
-          for (int i = 0; ok && i < first; ++i) ok = load_kv(cur, i);
+          for (int i = 0; ok && i < n && i < 2; ++i) ok = load_stage(cur, i);
         }
         if (!ok) break;
         Item next;
         const int next_w = claim(next);
         if (!publish(seq + 1, next_w)) { ok = false; break; }
-        for (int i = first; ok && i < n; ++i) ok = load_kv(cur, i);
+        for (int i = 2; ok && i < n; ++i) ok = load_stage(cur, i);
         if (!ok) break;
-        g += n;
         cur = next;
         cur_w = next_w;
       }
       if (!ok) do_abort(abort, p.error_word);
       // Never leave with copies in flight.
-      for (int t = 0; t < 2; ++t)
-        if (q_loads[t] > 0) mbar_wait(&bars.q_full[t], (q_loads[t] - 1) & 1);
-      for (int gi = max(0, k_issued - S); gi < k_issued; ++gi)
-        mbar_wait(&bars.k_full[gi % S], (gi / S) & 1);
-      for (int gi = max(0, v_issued - S); gi < v_issued; ++gi)
-        mbar_wait(&bars.v_full[gi % S], (gi / S) & 1);
+      if (q_loads > 0) mbar_wait(&bars.q_full, (q_loads - 1) & 1);
+      for (int gi = max(0, kv_issued - S); gi < kv_issued; ++gi)
+        mbar_wait(&bars.kv_full[gi % S], (gi / S) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
     constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(kBM, kBN, 0);
     constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(kBM, D, 1);
-    int g = 0;                          // key tiles consumed over all items
-    int q_seen[2] = {0, 0};             // Q loads consumed per tile
-    int s_issued[2] = {0, 0};           // S MMAs (= s_full commits) per tile
-    int p_seen[2] = {0, 0};             // p_full phases consumed per tile
-    int o_commits[2] = {0, 0};          // o_final commits per tile
+    int g_kv = 0;        // key tiles whose stage has been waited for, over all items
+    int g_pv = 0;        // key tiles whose P V has been issued, over all items
+    int q_seen = 0;      // Q loads consumed
+    int s_issued = 0;    // S tile pairs issued (buffer = count mod 2)
+    int o_commits = 0;   // o_final commits
     bool ok = true;
-    auto issue_s = [&](int t, int gi) {
+    // Shared-memory descriptors: the start address is the low field
+    // (address >> 4, 14 bits; every operand lies below 256 KB), so a
+    // descriptor at an offset is the base descriptor plus offset >> 4.
+    const uint64_t q_desc0 = tc::smem_desc_sw128(q_s(0), 16, 1024);
+    const uint64_t k_desc0 = tc::smem_desc_sw128(k_s(0), 16, 1024);
+    const uint64_t v_desc0 = tc::smem_desc_sw128(v_s(0), kBN * 128, 1024);
+    // S_A and S_B of the key tile in stage kst into the next score buffer.
+    auto issue_s = [&](int kst) {
+      const int b = s_issued & 1;
       if (lane == 0) {
-        const int st = gi % S;
-        const uint32_t d_tmem = tmem + C::kSCol + (uint32_t)(t * kBN);
+        const uint64_t kd = k_desc0 + (uint64_t)((kst * C::kStageBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qoff = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-          const uint32_t koff = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-          tc::mma_ss(d_tmem, tc::smem_desc_sw128(q_s(t) + qoff, 16, 1024),
-                     tc::smem_desc_sw128(k_s(st) + koff, 16, 1024), idesc_qk, kk > 0);
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t d_tmem = tmem + s_col(t, b);
+          const uint64_t qd = q_desc0 + (uint64_t)((t * C::kQBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t qoff = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
+            const uint32_t koff = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
+            tc::mma_ss(d_tmem, qd + (qoff >> 4), kd + (koff >> 4), idesc_qk, kk > 0);
+          }
         }
-        tc::commit(smem_u32(&bars.s_full[t]));
+        tc::commit(smem_u32(&bars.s_full[b]));
       }
       __syncwarp();
-      ++s_issued[t];
+      ++s_issued;
     };
-    auto issue_pv = [&](int t, int gi, bool first) {
+    // O_t (+)= P_t V for both tiles, P_t in the first 32 columns of buffer b.
+    auto issue_pv = [&](int vst, int b, bool first) {
       if (lane == 0) {
-        const int st = gi % S;
-        const uint32_t d_tmem = tmem + C::kOCol + (uint32_t)(t * D);
-        const uint32_t a_tmem = tmem + C::kSCol + (uint32_t)(t * kBN);
+        const uint64_t vd = v_desc0 + (uint64_t)((vst * C::kStageBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          tc::mma_ts(d_tmem, a_tmem + kk * 8,
-                     tc::smem_desc_sw128(v_s(st) + kk * (16 * 128), kBN * 128, 1024), idesc_pv,
-                     (!first || kk > 0) ? 1u : 0u);
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t d_tmem = tmem + C::kOCol + (uint32_t)(t * D);
+          const uint32_t a_tmem = tmem + s_col(t, b);
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            tc::mma_ts(d_tmem, a_tmem + kk * 8, vd + (uint64_t)((kk * (16 * 128)) >> 4),
+                       idesc_pv, (!first || kk > 0) ? 1u : 0u);
+        }
       }
       __syncwarp();
     };
     auto commit_to = [&](uint64_t* bar) {
       if (lane == 0) tc::commit(smem_u32(bar));
       __syncwarp();
+    };
+    auto wait_stage = [&]() -> bool {
+      if (!warp_wait(&bars.kv_full[g_kv % S], (g_kv / S) & 1, abort, p.error_word)) return false;
+      ++g_kv;
+      return true;
     };
     for (int seq = 0; ok; ++seq) {
       const int slot = seq & 1;
@@ -476,78 +494,67 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (w < 0) break;
       Item it;
       if (!decode_item(p, w, n_qpairs, tpt, false, it) || it.n_tiles == 0) continue;
-      const int nq = it.has_b ? 2 : 1;
       const int n = it.n_tiles;
-      for (int t = 0; t < nq && ok; ++t) {
-        ok = warp_wait(&bars.q_full[t], q_seen[t] & 1, abort, p.error_word);
-        ++q_seen[t];
+      ok = warp_wait(&bars.q_full, q_seen & 1, abort, p.error_word);
+      ++q_seen;
+      // S(0), S(1)
+      for (int j = 0; ok && j < n && j < 2; ++j) {
+        const int kst = g_kv % S;
+        if (!wait_stage()) { ok = false; break; }
+        tc::fence_after_sync();
+        issue_s(kst);
+        if (j + 1 == n) commit_to(&bars.q_empty);  // last S of this item
       }
-      if (ok) ok = warp_wait(&bars.k_full[g % S], (g / S) & 1, abort, p.error_word);
-      if (!ok) break;
-      tc::fence_after_sync();
-      for (int t = 0; t < nq; ++t) issue_s(t, g);
-      commit_to(&bars.k_empty[g % S]);
-      if (n == 1)
-        for (int t = 0; t < nq; ++t) commit_to(&bars.q_empty[t]);
       for (int i = 0; ok && i < n; ++i) {
-        const int gi = g + i;
-        const int st = gi % S;
-        const bool last = i + 1 == n;
-        for (int t = 0; t < nq; ++t) {
-          // P_t(i) V_i
-          if (!warp_wait(&bars.p_full[t], p_seen[t] & 1, abort, p.error_word)) { ok = false; break; }
-          ++p_seen[t];
-          if (t == 0) {
-            if (!warp_wait(&bars.v_full[st], (gi / S) & 1, abort, p.error_word)) { ok = false; break; }
-            tc::fence_after_sync();
-            const int key0 = tile_of(it, i) * kBN;
-            if (key0 + kBN > it.k_len) {
-              // zero value rows at or past k_len
-              const int r0 = max(0, it.k_len - key0);
-              const int chunks = (kBN - r0) * C::kBoxes * 8;
-              for (int idx = lane; idx < chunks; idx += 32) {
-                const int ch = idx & 7;
-                const int rb = idx >> 3;
-                const int bx = rb % C::kBoxes;
-                const int r = r0 + rb / C::kBoxes;
-                uint8_t* dst =
-                    smem + C::kVOff + st * C::kKVBytes + bx * (kBN * 128) + r * 128 + ch * 16;
-                *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-              }
-              fence_proxy_async_smem();
-              __syncwarp();
-            }
+        const int vst = g_pv % S;
+        const int pb = g_pv & 1;
+        // P_A(i) and P_B(i) written
+        if (!warp_wait(&bars.p_full[pb], (g_pv >> 1) & 1, abort, p.error_word)) { ok = false; break; }
+        const int key0 = tile_of(it, i) * kBN;
+        if (key0 + kBN > it.k_len) {
+          // zero value rows at or past k_len (the stage was waited for with S(i))
+          const int r0 = max(0, it.k_len - key0);
+          const int chunks = (kBN - r0) * C::kBoxes * 8;
+          for (int idx = lane; idx < chunks; idx += 32) {
+            const int ch = idx & 7;
+            const int rb = idx >> 3;
+            const int bx = rb % C::kBoxes;
+            const int r = r0 + rb / C::kBoxes;
+            uint8_t* dst = smem + C::kKVOff + vst * C::kStageBytes + C::kKVBytes +
+                           bx * (kBN * 128) + r * 128 + ch * 16;
+            *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
           }
-          tc::fence_after_sync();
-          if (i == 0 && o_commits[t] > 0) {
-            // O_t of the previous item has been read by its epilogue.
-            if (!warp_wait(&bars.o_empty[t], (o_commits[t] - 1) & 1, abort, p.error_word)) {
-              ok = false;
-              break;
-            }
-            tc::fence_after_sync();
-          }
-          issue_pv(t, gi, i == 0);
-          if (last) {
-            commit_to(&bars.o_final[t]);
-            ++o_commits[t];
-          } else {
-            // S_t(i+1) overwrites the columns P_t(i) lives in; the MMAs run in
-            // issue order, so P_t(i) V_i has read them by then.
-            if (t == 0) {
-              if (!warp_wait(&bars.k_full[(gi + 1) % S], ((gi + 1) / S) & 1, abort,
-                             p.error_word)) { ok = false; break; }
-              tc::fence_after_sync();
-            }
-            issue_s(t, gi + 1);
-            if (i + 2 == n) commit_to(&bars.q_empty[t]);  // last S_t of this item
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (i == 0 && o_commits > 0) {
+          // O of the previous item has been read by its epilogue.
+          if (!warp_wait(&bars.o_empty, (o_commits - 1) & 1, abort, p.error_word)) {
+            ok = false;
+            break;
           }
         }
-        if (!ok) break;
-        commit_to(&bars.v_empty[st]);
-        if (!last) commit_to(&bars.k_empty[(gi + 1) % S]);
+        int kst = -1;
+        if (i + 2 < n) {
+          kst = g_kv % S;
+          if (!wait_stage()) { ok = false; break; }
+        }
+        tc::fence_after_sync();
+        issue_pv(vst, pb, i == 0);
+        ++g_pv;
+        if (i + 2 == n) commit_to(&bars.pv_item[0]);  // P(n-2) V done: last-tile rescales
+        if (i + 1 == n) {
+          commit_to(&bars.o_final);
+          ++o_commits;
+        }
+        commit_to(&bars.kv_empty[vst]);
+        if (kst >= 0) {
+          // S(i+2) overwrites the buffer P(i) lives in; the MMAs run in issue
+          // order, so P(i) V_i has read it by then.
+          issue_s(kst);
+          if (i + 3 == n) commit_to(&bars.q_empty);  // last S of this item
+        }
       }
-      if (ok) g += n;
     }
     if (!ok) do_abort(abort, p.error_word);
     // Drain: every MMA issued above has completed before TMEM is freed.
@@ -563,10 +570,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qw = warp & 3;             // TMEM lane quarter of this warp
     const int r = qw * 32 + lane;        // row of this thread
     const uint32_t lane_base = (uint32_t)(qw * 32) << 16;
-    const uint32_t s_col = tmem + lane_base + C::kSCol + (uint32_t)(t * kBN);
     const uint32_t o_col = tmem + lane_base + C::kOCol + (uint32_t)(t * D);
     const float sl2 = p.scale_log2;
-    int s_seen = 0, o_seen = 0;
+    int s_seen = 0;      // score tiles consumed over all items
+    int o_seen = 0;      // items with keys consumed
+    int pv_items = 0;    // items with two or more key tiles consumed
     bool ok = true;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
     for (int seq = 0; ok; ++seq) {
@@ -581,7 +589,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (w < 0) break;
       Item it;
       if (!decode_item(p, w, n_qpairs, tpt, false, it)) continue;
-      if (t == 1 && !it.has_b) continue;
       const int tok = it.t_begin + t * tpt + r / G;
       const bool row_ok = r < rows_used && tok < it.q_len;
       const int pos = tok + it.k_len - it.q_len;
@@ -595,11 +602,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr bool kSinks = decltype(with_sinks)::value;
         float v[kBN];
         for (int i = 0; i < n; ++i) {
-          if (!warp_wait(&bars.s_full[t], s_seen & 1, abort, p.error_word)) { ok = false; break; }
-          ++s_seen;
+          const int b = s_seen & 1;
+          if (!warp_wait(&bars.s_full[b], (s_seen >> 1) & 1, abort, p.error_word)) {
+            ok = false;
+            break;
+          }
+          const int gt = s_seen++;  // this tile's index over all items
           tc::fence_after_sync();
+          const uint32_t sc = tmem + lane_base + s_col(t, b);
 #pragma unroll
-          for (int c = 0; c < kBN / 32; ++c) tc::tmem_ld32(s_col + c * 32, v + c * 32);
+          for (int c = 0; c < kBN / 32; ++c) tc::tmem_ld32(sc + c * 32, v + c * 32);
           tc::tmem_wait_ld();
           const int key0 = tile_of(it, i) * kBN;
           if constexpr (!kSinks) {
@@ -640,8 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
           mx *= sl2;  // scale > 0: max of the scaled scores
           // Running max: taken at once while empty, else only when it grows by
-          // more than the threshold (then O and l are rescaled). O_t holds
-          // P_t(i-1) V_{i-1} here: S_t(i) was issued after it and has completed.
+          // more than the threshold (then O and l are rescaled).
           float alpha = 1.f;
           bool rescale = false;
           if (m == -INFINITY) {
@@ -654,26 +665,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= alpha;
           const float neg_m = m == -INFINITY ? 0.f : -m;  // an empty row keeps P = 0
           float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
-          // P in two halves of 64 keys (32 packed columns each) to bound registers.
+          uint32_t pk[kBN / 2];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t pk[32];
-#pragma unroll
-            for (int c = 0; c < 64; c += 2) {
-              float x0, x1;
-              fma2(x0, x1, v[h * 64 + c], v[h * 64 + c + 1], sl2, neg_m);
-              const float w0 = fast_exp2(x0);
-              const float w1 = fast_exp2(x1);
-              const int k = (c >> 1) & 3;
-              add2(rs[2 * k], rs[2 * k + 1], w0, w1);
-              pk[c >> 1] = pack_bf16x2(w0, w1);
-            }
-            tc::tmem_st32(s_col + h * 32, reinterpret_cast<const float*>(pk));
+          for (int c = 0; c < kBN; c += 2) {
+            float x0, x1;
+            fma2(x0, x1, v[c], v[c + 1], sl2, neg_m);
+            const float w0 = fast_exp2(x0);
+            const float w1 = fast_exp2(x1);
+            const int k = (c >> 1) & 3;
+            add2(rs[2 * k], rs[2 * k + 1], w0, w1);
+            pk[c >> 1] = pack_bf16x2(w0, w1);
           }
+          tc::tmem_st32(sc, reinterpret_cast<const float*>(pk));
           l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
-          // Rescale O_t (after P, so that the scores are dead): it must finish
-          // before P_t(i) V_i is issued, i.e. before p_full.
+          // Rescale O_t after P(i-1) V_{i-1} has completed and before P(i) V_i
+          // is issued (before p_full): proven by S(i+1), or for the item's
+          // last tile by the per-item barrier (see the header).
           if (i > 0 && __any_sync(0xffffffffu, rescale)) {
+            const bool waited =
+                i + 1 < n
+                    ? warp_wait(&bars.s_full[(gt + 1) & 1], ((gt + 1) >> 1) & 1, abort,
+                                p.error_word)
+                    : warp_wait(&bars.pv_item[0], pv_items & 1, abort, p.error_word);
+            if (!waited) {
+              ok = false;
+              break;
+            }
+            tc::fence_after_sync();
             float o[32];
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
@@ -687,16 +705,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tmem_wait_st();
           tc::fence_before_sync();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bars.p_full[t]);
+          if (lane == 0) mbar_arrive(&bars.p_full[b]);
         }
       };
       if (p.sinks > 0) tile_loop(std::true_type{});
       else tile_loop(std::false_type{});
       if (!ok) break;
+      if (n >= 2) ++pv_items;
       // ---------------------------------------------------------- epilogue
       const bool have_o = n > 0;
       if (have_o) {
-        if (!warp_wait(&bars.o_final[t], o_seen & 1, abort, p.error_word)) { ok = false; break; }
+        if (!warp_wait(&bars.o_final, o_seen & 1, abort, p.error_word)) { ok = false; break; }
         ++o_seen;
         tc::fence_after_sync();
       }
@@ -712,10 +731,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tmem_ld32(o_col + c * 32, o);
           tc::tmem_wait_ld();
           if (c + 1 == D / 32) {
-            // O_t may now be overwritten by the next item's first P V.
+            // O may now be overwritten by the next item's first P V.
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.o_empty[t]);
+            if (lane == 0) mbar_arrive(&bars.o_empty);
           }
         }
         if (row_ok) {

@@ -260,7 +260,7 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
     if (!workspace || workspace_bytes < rpk::kPrefillWorkspaceBytes) return RPK_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return RPK_ERR_WORKSPACE;
     CUtensorMap q_map, k_map, v_map;
-    const int32_t box_rows = p.P < 128 ? p.P : 128;
+    const int32_t box_rows = p.P < rpk::kPrefillKeyTile ? p.P : rpk::kPrefillKeyTile;
     const int64_t pool_rows = (int64_t)p.num_pages * p.P;
     st = encode_rows_map(&q_map, q, head_dim, n_heads, total_q_tokens, p.G, tpt);
     if (st != RPK_OK) return st;
