@@ -186,6 +186,28 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
+// Bounded wait for two barriers at once (the second only when `need_b`): the
+// two try_waits are issued back to back, so a warp that finds both phases
+// complete pays one barrier round trip, not two.
+__device__ __forceinline__ bool warp_wait2(uint64_t* bar_a, uint32_t par_a, uint64_t* bar_b,
+                                           uint32_t par_b, bool need_b, volatile int* abort,
+                                           const int32_t* error_word) {
+  uint32_t ok_a, ok_b;
+  asm volatile(
+      "{\n\t.reg .pred pa, pb;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 pa, [%2], %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 pb, [%4], %5;\n\t"
+      "selp.u32 %0, 1, 0, pa;\n\t"
+      "selp.u32 %1, 1, 0, pb;\n\t}"
+      : "=r"(ok_a), "=r"(ok_b)
+      : "r"(smem_u32(bar_a)), "r"(par_a), "r"(smem_u32(need_b ? bar_b : bar_a)),
+        "r"(need_b ? par_b : par_a)
+      : "memory");
+  bool ok = (ok_a != 0 || thread_wait(bar_a, par_a, abort, error_word)) &&
+            (!need_b || ok_b != 0 || thread_wait(bar_b, par_b, abort, error_word));
+  return __all_sync(0xffffffffu, ok);
+}
+
 __device__ __forceinline__ void do_abort(volatile int* abort, int32_t* error_word) {
   if (!*abort) {
     *abort = 1;
@@ -430,26 +452,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     int s_issued = 0;    // S tile pairs issued (buffer = count mod 2)
     int o_commits = 0;   // o_final commits
     bool ok = true;
-    // Shared-memory descriptors: the start address is the low field
-    // (address >> 4, 14 bits; every operand lies below 256 KB), so a
-    // descriptor at an offset is the base descriptor plus offset >> 4.
+    // Shared-memory descriptors: the start address is the low field of the
+    // low word (address >> 4, 14 bits; every operand lies below 256 KB), so
+    // the descriptor of an operand at an offset is the base low word plus
+    // offset >> 4; the high word (stride offset, swizzle) is common.
     const uint64_t q_desc0 = tc::smem_desc_sw128(q_s(0), 16, 1024);
-    const uint64_t k_desc0 = tc::smem_desc_sw128(k_s(0), 16, 1024);
-    const uint64_t v_desc0 = tc::smem_desc_sw128(v_s(0), kBN * 128, 1024);
+    const uint32_t q_lo0 = (uint32_t)q_desc0;
+    const uint32_t k_lo0 = (uint32_t)tc::smem_desc_sw128(k_s(0), 16, 1024);
+    const uint32_t v_lo0 = (uint32_t)tc::smem_desc_sw128(v_s(0), kBN * 128, 1024);
+    const uint32_t desc_hi = (uint32_t)(q_desc0 >> 32);
     // S_A and S_B of the key tile in stage kst into the next score buffer.
     auto issue_s = [&](int kst) {
       const int b = s_issued & 1;
       if (lane == 0) {
-        const uint64_t kd = k_desc0 + (uint64_t)((kst * C::kStageBytes) >> 4);
+        const uint32_t kd = k_lo0 + (uint32_t)((kst * C::kStageBytes) >> 4);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           const uint32_t d_tmem = tmem + s_col(t, b);
-          const uint64_t qd = q_desc0 + (uint64_t)((t * C::kQBytes) >> 4);
+          const uint32_t qd = q_lo0 + (uint32_t)((t * C::kQBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t qoff = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
             const uint32_t koff = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-            tc::mma_ss(d_tmem, qd + (qoff >> 4), kd + (koff >> 4), idesc_qk, kk > 0);
+            tc::mma_ss_lo(d_tmem, qd + (qoff >> 4), kd + (koff >> 4), desc_hi, idesc_qk, kk > 0);
           }
         }
         tc::commit(smem_u32(&bars.s_full[b]));
@@ -460,15 +485,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // O_t (+)= P_t V for both tiles, P_t in the first 32 columns of buffer b.
     auto issue_pv = [&](int vst, int b, bool first) {
       if (lane == 0) {
-        const uint64_t vd = v_desc0 + (uint64_t)((vst * C::kStageBytes) >> 4);
+        const uint32_t vd = v_lo0 + (uint32_t)((vst * C::kStageBytes) >> 4);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           const uint32_t d_tmem = tmem + C::kOCol + (uint32_t)(t * D);
           const uint32_t a_tmem = tmem + s_col(t, b);
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
-            tc::mma_ts(d_tmem, a_tmem + kk * 8, vd + (uint64_t)((kk * (16 * 128)) >> 4),
-                       idesc_pv, (!first || kk > 0) ? 1u : 0u);
+            tc::mma_ts_lo(d_tmem, a_tmem + kk * 8, vd + (uint32_t)((kk * (16 * 128)) >> 4),
+                          desc_hi, idesc_pv, (!first || kk > 0) ? 1u : 0u);
         }
       }
       __syncwarp();
@@ -508,8 +533,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; ok && i < n; ++i) {
         const int vst = g_pv % S;
         const int pb = g_pv & 1;
-        // P_A(i) and P_B(i) written
-        if (!warp_wait(&bars.p_full[pb], (g_pv >> 1) & 1, abort, p.error_word)) { ok = false; break; }
+        // P_A(i) and P_B(i) written, and the stage of key tile i+2 (for S(i+2)) loaded
+        const bool more_s = i + 2 < n;
+        const int kst = more_s ? g_kv % S : -1;
+        if (!warp_wait2(&bars.p_full[pb], (g_pv >> 1) & 1, &bars.kv_full[g_kv % S],
+                        (g_kv / S) & 1, more_s, abort, p.error_word)) {
+          ok = false;
+          break;
+        }
+        if (more_s) ++g_kv;
         const int key0 = tile_of(it, i) * kBN;
         if (key0 + kBN > it.k_len) {
           // zero value rows at or past k_len (the stage was waited for with S(i))
@@ -533,11 +565,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-        }
-        int kst = -1;
-        if (i + 2 < n) {
-          kst = g_kv % S;
-          if (!wait_stage()) { ok = false; break; }
         }
         tc::fence_after_sync();
         issue_pv(vst, pb, i == 0);
