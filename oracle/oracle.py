@@ -14,7 +14,7 @@ import numpy as np
 
 from . import build as _build
 
-F32, BF16 = 0, 1
+F32, BF16, E4M3 = 0, 1, 2
 
 _lib = None
 
@@ -61,6 +61,17 @@ def _declare(L):
                                  _i32, _i32, _p, _i32, C.c_double, _i32, _i32, _p, _i64, _p,
                                  _p, C.c_int]
     L.rpko_attention.restype = C.c_int
+    L.rpko_e4m3_to_f64.argtypes = [C.c_uint8]
+    L.rpko_e4m3_to_f64.restype = C.c_double
+    L.rpko_f64_to_e4m3.argtypes = [C.c_double]
+    L.rpko_f64_to_e4m3.restype = C.c_uint8
+    L.rpko_cache_image_e4m3.argtypes = [_p, _p, C.c_int, _i32, _i32, _i32, _p, _i32, _p, _p,
+                                        _i32, _i32, _i32, _p, _p, _p, _p]
+    L.rpko_cache_image_e4m3.restype = C.c_int
+    L.rpko_attention_cache.argtypes = [_p, C.c_int, _p, _p, _i32, _i32, _i32, _i32, _i32, _p,
+                                       _p, C.c_int, _p, _p, _i32, _i32, _p, _i32, C.c_double,
+                                       _i32, _i32, _p, _i64, _p, _p, C.c_int]
+    L.rpko_attention_cache.restype = C.c_int
     L.rpko_flash_step.argtypes = [C.POINTER(C.c_double)] * 3 + [C.c_double, C.c_double]
     L.rpko_flash_step.restype = None
 
@@ -75,6 +86,8 @@ def _raw(x):
                 return x.view(torch.int16).numpy().view(np.uint16), BF16
             if x.dtype == torch.float32:
                 return x.numpy(), F32
+            if x.dtype == torch.float8_e4m3fn:
+                return x.view(torch.uint8).numpy(), E4M3
             raise TypeError(f"unsupported dtype {x.dtype}")
     except ImportError:  # pragma: no cover
         pass
@@ -83,6 +96,8 @@ def _raw(x):
         return x, F32
     if x.dtype == np.uint16:
         return x, BF16
+    if x.dtype == np.uint8:
+        return x, E4M3
     raise TypeError(f"unsupported dtype {x.dtype}")
 
 
@@ -100,6 +115,15 @@ def bf16_bits_to_f64(bits: int) -> float:
 
 def f64_to_bf16_bits(x: float) -> int:
     return int(lib().rpko_f64_to_bf16(float(x)))
+
+
+def e4m3_to_f64(code: int) -> float:
+    return lib().rpko_e4m3_to_f64(int(code))
+
+
+def f64_to_e4m3(x: float) -> int:
+    """One rounding to nearest, ties to even; beyond +-448 saturates."""
+    return int(lib().rpko_f64_to_e4m3(float(x)))
 
 
 def round_to(x: np.ndarray, dtype: int) -> np.ndarray:
@@ -159,24 +183,36 @@ def rope(x, row_offsets, cache_lens, position_ids, mrope_section, table, interle
 
 
 def cache_image(k_rot: np.ndarray, v_new, row_offsets, cache_lens, block_table, k_pages,
-                v_pages, inplace: bool = False):
+                v_pages, inplace: bool = False, k_scale=None, v_scale=None):
     """Return (k_pages', v_pages') raw arrays with the new tokens written in.
 
     k_rot is fp64 [T, n_kv_heads, d]; v_new, k_pages and v_pages are tensors or
-    raw arrays of the cache dtype. The inputs are copied first unless inplace
-    is set, in which case k_pages / v_pages must be raw numpy arrays and are
-    written directly.
+    raw arrays of the cache dtype, or, for an e4m3 cache (uint8 / float8_e4m3fn
+    pools), v_new of q's dtype and k_scale / v_scale the per-KV-head fp32
+    scales. The inputs are copied first unless inplace is set, in which case
+    k_pages / v_pages must be raw numpy arrays and are written directly.
     """
     vraw, code = _raw(v_new)
     kp, kcode = _raw(k_pages)
     vp, vcode = _raw(v_pages)
-    assert code == kcode == vcode
     if not inplace:
         kp, vp = kp.copy(), vp.copy()
     k_rot = np.ascontiguousarray(k_rot, dtype=np.float64)
     T, hk, d = k_rot.shape
     offs = _i32arr(row_offsets)
     bt = _i32arr(block_table)
+    if kcode == E4M3:
+        assert vcode == E4M3 and k_scale is not None and v_scale is not None
+        ks = np.ascontiguousarray(k_scale, dtype=np.float32)
+        vs = np.ascontiguousarray(v_scale, dtype=np.float32)
+        rc = lib().rpko_cache_image_e4m3(_ptr(k_rot), _ptr(vraw), code, T, hk, d, _ptr(offs),
+                                         len(offs) - 1, _ptr(_i32arr(cache_lens)), _ptr(bt),
+                                         bt.shape[1], kp.shape[0], kp.shape[1], _ptr(ks),
+                                         _ptr(vs), _ptr(kp), _ptr(vp))
+        if rc:
+            raise ValueError(f"rpko_cache_image_e4m3 failed ({rc})")
+        return kp, vp
+    assert code == kcode == vcode
     rc = lib().rpko_cache_image(_ptr(k_rot), _ptr(vraw), code, T, hk, d, _ptr(offs),
                                 len(offs) - 1, _ptr(_i32arr(cache_lens)), _ptr(bt), bt.shape[1],
                                 kp.shape[0], kp.shape[1], _ptr(kp), _ptr(vp))
@@ -199,7 +235,7 @@ def band(r: int, q_len: int, k_len: int, window: int) -> tuple[int, int]:
 
 def attention(q, q_offsets, kv_lens, k_pages, v_pages, block_table, n_kv_heads, scale,
               window, rows=None, n_threads: int | None = None, with_lse: bool = False,
-              sinks: int = 0):
+              sinks: int = 0, k_scale=None, v_scale=None):
     """fp64 attention rows.
 
     rows=None: all rows, shape [T, n_heads, head_dim]. Otherwise rows is an
@@ -207,11 +243,15 @@ def attention(q, q_offsets, kv_lens, k_pages, v_pages, block_table, n_kv_heads, 
     with_lse: return (out, lse), lse the natural log-sum-exp of each row's
     scores ([T, n_heads] or [n]; -inf for a row that sees no key).
     sinks: under a window, the first `sinks` keys stay visible (StreamingLLM).
+    k_scale, v_scale: per-KV-head fp32 scales of an e4m3 cache (uint8 /
+    float8_e4m3fn pools): key = code * k_scale[kvh], value = code * v_scale[kvh].
     """
     qraw, code = _raw(q)
     kp, kcode = _raw(k_pages)
     vp, vcode = _raw(v_pages)
-    assert code == kcode == vcode
+    assert kcode == vcode and (kcode == code or kcode == E4M3)
+    ks = None if k_scale is None else np.ascontiguousarray(k_scale, dtype=np.float32)
+    vs = None if v_scale is None else np.ascontiguousarray(v_scale, dtype=np.float32)
     T, H, d = qraw.shape
     offs = _i32arr(q_offsets)
     kvl = _i32arr(kv_lens)
@@ -227,13 +267,13 @@ def attention(q, q_offsets, kv_lens, k_pages, v_pages, block_table, n_kv_heads, 
         out = np.empty((rows.shape[0], d), dtype=np.float64)
         lse = np.empty(rows.shape[0], dtype=np.float64) if with_lse else None
         rptr, n = _ptr(rows), rows.shape[0]
-    rc = lib().rpko_attention(_ptr(qraw), code, _ptr(offs), _ptr(kvl), len(offs) - 1, T, H,
-                              int(n_kv_heads), d, _ptr(kp), _ptr(vp), kp.shape[1], kp.shape[0],
-                              _ptr(bt), bt.shape[1], float(scale), int(window), int(sinks),
-                              rptr, n,
-                              _ptr(out), None if lse is None else _ptr(lse), int(n_threads))
+    rc = lib().rpko_attention_cache(_ptr(qraw), code, _ptr(offs), _ptr(kvl), len(offs) - 1, T,
+                                    H, int(n_kv_heads), d, _ptr(kp), _ptr(vp), kcode, _ptr(ks),
+                                    _ptr(vs), kp.shape[1], kp.shape[0], _ptr(bt), bt.shape[1],
+                                    float(scale), int(window), int(sinks), rptr, n, _ptr(out),
+                                    None if lse is None else _ptr(lse), int(n_threads))
     if rc:
-        raise ValueError(f"rpko_attention failed ({rc})")
+        raise ValueError(f"rpko_attention_cache failed ({rc})")
     return (out, lse) if with_lse else out
 
 

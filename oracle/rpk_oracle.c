@@ -26,7 +26,11 @@
  *    r of q rows over k keys sits at position r + k - q, sees keys_before keys
  *    before it and keys_after after; rows that see no key are zeros.
  *  - NumKong "NumKong for Python" (conversion policy): narrowing rounds to
- *    nearest, ties to even.
+ *    nearest, ties to even; (low-precision scalar types): e4m3 is 1 sign,
+ *    4 exponent and 3 mantissa bits, range +-448, no infinity, with NaN.
+ *  - Mojo "generic_fused_qk_rope_bshd_paged_ragged_kernel_api" (Parameters:
+ *    cache_dtype; Args: kv_collection with a scale dtype and a quantization
+ *    granularity): the cache may hold a narrower type than q with scales.
  *
  * Readings where the pages are silent (the same list is kept in the design
  * notes): freqs_cis is fp32 [max_position, rotary_dim] with (cos, sin) per
@@ -34,7 +38,10 @@
  * multiplication by e^{i theta}: (a, b) -> (a cos - b sin, b cos + a sin);
  * M-RoPE sections count rotary pairs and pair j takes its section's position;
  * a window w > 0 means w keys including the row's own (keys_before = w - 1);
- * masked keys are left out of the softmax (not given -1e9).
+ * masked keys are left out of the softmax (not given -1e9); an e4m3 cache
+ * holds code = e4m3(x / scale) with one fp32 scale per KV head for K and one
+ * for V (stored value = code * scale), values beyond the largest finite
+ * saturating to +-448.
  */
 #include <math.h>
 #include <pthread.h>
@@ -44,6 +51,7 @@
 
 #define RPKO_F32 0
 #define RPKO_BF16 1
+#define RPKO_E4M3 2
 
 #define RPKO_OK 0
 #define RPKO_ERR_ARG 1
@@ -84,6 +92,43 @@ uint16_t rpko_f64_to_bf16(double x) {
   uint32_t u;
   memcpy(&u, &f, sizeof u);
   return sign | (uint16_t)(u >> 16);
+}
+
+/* e4m3 code -> fp64. The code is 1 sign bit, a 4-bit exponent with bias 7
+ * and a 3-bit mantissa (E4M3 without infinities): exponent 0 holds the
+ * subnormals m * 2^-9, exponent 15 with mantissa 7 is NaN, so the largest
+ * finite value is 1.75 * 2^8 = 448. */
+double rpko_e4m3_to_f64(uint8_t c) {
+  int e = (c >> 3) & 15, m = c & 7;
+  if (e == 15 && m == 7) return NAN;
+  double v = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+  return (c & 0x80) ? -v : v;
+}
+
+/* fp64 -> e4m3 code, one rounding to nearest with ties to even. Magnitudes
+ * from 448 up (including infinities) saturate to +-448: a value between 448
+ * and 464 rounds to 448, 464 is a tie that goes to the even 448, and
+ * anything larger has no finite code. NaN stays NaN. The value is scaled so
+ * that one unit in the last place at its binade (2^-9 below the normals) is
+ * 1, rounded with rint and scaled back, as for bf16. */
+uint8_t rpko_f64_to_e4m3(double x) {
+  if (isnan(x)) return 0x7F;
+  uint8_t sign = signbit(x) ? 0x80 : 0;
+  double a = fabs(x);
+  if (a >= 448.0) return sign | 0x7E;
+  if (a == 0.0) return sign;
+  int e2;
+  frexp(a, &e2);
+  int lead = e2 - 1;             /* a in [2^lead, 2^(lead+1)) */
+  if (lead < -6) lead = -6;      /* below the normals: fixed spacing 2^-9 */
+  double ulp = ldexp(1.0, lead - 3);
+  double units = rint(a / ulp);  /* whole units in the last place, ties to even */
+  double r = units * ulp;
+  if (r < ldexp(1.0, -6)) return sign | (uint8_t)(r * 512.0);  /* subnormal code m */
+  double mant = frexp(r, &e2);   /* r = mant * 2^e2, mant in [0.5, 1) */
+  int E = e2 - 1 + 7;            /* biased exponent, 1 .. 15 */
+  int M = (int)((mant * 2.0 - 1.0) * 8.0);  /* exact: r has at most 4 significant bits */
+  return sign | (uint8_t)((E << 3) | M);
 }
 
 /* fp64 -> fp32 with one rounding to nearest, ties to even (C conversion). */
@@ -270,6 +315,41 @@ int rpko_cache_image(const double* k_rot, const void* v_new, int dtype, int32_t 
   return RPKO_OK;
 }
 
+/*
+ * The same write into an e4m3 cache: K code = e4m3(k_rot / k_scale[kvh]) and
+ * V code = e4m3(v / v_scale[kvh]), v widened exactly from dtype (bf16 or
+ * fp32), each quotient formed in fp64 and rounded once.
+ */
+int rpko_cache_image_e4m3(const double* k_rot, const void* v_new, int dtype, int32_t T,
+                          int32_t n_kv_heads, int32_t head_dim, const int32_t* row_offsets,
+                          int32_t batch, const int32_t* cache_lens, const int32_t* block_table,
+                          int32_t max_pages_per_seq, int32_t num_pages, int32_t page_size,
+                          const float* k_scale, const float* v_scale, uint8_t* k_pages,
+                          uint8_t* v_pages) {
+  if (!k_rot || !v_new || !row_offsets || !cache_lens || !block_table || !k_pages || !v_pages ||
+      !k_scale || !v_scale)
+    return RPKO_ERR_ARG;
+  for (int32_t t = 0; t < T; ++t) {
+    int b = owner_of(row_offsets, batch, t);
+    if (b < 0) return RPKO_ERR_ARG;
+    int32_t slot = cache_lens[b] + (t - row_offsets[b]);
+    int32_t pi = slot / page_size;
+    if (pi >= max_pages_per_seq) return RPKO_ERR_PAGE;
+    int32_t page = block_table[(size_t)b * max_pages_per_seq + pi];
+    if (page < 0 || page >= num_pages) return RPKO_ERR_PAGE;
+    int32_t row = slot % page_size;
+    for (int32_t kh = 0; kh < n_kv_heads; ++kh) {
+      size_t src = ((size_t)t * n_kv_heads + kh) * head_dim;
+      size_t dst = (((size_t)page * page_size + row) * n_kv_heads + kh) * head_dim;
+      for (int32_t c = 0; c < head_dim; ++c) {
+        k_pages[dst + c] = rpko_f64_to_e4m3(k_rot[src + c] / (double)k_scale[kh]);
+        v_pages[dst + c] = rpko_f64_to_e4m3(load_elt(v_new, dtype, src + c) / (double)v_scale[kh]);
+      }
+    }
+  }
+  return RPKO_OK;
+}
+
 /* ------------------------------------------------------------- attention */
 
 /* Visible key range of row r of a sequence with q_len rows and k_len keys:
@@ -306,6 +386,9 @@ typedef struct {
   int32_t batch, T, n_heads, n_kv_heads, head_dim;
   const void* k_pages;
   const void* v_pages;
+  int cache_dtype;        /* dtype of the pools: q's dtype, or RPKO_E4M3 with scales */
+  const float* k_scale;   /* [n_kv_heads] for RPKO_E4M3 */
+  const float* v_scale;
   int32_t page_size, num_pages, max_pages_per_seq;
   const int32_t* block_table;
   double scale;
@@ -328,6 +411,14 @@ typedef struct {
  * With lse != NULL also its natural log-sum-exp of the scores, ln sum_j e^{s_j}
  * = m + ln sum_j e^{s_j - m} (NumKong attention_packed's log_sum_exp output);
  * -inf for a row that sees no key (an empty sum). */
+/* Element idx of a pool of KV head kvh as the key or value it stands for. */
+static double load_cache(const attn_job* J, const void* pool, const float* scale, int kvh,
+                         size_t idx) {
+  if (J->cache_dtype == RPKO_E4M3)
+    return rpko_e4m3_to_f64(((const uint8_t*)pool)[idx]) * (double)scale[kvh];
+  return load_elt(pool, J->cache_dtype, idx);
+}
+
 static int attention_row(const attn_job* J, int32_t t, int32_t h, double* o, double* w,
                          double* lse) {
   int d = J->head_dim;
@@ -357,7 +448,8 @@ static int attention_row(const attn_job* J, int32_t t, int32_t h, double* o, dou
     size_t kbase = (((size_t)page * J->page_size + j % J->page_size) * J->n_kv_heads + kvh) * d;
     double acc = 0.0;
     for (int c = 0; c < d; ++c)
-      acc += load_elt(J->q, J->dtype, qbase + c) * load_elt(J->k_pages, J->dtype, kbase + c);
+      acc += load_elt(J->q, J->dtype, qbase + c) * load_cache(J, J->k_pages, J->k_scale, kvh,
+                                                              kbase + c);
     double s = J->scale * acc;
     w[n++] = s;
     if (s > m) m = s;
@@ -376,7 +468,7 @@ static int attention_row(const attn_job* J, int32_t t, int32_t h, double* o, dou
     double wj = w[i++] / den;
     int32_t page = J->block_table[(size_t)b * J->max_pages_per_seq + j / J->page_size];
     size_t vbase = (((size_t)page * J->page_size + j % J->page_size) * J->n_kv_heads + kvh) * d;
-    for (int c = 0; c < d; ++c) o[c] += wj * load_elt(J->v_pages, J->dtype, vbase + c);
+    for (int c = 0; c < d; ++c) o[c] += wj * load_cache(J, J->v_pages, J->v_scale, kvh, vbase + c);
   }
   return RPKO_OK;
 }
@@ -413,21 +505,27 @@ static void* attention_worker(void* arg) {
  * q_len (rpko_band). Output fp64, one row of head_dim per requested (t, h),
  * in the order given (rows == NULL: all T * n_heads rows, t-major), and, when
  * lse != NULL, each row's natural log-sum-exp of its scores (-inf when empty).
+ * The pools hold q's dtype, or (cache_dtype RPKO_E4M3) e4m3 codes whose key
+ * or value is code * k_scale[kvh] or code * v_scale[kvh], formed in fp64.
  * n_threads > 1 splits the rows over POSIX threads.
  */
-int rpko_attention(const void* q, int dtype, const int32_t* q_offsets, const int32_t* kv_lens,
-                   int32_t batch, int32_t T, int32_t n_heads, int32_t n_kv_heads,
-                   int32_t head_dim, const void* k_pages, const void* v_pages,
-                   int32_t page_size, int32_t num_pages, const int32_t* block_table,
-                   int32_t max_pages_per_seq, double scale, int32_t window, int32_t sinks,
-                   const int32_t* rows, int64_t n_rows, double* out, double* lse,
-                   int n_threads) {
+int rpko_attention_cache(const void* q, int dtype, const int32_t* q_offsets,
+                         const int32_t* kv_lens, int32_t batch, int32_t T, int32_t n_heads,
+                         int32_t n_kv_heads, int32_t head_dim, const void* k_pages,
+                         const void* v_pages, int cache_dtype, const float* k_scale,
+                         const float* v_scale, int32_t page_size, int32_t num_pages,
+                         const int32_t* block_table, int32_t max_pages_per_seq, double scale,
+                         int32_t window, int32_t sinks, const int32_t* rows, int64_t n_rows,
+                         double* out, double* lse, int n_threads) {
   if (!q || !q_offsets || !kv_lens || !k_pages || !v_pages || !block_table || !out)
     return RPKO_ERR_ARG;
   if (n_kv_heads <= 0 || n_heads % n_kv_heads != 0 || head_dim <= 0 || page_size <= 0)
     return RPKO_ERR_ARG;
+  if (cache_dtype != dtype && !(cache_dtype == RPKO_E4M3 && k_scale && v_scale))
+    return RPKO_ERR_ARG;
   attn_job J = {q, dtype, q_offsets, kv_lens, batch, T, n_heads, n_kv_heads, head_dim,
-                k_pages, v_pages, page_size, num_pages, max_pages_per_seq, block_table,
+                k_pages, v_pages, cache_dtype, k_scale, v_scale, page_size, num_pages,
+                max_pages_per_seq, block_table,
                 scale, window, sinks, rows, rows ? n_rows : (int64_t)T * n_heads, out, lse, RPKO_OK};
   if (n_threads < 1) n_threads = 1;
   if (n_threads > 256) n_threads = 256;
@@ -450,6 +548,20 @@ int rpko_attention(const void* q, int dtype, const int32_t* q_offsets, const int
   for (int i = 0; i < n_threads; ++i)
     if (slices[i].status != RPKO_OK) return slices[i].status;
   return RPKO_OK;
+}
+
+/* rpko_attention_cache with the pools in q's dtype. */
+int rpko_attention(const void* q, int dtype, const int32_t* q_offsets, const int32_t* kv_lens,
+                   int32_t batch, int32_t T, int32_t n_heads, int32_t n_kv_heads,
+                   int32_t head_dim, const void* k_pages, const void* v_pages,
+                   int32_t page_size, int32_t num_pages, const int32_t* block_table,
+                   int32_t max_pages_per_seq, double scale, int32_t window, int32_t sinks,
+                   const int32_t* rows, int64_t n_rows, double* out, double* lse,
+                   int n_threads) {
+  return rpko_attention_cache(q, dtype, q_offsets, kv_lens, batch, T, n_heads, n_kv_heads,
+                              head_dim, k_pages, v_pages, dtype, NULL, NULL, page_size,
+                              num_pages, block_table, max_pages_per_seq, scale, window, sinks,
+                              rows, n_rows, out, lse, n_threads);
 }
 
 /* ------------------------------------------------- online-softmax state */

@@ -45,6 +45,14 @@ MUTATIONS = {
     "p_rope_tail_rotated": ("      if (j < rotated_pairs) {", "      if (j <= rotated_pairs) {"),
     "lse_log_base": ("if (lse) *lse = m + log(den);", "if (lse) *lse = m + log2(den);"),
     "lse_max_dropped": ("if (lse) *lse = m + log(den);", "if (lse) *lse = log(den);"),
+    "e4m3_exponent_bias": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
+    "e4m3_ties_away": ("double units = rint(a / ulp);", "double units = floor(a / ulp + 0.5);"),
+    "e4m3_no_saturation": ("if (a >= 448.0) return sign | 0x7E;",
+                           "if (a >= 480.0) return sign | 0x7E;"),
+    "e4m3_key_scale_multiplied": ("rpko_f64_to_e4m3(k_rot[src + c] / (double)k_scale[kh]);",
+                                  "rpko_f64_to_e4m3(k_rot[src + c] * (double)k_scale[kh]);"),
+    "e4m3_read_scale_dropped": ("return rpko_e4m3_to_f64(((const uint8_t*)pool)[idx]) * (double)scale[kvh];",
+                                "return rpko_e4m3_to_f64(((const uint8_t*)pool)[idx]);"),
 }
 
 

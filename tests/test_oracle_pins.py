@@ -682,3 +682,140 @@ def test_cache_image_logical_order_invariant():
             assert np.array_equal(kp[page, slot % P], O.round_to(k_rot[t], O.BF16))
     assert touched.sum() == wl.total_tokens
     assert np.array_equal(kp_new[~touched], kp0[~touched])
+
+
+# ------------------------------------------------------------- e4m3 cache
+# NumKong's scalar-type table fixes e4m3 as 1 sign, 4 exponent and 3 mantissa
+# bits, range +-448, no infinity, with NaN, and its conversion policy rounds
+# narrowing conversions to nearest with ties to even. torch's float8_e4m3fn is
+# the same format, so it serves as an independent reference for every code
+# and for rounding inside the finite range.
+
+
+def _torch_e4m3_values():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    return codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def test_e4m3_decode_matches_every_code():
+    ref = _torch_e4m3_values()
+    got = np.array([O.e4m3_to_f64(c) for c in range(256)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert np.nanmax(got) == 448.0 and np.nanmin(got) == -448.0
+    assert O.e4m3_to_f64(0x01) == 2.0 ** -9          # smallest subnormal
+    assert O.e4m3_to_f64(0x08) == 2.0 ** -6          # smallest normal
+
+
+def test_e4m3_encode_round_trips_every_finite_code():
+    for c in range(256):
+        v = O.e4m3_to_f64(c)
+        if not math.isnan(v):
+            assert O.f64_to_e4m3(v) == c, hex(c)
+
+
+def test_e4m3_rounding_matches_torch_in_range():
+    rng = np.random.default_rng(0)
+    x = np.concatenate([
+        rng.uniform(-464.0, 464.0, 20000),
+        rng.uniform(-0.03, 0.03, 20000),                 # subnormals and small normals
+        np.ldexp(rng.uniform(1.0, 2.0, 20000), rng.integers(-12, 9, 20000)) *
+        rng.choice([-1.0, 1.0], 20000),
+    ]).astype(np.float32)
+    x = x[np.abs(x) <= 464.0]   # beyond, torch gives NaN where the cache saturates
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([O.f64_to_e4m3(float(v)) for v in x], dtype=np.uint8)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("x,code", [
+    (17.0, 0x58), (19.0, 0x5A),          # ties between 16 / 18 and 18 / 20 go to the even mantissa
+    (1.0625, 0x38), (1.1875, 0x3A),      # 1 + 1/16 -> 1, 1 + 3/16 -> 1.25
+    (2.0 ** -10, 0x00), (3 * 2.0 ** -10, 0x02), (1.5 * 2.0 ** -10, 0x01),
+    (464.0, 0x7E),                       # tie between 448 and the missing 480: the even 448
+    (-0.0, 0x80),
+])
+def test_e4m3_ties_to_even(x, code):
+    assert O.f64_to_e4m3(x) == code
+
+
+@pytest.mark.parametrize("x", [448.5, 470.0, 480.0, 1e6, math.inf])
+def test_e4m3_saturates_beyond_largest_finite(x):
+    assert O.f64_to_e4m3(x) == 0x7E
+    assert O.f64_to_e4m3(-x) == 0xFE
+
+
+def test_e4m3_nan_stays_nan():
+    assert math.isnan(O.e4m3_to_f64(O.f64_to_e4m3(math.nan)))
+
+
+def _e4m3_case(seed=0, Hk=2, d=8, P=4, lens=(5, 3), cache=(2, 0)):
+    rng = np.random.default_rng(seed)
+    B = len(lens)
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(offs[-1])
+    n_pages = sum((c + l + P - 1) // P for c, l in zip(cache, lens)) + 2
+    perm = rng.permutation(n_pages)
+    bt = np.full((B, 4), -1, dtype=np.int32)
+    cur = 0
+    for b in range(B):
+        for i in range((cache[b] + lens[b] + P - 1) // P):
+            bt[b, i] = perm[cur]
+            cur += 1
+    k_rot = rng.standard_normal((T, Hk, d)) * 3.0
+    v = rng.standard_normal((T, Hk, d)).astype(np.float32)
+    ks = np.array([0.02, 0.037], dtype=np.float32)[:Hk]
+    vs = np.array([0.011, 0.05], dtype=np.float32)[:Hk]
+    kp = np.full((n_pages, P, Hk, d), 0x7F, dtype=np.uint8)   # NaN code sentinel
+    vp = np.full((n_pages, P, Hk, d), 0x7F, dtype=np.uint8)
+    return offs, np.array(cache, dtype=np.int32), bt, k_rot, v, ks, vs, kp, vp
+
+
+def test_e4m3_cache_image_codes_and_slots():
+    offs, cl, bt, k_rot, v, ks, vs, kp, vp = _e4m3_case()
+    k2, v2 = O.cache_image(k_rot, v, offs, cl, bt, kp, vp, k_scale=ks, v_scale=vs)
+    P = kp.shape[1]
+    written = np.zeros(kp.shape[:3], dtype=bool)
+    for b in range(len(offs) - 1):
+        for i in range(offs[b + 1] - offs[b]):
+            t = offs[b] + i
+            slot = cl[b] + i
+            page, row = bt[b, slot // P], slot % P
+            written[page, row] = True
+            for h in range(kp.shape[2]):
+                for c in range(kp.shape[3]):
+                    assert k2[page, row, h, c] == O.f64_to_e4m3(k_rot[t, h, c] / float(ks[h]))
+                    assert v2[page, row, h, c] == O.f64_to_e4m3(float(v[t, h, c]) / float(vs[h]))
+    assert np.all(k2[~written] == 0x7F) and np.all(v2[~written] == 0x7F)
+    # the stored value is code * scale within half an e4m3 step of the exact one
+    t, h = 0, 1
+    page, row = bt[0, cl[0] // P], cl[0] % P
+    back = np.array([O.e4m3_to_f64(c) for c in k2[page, row, h]]) * float(ks[h])
+    assert np.all(np.abs(back - k_rot[t, h]) <= 2.0 ** -4 * np.abs(k_rot[t, h]) + 2.0 ** -10 * ks[h])
+
+
+def test_e4m3_attention_reads_code_times_scale():
+    # Power-of-two scales make code * scale exact in fp32, so the e4m3 read must
+    # equal the plain attention over those fp32 values to the last bit.
+    rng = np.random.default_rng(3)
+    Hk, d, P, H = 2, 8, 4, 4
+    lens = [6, 9]
+    kd = [rng.integers(0, 256, (n, Hk, d)).astype(np.uint8) for n in lens]
+    vd = [rng.integers(0, 256, (n, Hk, d)).astype(np.uint8) for n in lens]
+    for arr in kd + vd:
+        arr[(arr & 0x7F) == 0x7F] = 0x3C   # no NaN codes in used slots
+    ks = np.array([0.25, 2.0 ** -5], dtype=np.float32)
+    vs = np.array([2.0 ** -3, 4.0], dtype=np.float32)
+    kp8, vp8, bt = paged(kd, vd, P, dtype=np.uint8)
+    dec = np.vectorize(O.e4m3_to_f64)
+    kf = [(dec(k) * ks[None, :, None]).astype(np.float32) for k in kd]
+    vf = [(dec(v) * vs[None, :, None]).astype(np.float32) for v in vd]
+    kpf, vpf, bt2 = paged(kf, vf, P)
+    assert np.array_equal(bt, bt2)
+    q = rng.standard_normal((sum(lens), H, d)).astype(np.float32)
+    offs = np.array([0, lens[0], sum(lens)], dtype=np.int32)
+    for w in (0, 3):
+        got = O.attention(q, offs, lens, kp8, vp8, bt, Hk, 0.3, w, k_scale=ks, v_scale=vs)
+        ref = O.attention(q, offs, lens, kpf, vpf, bt, Hk, 0.3, w)
+        assert np.array_equal(got, ref)
