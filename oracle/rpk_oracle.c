@@ -337,7 +337,7 @@ int rpko_cache_image_e4m3(const double* k_rot, const void* v_new, int dtype, int
     if (pi >= max_pages_per_seq) return RPKO_ERR_PAGE;
     int32_t page = block_table[(size_t)b * max_pages_per_seq + pi];
     if (page < 0 || page >= num_pages) return RPKO_ERR_PAGE;
-    int32_t row = slot % page_size;
+    int32_t row = slot - pi * page_size;
     for (int32_t kh = 0; kh < n_kv_heads; ++kh) {
       size_t src = ((size_t)t * n_kv_heads + kh) * head_dim;
       size_t dst = (((size_t)page * page_size + row) * n_kv_heads + kh) * head_dim;

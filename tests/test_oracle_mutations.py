@@ -51,6 +51,8 @@ MUTATIONS = {
                            "if (a >= 480.0) return sign | 0x7E;"),
     "e4m3_key_scale_multiplied": ("rpko_f64_to_e4m3(k_rot[src + c] / (double)k_scale[kh]);",
                                   "rpko_f64_to_e4m3(k_rot[src + c] * (double)k_scale[kh]);"),
+    "e4m3_slot_row": ("int32_t row = slot - pi * page_size;",
+                      "int32_t row = (slot + 1) % page_size;"),
     "e4m3_read_scale_dropped": ("return rpko_e4m3_to_f64(((const uint8_t*)pool)[idx]) * (double)scale[kvh];",
                                 "return rpko_e4m3_to_f64(((const uint8_t*)pool)[idx]);"),
 }
