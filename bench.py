@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cache-dtype", default=None, choices=["e4m3"],
+                    help="hold the KV cache as e4m3 codes with per-head scales")
     return ap.parse_args()
 
 
@@ -253,8 +255,11 @@ class Step:
         self.kv_lens = i32(wl.kv_lens)
         self.position_ids = None if wl.position_ids is None else i32(wl.position_ids)
         self.error_word = torch.zeros(1, dtype=torch.int32, device=device)
+        f32 = lambda a: None if a is None else torch.from_numpy(
+            np.ascontiguousarray(a, dtype=np.float32)).to(device)
         self.cache = R.PagedKVCache(wl.k_pages.to(device), wl.v_pages.to(device),
-                                    i32(wl.block_table), i32(wl.cache_lens), self.error_word)
+                                    i32(wl.block_table), i32(wl.cache_lens), self.error_word,
+                                    k_scale=f32(wl.k_scale), v_scale=f32(wl.v_scale))
         self.table = R.freqs_cis(wl.max_position, sp.rotary_dim, sp.theta, device=device)
         self.q_rot = torch.empty_like(self.q)
         self.out = torch.empty_like(self.q)
@@ -396,13 +401,20 @@ def is_decode(wl: W.Workload) -> bool:
     return sp.dtype == "bf16" and int(wl.q_lens.max()) * (sp.n_heads // sp.n_kv_heads) <= 16
 
 
+def cache_elt(wl: W.Workload) -> int:
+    """Bytes per cached K or V element: 1 for an e4m3 cache, else q's element size."""
+    if wl.spec.cache_dtype == "e4m3":
+        return 1
+    return 2 if wl.spec.dtype == "bf16" else 4
+
+
 def metric_of(wl: W.Workload):
     """(metric, unit, amount per step, scale to the unit) of a workload: K/V
     bytes read for decode (GB/s, HBM-bound), visible-pair FLOPs for prefill
     (TFLOP/s, tensor-bound)."""
     sp = wl.spec
     if is_decode(wl):
-        elt = 2
+        elt = cache_elt(wl)
         return ("decode_attention_kv_GBps", "GB/s",
                 M.attention_kv_bytes(wl.q_lens, wl.kv_lens, sp.window, sp.n_kv_heads,
                                      sp.head_dim, elt), 1e9)
@@ -435,7 +447,7 @@ def oracle_sample_time(wl: W.Workload, max_seconds: float = 20.0):
     # attention one sequence at a time until the time budget is used
     done_b, kv_bytes, flops, toks = 0, 0, 0, 0
     t1 = time.perf_counter()
-    elt = 2 if sp.dtype == "bf16" else 4
+    elt = cache_elt(wl)
     for b in range(sp.batch):
         lo, hi = int(wl.q_offsets[b]), int(wl.q_offsets[b + 1])
         rows = np.array([[t, h] for t in range(lo, hi) for h in range(sp.n_heads)], np.int32)
@@ -469,10 +481,12 @@ def main():
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     over = {} if args.batch is None else {"batch": args.batch}
+    if args.cache_dtype:
+        over["cache_dtype"] = args.cache_dtype
     wl = W.make(args.workload, seed=rank_seed(args.seed, rank), **over)
     sp = wl.spec
     step = Step(wl, device)
-    elt = 2 if sp.dtype == "bf16" else 4
+    elt = cache_elt(wl)
     kv_bytes = M.attention_kv_bytes(wl.q_lens, wl.kv_lens, sp.window, sp.n_kv_heads,
                                     sp.head_dim, elt)
     metric, unit, amount, scale = metric_of(wl)
@@ -489,7 +503,8 @@ def main():
     peaks = load_peaks()
     value = job_amount / (step_ms * 1e-3) / scale
     achieved = amount / (attn_ms_mean * 1e-3) / scale
-    traffic = load_traffic("attn_decode") if decode else None
+    # the committed DRAM capture is of the bf16-cache decode kernel
+    traffic = load_traffic("attn_decode") if decode and sp.cache_dtype is None else None
     if decode:
         roofline = {"bound": "hbm", "kernel": "ragged_paged_attention (split-KV decode + combine)",
                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": unit,
@@ -537,6 +552,7 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": sp.dtype,
         "data": "synthetic (seeded N(0,1) values, shuffled page tables)",
         "config": {"workload": sp.name, "description": sp.description,
+                   "cache_dtype": sp.cache_dtype or sp.dtype,
                    "batch_per_gpu": sp.batch, "new_tokens_per_step": wl.total_tokens,
                    "kv_bytes_per_step": kv_bytes,
                    "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V per step "
@@ -566,6 +582,8 @@ def reference_arm(args, world, rank):
             torch.distributed.destroy_process_group()
         return
     over = {} if args.batch is None else {"batch": args.batch}
+    if args.cache_dtype:
+        over["cache_dtype"] = args.cache_dtype
     wl = W.make(args.workload, seed=args.seed, **over)
     sp = wl.spec
     metric, unit, _, scale = metric_of(wl)

@@ -24,7 +24,9 @@
  *           and no silent change of path (aria_kernel crate index,
  *           resolve_compute: CUDA never falls back to the CPU).
  * Dtypes.   RPK_BF16 or RPK_F32 for q, k, v, out and the cache; all arithmetic
- *           is fp32 with one round-to-nearest-even narrowing at the end.
+ *           is fp32 with one round-to-nearest-even narrowing at the end. The
+ *           cache may instead be RPK_E4M3 (see rpk_paged_kv) under bf16 or
+ *           fp32 tensors.
  */
 #ifndef RPK_H
 #define RPK_H
@@ -46,7 +48,10 @@ typedef enum {
   RPK_ERR_WORKSPACE = 6     /* workspace missing, too small or misaligned           */
 } rpk_status;
 
-typedef enum { RPK_F32 = 0, RPK_BF16 = 1 } rpk_dtype;
+/* RPK_E4M3 is a cache dtype only: 1 sign, 4 exponent (bias 7) and 3 mantissa
+ * bits, no infinity, NaN = S.1111.111, largest finite 448 (NumKong "NumKong for
+ * Python", scalar types: float8_e4m3). */
+typedef enum { RPK_F32 = 0, RPK_BF16 = 1, RPK_E4M3 = 2 } rpk_dtype;
 
 /* Bits OR-ed into *error_word by the kernels. */
 #define RPK_DEVERR_PAGE 0x1u     /* page id outside [0, num_pages) or slot beyond the block table */
@@ -77,6 +82,17 @@ typedef enum { RPK_F32 = 0, RPK_BF16 = 1 } rpk_dtype;
  *                      only, sharing block_table and cache_lens with the other
  *                      layers. num_layers 0 (a zero-initialised struct) means 1.
  *                      layer_idx outside [0, num_layers): RPK_ERR_SHAPE.
+ *   cache_dtype        RPK_BF16 / RPK_F32 (the dtype of q, k, v), or RPK_E4M3: a
+ *                      quantised cache (Mojo's kv_collection with a cache dtype,
+ *                      a scale dtype and a quantisation granularity) holding
+ *                      code = e4m3(x / scale) with one fp32 scale per KV head
+ *                      for K and one for V; the key or value is code * scale.
+ *                      rope_qk_paged_ragged rounds the fp32 quotient once to
+ *                      nearest (ties to even) and saturates magnitudes beyond
+ *                      448 to +-448.
+ *   k_scale, v_scale   fp32 [n_kv_heads] (device), finite and > 0: the scales of
+ *                      an RPK_E4M3 cache (required then: NULL is RPK_ERR_NULL);
+ *                      not read for other cache dtypes.
  */
 typedef struct {
   void* k_pages;
@@ -93,6 +109,8 @@ typedef struct {
   int32_t* error_word;
   int32_t num_layers;
   int32_t layer_idx;
+  const float* k_scale;
+  const float* v_scale;
 } rpk_paged_kv;
 
 /*
@@ -128,8 +146,10 @@ typedef struct {
  *                      position of its section's row of position_ids
  *
  * Each pair (a, b) becomes (a cos - b sin, b cos + a sin), computed in fp32
- * and rounded once to the output dtype. Requirements: dtype == cache dtype,
- * n_heads % n_kv_heads == 0, (R/2) a multiple of 8 (bf16) or 4 (f32).
+ * and rounded once to the output dtype. Requirements: dtype == cache dtype
+ * (or an RPK_E4M3 cache, which receives e4m3(k' / k_scale) and e4m3(v / v_scale)
+ * of the fp32 values, see rpk_paged_kv), n_heads % n_kv_heads == 0, (R/2) a
+ * multiple of 8 (bf16) or 4 (f32).
  */
 rpk_status rope_qk_paged_ragged(const void* q_proj, const int32_t* input_row_offsets,
                                 const void* k_new, const void* v_new,
@@ -232,6 +252,9 @@ size_t ragged_paged_attention_workspace_size(int32_t total_q_tokens, int32_t n_h
  *   bf16, otherwise                -> tcgen05 prefill kernel (head_dim 64/128,
  *                                     group <= 128; other shapes run on the
  *                                     CUDA-core kernel)
+ * An RPK_E4M3 cache takes the same decode path (the kernel widens each tile
+ * to f16 in shared memory, exactly, and folds k_scale into the score scale and
+ * v_scale into the output); its other shapes run on the CUDA-core kernel.
  */
 rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
                                   const int32_t* kv_lens, const rpk_paged_kv* page_table,

@@ -28,7 +28,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "librpk.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "rpk.h")
 
-RPK_F32, RPK_BF16 = 0, 1
+RPK_F32, RPK_BF16, RPK_E4M3 = 0, 1, 2
 STATUS = {0: "RPK_OK", 1: "RPK_ERR_NULL", 2: "RPK_ERR_SHAPE", 3: "RPK_ERR_DTYPE",
           4: "RPK_ERR_UNSUPPORTED", 5: "RPK_ERR_CUDA", 6: "RPK_ERR_WORKSPACE"}
 DEVERR_PAGE, DEVERR_POSITION, DEVERR_LENGTH, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
@@ -53,6 +53,7 @@ class PagedKV(C.Structure):
         ("block_table", C.c_void_p), ("max_pages_per_seq", C.c_int32), ("batch", C.c_int32),
         ("cache_lens", C.c_void_p), ("error_word", C.c_void_p),
         ("num_layers", C.c_int32), ("layer_idx", C.c_int32),
+        ("k_scale", C.c_void_p), ("v_scale", C.c_void_p),
     ]
 
 
@@ -113,6 +114,13 @@ def _dtype_code(t: torch.dtype) -> int:
     raise RpkError(f"unsupported dtype {t}")
 
 
+def _cache_dtype_code(t: torch.dtype) -> int:
+    """Cache pools may also hold e4m3 codes (torch.float8_e4m3fn or raw uint8)."""
+    if t in (torch.float8_e4m3fn, torch.uint8):
+        return RPK_E4M3
+    return _dtype_code(t)
+
+
 def _dev(t: torch.Tensor, name: str, dtype=None, ndim=None) -> int:
     if not isinstance(t, torch.Tensor):
         raise RpkError(f"{name} must be a torch.Tensor")
@@ -142,6 +150,8 @@ class PagedKVCache:
     The pools are [num_pages, page_size, n_kv_heads, head_dim], or, for a
     multi-layer collection, [num_layers, num_pages, page_size, n_kv_heads,
     head_dim] with layer_idx choosing the layer the calls read and write.
+    Pools of torch.float8_e4m3fn (or raw uint8) hold e4m3 codes of x / scale,
+    with k_scale / v_scale the fp32 [n_kv_heads] scales of K and V.
     """
 
     k_pages: torch.Tensor
@@ -150,6 +160,8 @@ class PagedKVCache:
     cache_lens: torch.Tensor | None = None   # int32 [batch]
     error_word: torch.Tensor | None = None   # int32 [1]
     layer_idx: int = 0
+    k_scale: torch.Tensor | None = None      # fp32 [n_kv_heads], e4m3 pools only
+    v_scale: torch.Tensor | None = None
 
     def struct(self) -> PagedKV:
         kp, vp = self.k_pages, self.v_pages
@@ -166,7 +178,12 @@ class PagedKVCache:
         s.num_layers = shape[0] if len(shape) == 5 else 1
         s.layer_idx = int(self.layer_idx)
         s.num_pages, s.page_size, s.n_kv_heads, s.head_dim = shape[-4:]
-        s.cache_dtype = _dtype_code(kp.dtype)
+        s.cache_dtype = _cache_dtype_code(kp.dtype)
+        if s.cache_dtype == RPK_E4M3:
+            if self.k_scale is None or self.v_scale is None:
+                raise RpkError("an e4m3 cache needs k_scale and v_scale")
+            s.k_scale = _dev(self.k_scale, "k_scale", torch.float32, 1)
+            s.v_scale = _dev(self.v_scale, "v_scale", torch.float32, 1)
         s.block_table = self.block_table.data_ptr()
         s.batch, s.max_pages_per_seq = (int(x) for x in self.block_table.shape)
         s.cache_lens = (_dev(self.cache_lens, "cache_lens", torch.int32, 1)

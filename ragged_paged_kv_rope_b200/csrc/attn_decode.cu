@@ -28,6 +28,15 @@
 // at p = r + k_len - q_len and sees [p - (window - 1), p]; masked keys are left
 // out (score -inf, weight 0) and value rows past k_len are zeroed in shared
 // memory before use so that stale or sentinel bytes never reach P V.
+//
+// An e4m3 cache (codes of x / scale, one scale per KV head for K and for V)
+// halves the bytes per key. The stages then hold raw codes (no swizzle); each
+// consumer warp widens its own 16 key rows of K and V to f16 (exact for every
+// e4m3 value) into a private swizzled tile, releases the stage, and runs the
+// same ldmatrix / mma.sync code in f16. Q is scaled by a power of two 2^-qs
+// that brings its largest magnitude into [2^14, 2^15) before the f16
+// narrowing; 2^qs and k_scale join the score scale, v_scale multiplies the
+// merged output. P is f16 (values in [0, 1]).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -111,7 +120,16 @@ __device__ __forceinline__ void mma_bf16(float* d, const uint32_t* a, uint32_t b
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <int D>
+// D += A(16x16 f16, row) * B(16x8 f16, col), fp32 accumulators.
+__device__ __forceinline__ void mma_f16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int D, bool kFp8 = false>
 struct DecodeCfg {
   static constexpr int kBoxes = D / 64;                      // 128-byte column boxes per row
   static constexpr int kTileBytes = kDecodeTile * D * 2;     // one of K or V
@@ -121,12 +139,31 @@ struct DecodeCfg {
   static_assert(kConsumerWarps * 16 * D * 4 <= kStages * kStageBytes, "merge buffer");
 };
 
+// e4m3 cache: stages of raw codes [64 keys][D bytes] for K then V, and one
+// f16 tile of 16 rows (kBoxes 128-byte swizzled boxes) for K and for V per
+// consumer warp.
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+struct DecodeCfg<D, true> {
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kTileBytes = kDecodeTile * D;          // raw codes of K or V
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kStages = D == 256 ? 2 : (D == 128 ? 4 : 8);
+  static constexpr int kConvTileBytes = 16 * D * 2;           // 16 rows of f16
+  static constexpr int kConvOff = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kConvOff + kConsumerWarps * 2 * kConvTileBytes + 1024;
+  static_assert(kConsumerWarps * 16 * D * 4 <= kSmemBytes - 1024, "merge buffer");
+};
+
+// Two CTAs share an SM when each warp holds at most 168 registers: ten warps
+// put three on some sub-partition, whose register file is a quarter of the
+// SM's (3 * 168 * 32 <= 16384). The bf16 kernel needs no cap for that; the
+// e4m3 kernel's widening would otherwise take it past the limit.
+template <int D, bool kFp8>
+__global__ void __launch_bounds__(kThreads, 1) __maxnreg__(kFp8 && D <= 128 ? 168 : 255)
     attn_decode_kernel(const AttnParams p, const __grid_constant__ CUtensorMap k_map,
                        const __grid_constant__ CUtensorMap v_map, const DecodePlan plan,
                        const DecodeWorkspace ws) {
-  using Cfg = DecodeCfg<D>;
+  using Cfg = DecodeCfg<D, kFp8>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t full_bar[S], empty_bar[S];
@@ -172,6 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&k_map);
       prefetch_tensormap(&v_map);
       const int box_rows = p.P < kDecodeTile ? p.P : kDecodeTile;
+      // bf16: boxes of 64 channels (128 bytes) per row; e4m3: one box of D bytes per row.
       const uint32_t box_bytes = box_rows * 128u;
       int issued = 0;
       bool ok = true;
@@ -186,7 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (key >= k_len) break;
           const int pi = key / p.P;
           const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
-          if (page >= 0 && page < p.num_pages) bytes += 2u * Cfg::kBoxes * box_bytes;
+          if (page >= 0 && page < p.num_pages)
+            bytes += kFp8 ? 2u * box_rows * D : 2u * Cfg::kBoxes * box_bytes;
         }
         mbar_arrive_expect_tx(&full_bar[s], bytes);
         for (int r = 0; r < kDecodeTile; r += box_rows) {
@@ -199,12 +238,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             continue;
           }
           const int grow = page * p.P + (key - pi * p.P);
+          if constexpr (kFp8) {
+            tma_load_3d(k_stage(s) + r * D, &k_map, 0, kvh, grow, &full_bar[s]);
+            tma_load_3d(v_stage(s) + r * D, &v_map, 0, kvh, grow, &full_bar[s]);
+          } else {
 #pragma unroll
-          for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-            tma_load_3d(k_stage(s) + bx * (kDecodeTile * 128) + r * 128, &k_map, bx * 64, kvh,
-                        grow, &full_bar[s]);
-            tma_load_3d(v_stage(s) + bx * (kDecodeTile * 128) + r * 128, &v_map, bx * 64, kvh,
-                        grow, &full_bar[s]);
+            for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+              tma_load_3d(k_stage(s) + bx * (kDecodeTile * 128) + r * 128, &k_map, bx * 64, kvh,
+                          grow, &full_bar[s]);
+              tma_load_3d(v_stage(s) + bx * (kDecodeTile * 128) + r * 128, &v_map, bx * 64, kvh,
+                          grow, &full_bar[s]);
+            }
           }
         }
         ++issued;
@@ -257,6 +301,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
+  float sl2 = p.scale_log2;   // score scale in log2 units
+  float v_mul = 1.f;          // applied to the merged output
+  if constexpr (kFp8) {
+    // Largest |q| of the group's rows (every consumer warp holds all of them,
+    // so every warp finds the same power of two).
+    float mx = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(&qa[ks][k]);
+        mx = fmaxf(mx, fmaxf(fabsf(__low2float(v2)), fabsf(__high2float(v2))));
+      }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    int qs = 0;
+    if (mx > 0.f && mx <= 3.0e38f) qs = min(64, max(-64, ilogbf(mx) - 14));
+    const float down = __int_as_float((127 - qs) << 23);  // 2^-qs
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(&qa[ks][k]);
+        qa[ks][k] = pack_f16x2(__low2float(v2) * down, __high2float(v2) * down);
+      }
+    sl2 = p.scale_log2 * __ldg(p.k_scale + kvh) * __int_as_float((127 + qs) << 23);
+    v_mul = __ldg(p.v_scale + kvh);
+  }
 
   float o[D / 8][4];
 #pragma unroll
@@ -269,13 +341,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int s = i % S;
     if (!mbar_wait(&full_bar[s], (i / S) & 1)) { ok = false; break; }
     const int key0 = ss.tile_at(v_begin + i) * kDecodeTile + warp * 16;  // this warp's 16 keys
-    const uint32_t kbase = smem_u32(k_stage(s));
-    const uint32_t vbase = smem_u32(v_stage(s));
-    const int wrow0 = warp * 16;  // row of this warp's first key inside the tile
-
-    // Zero value rows at or past k_len (stale or never written bytes).
+    uint32_t kbase = smem_u32(k_stage(s));
+    uint32_t vbase = smem_u32(v_stage(s));
+    int wrow0 = warp * 16;  // row of this warp's first key inside the tile
+    constexpr int kBoxStride = (kFp8 ? 16 : kDecodeTile) * 128;  // bytes between 64-channel boxes
     const bool tail = key0 + 15 >= k_len;
-    if (tail) {
+    if constexpr (kFp8) {
+      // Widen this warp's 16 rows of K and V from e4m3 codes to f16 in its own
+      // tiles (value rows at or past k_len become zeros), then release the stage.
+      uint8_t* ck = smem + Cfg::kConvOff + warp * 2 * Cfg::kConvTileBytes;
+      uint8_t* cv = ck + Cfg::kConvTileBytes;
+      constexpr int kChunks = D / 16;  // 16-code chunks per row
+      // K, then V (one tile at a time keeps fewer registers live under the
+      // 168-register cap; head_dim 256 runs one CTA per SM and unrolls both)
+      constexpr int kUnrollKV = D == 256 ? 2 : 1;
+#pragma unroll kUnrollKV
+      for (int kv = 0; kv < 2; ++kv) {
+        const uint8_t* raw = kv ? v_stage(s) : k_stage(s);
+        uint8_t* conv = kv ? cv : ck;
+#pragma unroll
+        for (int it = 0; it < (16 * kChunks) / 32; ++it) {
+          const int idx = lane + 32 * it;
+          const int kr = idx / kChunks;
+          const int j = idx - kr * kChunks;
+          uint4 r4 = *reinterpret_cast<const uint4*>(raw + (wrow0 + kr) * D + j * 16);
+          if (kv && key0 + kr >= k_len) r4 = make_uint4(0, 0, 0, 0);
+          const uint32_t w[4] = {r4.x, r4.y, r4.z, r4.w};
+          uint32_t h[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            h[2 * q] = f16x2_from_e4m3x2(w[q] & 0xFFFFu);
+            h[2 * q + 1] = f16x2_from_e4m3x2(w[q] >> 16);
+          }
+          // f16 channels 16j .. 16j+15 are the 16-byte chunks 2j and 2j+1 of the row.
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int ch = 2 * j + hh;
+            *reinterpret_cast<uint4*>(conv + (ch >> 3) * kBoxStride + swz128(kr, ch & 7)) =
+                make_uint4(h[4 * hh], h[4 * hh + 1], h[4 * hh + 2], h[4 * hh + 3]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[s]);
+      kbase = smem_u32(ck);
+      vbase = smem_u32(cv);
+      wrow0 = 0;
+    } else if (tail) {
+      // Zero value rows at or past k_len (stale or never written bytes).
       for (int idx = lane; idx < 16 * (D / 8); idx += 32) {
         const int kr = idx / (D / 8);
         if (key0 + kr < k_len) continue;
@@ -294,11 +407,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mi = lane >> 3;
       const int krow = wrow0 + (mi >> 1) * 8 + (lane & 7);
       const int chunk = ks * 2 + (mi & 1);
-      const uint32_t addr = kbase + (chunk >> 3) * (kDecodeTile * 128) + swz128(krow, chunk & 7);
+      const uint32_t addr = kbase + (chunk >> 3) * kBoxStride + swz128(krow, chunk & 7);
       uint32_t b0, b1, b2, b3;
       ldsm_x4(addr, b0, b1, b2, b3);
-      mma_bf16(sc[0], qa[ks], b0, b1);
-      mma_bf16(sc[1], qa[ks], b2, b3);
+      if constexpr (kFp8) {
+        mma_f16(sc[0], qa[ks], b0, b1);
+        mma_f16(sc[1], qa[ks], b2, b3);
+      } else {
+        mma_bf16(sc[0], qa[ks], b0, b1);
+        mma_bf16(sc[1], qa[ks], b2, b3);
+      }
     }
 
     // Mask, scale to log2 units, online-softmax update of both rows.
@@ -311,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int key = key0 + nt * 8 + 2 * c + (e & 1);
         const bool vis =
             row_ok[hr] && key <= row_hi[hr] && (key >= row_lo[hr] || key < p.sinks);
-        const float v = vis ? sc[nt][e] * p.scale_log2 : -INFINITY;
+        const float v = vis ? sc[nt][e] * sl2 : -INFINITY;
         sc[nt][e] = v;
         tmax[hr] = fmaxf(tmax[hr], v);
       }
@@ -345,10 +463,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // O += P V: P (16 rows x 16 keys) as the A operand straight from registers.
     uint32_t pa[4];
-    pa[0] = pack_bf16x2(sc[0][0], sc[0][1]);
-    pa[1] = pack_bf16x2(sc[0][2], sc[0][3]);
-    pa[2] = pack_bf16x2(sc[1][0], sc[1][1]);
-    pa[3] = pack_bf16x2(sc[1][2], sc[1][3]);
+    if constexpr (kFp8) {
+      pa[0] = pack_f16x2(sc[0][0], sc[0][1]);
+      pa[1] = pack_f16x2(sc[0][2], sc[0][3]);
+      pa[2] = pack_f16x2(sc[1][0], sc[1][1]);
+      pa[3] = pack_f16x2(sc[1][2], sc[1][3]);
+    } else {
+      pa[0] = pack_bf16x2(sc[0][0], sc[0][1]);
+      pa[1] = pack_bf16x2(sc[0][2], sc[0][3]);
+      pa[2] = pack_bf16x2(sc[1][0], sc[1][1]);
+      pa[3] = pack_bf16x2(sc[1][2], sc[1][3]);
+    }
 #pragma unroll
     for (int dn = 0; dn < D / 16; ++dn) {
       // matrices (transposed): (keys 0-7, d n0), (keys 8-15, d n0), (keys 0-7, d n0+8),
@@ -356,16 +481,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mi = lane >> 3;
       const int vrow = wrow0 + (mi & 1) * 8 + (lane & 7);
       const int chunk = dn * 2 + (mi >> 1);
-      const uint32_t addr = vbase + (chunk >> 3) * (kDecodeTile * 128) + swz128(vrow, chunk & 7);
+      const uint32_t addr = vbase + (chunk >> 3) * kBoxStride + swz128(vrow, chunk & 7);
       uint32_t b0, b1, b2, b3;
       ldsm_x4_t(addr, b0, b1, b2, b3);
-      mma_bf16(o[2 * dn], pa, b0, b1);
-      mma_bf16(o[2 * dn + 1], pa, b2, b3);
+      if constexpr (kFp8) {
+        mma_f16(o[2 * dn], pa, b0, b1);
+        mma_f16(o[2 * dn + 1], pa, b2, b3);
+      } else {
+        mma_bf16(o[2 * dn], pa, b0, b1);
+        mma_bf16(o[2 * dn + 1], pa, b2, b3);
+      }
     }
 
     __syncwarp();
-    if (tail) fence_proxy_async_smem();  // generic zero-writes before the next TMA into s
-    if (lane == 0) mbar_arrive(&empty_bar[s]);
+    if constexpr (!kFp8) {
+      if (tail) fence_proxy_async_smem();  // generic zero-writes before the next TMA into s
+      if (lane == 0) mbar_arrive(&empty_bar[s]);
+    }
   }
   if (!ok) raise_error(p.error_word, RPK_DEVERR_TIMEOUT);
   // Let the combine kernel launch now (it waits for this grid's completion
@@ -421,6 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float4 v = *reinterpret_cast<const float4*>(obuf + ((size_t)w * 16 + rr) * D + e4);
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
+    acc.x *= v_mul; acc.y *= v_mul; acc.z *= v_mul; acc.w *= v_mul;
     const int t = q0 + rr / p.G;
     const int h = kvh * p.G + rr % p.G;
     const size_t orow = (size_t)t * p.H + h;
@@ -486,16 +619,17 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p,
   for (int e = 0; e < E; e += 2) *reinterpret_cast<uint32_t*>(out + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
 }
 
-template <int D>
+template <int D, bool kFp8>
 cudaError_t launch_d(const AttnParams& p, const CUtensorMap& k_map, const CUtensorMap& v_map,
                      const DecodePlan& plan, const DecodeWorkspace& ws, cudaStream_t stream) {
-  using Cfg = DecodeCfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<D>,
+  using Cfg = DecodeCfg<D, kFp8>;
+  cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<D, kFp8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.max_splits, p.Hk, p.batch);
-  attn_decode_kernel<D><<<grid, kThreads, Cfg::kSmemBytes, stream>>>(p, k_map, v_map, plan, ws);
+  attn_decode_kernel<D, kFp8><<<grid, kThreads, Cfg::kSmemBytes, stream>>>(p, k_map, v_map, plan,
+                                                                          ws);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (plan.max_splits > 1) {
@@ -521,10 +655,18 @@ cudaError_t launch_attn_decode(const AttnParams& p, const CUtensorMap& k_map,
                                const CUtensorMap& v_map, const DecodePlan& plan,
                                const DecodeWorkspace& ws, cudaStream_t stream) {
   if ((long long)p.T * p.H == 0 || p.batch == 0) return cudaSuccess;
+  if (p.cache_fp8) {
+    switch (p.d) {
+      case 64: return launch_d<64, true>(p, k_map, v_map, plan, ws, stream);
+      case 128: return launch_d<128, true>(p, k_map, v_map, plan, ws, stream);
+      case 256: return launch_d<256, true>(p, k_map, v_map, plan, ws, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (p.d) {
-    case 64: return launch_d<64>(p, k_map, v_map, plan, ws, stream);
-    case 128: return launch_d<128>(p, k_map, v_map, plan, ws, stream);
-    case 256: return launch_d<256>(p, k_map, v_map, plan, ws, stream);
+    case 64: return launch_d<64, false>(p, k_map, v_map, plan, ws, stream);
+    case 128: return launch_d<128, false>(p, k_map, v_map, plan, ws, stream);
+    case 256: return launch_d<256, false>(p, k_map, v_map, plan, ws, stream);
     default: return cudaErrorInvalidValue;
   }
 }

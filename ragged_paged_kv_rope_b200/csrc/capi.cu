@@ -33,7 +33,9 @@ bool supported_page(int32_t P) { return P == 16 || P == 32 || P == 64 || P == 12
 rpk_status check_cache(const rpk_paged_kv* c) {
   if (!c) return RPK_ERR_NULL;
   if (!c->k_pages || !c->v_pages || !c->block_table) return RPK_ERR_NULL;
-  if (c->cache_dtype != RPK_BF16 && c->cache_dtype != RPK_F32) return RPK_ERR_DTYPE;
+  if (c->cache_dtype != RPK_BF16 && c->cache_dtype != RPK_F32 && c->cache_dtype != RPK_E4M3)
+    return RPK_ERR_DTYPE;
+  if (c->cache_dtype == RPK_E4M3 && (!c->k_scale || !c->v_scale)) return RPK_ERR_NULL;
   if (c->num_pages <= 0 || c->n_kv_heads <= 0 || c->max_pages_per_seq <= 0 || c->batch <= 0)
     return RPK_ERR_SHAPE;
   if (!supported_page(c->page_size) || !supported_head_dim(c->head_dim))
@@ -58,6 +60,35 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   });
   return fn;
+}
+
+// q / k / v dtype and a cache dtype agree, or the cache holds e4m3 codes.
+bool cache_dtype_ok(rpk_dtype dtype, rpk_dtype cache) {
+  return cache == dtype || cache == RPK_E4M3;
+}
+
+// 3-D byte map over rows of an e4m3 pool [rows, heads, d]: box (d, 1, box_rows)
+// = whole rows of one head, no swizzle (the decode kernel widens them itself).
+rpk_status encode_rows_map_u8(CUtensorMap* map, const void* base, int32_t d, int32_t heads,
+                              int64_t rows, int32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) {
+    snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled unavailable");
+    return RPK_ERR_CUDA;
+  }
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)heads * d};
+  cuuint32_t box[3] = {(cuuint32_t)d, 1u, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled failed (%d)",
+             (int)r);
+    return RPK_ERR_CUDA;
+  }
+  return RPK_OK;
 }
 
 // 3-D bf16 map over rows of [rows, heads, d]: dims (d, heads, rows), box
@@ -116,7 +147,7 @@ rpk_status rope_qk_paged_ragged(const void* q_proj, const int32_t* input_row_off
   if (st != RPK_OK) return st;
   if (!page_table->cache_lens) return RPK_ERR_NULL;
   if (dtype != RPK_BF16 && dtype != RPK_F32) return RPK_ERR_DTYPE;
-  if (dtype != page_table->cache_dtype) return RPK_ERR_DTYPE;
+  if (!cache_dtype_ok(dtype, page_table->cache_dtype)) return RPK_ERR_DTYPE;
   const int32_t d = page_table->head_dim, Hk = page_table->n_kv_heads;
   if (total_tokens < 0 || n_heads <= 0 || max_position <= 0) return RPK_ERR_SHAPE;
   if (n_heads % Hk != 0) return RPK_ERR_SHAPE;
@@ -148,6 +179,9 @@ rpk_status rope_qk_paged_ragged(const void* q_proj, const int32_t* input_row_off
   p.sec_end0 = mrope_section ? mrope_section[0] : rotary_dim;
   p.sec_end1 = mrope_section ? mrope_section[0] + mrope_section[1] : rotary_dim;
   p.tokens_per_cta = 1;
+  p.cache_fp8 = page_table->cache_dtype == RPK_E4M3;
+  p.k_scale = page_table->k_scale;
+  p.v_scale = page_table->v_scale;
   return cuda_status(rpk::launch_rope(p, dtype, interleaved != 0,
                                       static_cast<cudaStream_t>(stream)));
 }
@@ -196,7 +230,7 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
   rpk_status st = check_cache(page_table);
   if (st != RPK_OK) return st;
   if (dtype != RPK_BF16 && dtype != RPK_F32) return RPK_ERR_DTYPE;
-  if (dtype != page_table->cache_dtype) return RPK_ERR_DTYPE;
+  if (!cache_dtype_ok(dtype, page_table->cache_dtype)) return RPK_ERR_DTYPE;
   if (n_kv_heads != page_table->n_kv_heads || head_dim != page_table->head_dim)
     return RPK_ERR_SHAPE;
   if (n_heads <= 0 || n_heads % n_kv_heads != 0) return RPK_ERR_SHAPE;
@@ -227,6 +261,9 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
   p.window = window > 0 ? window : 0; p.max_q_len = max_q_len; p.max_kv_len = max_kv_len;
   p.scale = scale;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  p.cache_fp8 = page_table->cache_dtype == RPK_E4M3;
+  p.k_scale = page_table->k_scale;
+  p.v_scale = page_table->v_scale;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   if (dtype == RPK_F32) return cuda_status(rpk::launch_attn_simt(p, dtype, s));
@@ -247,12 +284,20 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
     CUtensorMap k_map, v_map;
     const int32_t box_rows = p.P < rpk::kDecodeTile ? p.P : rpk::kDecodeTile;
     const int64_t pool_rows = (int64_t)p.num_pages * p.P;
-    st = encode_rows_map(&k_map, p.k_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
-    if (st != RPK_OK) return st;
-    st = encode_rows_map(&v_map, p.v_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
+    if (p.cache_fp8) {
+      st = encode_rows_map_u8(&k_map, p.k_pages, head_dim, n_kv_heads, pool_rows, box_rows);
+      if (st != RPK_OK) return st;
+      st = encode_rows_map_u8(&v_map, p.v_pages, head_dim, n_kv_heads, pool_rows, box_rows);
+    } else {
+      st = encode_rows_map(&k_map, p.k_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
+      if (st != RPK_OK) return st;
+      st = encode_rows_map(&v_map, p.v_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
+    }
     if (st != RPK_OK) return st;
     return cuda_status(rpk::launch_attn_decode(p, k_map, v_map, plan, ws, s));
   }
+  // An e4m3 cache under prefill shapes: CUDA-core kernel.
+  if (p.cache_fp8) return cuda_status(rpk::launch_attn_simt(p, dtype, s));
 
   // Prefill shapes: tcgen05 kernel for head_dim 64 / 128 and groups up to 128.
   const int tpt = rpk::prefill_rows_per_tile(p.G);

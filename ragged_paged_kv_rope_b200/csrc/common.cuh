@@ -8,6 +8,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -68,7 +69,37 @@ __device__ __forceinline__ void store16(T* p, const float* in) {
   *reinterpret_cast<uint4*>(p) = raw;
 }
 
-// 2^x by the MUFU approximation (relative error ~2^-22; 2^-inf = +0).
+// ------------------------------------------------------------------- e4m3
+
+// Two fp32 values -> two e4m3 codes, lo in bits 0-7 and hi in bits 8-15:
+// rounded to nearest with ties to even, magnitudes beyond 448 saturating to
+// +-448 (the largest finite code), NaN kept (PTX cvt .satfinite .e4m3x2).
+__device__ __forceinline__ uint32_t e4m3x2_from_f32(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two e4m3 codes (bits 0-7, 8-15) -> two f16 values (bits 0-15, 16-31); every
+// e4m3 value is exactly representable in f16.
+__device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint32_t codes) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"((uint16_t)codes));
+  return r;
+}
+
+// One e4m3 code -> fp32 (exact).
+__device__ __forceinline__ float f32_from_e4m3(uint8_t code) {
+  const uint32_t h2 = f16x2_from_e4m3x2(code);
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// Two fp32 values -> f16x2 (round to nearest even), lo in bits 0-15.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 // Natural log-sum-exp of a row from its running state in log2 units: the
 // scores' maximum m (times log2 e) and the sum l of 2^(score - m); -inf for a
 // row with no key (l = 0).
@@ -76,6 +107,7 @@ __device__ __forceinline__ float lse_from_log2_state(float m, float l) {
   return l > 0.f ? (m + log2f(l)) * 0.693147180559945309f : -INFINITY;
 }
 
+// 2^x by the MUFU approximation (relative error ~2^-22; 2^-inf = +0).
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -16,7 +16,7 @@ namespace rpk {
 inline bool layer_pools(const rpk_paged_kv* c, void** k, void** v) {
   const int32_t layers = c->num_layers > 0 ? c->num_layers : 1;
   if (c->num_layers < 0 || c->layer_idx < 0 || c->layer_idx >= layers) return false;
-  const size_t elt = c->cache_dtype == RPK_F32 ? 4 : 2;
+  const size_t elt = c->cache_dtype == RPK_F32 ? 4 : (c->cache_dtype == RPK_E4M3 ? 1 : 2);
   const size_t per_layer =
       (size_t)c->num_pages * c->page_size * c->n_kv_heads * c->head_dim * elt;
   *k = static_cast<char*>(c->k_pages) + (size_t)c->layer_idx * per_layer;
@@ -41,6 +41,9 @@ struct RopeParams {
   int32_t sec_end0, sec_end1;   // M-RoPE: pair j < sec_end0 -> section 0, < sec_end1 -> 1, else 2
   int32_t has_mrope;
   int32_t tokens_per_cta;       // 1..4, chosen by the launcher
+  int32_t cache_fp8;            // the pools hold e4m3 codes of x / scale
+  const float* k_scale;         // [Hk] when cache_fp8
+  const float* v_scale;
 };
 
 cudaError_t launch_rope(const RopeParams& p, rpk_dtype dtype, bool interleaved,
@@ -62,6 +65,9 @@ struct AttnParams {
   float scale_log2;            // scale * log2(e)
   float* lse = nullptr;        // [T, H] natural log-sum-exp of each row's scores, or null
   int32_t sinks = 0;           // under a window: the first `sinks` keys stay visible
+  int32_t cache_fp8 = 0;       // the pools hold e4m3 codes; key = code * k_scale[kvh] etc.
+  const float* k_scale = nullptr;
+  const float* v_scale = nullptr;
 };
 
 // fp32 / bf16 CUDA-core attention: one warp per (token, head) row.

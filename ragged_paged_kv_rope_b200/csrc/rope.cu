@@ -16,7 +16,12 @@
 // kVec pairs (kVec channels from each half), one of the interleaved layout a
 // 16-byte chunk of kVec/2 adjacent pairs, whose (cos, sin) entries are the
 // same 16-byte-aligned run of the table row. Channels >= rotary_dim and V rows
-// are 16-byte copies. Every global access is a 16-byte vector.
+// are 16-byte copies. Every global load is a 16-byte vector.
+//
+// An e4m3 cache (Mojo's cache_dtype with per-head scales) receives
+// e4m3(k' / k_scale[kvh]) and e4m3(v / v_scale[kvh]) of the fp32 values: the
+// quotient is an IEEE fp32 division, rounded once to the nearest code with
+// ties to even and saturated to +-448; a unit of V elements becomes V bytes.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -33,7 +38,22 @@ struct TokenInfo {
   int pos_ok;
 };
 
-template <typename T, bool kInterleaved>
+// V fp32 values divided by `scale` -> V e4m3 codes at dst (V = 4 or 8 bytes).
+template <int V>
+__device__ __forceinline__ void store_e4m3(uint8_t* dst, const float* x, float scale) {
+  uint32_t w[V / 4];
+#pragma unroll
+  for (int i = 0; i < V / 4; ++i) {
+    const uint32_t lo = e4m3x2_from_f32(__fdiv_rn(x[4 * i], scale), __fdiv_rn(x[4 * i + 1], scale));
+    const uint32_t hi =
+        e4m3x2_from_f32(__fdiv_rn(x[4 * i + 2], scale), __fdiv_rn(x[4 * i + 3], scale));
+    w[i] = lo | (hi << 16);
+  }
+  if constexpr (V == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+  else *reinterpret_cast<uint32_t*>(dst) = w[0];
+}
+
+template <typename T, bool kInterleaved, bool kFp8>
 __global__ void __launch_bounds__(kThreads) rope_scatter_kernel(const RopeParams p) {
   constexpr int V = Elt<T>::kVec;
   __shared__ TokenInfo info[kTokens];
@@ -90,6 +110,8 @@ __global__ void __launch_bounds__(kThreads) rope_scatter_kernel(const RopeParams
   T* out_q = static_cast<T*>(p.out_q);
   T* kp = static_cast<T*>(p.k_pages);
   T* vp = static_cast<T*>(p.v_pages);
+  uint8_t* kp8 = static_cast<uint8_t*>(p.k_pages);
+  uint8_t* vp8 = static_cast<uint8_t*>(p.v_pages);
 
   for (int uu = threadIdx.x; uu < total; uu += kThreads) {
     const int tk = uu / per_token;
@@ -106,6 +128,9 @@ __global__ void __launch_bounds__(kThreads) rope_scatter_kernel(const RopeParams
     int unit;
     if (u < q_units + k_units) {
       int row;
+      bool to_cache = false;  // a K row of an e4m3 cache
+      size_t crow = 0;        // its element offset in the pool
+      float kscale = 1.f;
       if (u < q_units) {
         row = u / units_row;
         unit = u - row * units_row;
@@ -117,11 +142,27 @@ __global__ void __launch_bounds__(kThreads) rope_scatter_kernel(const RopeParams
         row = uk / units_row;
         unit = uk - row * units_row;
         src = kn + ((size_t)t * p.Hk + row) * p.d;
-        dst = kp + (((size_t)page * p.P + row_in_page) * p.Hk + row) * p.d;
+        crow = (((size_t)page * p.P + row_in_page) * p.Hk + row) * p.d;
+        dst = kp + crow;
+        if constexpr (kFp8) {
+          to_cache = true;
+          kscale = __ldg(p.k_scale + row);
+        }
       }
+      // V elements at channel `off` of the row: to the output dtype, or to e4m3 codes.
+      auto put = [&](int off, const float* x) {
+        if (kFp8 && to_cache) store_e4m3<V>(kp8 + crow + off, x, kscale);
+        else store16(dst + off, x);
+      };
       if (unit >= rot_units) {  // channels >= rotary_dim: copy
         const int off = p.R + (unit - rot_units) * V;
-        *reinterpret_cast<uint4*>(dst + off) = *reinterpret_cast<const uint4*>(src + off);
+        if (kFp8 && to_cache) {
+          float x[V];
+          load16(src + off, x);
+          put(off, x);
+        } else {
+          *reinterpret_cast<uint4*>(dst + off) = *reinterpret_cast<const uint4*>(src + off);
+        }
         continue;
       }
       if (!pos_ok) continue;
@@ -158,7 +199,7 @@ __global__ void __launch_bounds__(kThreads) rope_scatter_kernel(const RopeParams
           x[2 * k] = fmaf(a, c, -bb * s);
           x[2 * k + 1] = fmaf(bb, c, a * s);
         }
-        store16(dst + 2 * j0, x);
+        put(2 * j0, x);
       } else {
         float x1[V], x2[V];
         load16(src + j0, x1);
@@ -169,8 +210,8 @@ __global__ void __launch_bounds__(kThreads) rope_scatter_kernel(const RopeParams
           x1[k] = fmaf(a, c, -bb * s);
           x2[k] = fmaf(bb, c, a * s);
         }
-        store16(dst + j0, x1);
-        store16(dst + half + j0, x2);
+        put(j0, x1);
+        put(half + j0, x2);
       }
     } else {  // V rows: copy into the cache slot
       if (!page_ok) continue;
@@ -178,8 +219,14 @@ __global__ void __launch_bounds__(kThreads) rope_scatter_kernel(const RopeParams
       const int row = uv / (p.d / V);
       const int off = (uv - row * (p.d / V)) * V;
       src = vn + ((size_t)t * p.Hk + row) * p.d + off;
-      dst = vp + (((size_t)page * p.P + row_in_page) * p.Hk + row) * p.d + off;
-      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+      const size_t crow = (((size_t)page * p.P + row_in_page) * p.Hk + row) * p.d + off;
+      if constexpr (kFp8) {
+        float x[V];
+        load16(src, x);
+        store_e4m3<V>(vp8 + crow, x, __ldg(p.v_scale + row));
+      } else {
+        *reinterpret_cast<uint4*>(vp + crow) = *reinterpret_cast<const uint4*>(src);
+      }
     }
   }
 }
@@ -214,12 +261,23 @@ cudaError_t launch_rope(const RopeParams& p, rpk_dtype dtype, bool interleaved,
   RopeParams q = p;
   q.tokens_per_cta = p.T >= 8 * 148 * kTokens ? kTokens : 1;
   dim3 grid((p.T + q.tokens_per_cta - 1) / q.tokens_per_cta), block(kThreads);
+  auto go = [&](auto kernel) { kernel<<<grid, block, 0, stream>>>(q); };
   if (dtype == RPK_BF16) {
-    if (interleaved) rope_scatter_kernel<__nv_bfloat16, true><<<grid, block, 0, stream>>>(q);
-    else rope_scatter_kernel<__nv_bfloat16, false><<<grid, block, 0, stream>>>(q);
+    if (p.cache_fp8) {
+      if (interleaved) go(rope_scatter_kernel<__nv_bfloat16, true, true>);
+      else go(rope_scatter_kernel<__nv_bfloat16, false, true>);
+    } else {
+      if (interleaved) go(rope_scatter_kernel<__nv_bfloat16, true, false>);
+      else go(rope_scatter_kernel<__nv_bfloat16, false, false>);
+    }
   } else {
-    if (interleaved) rope_scatter_kernel<float, true><<<grid, block, 0, stream>>>(q);
-    else rope_scatter_kernel<float, false><<<grid, block, 0, stream>>>(q);
+    if (p.cache_fp8) {
+      if (interleaved) go(rope_scatter_kernel<float, true, true>);
+      else go(rope_scatter_kernel<float, false, true>);
+    } else {
+      if (interleaved) go(rope_scatter_kernel<float, true, false>);
+      else go(rope_scatter_kernel<float, false, false>);
+    }
   }
   return cudaGetLastError();
 }

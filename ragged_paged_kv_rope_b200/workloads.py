@@ -21,6 +21,12 @@ Values are drawn as float32 N(0, 1) with numpy's PCG64 and narrowed to
 bfloat16 by torch's own conversion (round to nearest, ties to even) where the
 workload is bf16. Slots of the page pool that hold no token are filled with a
 NaN sentinel so that any read of them by a kernel shows up in the result.
+
+With ``cache_dtype="e4m3"`` the pools hold e4m3 codes: one fp32 scale per KV
+head for K and one for V, drawn uniformly in [1/64, 1/32] from a separate
+seeded stream, and the tokens already in the cache are stored as torch's
+float8_e4m3fn conversion of value / scale (the new tokens are q's dtype and
+reach the cache through the kernels).
 """
 
 from __future__ import annotations
@@ -34,6 +40,7 @@ import torch
 
 BF16_SENTINEL_BITS = 0x7FC1          # a quiet NaN with a payload
 F32_SENTINEL_BITS = 0x7FC01234       # a quiet NaN with a payload
+E4M3_SENTINEL_BITS = 0x7F            # the e4m3 NaN code
 
 
 @dataclass(frozen=True)
@@ -58,6 +65,7 @@ class Spec:
     mrope_section: tuple | None = None
     rms_norm: bool = False           # RMS-normalise q, k_new and cached K per head
     spare_pages: int = 8
+    cache_dtype: str | None = None   # None: dtype; "e4m3": codes of value / per-head scale
     description: str = ""
 
     @property
@@ -127,6 +135,8 @@ class Workload:
     k_pages: torch.Tensor
     v_pages: torch.Tensor
     extra: dict = field(default_factory=dict)
+    k_scale: np.ndarray | None = None   # fp32 [n_kv_heads] of an e4m3 cache
+    v_scale: np.ndarray | None = None
 
     @property
     def total_tokens(self) -> int:
@@ -182,11 +192,31 @@ def sentinel_pool(num_pages: int, page_size: int, n_kv_heads: int, head_dim: int
                   dtype: str) -> torch.Tensor:
     """A pool whose every slot holds the NaN sentinel."""
     shape = (num_pages, page_size, n_kv_heads, head_dim)
+    if dtype == "e4m3":
+        return torch.full(shape, E4M3_SENTINEL_BITS, dtype=torch.uint8).view(torch.float8_e4m3fn)
     if dtype == "bf16":
         bits = torch.full(shape, BF16_SENTINEL_BITS, dtype=torch.int16)
         return bits.view(torch.bfloat16)
     bits = torch.full(shape, F32_SENTINEL_BITS, dtype=torch.int32)
     return bits.view(torch.float32)
+
+
+def _cache_scales(sp: Spec, seed: int):
+    """Per-KV-head (k_scale, v_scale) of an e4m3 cache, else (None, None)."""
+    if sp.cache_dtype != "e4m3":
+        return None, None
+    srng = np.random.default_rng([seed, 0xE4])
+    ks = srng.uniform(1.0 / 64, 1.0 / 32, size=sp.n_kv_heads).astype(np.float32)
+    vs = srng.uniform(1.0 / 64, 1.0 / 32, size=sp.n_kv_heads).astype(np.float32)
+    return ks, vs
+
+
+def _cache_rows(x: np.ndarray, sp: Spec, scale: np.ndarray | None) -> torch.Tensor:
+    """Rows [n, Hk, d] as stored in the cache: q's dtype, or e4m3 codes of x / scale."""
+    if scale is None:
+        return _narrow(x, sp.dtype)
+    q = (x / scale[None, :, None]).astype(np.float32)
+    return torch.from_numpy(np.ascontiguousarray(q)).to(torch.float8_e4m3fn)
 
 
 def make(spec_or_name, seed: int = 0, **overrides) -> Workload:
@@ -242,8 +272,9 @@ def make(spec_or_name, seed: int = 0, **overrides) -> Workload:
         q = _rms_normalise(q)
         k_new = _rms_normalise(k_new)
 
-    k_pages = sentinel_pool(num_pages, P, Hk, d, sp.dtype)
-    v_pages = sentinel_pool(num_pages, P, Hk, d, sp.dtype)
+    ks, vs = _cache_scales(sp, seed)
+    k_pages = sentinel_pool(num_pages, P, Hk, d, sp.cache_dtype or sp.dtype)
+    v_pages = sentinel_pool(num_pages, P, Hk, d, sp.cache_dtype or sp.dtype)
     # Tokens already in the cache: N(0, 1) in slots [0, cache_len) of each sequence.
     for b in range(B):
         n = int(cache_lens[b])
@@ -253,8 +284,8 @@ def make(spec_or_name, seed: int = 0, **overrides) -> Workload:
         vc = _normal(rng, (n, Hk, d))
         if sp.rms_norm:
             kc = _rms_normalise(kc)
-        kc_t = _narrow(kc, sp.dtype)
-        vc_t = _narrow(vc, sp.dtype)
+        kc_t = _cache_rows(kc, sp, ks)
+        vc_t = _cache_rows(vc, sp, vs)
         for pg in range((n + P - 1) // P):
             page = int(block_table[b, pg])
             rows = min(P, n - pg * P)
@@ -269,7 +300,7 @@ def make(spec_or_name, seed: int = 0, **overrides) -> Workload:
         position_ids=None if position_ids is None else position_ids.astype(np.int32),
         max_position=max_position,
         q=_narrow(q, sp.dtype), k_new=_narrow(k_new, sp.dtype), v_new=_narrow(v_new, sp.dtype),
-        k_pages=k_pages, v_pages=v_pages)
+        k_pages=k_pages, v_pages=v_pages, k_scale=ks, v_scale=vs)
 
 
 def attention_only(sp: Spec, seed: int, q_lens, kv_lens) -> Workload:
@@ -301,8 +332,9 @@ def attention_only(sp: Spec, seed: int, q_lens, kv_lens) -> Workload:
     q = _normal(rng, (T, H, d))
     if sp.rms_norm:
         q = _rms_normalise(q)
-    k_pages = sentinel_pool(num_pages, P, Hk, d, sp.dtype)
-    v_pages = sentinel_pool(num_pages, P, Hk, d, sp.dtype)
+    ks, vs = _cache_scales(sp, seed)
+    k_pages = sentinel_pool(num_pages, P, Hk, d, sp.cache_dtype or sp.dtype)
+    v_pages = sentinel_pool(num_pages, P, Hk, d, sp.cache_dtype or sp.dtype)
     for b in range(B):
         n = int(kv_lens[b])
         if n == 0:
@@ -311,7 +343,7 @@ def attention_only(sp: Spec, seed: int, q_lens, kv_lens) -> Workload:
         vc = _normal(rng, (n, Hk, d))
         if sp.rms_norm:
             kc = _rms_normalise(kc)
-        kc_t, vc_t = _narrow(kc, sp.dtype), _narrow(vc, sp.dtype)
+        kc_t, vc_t = _cache_rows(kc, sp, ks), _cache_rows(vc, sp, vs)
         for pg in range((n + P - 1) // P):
             page = int(block_table[b, pg])
             rows = min(P, n - pg * P)
@@ -325,4 +357,4 @@ def attention_only(sp: Spec, seed: int, q_lens, kv_lens) -> Workload:
         block_table=block_table.astype(np.int32), num_pages=num_pages,
         position_ids=None, max_position=int(kv_lens.max()) if B else 1,
         q=_narrow(q, sp.dtype), k_new=empty, v_new=empty,
-        k_pages=k_pages, v_pages=v_pages)
+        k_pages=k_pages, v_pages=v_pages, k_scale=ks, v_scale=vs)

@@ -54,9 +54,12 @@ class Dev:
 def to_device(wl: W.Workload, device="cuda") -> Dev:
     i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
+    f32 = lambda a: None if a is None else torch.from_numpy(
+        np.ascontiguousarray(a, dtype=np.float32)).to(device)
     cache = R.PagedKVCache(
         k_pages=wl.k_pages.to(device), v_pages=wl.v_pages.to(device),
-        block_table=i32(wl.block_table), cache_lens=i32(wl.cache_lens), error_word=err)
+        block_table=i32(wl.block_table), cache_lens=i32(wl.cache_lens), error_word=err,
+        k_scale=f32(wl.k_scale), v_scale=f32(wl.v_scale))
     return Dev(
         q=wl.q.to(device), k_new=wl.k_new.to(device), v_new=wl.v_new.to(device),
         offsets=i32(wl.q_offsets), cache_lens=i32(wl.cache_lens), kv_lens=i32(wl.kv_lens),

@@ -58,6 +58,8 @@ def cache(**kw):
     s.error_word = None
     s.num_layers = kw.get("num_layers", 0)
     s.layer_idx = kw.get("layer_idx", 0)
+    s.k_scale = kw.get("k_scale", None)
+    s.v_scale = kw.get("v_scale", None)
     return s
 
 
@@ -125,6 +127,26 @@ def test_rope_rejects_cache(L, ckw, status):
 ])
 def test_attention_rejects(L, kw, status):
     assert attn(L, cache(max_pages_per_seq=16), **kw) == status
+
+
+@host_only
+def test_e4m3_cache_needs_both_scales(L):
+    for ks, vs in ((None, FAKE), (FAKE, None), (None, None)):
+        c = cache(cache_dtype=B.RPK_E4M3, k_scale=ks, v_scale=vs, max_pages_per_seq=16)
+        assert rope(L, c) == 1
+        assert attn(L, c) == 1
+
+
+@host_only
+def test_e4m3_cache_takes_bf16_and_f32_tensors_only(L):
+    c = cache(cache_dtype=B.RPK_E4M3, k_scale=FAKE, v_scale=FAKE, max_pages_per_seq=16)
+    assert rope(L, c, dtype=B.RPK_E4M3) == 3       # e4m3 is a cache dtype only
+    assert attn(L, c, dtype=B.RPK_E4M3) == 3
+    assert rope(L, c, R=6, dtype=B.RPK_F32) == 4    # validation continues past the dtype
+    # the no-allocation decode entry point does not take e4m3 caches
+    assert L.ragged_paged_attention_noalloc(
+        C.c_void_p(FAKE), C.c_void_p(FAKE), C.c_void_p(FAKE), C.byref(c), 32, 8, 128,
+        C.c_float(0.1), 0, C.c_void_p(FAKE), 2, 2, 1, 200, B.RPK_BF16, None) == 3
 
 
 @host_only
