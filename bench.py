@@ -287,9 +287,17 @@ class Step:
         sp, wl = self.sp, self.wl
         decode = wl.max_q_len * (sp.n_heads // sp.n_kv_heads) <= 16 and sp.dtype == "bf16"
         if decode:
+            # the library's launch plan: about two waves of CTAs, 8..24 tiles per split
             max_tiles = (wl.max_kv_len + 63) // 64 + 1
-            tps = max(8, (max_tiles + 63) // 64)
-            return 2 + (1 if (max_tiles + tps - 1) // tps > 1 else 0)
+            most = max(8, (max_tiles + 63) // 64)
+            units = max(1, sp.batch * sp.n_kv_heads)
+            sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+            slots = 2 * sms * (2 if sp.head_dim <= 128 else 1)
+            per_unit = max(1, -(-slots // units))
+            tps = -(-max_tiles // per_unit)
+            tps = min(max(tps, most), max(24 if sp.head_dim <= 128 else 16, most))
+            splits = -(-max_tiles // tps)
+            return 2 + (1 if splits > 1 else 0)
         return 2
 
 

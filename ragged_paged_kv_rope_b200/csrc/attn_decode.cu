@@ -37,20 +37,59 @@
 // that brings its largest magnitude into [2^14, 2^15) before the f16
 // narrowing; 2^qs and k_scale join the score scale, v_scale multiplies the
 // merged output. P is f16 (values in [0, 1]).
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace rpk {
 
+namespace {
+// Tiles of the longest band (one extra for a window start inside a tile).
+int32_t band_tiles(int32_t max_kv_len) { return (max_kv_len + kDecodeTile - 1) / kDecodeTile + 1; }
+
+int device_sm_count() {
+  static int n[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (n[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    n[dev] = v;
+  }
+  return n[dev];
+}
+}  // namespace
+
 DecodePlan decode_plan(int32_t max_kv_len) {
-  // Tiles of the longest band (one extra for a window start inside a tile).
-  const int32_t max_tiles = (max_kv_len + kDecodeTile - 1) / kDecodeTile + 1;
+  const int32_t max_tiles = band_tiles(max_kv_len);
   int32_t tps = 8;  // 512 keys per split
   if ((max_tiles + tps - 1) / tps > kDecodeMaxSplits)
     tps = (max_tiles + kDecodeMaxSplits - 1) / kDecodeMaxSplits;
   DecodePlan plan;
   plan.tiles_per_split = tps;
   plan.max_splits = (max_tiles + tps - 1) / tps;
+  return plan;
+}
+
+DecodePlan decode_launch_plan(int32_t max_kv_len, int32_t units, int32_t head_dim) {
+  // Longer splits stream more bytes per CTA for the same start-up and merge,
+  // but a launch needs enough CTAs to fill the GPU: aim at two waves (two CTAs
+  // per SM for head_dim <= 128, one for 256), never go below the sizing plan's
+  // split and never above 24 tiles (16 for head_dim 256), then even out the
+  // splits of the longest band.
+  const DecodePlan most = decode_plan(max_kv_len);
+  const int32_t max_tiles = band_tiles(max_kv_len);
+  const long long slots = 2LL * device_sm_count() * (head_dim <= 128 ? 2 : 1);
+  const long long per_unit = std::max(1LL, (slots + std::max(1, units) - 1) / std::max(1, units));
+  long long tps = (max_tiles + per_unit - 1) / per_unit;
+  const int32_t cap = std::max(head_dim <= 128 ? 24 : 16, most.tiles_per_split);
+  tps = std::min<long long>(std::max<long long>(tps, most.tiles_per_split), cap);
+  const int32_t splits = (int32_t)((max_tiles + tps - 1) / tps);
+  DecodePlan plan;
+  plan.tiles_per_split = std::max(most.tiles_per_split, (max_tiles + splits - 1) / splits);
+  plan.max_splits = (max_tiles + plan.tiles_per_split - 1) / plan.tiles_per_split;
   return plan;
 }
 
@@ -134,7 +173,8 @@ struct DecodeCfg {
   static constexpr int kBoxes = D / 64;                      // 128-byte column boxes per row
   static constexpr int kTileBytes = kDecodeTile * D * 2;     // one of K or V
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = D == 256 ? 2 : (D == 128 ? 3 : 6);
+  // head_dim 256 runs one CTA per SM: three 64 KB stages keep two in flight
+  static constexpr int kStages = D == 256 ? 3 : (D == 128 ? 3 : 6);
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024;  // + alignment slack
   static_assert(kConsumerWarps * 16 * D * 4 <= kStages * kStageBytes, "merge buffer");
 };
@@ -147,7 +187,7 @@ struct DecodeCfg<D, true> {
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = kDecodeTile * D;          // raw codes of K or V
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = D == 256 ? 2 : (D == 128 ? 4 : 8);
+  static constexpr int kStages = D == 256 ? 4 : (D == 128 ? 4 : 8);
   static constexpr int kConvTileBytes = 16 * D * 2;           // 16 rows of f16
   static constexpr int kConvOff = kStages * kStageBytes;
   static constexpr int kSmemBytes = kConvOff + kConsumerWarps * 2 * kConvTileBytes + 1024;

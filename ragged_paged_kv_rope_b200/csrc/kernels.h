@@ -82,7 +82,11 @@ struct DecodePlan {
   int32_t tiles_per_split;
   int32_t max_splits;
 };
+// The plan with the most splits any launch uses (sizes the workspace).
 DecodePlan decode_plan(int32_t max_kv_len);
+// The plan a launch uses for `units` (sequence, KV head) pairs: never more
+// splits than decode_plan.
+DecodePlan decode_launch_plan(int32_t max_kv_len, int32_t units, int32_t head_dim);
 size_t decode_workspace_bytes(int32_t total_q_tokens, int32_t n_heads, int32_t head_dim,
                               int32_t max_kv_len);
 
