@@ -287,15 +287,22 @@ class Step:
         sp, wl = self.sp, self.wl
         decode = wl.max_q_len * (sp.n_heads // sp.n_kv_heads) <= 16 and sp.dtype == "bf16"
         if decode:
-            # the library's launch plan: about two waves of CTAs, 8..24 tiles per split
-            max_tiles = (wl.max_kv_len + 63) // 64 + 1
-            most = max(8, (max_tiles + 63) // 64)
+            # the library's launch plan: one wave when the units fit, else about two
+            # waves of CTAs with 8..24 tiles per split
+            most = max(8, ((wl.max_kv_len + 63) // 64 + 1 + 63) // 64)
+            band = wl.max_kv_len
+            if sp.window > 0:
+                band = min(band, sp.window + wl.max_q_len - 1)
+            max_tiles = (band + 63) // 64 + 1
             units = max(1, sp.batch * sp.n_kv_heads)
             sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
-            slots = 2 * sms * (2 if sp.head_dim <= 128 else 1)
-            per_unit = max(1, -(-slots // units))
-            tps = -(-max_tiles // per_unit)
-            tps = min(max(tps, most), max(24 if sp.head_dim <= 128 else 16, most))
+            wave = sms * (2 if sp.head_dim <= 128 else 1)
+            if units <= wave:
+                tps = max(-(-max_tiles // (wave // units)), most)
+            else:
+                per_unit = max(1, -(-2 * wave // units))
+                tps = -(-max_tiles // per_unit)
+                tps = min(max(tps, most), max(24 if sp.head_dim <= 128 else 16, most))
             splits = -(-max_tiles // tps)
             return 2 + (1 if splits > 1 else 0)
         return 2

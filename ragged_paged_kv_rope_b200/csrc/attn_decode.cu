@@ -73,19 +73,37 @@ DecodePlan decode_plan(int32_t max_kv_len) {
   return plan;
 }
 
-DecodePlan decode_launch_plan(int32_t max_kv_len, int32_t units, int32_t head_dim) {
+DecodePlan decode_launch_plan(int32_t max_kv_len, int32_t units, int32_t head_dim, int32_t window,
+                              int32_t max_q_len, int32_t sinks) {
   // Longer splits stream more bytes per CTA for the same start-up and merge,
-  // but a launch needs enough CTAs to fill the GPU: aim at two waves (two CTAs
-  // per SM for head_dim <= 128, one for 256), never go below the sizing plan's
-  // split and never above 24 tiles (16 for head_dim 256), then even out the
-  // splits of the longest band.
+  // but a launch needs enough CTAs to fill the GPU, and a last wave with few
+  // CTAs cannot keep HBM busy. When every (sequence, KV head) unit fits in one
+  // wave (two CTAs per SM for head_dim <= 128, one for 256), the splits fill
+  // exactly one wave. Otherwise aim at two waves and keep splits between the
+  // sizing plan's and 24 tiles (16 for head_dim 256). Then even out the splits
+  // of the longest band.
   const DecodePlan most = decode_plan(max_kv_len);
-  const int32_t max_tiles = band_tiles(max_kv_len);
-  const long long slots = 2LL * device_sm_count() * (head_dim <= 128 ? 2 : 1);
-  const long long per_unit = std::max(1LL, (slots + std::max(1, units) - 1) / std::max(1, units));
-  long long tps = (max_tiles + per_unit - 1) / per_unit;
-  const int32_t cap = std::max(head_dim <= 128 ? 24 : 16, most.tiles_per_split);
-  tps = std::min<long long>(std::max<long long>(tps, most.tiles_per_split), cap);
+  // Keys a sequence's rows can see: under a window at most window + max_q_len - 1
+  // (plus the attention sinks' tiles), else all max_kv_len.
+  long long band = max_kv_len;
+  if (window > 0)
+    band = std::min<long long>(band, (long long)window + std::max(0, max_q_len - 1) +
+                                         (long long)(sinks + kDecodeTile - 1) / kDecodeTile *
+                                             kDecodeTile);
+  const int32_t max_tiles = band_tiles((int32_t)band);
+  const long long wave = (long long)device_sm_count() * (head_dim <= 128 ? 2 : 1);
+  const long long n_units = std::max(1, units);
+  long long tps;
+  if (n_units <= wave) {
+    const long long per_unit = wave / n_units;
+    tps = std::max<long long>((max_tiles + per_unit - 1) / per_unit, most.tiles_per_split);
+  } else {
+    const long long slots = 2 * wave;
+    const long long per_unit = std::max(1LL, (slots + n_units - 1) / n_units);
+    tps = (max_tiles + per_unit - 1) / per_unit;
+    const int32_t cap = std::max(head_dim <= 128 ? 24 : 16, most.tiles_per_split);
+    tps = std::min<long long>(std::max<long long>(tps, most.tiles_per_split), cap);
+  }
   const int32_t splits = (int32_t)((max_tiles + tps - 1) / tps);
   DecodePlan plan;
   plan.tiles_per_split = std::max(most.tiles_per_split, (max_tiles + splits - 1) / splits);

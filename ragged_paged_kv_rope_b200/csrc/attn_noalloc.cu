@@ -135,7 +135,8 @@ extern "C" rpk_status ragged_paged_attention_noalloc(
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
 
   // Partials layout inside the scratch: O [splits, T, H, d] fp32, then (m, l).
-  const rpk::DecodePlan plan = rpk::decode_launch_plan(max_kv_len, batch * n_kv_heads, head_dim);
+  const rpk::DecodePlan plan = rpk::decode_launch_plan(max_kv_len, batch * n_kv_heads, head_dim,
+                                                       p.window, max_q_len, 0);
   const size_t rows = (size_t)plan.max_splits * total_q_tokens * n_heads;
   const size_t o_bytes = (rows * head_dim * sizeof(float) + 255) & ~size_t(255);
   rpk::DecodeWorkspace ws;

@@ -86,7 +86,8 @@ struct DecodePlan {
 DecodePlan decode_plan(int32_t max_kv_len);
 // The plan a launch uses for `units` (sequence, KV head) pairs: never more
 // splits than decode_plan.
-DecodePlan decode_launch_plan(int32_t max_kv_len, int32_t units, int32_t head_dim);
+DecodePlan decode_launch_plan(int32_t max_kv_len, int32_t units, int32_t head_dim, int32_t window,
+                              int32_t max_q_len, int32_t sinks);
 size_t decode_workspace_bytes(int32_t total_q_tokens, int32_t n_heads, int32_t head_dim,
                               int32_t max_kv_len);
 
