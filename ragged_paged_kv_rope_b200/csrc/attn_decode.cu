@@ -168,6 +168,15 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
+// Transpose of an 8x8 matrix of 16-bit elements held one row pair per lane
+// (lane t: row t / 4, columns 2 (t % 4), +1): lane t receives the same
+// positions of the transposed matrix.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 // D += A(16x16 bf16, row) * B(16x8 bf16, col), fp32 accumulators.
 __device__ __forceinline__ void mma_bf16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -214,10 +223,9 @@ struct DecodeCfg<D, true> {
 
 // Two CTAs share an SM when each warp holds at most 168 registers: ten warps
 // put three on some sub-partition, whose register file is a quarter of the
-// SM's (3 * 168 * 32 <= 16384). The bf16 kernel needs no cap for that; the
-// e4m3 kernel's widening would otherwise take it past the limit.
-template <int D, bool kFp8>
-__global__ void __launch_bounds__(kThreads, 1) __maxnreg__(kFp8 && D <= 128 ? 168 : 255)
+// SM's (3 * 168 * 32 <= 16384). head_dim 256 runs one CTA per SM anyway.
+template <int D, bool kFp8, int NT>
+__global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
     attn_decode_kernel(const AttnParams p, const __grid_constant__ CUtensorMap k_map,
                        const __grid_constant__ CUtensorMap v_map, const DecodePlan plan,
                        const DecodeWorkspace ws) {
@@ -320,32 +328,40 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(kFp8 && D <= 128 ? 16
   }
 
   // ------------------------------------------------------------- consumers
+  // Scores are computed transposed, S^T = K Q^T: this warp's 16 keys are the
+  // MMA's M and the group's rows its N (8 per n-tile, NT n-tiles), so a group
+  // of at most 8 rows fills one m16n8k16 per 16 channels. O^T = V^T P^T the
+  // same way, P^T going from the score accumulators to the B operand through
+  // an 8x8 transpose (movmatrix). Lane (g, c) = (lane / 4, lane % 4) holds
+  // keys g and g + 8 of rows nt * 8 + 2c and 2c + 1.
   const int g = lane >> 2, c = lane & 3;
-  // Row ids of this lane's two accumulator rows and their visible key ranges.
-  int row_lo[2], row_hi[2];
-  bool row_ok[2];
+  int row_lo[NT][2], row_hi[NT][2];
+  bool row_ok[NT][2];
 #pragma unroll
-  for (int hr = 0; hr < 2; ++hr) {
-    const int rr = g + hr * 8;
-    row_ok[hr] = rr < rows;
-    const int tok = rr / p.G;                 // token index in the sequence
-    const int pos = tok + k_len - q_len;      // its position
-    row_hi[hr] = pos;
-    row_lo[hr] = p.window > 0 ? pos - p.window + 1 : 0;
-  }
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int rr = nt * 8 + 2 * c + j;
+      row_ok[nt][j] = rr < rows;
+      const int tok = rr / p.G;                 // token index in the sequence
+      const int pos = tok + k_len - q_len;      // its position
+      row_hi[nt][j] = pos;
+      row_lo[nt][j] = p.window > 0 ? pos - p.window + 1 : 0;
+    }
 
-  // Q as the A operand (16 rows x D), rows past `rows` are zero.
-  uint32_t qa[D / 16][4];
+  // Q^T as the B operand: for channel step ks and n-tile nt, b0 = q[row][16ks + 2c, +1]
+  // and b1 = q[row][16ks + 8 + 2c, +1] of row nt * 8 + g; rows past `rows` are zero.
+  uint32_t qb[D / 16][NT][2];
   {
-    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.q);
+    const __nv_bfloat16* qbase = static_cast<const __nv_bfloat16*>(p.q);
 #pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      const int rr = g + hr * 8;
+    for (int nt = 0; nt < NT; ++nt) {
+      const int rr = nt * 8 + g;
       const __nv_bfloat16* qrow = nullptr;
       if (rr < rows) {
         const int t = q0 + rr / p.G;
         const int h = kvh * p.G + rr % p.G;
-        qrow = qb + ((size_t)t * p.H + h) * D;
+        qrow = qbase + ((size_t)t * p.H + h) * D;
       }
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
@@ -354,8 +370,8 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(kFp8 && D <= 128 ? 16
           lo = *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * c);
           hi = *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * c);
         }
-        qa[ks][hr] = lo;       // a0 (row g) / a1 (row g+8)
-        qa[ks][2 + hr] = hi;   // a2 / a3
+        qb[ks][nt][0] = lo;
+        qb[ks][nt][1] = hi;
       }
     }
   }
@@ -368,10 +384,12 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(kFp8 && D <= 128 ? 16
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks)
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(&qa[ks][k]);
-        mx = fmaxf(mx, fmaxf(fabsf(__low2float(v2)), fabsf(__high2float(v2))));
-      }
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(&qb[ks][nt][k]);
+          mx = fmaxf(mx, fmaxf(fabsf(__low2float(v2)), fabsf(__high2float(v2))));
+        }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     int qs = 0;
@@ -380,19 +398,31 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(kFp8 && D <= 128 ? 16
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks)
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(&qa[ks][k]);
-        qa[ks][k] = pack_f16x2(__low2float(v2) * down, __high2float(v2) * down);
-      }
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(&qb[ks][nt][k]);
+          qb[ks][nt][k] = pack_f16x2(__low2float(v2) * down, __high2float(v2) * down);
+        }
     sl2 = p.scale_log2 * __ldg(p.k_scale + kvh) * __int_as_float((127 + qs) << 23);
     v_mul = __ldg(p.v_scale + kvh);
   }
 
-  float o[D / 8][4];
+  // O^T accumulators per 16-channel step and n-tile: (channel g, row 2c),
+  // (g, 2c + 1), (g + 8, 2c), (g + 8, 2c + 1).
+  float o[D / 16][NT][4];
 #pragma unroll
-  for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-  float m_run[2] = {-INFINITY, -INFINITY};
-  float l_run[2] = {0.f, 0.f};
+  for (int dc = 0; dc < D / 16; ++dc)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) o[dc][nt][0] = o[dc][nt][1] = o[dc][nt][2] = o[dc][nt][3] = 0.f;
+  float m_run[NT][2], l_run[NT][2];  // l_run: this lane's keys only, summed at the end
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      m_run[nt][j] = -INFINITY;
+      l_run[nt][j] = 0.f;
+    }
   bool ok = true;
 
   for (int i = 0; i < n_tiles; ++i) {
@@ -457,97 +487,102 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(kFp8 && D <= 128 ? 16
       __syncwarp();
     }
 
-    // S = Q K^T for 16 keys: two n-tiles of 8 keys.
-    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    // S^T = K Q^T: A = this warp's 16 keys (rows) x 16 channels per step.
+    float sc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
-      // matrices: (keys 0-7, d lo), (keys 0-7, d hi), (keys 8-15, d lo), (keys 8-15, d hi)
+      // matrices: (keys 0-7, d lo), (keys 8-15, d lo), (keys 0-7, d hi), (keys 8-15, d hi)
       const int mi = lane >> 3;
-      const int krow = wrow0 + (mi >> 1) * 8 + (lane & 7);
-      const int chunk = ks * 2 + (mi & 1);
+      const int krow = wrow0 + (mi & 1) * 8 + (lane & 7);
+      const int chunk = ks * 2 + (mi >> 1);
       const uint32_t addr = kbase + (chunk >> 3) * kBoxStride + swz128(krow, chunk & 7);
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4(addr, b0, b1, b2, b3);
-      if constexpr (kFp8) {
-        mma_f16(sc[0], qa[ks], b0, b1);
-        mma_f16(sc[1], qa[ks], b2, b3);
-      } else {
-        mma_bf16(sc[0], qa[ks], b0, b1);
-        mma_bf16(sc[1], qa[ks], b2, b3);
+      uint32_t a[4];
+      ldsm_x4(addr, a[0], a[1], a[2], a[3]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        if constexpr (kFp8) mma_f16(sc[nt], a, qb[ks][nt][0], qb[ks][nt][1]);
+        else mma_bf16(sc[nt], a, qb[ks][nt][0], qb[ks][nt][1]);
       }
     }
 
-    // Mask, scale to log2 units, online-softmax update of both rows.
-    float tmax[2] = {-INFINITY, -INFINITY};
+    // Mask, scale to log2 units, online-softmax update of this lane's rows;
+    // the 16 keys of a row sit on the 8 lanes that share c.
+    float tmax[NT][2];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) tmax[nt][j] = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int hr = e >> 1;
-        const int key = key0 + nt * 8 + 2 * c + (e & 1);
-        const bool vis =
-            row_ok[hr] && key <= row_hi[hr] && (key >= row_lo[hr] || key < p.sinks);
+        const int j = e & 1;
+        const int key = key0 + g + (e >> 1) * 8;
+        const bool vis = row_ok[nt][j] && key <= row_hi[nt][j] &&
+                         (key >= row_lo[nt][j] || key < p.sinks);
         const float v = vis ? sc[nt][e] * sl2 : -INFINITY;
         sc[nt][e] = v;
-        tmax[hr] = fmaxf(tmax[hr], v);
+        tmax[nt][j] = fmaxf(tmax[nt][j], v);
       }
-    float alpha[2], m_use[2];
+    float alpha[NT][2], m_use[NT][2];
 #pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      tmax[hr] = fmaxf(tmax[hr], __shfl_xor_sync(0xffffffffu, tmax[hr], 1));
-      tmax[hr] = fmaxf(tmax[hr], __shfl_xor_sync(0xffffffffu, tmax[hr], 2));
-      const float m_new = fmaxf(m_run[hr], tmax[hr]);
-      m_use[hr] = m_new == -INFINITY ? 0.f : m_new;
-      alpha[hr] = fast_exp2(m_run[hr] - m_use[hr]);
-      m_run[hr] = m_new;
-    }
-    float rsum[2] = {0.f, 0.f};
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int hr = e >> 1;
-        const float w = fast_exp2(sc[nt][e] - m_use[hr]);
-        sc[nt][e] = w;
-        rsum[hr] += w;
+      for (int j = 0; j < 2; ++j) {
+        float t = tmax[nt][j];
+        t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 4));
+        t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 8));
+        t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, 16));
+        const float m_new = fmaxf(m_run[nt][j], t);
+        m_use[nt][j] = m_new == -INFINITY ? 0.f : m_new;
+        alpha[nt][j] = fast_exp2(m_run[nt][j] - m_use[nt][j]);
+        m_run[nt][j] = m_new;
       }
+    uint32_t pb[NT][2];  // P^T as the B operand of O^T = V^T P^T
 #pragma unroll
-    for (int hr = 0; hr < 2; ++hr) l_run[hr] = l_run[hr] * alpha[hr] + rsum[hr];
+    for (int nt = 0; nt < NT; ++nt) {
+      float w[4];
 #pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      o[n][0] *= alpha[0]; o[n][1] *= alpha[0];
-      o[n][2] *= alpha[1]; o[n][3] *= alpha[1];
-    }
-
-    // O += P V: P (16 rows x 16 keys) as the A operand straight from registers.
-    uint32_t pa[4];
-    if constexpr (kFp8) {
-      pa[0] = pack_f16x2(sc[0][0], sc[0][1]);
-      pa[1] = pack_f16x2(sc[0][2], sc[0][3]);
-      pa[2] = pack_f16x2(sc[1][0], sc[1][1]);
-      pa[3] = pack_f16x2(sc[1][2], sc[1][3]);
-    } else {
-      pa[0] = pack_bf16x2(sc[0][0], sc[0][1]);
-      pa[1] = pack_bf16x2(sc[0][2], sc[0][3]);
-      pa[2] = pack_bf16x2(sc[1][0], sc[1][1]);
-      pa[3] = pack_bf16x2(sc[1][2], sc[1][3]);
-    }
+      for (int e = 0; e < 4; ++e) w[e] = fast_exp2(sc[nt][e] - m_use[nt][e & 1]);
 #pragma unroll
-    for (int dn = 0; dn < D / 16; ++dn) {
-      // matrices (transposed): (keys 0-7, d n0), (keys 8-15, d n0), (keys 0-7, d n0+8),
-      // (keys 8-15, d n0+8)
-      const int mi = lane >> 3;
-      const int vrow = wrow0 + (mi & 1) * 8 + (lane & 7);
-      const int chunk = dn * 2 + (mi >> 1);
-      const uint32_t addr = vbase + (chunk >> 3) * kBoxStride + swz128(vrow, chunk & 7);
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(addr, b0, b1, b2, b3);
+      for (int j = 0; j < 2; ++j) l_run[nt][j] = l_run[nt][j] * alpha[nt][j] + (w[j] + w[2 + j]);
+      // P^T blocks (keys 0-7 and 8-15) x (rows 2c, 2c+1), transposed to rows x keys.
+      uint32_t blk0, blk1;
       if constexpr (kFp8) {
-        mma_f16(o[2 * dn], pa, b0, b1);
-        mma_f16(o[2 * dn + 1], pa, b2, b3);
+        blk0 = pack_f16x2(w[0], w[1]);
+        blk1 = pack_f16x2(w[2], w[3]);
       } else {
-        mma_bf16(o[2 * dn], pa, b0, b1);
-        mma_bf16(o[2 * dn + 1], pa, b2, b3);
+        blk0 = pack_bf16x2(w[0], w[1]);
+        blk1 = pack_bf16x2(w[2], w[3]);
+      }
+      pb[nt][0] = movmatrix_trans(blk0);
+      pb[nt][1] = movmatrix_trans(blk1);
+    }
+#pragma unroll
+    for (int dc = 0; dc < D / 16; ++dc)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        o[dc][nt][0] *= alpha[nt][0]; o[dc][nt][1] *= alpha[nt][1];
+        o[dc][nt][2] *= alpha[nt][0]; o[dc][nt][3] *= alpha[nt][1];
+      }
+
+    // O^T += V^T P^T: A = V^T (16 channels x 16 keys) by a transposing load.
+#pragma unroll
+    for (int dc = 0; dc < D / 16; ++dc) {
+      // matrices (transposed): (keys 0-7, d lo), (keys 0-7, d hi), (keys 8-15, d lo),
+      // (keys 8-15, d hi)
+      const int mi = lane >> 3;
+      const int vrow = wrow0 + (mi >> 1) * 8 + (lane & 7);
+      const int chunk = dc * 2 + (mi & 1);
+      const uint32_t addr = vbase + (chunk >> 3) * kBoxStride + swz128(vrow, chunk & 7);
+      uint32_t a[4];
+      ldsm_x4_t(addr, a[0], a[1], a[2], a[3]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        if constexpr (kFp8) mma_f16(o[dc][nt], a, pb[nt][0], pb[nt][1]);
+        else mma_bf16(o[dc][nt], a, pb[nt][0], pb[nt][1]);
       }
     }
 
@@ -564,34 +599,44 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(kFp8 && D <= 128 ? 16
 
   // ----------------------------------------------- merge the four warps' states
 #pragma unroll
-  for (int hr = 0; hr < 2; ++hr) {
-    l_run[hr] += __shfl_xor_sync(0xffffffffu, l_run[hr], 1);
-    l_run[hr] += __shfl_xor_sync(0xffffffffu, l_run[hr], 2);
-  }
-  if (c == 0) {
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      m_part[warp][g + hr * 8] = m_run[hr];
-      l_part[warp][g + hr * 8] = l_run[hr];
+    for (int j = 0; j < 2; ++j) {
+      float l = l_run[nt][j];
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      l_run[nt][j] = l;
     }
+  if (g == 0) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        m_part[warp][nt * 8 + 2 * c + j] = m_run[nt][j];
+        l_part[warp][nt * 8 + 2 * c + j] = l_run[nt][j];
+      }
   }
   // All consumers are past the tile loop, so every stage's TMA has landed and
   // the ring can be reused as the merge buffer.
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
   float* obuf = reinterpret_cast<float*>(smem);  // [warp][16][D]
 #pragma unroll
-  for (int hr = 0; hr < 2; ++hr) {
-    const int rr = g + hr * 8;
-    float mx = -INFINITY;
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) mx = fmaxf(mx, m_part[w][rr]);
-    const float f = m_run[hr] == -INFINITY ? 0.f : fast_exp2(m_run[hr] - mx);
+    for (int j = 0; j < 2; ++j) {
+      const int rr = nt * 8 + 2 * c + j;
+      float mx = -INFINITY;
 #pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      float2 v = make_float2(o[n][2 * hr] * f, o[n][2 * hr + 1] * f);
-      *reinterpret_cast<float2*>(obuf + ((size_t)warp * 16 + rr) * D + n * 8 + 2 * c) = v;
+      for (int w = 0; w < kConsumerWarps; ++w) mx = fmaxf(mx, m_part[w][rr]);
+      const float f = m_run[nt][j] == -INFINITY ? 0.f : fast_exp2(m_run[nt][j] - mx);
+      float* orow = obuf + ((size_t)warp * 16 + rr) * D + g;
+#pragma unroll
+      for (int dc = 0; dc < D / 16; ++dc) {
+        orow[dc * 16] = o[dc][nt][j] * f;
+        orow[dc * 16 + 8] = o[dc][nt][2 + j] * f;
+      }
     }
-  }
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 
   const bool single = ss.n_splits == 1;
@@ -681,13 +726,14 @@ template <int D, bool kFp8>
 cudaError_t launch_d(const AttnParams& p, const CUtensorMap& k_map, const CUtensorMap& v_map,
                      const DecodePlan& plan, const DecodeWorkspace& ws, cudaStream_t stream) {
   using Cfg = DecodeCfg<D, kFp8>;
-  cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<D, kFp8>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Cfg::kSmemBytes);
+  // One n-tile of 8 rows when the group's rows fit, else two.
+  auto kernel = p.max_q_len * p.G <= 8 ? attn_decode_kernel<D, kFp8, 1>
+                                       : attn_decode_kernel<D, kFp8, 2>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.max_splits, p.Hk, p.batch);
-  attn_decode_kernel<D, kFp8><<<grid, kThreads, Cfg::kSmemBytes, stream>>>(p, k_map, v_map, plan,
-                                                                          ws);
+  kernel<<<grid, kThreads, Cfg::kSmemBytes, stream>>>(p, k_map, v_map, plan, ws);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (plan.max_splits > 1) {

@@ -89,6 +89,7 @@ EDGE = [
     ("head_dim 64", {"head_dim": 64, "rotary_dim": 64}, [1, 9], [70, 30], 0),
     ("head_dim 256", {"head_dim": 256, "rotary_dim": 128}, [1, 2], [513, 200], 0),
     ("chunked prefill rows", {}, [3, 2], [100, 5], 0),
+    ("head_dim 256, 12 rows", {"head_dim": 256, "rotary_dim": 128}, [3, 2], [300, 77], 0),
 ]
 
 

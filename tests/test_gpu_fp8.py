@@ -142,6 +142,20 @@ def test_decode_over_e4m3_cache_head_dims(d):
     check_attention(out.cpu(), ref, "bf16", f"d={d} e4m3")
 
 
+@pytest.mark.parametrize("d", [128, 256])
+def test_decode_over_e4m3_cache_more_rows(d):
+    # 3 and 4 tokens of a group of 4: 12 and 16 rows per KV head (two n-tiles)
+    sp = W.spec("llama3_8b_decode", cache_dtype="e4m3", head_dim=d, rotary_dim=d, batch=3)
+    wl = W.attention_only(sp, 6, [3, 4, 1], [200, 700, 64])
+    dev = to_device(wl)
+    out = gpu_attention(wl, dev, dev.q)
+    torch.cuda.synchronize()
+    assert int(dev.error_word.item()) == 0
+    ref = O.attention(wl.q, wl.q_offsets, wl.kv_lens, wl.k_pages, wl.v_pages, wl.block_table,
+                      sp.n_kv_heads, sp.softmax_scale, 0, k_scale=wl.k_scale, v_scale=wl.v_scale)
+    check_attention(out.cpu(), ref, "bf16", f"d={d} e4m3, 12 and 16 rows")
+
+
 def test_decode_e4m3_large_and_small_queries():
     # Q far outside f16's range in both directions: the kernel's power-of-two
     # pre-scale keeps the scores right.
