@@ -36,7 +36,12 @@
 // same ldmatrix / mma.sync code in f16. Q is scaled by a power of two 2^-qs
 // that brings its largest magnitude into [2^14, 2^15) before the f16
 // narrowing; 2^qs and k_scale join the score scale, v_scale multiplies the
-// merged output. P is f16 (values in [0, 1]).
+// merged output. P is f16 (values in [0, 1]). For head_dim >= 128 the raw
+// stages are written with the 128-byte swizzle, only V is widened, and the
+// score MMAs take K straight from the codes: lane (g, c) loads the four codes
+// of channels 4c .. 4c+3 of each 16-channel step as the A operand's logical
+// channels 2c, 2c+1, 2c+8, 2c+9, and Q's B operand uses the same order (a
+// dot product does not depend on the order of its channels).
 #include <algorithm>
 
 #include "common.cuh"
@@ -231,6 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
                        const DecodeWorkspace ws) {
   using Cfg = DecodeCfg<D, kFp8>;
   constexpr int S = Cfg::kStages;
+  // e4m3 with head_dim >= 128: K fragments straight from the swizzled raw codes
+  constexpr bool kKDirect = kFp8 && D >= 128;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t full_bar[S], empty_bar[S];
   __shared__ float m_part[kConsumerWarps][kDecodeMaxRows];
@@ -304,7 +311,15 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
             continue;
           }
           const int grow = page * p.P + (key - pi * p.P);
-          if constexpr (kFp8) {
+          if constexpr (kKDirect) {
+#pragma unroll
+            for (int bx = 0; bx < D / 128; ++bx) {
+              tma_load_3d(k_stage(s) + bx * (kDecodeTile * 128) + r * 128, &k_map, bx * 128, kvh,
+                          grow, &full_bar[s]);
+              tma_load_3d(v_stage(s) + bx * (kDecodeTile * 128) + r * 128, &v_map, bx * 128, kvh,
+                          grow, &full_bar[s]);
+            }
+          } else if constexpr (kFp8) {
             tma_load_3d(k_stage(s) + r * D, &k_map, 0, kvh, grow, &full_bar[s]);
             tma_load_3d(v_stage(s) + r * D, &v_map, 0, kvh, grow, &full_bar[s]);
           } else {
@@ -367,8 +382,12 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
       for (int ks = 0; ks < D / 16; ++ks) {
         uint32_t lo = 0, hi = 0;
         if (qrow) {
-          lo = *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * c);
-          hi = *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * c);
+          // logical channels (2c, 2c+1) and (2c+8, 2c+9) of the step; with K
+          // read straight from the codes they sit at 4c, 4c+1 and 4c+2, 4c+3
+          const int c_lo = kKDirect ? 4 * c : 2 * c;
+          const int c_hi = kKDirect ? 4 * c + 2 : 8 + 2 * c;
+          lo = *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + c_lo);
+          hi = *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + c_hi);
         }
         qb[ks][nt][0] = lo;
         qb[ks][nt][1] = hi;
@@ -431,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
     const int key0 = ss.tile_at(v_begin + i) * kDecodeTile + warp * 16;  // this warp's 16 keys
     uint32_t kbase = smem_u32(k_stage(s));
     uint32_t vbase = smem_u32(v_stage(s));
-    int wrow0 = warp * 16;  // row of this warp's first key inside the tile
+    const int wrow0 = warp * 16;  // row of this warp's first key inside the tile
     constexpr int kBoxStride = (kFp8 ? 16 : kDecodeTile) * 128;  // bytes between 64-channel boxes
     const bool tail = key0 + 15 >= k_len;
     if constexpr (kFp8) {
@@ -444,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
       // 168-register cap; head_dim 256 runs one CTA per SM and unrolls both)
       constexpr int kUnrollKV = D == 256 ? 2 : 1;
 #pragma unroll kUnrollKV
-      for (int kv = 0; kv < 2; ++kv) {
+      for (int kv = kKDirect ? 1 : 0; kv < 2; ++kv) {
         const uint8_t* raw = kv ? v_stage(s) : k_stage(s);
         uint8_t* conv = kv ? cv : ck;
 #pragma unroll
@@ -452,7 +471,11 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
           const int idx = lane + 32 * it;
           const int kr = idx / kChunks;
           const int j = idx - kr * kChunks;
-          uint4 r4 = *reinterpret_cast<const uint4*>(raw + (wrow0 + kr) * D + j * 16);
+          // raw row: swizzled 128-byte boxes (kKDirect) or plain D-byte rows
+          const uint8_t* src =
+              kKDirect ? raw + (j >> 3) * (kDecodeTile * 128) + swz128(wrow0 + kr, j & 7)
+                       : raw + (wrow0 + kr) * D + j * 16;
+          uint4 r4 = *reinterpret_cast<const uint4*>(src);
           if (kv && key0 + kr >= k_len) r4 = make_uint4(0, 0, 0, 0);
           const uint32_t w[4] = {r4.x, r4.y, r4.z, r4.w};
           uint32_t h[8];
@@ -471,10 +494,11 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[s]);
-      kbase = smem_u32(ck);
+      if constexpr (!kKDirect) {
+        if (lane == 0) mbar_arrive(&empty_bar[s]);
+        kbase = smem_u32(ck);
+      }
       vbase = smem_u32(cv);
-      wrow0 = 0;
     } else if (tail) {
       // Zero value rows at or past k_len (stale or never written bytes).
       for (int idx = lane; idx < 16 * (D / 8); idx += 32) {
@@ -491,20 +515,38 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
     float sc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+    const int krow0 = kFp8 && !kKDirect ? 0 : wrow0;  // first key row in the K buffer read
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
-      // matrices: (keys 0-7, d lo), (keys 8-15, d lo), (keys 0-7, d hi), (keys 8-15, d hi)
-      const int mi = lane >> 3;
-      const int krow = wrow0 + (mi & 1) * 8 + (lane & 7);
-      const int chunk = ks * 2 + (mi >> 1);
-      const uint32_t addr = kbase + (chunk >> 3) * kBoxStride + swz128(krow, chunk & 7);
       uint32_t a[4];
-      ldsm_x4(addr, a[0], a[1], a[2], a[3]);
+      if constexpr (kKDirect) {
+        // codes of channels 4c .. 4c+3 of step ks, keys g and g + 8
+        const uint8_t* kb = k_stage(s) + (ks >> 3) * (kDecodeTile * 128) + 4 * c;
+        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(kb + swz128(krow0 + g, ks & 7));
+        const uint32_t w1 =
+            *reinterpret_cast<const uint32_t*>(kb + swz128(krow0 + g + 8, ks & 7));
+        a[0] = f16x2_from_e4m3x2(w0 & 0xFFFFu);
+        a[2] = f16x2_from_e4m3x2(w0 >> 16);
+        a[1] = f16x2_from_e4m3x2(w1 & 0xFFFFu);
+        a[3] = f16x2_from_e4m3x2(w1 >> 16);
+      } else {
+        // matrices: (keys 0-7, d lo), (keys 8-15, d lo), (keys 0-7, d hi), (keys 8-15, d hi)
+        const int mi = lane >> 3;
+        const int krow = krow0 + (mi & 1) * 8 + (lane & 7);
+        const int chunk = ks * 2 + (mi >> 1);
+        const uint32_t addr = kbase + (chunk >> 3) * kBoxStride + swz128(krow, chunk & 7);
+        ldsm_x4(addr, a[0], a[1], a[2], a[3]);
+      }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         if constexpr (kFp8) mma_f16(sc[nt], a, qb[ks][nt][0], qb[ks][nt][1]);
         else mma_bf16(sc[nt], a, qb[ks][nt][0], qb[ks][nt][1]);
       }
+    }
+
+    if constexpr (kKDirect) {
+      __syncwarp();  // every lane has read its K codes and V is widened
+      if (lane == 0) mbar_arrive(&empty_bar[s]);
     }
 
     // Mask, scale to log2 units, online-softmax update of this lane's rows;
@@ -574,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
       // matrices (transposed): (keys 0-7, d lo), (keys 0-7, d hi), (keys 8-15, d lo),
       // (keys 8-15, d hi)
       const int mi = lane >> 3;
-      const int vrow = wrow0 + (mi >> 1) * 8 + (lane & 7);
+      const int vrow = (kFp8 ? 0 : wrow0) + (mi >> 1) * 8 + (lane & 7);
       const int chunk = dc * 2 + (mi & 1);
       const uint32_t addr = vbase + (chunk >> 3) * kBoxStride + swz128(vrow, chunk & 7);
       uint32_t a[4];

@@ -67,8 +67,10 @@ bool cache_dtype_ok(rpk_dtype dtype, rpk_dtype cache) {
   return cache == dtype || cache == RPK_E4M3;
 }
 
-// 3-D byte map over rows of an e4m3 pool [rows, heads, d]: box (d, 1, box_rows)
-// = whole rows of one head, no swizzle (the decode kernel widens them itself).
+// 3-D byte map over rows of an e4m3 pool [rows, heads, d]: for head_dim >= 128
+// boxes of (128 codes, 1, box_rows) with the 128-byte swizzle (the decode
+// kernel reads K fragments straight from them), for head_dim 64 whole rows,
+// no swizzle.
 rpk_status encode_rows_map_u8(CUtensorMap* map, const void* base, int32_t d, int32_t heads,
                               int64_t rows, int32_t box_rows) {
   auto fn = encode_fn();
@@ -78,10 +80,12 @@ rpk_status encode_rows_map_u8(CUtensorMap* map, const void* base, int32_t d, int
   }
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)heads * d};
-  cuuint32_t box[3] = {(cuuint32_t)d, 1u, (cuuint32_t)box_rows};
+  const bool swizzled = d >= 128;
+  cuuint32_t box[3] = {swizzled ? 128u : (cuuint32_t)d, 1u, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzled ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled failed (%d)",
