@@ -72,6 +72,10 @@ def _declare(L):
                                        _p, C.c_int, _p, _p, _i32, _i32, _p, _i32, C.c_double,
                                        _i32, _i32, _p, _i64, _p, _p, C.c_int]
     L.rpko_attention_cache.restype = C.c_int
+    L.rpko_attention_backward.argtypes = [_p, _p, C.c_int, _p, _p, _i32, _i32, _i32, _i32,
+                                          _i32, _p, _p, C.c_int, _p, _p, _i32, _i32, _p, _i32,
+                                          C.c_double, _i32, _i32, _p, _p, _p]
+    L.rpko_attention_backward.restype = C.c_int
     L.rpko_flash_step.argtypes = [C.POINTER(C.c_double)] * 3 + [C.c_double, C.c_double]
     L.rpko_flash_step.restype = None
 
@@ -275,6 +279,35 @@ def attention(q, q_offsets, kv_lens, k_pages, v_pages, block_table, n_kv_heads, 
     if rc:
         raise ValueError(f"rpko_attention_cache failed ({rc})")
     return (out, lse) if with_lse else out
+
+
+def attention_backward(q, d_out, q_offsets, kv_lens, k_pages, v_pages, block_table, n_kv_heads,
+                       scale, window, sinks: int = 0, k_scale=None, v_scale=None):
+    """fp64 (d_q [T, n_heads, d], d_k, d_v [num_pages, page_size, n_kv_heads, d]) of the
+    attention output for the output gradient d_out (q's dtype)."""
+    qraw, code = _raw(q)
+    draw, dcode = _raw(d_out)
+    assert dcode == code
+    kp, kcode = _raw(k_pages)
+    vp, vcode = _raw(v_pages)
+    assert kcode == vcode and (kcode == code or kcode == E4M3)
+    ks = None if k_scale is None else np.ascontiguousarray(k_scale, dtype=np.float32)
+    vs = None if v_scale is None else np.ascontiguousarray(v_scale, dtype=np.float32)
+    T, H, d = qraw.shape
+    offs = _i32arr(q_offsets)
+    kvl = _i32arr(kv_lens)
+    bt = _i32arr(block_table)
+    dq = np.empty((T, H, d), dtype=np.float64)
+    dk = np.empty(kp.shape, dtype=np.float64)
+    dv = np.empty(vp.shape, dtype=np.float64)
+    rc = lib().rpko_attention_backward(_ptr(qraw), _ptr(draw), code, _ptr(offs), _ptr(kvl),
+                                       len(offs) - 1, T, H, int(n_kv_heads), d, _ptr(kp),
+                                       _ptr(vp), kcode, _ptr(ks), _ptr(vs), kp.shape[1],
+                                       kp.shape[0], _ptr(bt), bt.shape[1], float(scale),
+                                       int(window), int(sinks), _ptr(dq), _ptr(dk), _ptr(dv))
+    if rc:
+        raise ValueError(f"rpko_attention_backward failed ({rc})")
+    return dq, dk, dv
 
 
 def flash_step(m: float, l: float, o: float, s: float, v: float) -> tuple[float, float, float]:

@@ -564,6 +564,108 @@ int rpko_attention(const void* q, int dtype, const int32_t* q_offsets, const int
                               rows, n_rows, out, lse, n_threads);
 }
 
+/* --------------------------------------------------------- gradients */
+
+/*
+ * Gradients of rpko_attention_cache's output (NumKong "Attention with a
+ * Pre-Packed KV-Cache": attention_packed_gradients turns the output gradient
+ * into query, key and value gradients under the same band). For each row i
+ * (token t, head h) and each key j it sees, written out from the definition
+ * of softmax attention: s_ij = scale q_i.k_j, P_ij = e^{s_ij} / sum_j' e^{s_ij'}
+ * (two-pass, as the forward oracle), dP_ij = dO_i.v_j, D_i = sum_j P_ij dP_ij,
+ * dS_ij = P_ij (dP_ij - D_i); then dQ_i = scale sum_j dS_ij k_j,
+ * dK_j += scale dS_ij q_i and dV_j += P_ij dO_i, summed over every row and
+ * query head that sees key j. dK and dV have the pools' shape
+ * [num_pages, page_size, n_kv_heads, head_dim] and are zero where no row
+ * looks; dQ is [T, n_heads, head_dim]; d_out is [T, n_heads, head_dim] of
+ * dtype (q's). All fp64, single-threaded.
+ */
+int rpko_attention_backward(const void* q, const void* d_out, int dtype, const int32_t* q_offsets,
+                            const int32_t* kv_lens, int32_t batch, int32_t T, int32_t n_heads,
+                            int32_t n_kv_heads, int32_t head_dim, const void* k_pages,
+                            const void* v_pages, int cache_dtype, const float* k_scale,
+                            const float* v_scale, int32_t page_size, int32_t num_pages,
+                            const int32_t* block_table, int32_t max_pages_per_seq, double scale,
+                            int32_t window, int32_t sinks, double* d_q, double* d_k, double* d_v) {
+  if (!q || !d_out || !q_offsets || !kv_lens || !k_pages || !v_pages || !block_table || !d_q ||
+      !d_k || !d_v)
+    return RPKO_ERR_ARG;
+  if (n_kv_heads <= 0 || n_heads % n_kv_heads != 0 || head_dim <= 0 || page_size <= 0)
+    return RPKO_ERR_ARG;
+  if (cache_dtype != dtype && !(cache_dtype == RPKO_E4M3 && k_scale && v_scale))
+    return RPKO_ERR_ARG;
+  attn_job J = {q, dtype, q_offsets, kv_lens, batch, T, n_heads, n_kv_heads, head_dim,
+                k_pages, v_pages, cache_dtype, k_scale, v_scale, page_size, num_pages,
+                max_pages_per_seq, block_table, scale, window, sinks, NULL, 0, NULL, NULL,
+                RPKO_OK};
+  const int d = head_dim;
+  const size_t pool = (size_t)num_pages * page_size * n_kv_heads * d;
+  for (size_t e = 0; e < pool; ++e) d_k[e] = d_v[e] = 0.0;
+  for (size_t e = 0; e < (size_t)T * n_heads * d; ++e) d_q[e] = 0.0;
+  const int group = n_heads / n_kv_heads;
+  int32_t maxk = max_kv(&J);
+  double* p = (double*)malloc(sizeof(double) * (size_t)maxk);
+  double* dp = (double*)malloc(sizeof(double) * (size_t)maxk);
+  size_t* base = (size_t*)malloc(sizeof(size_t) * (size_t)maxk);
+  if (!p || !dp || !base) { free(p); free(dp); free(base); return RPKO_ERR_ARG; }
+  int status = RPKO_OK;
+  for (int32_t t = 0; t < T && status == RPKO_OK; ++t) {
+    int b = owner_of(q_offsets, batch, t);
+    if (b < 0) { status = RPKO_ERR_ARG; break; }
+    int32_t q_len = q_offsets[b + 1] - q_offsets[b];
+    int32_t k_len = kv_lens[b];
+    int32_t r = t - q_offsets[b];
+    for (int32_t h = 0; h < n_heads && status == RPKO_OK; ++h) {
+      int kvh = h / group;
+      size_t qb = ((size_t)t * n_heads + h) * d;
+      /* visible keys: scores, then weights */
+      int64_t n = 0;
+      double m = -INFINITY;
+      for (int32_t j = 0; j < k_len; ++j) {
+        if (!rpko_visible(r, q_len, k_len, window, sinks, j)) continue;
+        int32_t pi = j / page_size;
+        if (pi >= max_pages_per_seq) { status = RPKO_ERR_PAGE; break; }
+        int32_t page = block_table[(size_t)b * max_pages_per_seq + pi];
+        if (page < 0 || page >= num_pages) { status = RPKO_ERR_PAGE; break; }
+        base[n] = (((size_t)page * page_size + j % page_size) * n_kv_heads + kvh) * d;
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c)
+          acc += load_elt(q, dtype, qb + c) * load_cache(&J, k_pages, k_scale, kvh, base[n] + c);
+        p[n] = scale * acc;
+        if (p[n] > m) m = p[n];
+        ++n;
+      }
+      if (status != RPKO_OK || n == 0) continue;
+      double den = 0.0;
+      for (int64_t i = 0; i < n; ++i) {
+        p[i] = exp(p[i] - m);
+        den += p[i];
+      }
+      double D = 0.0;
+      for (int64_t i = 0; i < n; ++i) {
+        p[i] /= den;
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c)
+          acc += load_elt(d_out, dtype, qb + c) * load_cache(&J, v_pages, v_scale, kvh, base[i] + c);
+        dp[i] = acc;
+        D += p[i] * dp[i];
+      }
+      for (int64_t i = 0; i < n; ++i) {
+        double ds = p[i] * (dp[i] - D);
+        for (int c = 0; c < d; ++c) {
+          d_q[qb + c] += scale * ds * load_cache(&J, k_pages, k_scale, kvh, base[i] + c);
+          d_k[base[i] + c] += scale * ds * load_elt(q, dtype, qb + c);
+          d_v[base[i] + c] += p[i] * load_elt(d_out, dtype, qb + c);
+        }
+      }
+    }
+  }
+  free(p);
+  free(dp);
+  free(base);
+  return status;
+}
+
 /* ------------------------------------------------- online-softmax state */
 
 /*

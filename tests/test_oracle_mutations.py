@@ -53,6 +53,11 @@ MUTATIONS = {
                                   "rpko_f64_to_e4m3(k_rot[src + c] * (double)k_scale[kh]);"),
     "e4m3_slot_row": ("int32_t row = slot - pi * page_size;",
                       "int32_t row = (slot + 1) % page_size;"),
+    "backward_delta_dropped": ("double ds = p[i] * (dp[i] - D);", "double ds = p[i] * dp[i];"),
+    "backward_key_scale_dropped": ("d_k[base[i] + c] += scale * ds * load_elt(q, dtype, qb + c);",
+                                   "d_k[base[i] + c] += ds * load_elt(q, dtype, qb + c);"),
+    "backward_value_weight_dropped": ("d_v[base[i] + c] += p[i] * load_elt(d_out, dtype, qb + c);",
+                                      "d_v[base[i] + c] += load_elt(d_out, dtype, qb + c);"),
     "e4m3_read_scale_dropped": ("return rpko_e4m3_to_f64(((const uint8_t*)pool)[idx]) * (double)scale[kvh];",
                                 "return rpko_e4m3_to_f64(((const uint8_t*)pool)[idx]);"),
 }

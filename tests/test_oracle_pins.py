@@ -819,3 +819,83 @@ def test_e4m3_attention_reads_code_times_scale():
         got = O.attention(q, offs, lens, kp8, vp8, bt, Hk, 0.3, w, k_scale=ks, v_scale=vs)
         ref = O.attention(q, offs, lens, kpf, vpf, bt, Hk, 0.3, w)
         assert np.array_equal(got, ref)
+
+
+# ----------------------------------------------------------------- gradients
+# attention_packed_gradients (NumKong "Attention with a Pre-Packed KV-Cache")
+# gives the query, key and value gradients of the output under the same band.
+# The oracle writes out the definition; here it is pinned to central finite
+# differences of the (separately pinned) forward oracle, to the single-key
+# case and to a conservation law.
+
+
+def _grad_case(seed=0, window=0, sinks=0):
+    rng = np.random.default_rng(seed)
+    Hk, H, d, P = 2, 4, 8, 4
+    q_lens, kv_lens = [4, 2], [6, 3]
+    # values on a 2^-6 grid in [-2, 2]: +- 2^-10 perturbations stay exact in fp32
+    grid = lambda shape: (rng.integers(-128, 129, shape) / 64.0).astype(np.float32)
+    kd = [grid((n, Hk, d)) for n in kv_lens]
+    vd = [grid((n, Hk, d)) for n in kv_lens]
+    kp, vp, bt = paged(kd, vd, P, seed=seed)
+    kp = np.nan_to_num(kp, nan=0.0)   # unused slots: any finite value
+    vp = np.nan_to_num(vp, nan=0.0)
+    T = sum(q_lens)
+    q = grid((T, H, d))
+    dout = grid((T, H, d))
+    offs = np.array([0, q_lens[0], T], dtype=np.int32)
+    return q, dout, offs, np.array(kv_lens, np.int32), kp, vp, bt, Hk
+
+
+@pytest.mark.parametrize("window,sinks", [(0, 0), (3, 0), (2, 1)])
+def test_gradients_match_finite_differences(window, sinks):
+    q, dout, offs, kvl, kp, vp, bt, Hk = _grad_case(window=window, sinks=sinks)
+    scale = 0.37
+    dq, dk, dv = O.attention_backward(q, dout, offs, kvl, kp, vp, bt, Hk, scale, window, sinks)
+    h = 2.0 ** -10
+
+    def loss(qq, kk, vv):
+        out = O.attention(qq, offs, kvl, kk, vv, bt, Hk, scale, window, sinks=sinks, n_threads=1)
+        return float(np.sum(out * dout.astype(np.float64)))
+
+    def fd(arr, idx, other):
+        plus, minus = arr.copy(), arr.copy()
+        plus[idx] += np.float32(h)
+        minus[idx] -= np.float32(h)
+        return (loss(*other(plus)) - loss(*other(minus))) / (2 * h)
+
+    for idx in np.ndindex(q.shape):
+        want = fd(q, idx, lambda a: (a, kp, vp))
+        assert abs(dq[idx] - want) <= 1e-6 + 1e-5 * abs(want), ("dq", idx, dq[idx], want)
+    used = np.unique(bt[bt >= 0])
+    for page in used:
+        for idx in np.ndindex(kp.shape[1:]):
+            full = (page,) + idx
+            want_k = fd(kp, full, lambda a: (q, a, vp))
+            want_v = fd(vp, full, lambda a: (q, kp, a))
+            assert abs(dk[full] - want_k) <= 1e-6 + 1e-5 * abs(want_k), ("dk", full, dk[full], want_k)
+            assert abs(dv[full] - want_v) <= 1e-6 + 1e-5 * abs(want_v), ("dv", full, dv[full], want_v)
+
+
+def test_gradients_of_a_single_visible_key():
+    # one key: the output is its value whatever q and k are, so dQ = dK = 0 and dV = dO
+    rng = np.random.default_rng(1)
+    d = 8
+    q = rng.standard_normal((1, 2, d)).astype(np.float32)
+    dout = rng.standard_normal((1, 2, d)).astype(np.float32)
+    k = rng.standard_normal((1, 1, d)).astype(np.float32)
+    v = rng.standard_normal((1, 1, d)).astype(np.float32)
+    kp, vp, bt = paged([k], [v], page_size=2)
+    dq, dk, dv = O.attention_backward(q, dout, [0, 1], [1], kp, vp, bt, 1, 0.5, 0)
+    assert np.all(dq == 0.0) and np.all(dk[bt[0, 0], 0] == 0.0)
+    assert np.allclose(dv[bt[0, 0], 0, 0], dout[0].astype(np.float64).sum(axis=0), rtol=0,
+                       atol=1e-15)
+
+
+def test_key_gradients_sum_to_zero():
+    # each row's dS sums to zero (its weights sum to one), so sum_j dK_j = 0 for
+    # every KV head
+    q, dout, offs, kvl, kp, vp, bt, Hk = _grad_case(seed=4, window=3, sinks=1)
+    dq, dk, dv = O.attention_backward(q, dout, offs, kvl, kp, vp, bt, Hk, 0.8, 3, 1)
+    assert np.max(np.abs(dk.sum(axis=(0, 1)))) <= 1e-12
+    assert np.any(dk != 0.0)
