@@ -266,6 +266,45 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
                                   int32_t sink_tokens, void* stream);
 
 /*
+ * ragged_paged_attention_backward -- gradients of ragged_paged_attention's
+ * output (NumKong "Attention with a Pre-Packed KV-Cache":
+ * attention_packed_gradients turns the forward's log-sum-exp, its output and
+ * the output gradient into query, key and value gradients under the same
+ * band).
+ *
+ * With s_ij = scale q_i.k_j, P_ij = e^(s_ij - lse_i), dP_ij = d_out_i.v_j,
+ * D_i = d_out_i.out_i and dS_ij = P_ij (dP_ij - D_i):
+ *   d_q_i = scale sum_j dS_ij k_j, d_k_j = scale sum_i dS_ij q_i,
+ *   d_v_j = sum_i P_ij d_out_i,
+ * the sums running over the (row, key) pairs the forward's band (window,
+ * sinks) makes visible, and over every query head of a KV head's group.
+ *
+ *   q, q_row_offsets, kv_lens, page_table, n_heads ... dtype, sink_tokens:
+ *                   as in the forward call whose gradient this is (the cache
+ *                   unchanged since; an RPK_E4M3 cache is read as code * scale)
+ *   out             the forward's output [total_q_tokens, n_heads, head_dim] dtype
+ *   d_out           [total_q_tokens, n_heads, head_dim] dtype, the output gradient
+ *   log_sum_exp     float32 [total_q_tokens, n_heads], the forward's log_sum_exp
+ *   d_q             float32 [total_q_tokens, n_heads, head_dim] (written)
+ *   d_k_pages,      float32, the shape of one layer's pools
+ *   d_v_pages       [num_pages, page_size, n_kv_heads, head_dim]: the entry of
+ *                   every key below kv_lens[b] of each sequence is written (the
+ *                   gradient of that cached key or value; for an e4m3 cache,
+ *                   of its dequantised value); other entries are left as they
+ *                   were, so a caller that sums over the pool zeroes them first.
+ *
+ * CUDA-core kernels in fp32 (a row-parallel one for d_q, a key-parallel one
+ * for d_k and d_v; no atomics). Errors as ragged_paged_attention; every pointer
+ * is 16-byte aligned device memory; buffers must not overlap.
+ */
+rpk_status ragged_paged_attention_backward(
+    const void* q, const int32_t* q_row_offsets, const int32_t* kv_lens,
+    const rpk_paged_kv* page_table, int32_t n_heads, int32_t n_kv_heads, int32_t head_dim,
+    float scale, int32_t window, const void* out, const void* d_out, const float* log_sum_exp,
+    float* d_q, float* d_k_pages, float* d_v_pages, int32_t batch, int32_t total_q_tokens,
+    int32_t max_q_len, int32_t max_kv_len, rpk_dtype dtype, int32_t sink_tokens, void* stream);
+
+/*
  * ragged_paged_attention_noalloc -- ragged_paged_attention for callers that
  * cannot allocate device memory at call time. The pages have no counterpart
  * for it; it is a convenience of this library.

@@ -20,6 +20,7 @@ from .binding import (  # noqa: F401
     freqs_cis_proportional,
     lib,
     ragged_paged_attention,
+    ragged_paged_attention_backward,
     ragged_paged_attention_workspace_size,
     rope_qk_paged_ragged,
 )

@@ -9,6 +9,7 @@ Entry points keep the C names:
 
 * ``rope_qk_paged_ragged``  fused RoPE on Q and new K, K/V written into the cache
 * ``ragged_paged_attention`` ragged causal GQA attention over the paged cache
+* ``ragged_paged_attention_backward`` its query, key and value gradients
 * ``ragged_paged_attention_workspace_size``
 * ``freqs_cis``             builds the fp32 (cos, sin) table with ``rope_freqs_cis``
 * ``freqs_cis_proportional`` builds the p-RoPE table with ``rope_freqs_cis_proportional``
@@ -302,6 +303,51 @@ def ragged_paged_attention(q, q_row_offsets, kv_lens, page_table: PagedKVCache, 
         qp, off, kvl, C.byref(pk), int(n_heads), int(n_kv_heads), int(head_dim), float(scale),
         int(window), op, batch, T, int(max_q_len), int(max_kv_len), _dtype_code(q.dtype), ws,
         ws_bytes, lp, int(sink_tokens), _stream(stream)))
+
+
+def ragged_paged_attention_backward(q, q_row_offsets, kv_lens, page_table: PagedKVCache,
+                                    n_heads: int, n_kv_heads: int, head_dim: int,
+                                    scale: float | None, window: int, out, d_out, log_sum_exp,
+                                    d_q, d_k_pages, d_v_pages, *, max_q_len: int, max_kv_len: int,
+                                    sink_tokens: int = 0, stream=None) -> None:
+    """Gradients of ragged_paged_attention: d_q [tokens, n_heads, head_dim] and the
+    pool-shaped d_k_pages / d_v_pages (float32) from the forward's out and
+    log_sum_exp and the output gradient d_out. Entries of d_k_pages / d_v_pages
+    that hold no key of any sequence are left as they were."""
+    L = lib()
+    fn = L.ragged_paged_attention_backward
+    if fn.argtypes is None:
+        _p, _i32 = C.c_void_p, C.c_int32
+        fn.argtypes = [_p, _p, _p, C.POINTER(PagedKV), _i32, _i32, _i32, C.c_float, _i32, _p, _p,
+                       _p, _p, _p, _p, _i32, _i32, _i32, _i32, C.c_int, _i32, _p]
+        fn.restype = C.c_int
+    pk = page_table.struct()
+    if q.dim() != 3:
+        raise RpkError("q must be [tokens, n_heads, head_dim]")
+    T = int(q.shape[0])
+    qp = _dev(q, "q")
+    op = _dev(out, "out", q.dtype, 3)
+    gp = _dev(d_out, "d_out", q.dtype, 3)
+    lp = _dev(log_sum_exp, "log_sum_exp", torch.float32, 2)
+    dq = _dev(d_q, "d_q", torch.float32, 3)
+    pool_shape = (pk.num_pages, pk.page_size, pk.n_kv_heads, pk.head_dim)
+    for t, name in ((d_k_pages, "d_k_pages"), (d_v_pages, "d_v_pages")):
+        _dev(t, name, torch.float32, 4)
+        if tuple(t.shape) != pool_shape:
+            raise RpkError(f"{name} must be {pool_shape}")
+    for t, name in ((out, "out"), (d_out, "d_out"), (d_q, "d_q")):
+        if tuple(t.shape) != tuple(q.shape):
+            raise RpkError(f"{name} must have q's shape")
+    if tuple(log_sum_exp.shape) != (T, int(n_heads)):
+        raise RpkError("log_sum_exp must be [tokens, n_heads]")
+    off = _dev(q_row_offsets, "q_row_offsets", torch.int32, 1)
+    kvl = _dev(kv_lens, "kv_lens", torch.int32, 1)
+    if scale is None:
+        scale = float(head_dim) ** -0.5
+    _check(fn(qp, off, kvl, C.byref(pk), int(n_heads), int(n_kv_heads), int(head_dim),
+              float(scale), int(window), op, gp, lp, dq, d_k_pages.data_ptr(),
+              d_v_pages.data_ptr(), int(kv_lens.shape[0]), T, int(max_q_len), int(max_kv_len),
+              _dtype_code(q.dtype), int(sink_tokens), _stream(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024

@@ -325,4 +325,54 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
   return cuda_status(rpk::launch_attn_simt(p, dtype, s));
 }
 
+rpk_status ragged_paged_attention_backward(
+    const void* q, const int32_t* q_row_offsets, const int32_t* kv_lens,
+    const rpk_paged_kv* page_table, int32_t n_heads, int32_t n_kv_heads, int32_t head_dim,
+    float scale, int32_t window, const void* out, const void* d_out, const float* log_sum_exp,
+    float* d_q, float* d_k_pages, float* d_v_pages, int32_t batch, int32_t total_q_tokens,
+    int32_t max_q_len, int32_t max_kv_len, rpk_dtype dtype, int32_t sink_tokens, void* stream) {
+  if (!q || !q_row_offsets || !kv_lens || !out || !d_out || !log_sum_exp || !d_q || !d_k_pages ||
+      !d_v_pages)
+    return RPK_ERR_NULL;
+  rpk_status st = check_cache(page_table);
+  if (st != RPK_OK) return st;
+  if (dtype != RPK_BF16 && dtype != RPK_F32) return RPK_ERR_DTYPE;
+  if (!cache_dtype_ok(dtype, page_table->cache_dtype)) return RPK_ERR_DTYPE;
+  if (n_kv_heads != page_table->n_kv_heads || head_dim != page_table->head_dim)
+    return RPK_ERR_SHAPE;
+  if (n_heads <= 0 || n_heads % n_kv_heads != 0) return RPK_ERR_SHAPE;
+  if (batch <= 0 || batch != page_table->batch || batch > 65535) return RPK_ERR_SHAPE;
+  if (total_q_tokens < 0 || max_q_len < 0 || max_kv_len < 0) return RPK_ERR_SHAPE;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return RPK_ERR_SHAPE;
+  if (sink_tokens < 0) return RPK_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(d_out) || !aligned16(log_sum_exp) ||
+      !aligned16(d_q) || !aligned16(d_k_pages) || !aligned16(d_v_pages))
+    return RPK_ERR_SHAPE;
+  if ((long long)max_kv_len > (long long)page_table->max_pages_per_seq * page_table->page_size)
+    return RPK_ERR_SHAPE;
+  if ((long long)max_kv_len > 65535LL * 8) return RPK_ERR_UNSUPPORTED;
+  if (total_q_tokens == 0) return RPK_OK;
+
+  rpk::BackwardParams p;
+  p.q = q; p.out = out; p.d_out = d_out; p.lse = log_sum_exp;
+  {
+    void *k, *v;
+    rpk::layer_pools(page_table, &k, &v);
+    p.k_pages = k; p.v_pages = v;
+  }
+  p.offsets = q_row_offsets; p.kv_lens = kv_lens; p.block_table = page_table->block_table;
+  p.error_word = page_table->error_word;
+  p.d_q = d_q; p.d_k = d_k_pages; p.d_v = d_v_pages;
+  p.T = total_q_tokens; p.batch = batch; p.H = n_heads; p.Hk = n_kv_heads;
+  p.G = n_heads / n_kv_heads; p.d = head_dim; p.P = page_table->page_size;
+  p.num_pages = page_table->num_pages; p.max_pages = page_table->max_pages_per_seq;
+  p.window = window > 0 ? window : 0; p.max_q_len = max_q_len; p.max_kv_len = max_kv_len;
+  p.sinks = window > 0 ? sink_tokens : 0;
+  p.scale = scale;
+  p.cache_fp8 = page_table->cache_dtype == RPK_E4M3;
+  p.k_scale = page_table->k_scale;
+  p.v_scale = page_table->v_scale;
+  return cuda_status(rpk::launch_attn_backward(p, dtype, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -110,4 +110,27 @@ cudaError_t launch_attn_prefill(const AttnParams& p, const CUtensorMap& q_map,
                                 int* work_counter, cudaStream_t stream);
 int prefill_rows_per_tile(int group);
 
+// Gradients of ragged_paged_attention (CUDA-core, fp32 math).
+struct BackwardParams {
+  const void* q;
+  const void* out;
+  const void* d_out;
+  const float* lse;            // [T, H] natural log-sum-exp of the forward
+  const void* k_pages;
+  const void* v_pages;
+  const int32_t* offsets;      // [batch + 1]
+  const int32_t* kv_lens;      // [batch]
+  const int32_t* block_table;  // [batch, max_pages]
+  int32_t* error_word;
+  float* d_q;                  // [T, H, d]
+  float* d_k;                  // pool-shaped [num_pages, P, Hk, d]
+  float* d_v;
+  int32_t T, batch, H, Hk, G, d, P, num_pages, max_pages, window, max_q_len, max_kv_len, sinks;
+  float scale;
+  int32_t cache_fp8;
+  const float* k_scale;
+  const float* v_scale;
+};
+cudaError_t launch_attn_backward(const BackwardParams& p, rpk_dtype dtype, cudaStream_t stream);
+
 }  // namespace rpk

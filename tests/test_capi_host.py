@@ -150,6 +150,30 @@ def test_e4m3_cache_takes_bf16_and_f32_tensors_only(L):
 
 
 @host_only
+def test_backward_rejects(L):
+    fn = L.ragged_paged_attention_backward
+    fn.restype = C.c_int
+    P = C.c_void_p
+    base = dict(q=FAKE, off=FAKE, kvl=FAKE, H=32, Hk=8, d=128, scale=0.1, w=0, out=FAKE,
+                dout=FAKE, lse=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, batch=2, T=5, mq=4, mk=200,
+                dtype=B.RPK_BF16, sinks=0)
+
+    def call(c, **kw):
+        a = dict(base, **kw)
+        return fn(P(a["q"]), P(a["off"]), P(a["kvl"]), C.byref(c), a["H"], a["Hk"], a["d"],
+                  C.c_float(a["scale"]), a["w"], P(a["out"]), P(a["dout"]), P(a["lse"]),
+                  P(a["dq"]), P(a["dk"]), P(a["dv"]), a["batch"], a["T"], a["mq"], a["mk"],
+                  a["dtype"], a["sinks"], None)
+
+    c = cache(max_pages_per_seq=16)
+    for kw, status in [({"dout": None}, 1), ({"lse": None}, 1), ({"dk": None}, 1),
+                       ({"Hk": 6}, 2), ({"scale": 0.0}, 2), ({"sinks": -1}, 2),
+                       ({"dq": FAKE + 4}, 2), ({"dtype": B.RPK_F32}, 3), ({"mk": 1025}, 2)]:
+        assert call(c, **kw) == status, kw
+    assert call(cache(cache_dtype=B.RPK_E4M3, max_pages_per_seq=16)) == 1   # scales missing
+
+
+@host_only
 def test_attention_rejects_layer_out_of_range(L):
     assert attn(L, cache(max_pages_per_seq=16, num_layers=2, layer_idx=2)) == 2
     assert L.ragged_paged_attention_noalloc(
