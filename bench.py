@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the attention backward on the ragged prefill workload")
     ap.add_argument("--cache-dtype", default=None, choices=["e4m3"],
                     help="hold the KV cache as e4m3 codes with per-head scales")
     return ap.parse_args()
@@ -407,6 +409,60 @@ def prefill_measure(device, world, steps=5, warmup=3):
     }
 
 
+def backward_measure(device, world, steps=5, warmup=3):
+    """The attention backward (its two kernels) on the ragged prefill workload:
+    the forward runs once for the output and log-sum-exp, then the backward is
+    timed with a seeded N(0, 1) output gradient. Algorithmic FLOPs are 2.5x the
+    forward's visible-pair FLOPs: five products of 2 d FLOP per visible (row,
+    key) pair and head (S, dP, dQ, dK, dV); the kernels recompute S and dP in
+    each of their two passes, which is not counted."""
+    wl = W.make("ragged_prefill", seed=0)
+    sp = wl.spec
+    step = Step(wl, device)
+    step.rope()
+    T, H, d = wl.q.shape
+    lse = torch.empty((T, H), dtype=torch.float32, device=device)
+    R.ragged_paged_attention(step.q_rot, step.offsets, step.kv_lens, step.cache, sp.n_heads,
+                             sp.n_kv_heads, sp.head_dim, sp.softmax_scale, sp.window, step.out,
+                             max_q_len=wl.max_q_len, max_kv_len=wl.max_kv_len,
+                             workspace=step.workspace, log_sum_exp=lse)
+    gen = torch.Generator().manual_seed(1)
+    d_out = torch.randn((T, H, d), generator=gen).to(step.q.dtype).to(device)
+    d_q = torch.empty((T, H, d), dtype=torch.float32, device=device)
+    d_k = torch.zeros(tuple(step.cache.k_pages.shape), dtype=torch.float32, device=device)
+    d_v = torch.zeros_like(d_k)
+
+    def run():
+        R.ragged_paged_attention_backward(step.q_rot, step.offsets, step.kv_lens, step.cache,
+                                          sp.n_heads, sp.n_kv_heads, sp.head_dim,
+                                          sp.softmax_scale, sp.window, step.out, d_out, lse,
+                                          d_q, d_k, d_v, max_q_len=wl.max_q_len,
+                                          max_kv_len=wl.max_kv_len)
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for a, b in ev:
+        a.record()
+        run()
+        b.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev), world)
+    flops = 2.5 * M.attention_flops(wl.q_lens, wl.kv_lens, sp.window, sp.n_heads, sp.head_dim)
+    peaks = load_peaks()
+    tflops = flops / (ms * 1e-3) / 1e12
+    kernel = ("tensor-core (mma.sync) dQ and dK/dV kernels"
+              if sp.dtype == "bf16" and sp.n_heads // sp.n_kv_heads <= 16
+              else "CUDA-core dQ and dK/dV kernels")
+    return {"workload": "ragged_prefill", "kernel": kernel, "backward_ms": ms,
+            "algorithmic_flops": flops, "tflops": tflops,
+            "tensor_peak_tflops": peaks["bf16_tflops"], "frac": tflops / peaks["bf16_tflops"],
+            "error_word": int(step.error_word.item())}
+
+
 # ------------------------------------------------------------ the metric
 
 def is_decode(wl: W.Workload) -> bool:
@@ -548,6 +604,7 @@ def main():
                "note": "pinned host inputs copied in, output copied out, inside the timed region"}
 
     prefill = None if args.no_prefill else prefill_measure(device, world)
+    backward = backward_measure(device, world) if args.backward else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -582,6 +639,7 @@ def main():
         "gpu_launches": step.launches_per_step() * args.steps,
         "error_word": err,
         "prefill": prefill,
+        "backward": backward,
         "cpu_baseline": cpu,
     }
     if rank == 0:

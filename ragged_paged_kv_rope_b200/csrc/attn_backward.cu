@@ -1,5 +1,7 @@
 // attn_backward.cu -- gradients of ragged paged causal GQA attention on CUDA
-// cores, fp32 math (NumKong "Attention with a Pre-Packed KV-Cache":
+// cores, fp32 math, for the shapes the tensor-core kernels (attn_backward_mma.cu)
+// do not take: fp32 tensors, e4m3 caches, groups of more than 16 query heads
+// (NumKong "Attention with a Pre-Packed KV-Cache":
 // attention_packed_gradients turns the forward's log-sum-exp, its output and
 // the output gradient into query, key and value gradients under the same
 // band).
@@ -205,6 +207,7 @@ cudaError_t launch_t(const BackwardParams& p, cudaStream_t stream) {
 
 cudaError_t launch_attn_backward(const BackwardParams& p, rpk_dtype dtype, cudaStream_t stream) {
   if (p.batch == 0) return cudaSuccess;
+  if (attn_backward_mma_supported(p, dtype)) return launch_attn_backward_mma(p, stream);
   if (dtype == RPK_BF16)
     return p.cache_fp8 ? launch_t<__nv_bfloat16, true>(p, stream)
                        : launch_t<__nv_bfloat16, false>(p, stream);

@@ -132,5 +132,9 @@ struct BackwardParams {
   const float* v_scale;
 };
 cudaError_t launch_attn_backward(const BackwardParams& p, rpk_dtype dtype, cudaStream_t stream);
+// Tensor-core (mma.sync) kernels: bf16 tensors over a bf16 cache, groups of at
+// most 16 query heads, head_dim 64 / 128 / 256.
+bool attn_backward_mma_supported(const BackwardParams& p, rpk_dtype dtype);
+cudaError_t launch_attn_backward_mma(const BackwardParams& p, cudaStream_t stream);
 
 }  // namespace rpk

@@ -7,7 +7,15 @@ kernel takes D_i = d_out_i . out_i from the forward's rounded output and P_ij
 from its fp32 log-sum-exp, as the API defines, so the comparison is relative
 to each gradient's scale: for bf16, max |got - ref| <= 2e-2 max|ref| and
 mean |got - ref| <= 2e-3 max|ref| (the output's bf16 rounding, 2^-9, enters
-D_i and so every dS_ij); for fp32, 1e-4 max|ref|.
+D_i and so every dS_ij; the tensor-core kernels also round P_ij and dS_ij to
+bf16, relative 2^-9, as operands of their second products); for fp32,
+1e-4 max|ref|.
+
+bf16 shapes with groups of up to 16 query heads run on the tensor-core
+kernels, the others (fp32, an e4m3 cache, larger groups) on the CUDA-core
+ones; the cases cover both, several 64-key tiles and 64-row blocks with
+ragged tails, windows with sinks across tiles, groups that do not divide 64,
+and rows that see no key.
 """
 
 import numpy as np
@@ -50,6 +58,19 @@ CASES = [
     ("fp32", "tiny_prefill_f32", {}, [5, 11], [5, 11], 0, 0),
     ("e4m3 cache", "llama3_8b_decode", dict(n_heads=8, n_kv_heads=2, cache_dtype="e4m3"),
      [3, 1], [200, 90], 0, 0),
+    ("tiles and ragged tails", "ragged_prefill", dict(n_heads=8, n_kv_heads=2, page_size=64),
+     [200, 64, 1], [330, 64, 129], 0, 0),
+    ("window and sinks across tiles", "ragged_prefill",
+     dict(n_heads=8, n_kv_heads=2, page_size=32), [150, 30], [400, 100], 70, 5),
+    ("group of 3", "ragged_prefill", dict(n_heads=6, n_kv_heads=2), [50, 7], [120, 7], 0, 0),
+    ("group of 16", "ragged_prefill",
+     dict(n_heads=16, n_kv_heads=1, head_dim=64, rotary_dim=64), [9, 20], [70, 20], 0, 0),
+    ("group of 32 (CUDA cores)", "ragged_prefill",
+     dict(n_heads=32, n_kv_heads=1, head_dim=64, rotary_dim=64), [3, 5], [50, 5], 0, 0),
+    ("rows without keys", "ragged_prefill", dict(n_heads=4, n_kv_heads=2), [12, 3], [5, 40],
+     0, 0),
+    ("head_dim 256 prefill, window and sinks", "gemma_swa_decode",
+     dict(n_heads=4, n_kv_heads=2), [100, 1], [300, 77], 128, 4),
 ]
 
 
