@@ -12,15 +12,18 @@
 // packed row rho of a block holds token rho / G and head rho % G, 64 rows per
 // block (64 / G tokens), as the forward packs its query tiles.
 //
-// Two kernels, no atomics (each output element has one writer):
-//   dQ  -- one CTA per 64 packed rows; its four warps own 16 rows each and walk
-//          the key tiles of the rows' band (sink tiles, then the window):
-//          S = Q K^T and dP = dO V^T from shared memory, P and dS in registers,
-//          dQ += dS K with dS reused as the A operand (bf16).
+// Three kernels, no atomics (each output element has one writer), in launch
+// order:
+//   D   -- D_i of every row, kept in d_q's memory until the dQ kernel
+//          overwrites it.
 //   dKV -- one CTA per 64 keys; its four warps own 16 keys each and walk the
 //          row blocks that see them: S^T = K Q^T, dP^T = V dO^T,
 //          dV += P^T dO and dK += dS^T Q. For head_dim 256 two CTAs share a key
 //          block, each accumulating half of the output channels.
+//   dQ  -- one CTA per 64 packed rows; its four warps own 16 rows each and walk
+//          the key tiles of the rows' band (sink tiles, then the window):
+//          S = Q K^T and dP = dO V^T from shared memory, P and dS in registers,
+//          dQ += dS K with dS reused as the A operand (bf16).
 // Tiles are staged in shared memory by cp.async (16-byte chunks, XOR-swizzled
 // by row so that ldmatrix reads are conflict-free), two stages deep. P and dS
 // are rounded to bf16 as operands of the second products; every sum is fp32.
@@ -46,6 +49,12 @@ __device__ __forceinline__ uint32_t toff(int r, int c) {
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
                "r"(valid ? 16 : 0)
+               : "memory");
+}
+// 4 bytes global -> shared, or 4 zero bytes when !valid (no global read).
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 4 : 0)
                : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -151,6 +160,21 @@ __device__ __forceinline__ float row_delta(const BackwardParams& p, size_t row_e
     }
   }
   return acc;
+}
+
+// ------------------------------------------------------------------- D
+
+// D_i of every (token, head) row into delta[t * H + h]; eight lanes per row.
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const BackwardParams p,
+                                                             float* __restrict__ delta) {
+  const long long row = ((long long)blockIdx.x * 256 + threadIdx.x) >> 3;
+  const bool ok = row < (long long)p.T * p.H;
+  float v = ok ? row_delta<D>(p, (size_t)row * D, threadIdx.x & 7, 8) : 0.f;
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  v += __shfl_xor_sync(0xffffffffu, v, 4);
+  if (ok && (threadIdx.x & 7) == 0) delta[row] = v;
 }
 
 // ------------------------------------------------------------------- dQ
@@ -302,15 +326,16 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_dq_mma_kernel(const Backwar
 // ------------------------------------------------------------------ dK, dV
 
 template <int D, int DC>
-__global__ void __launch_bounds__(kThreads) attn_bwd_dkv_mma_kernel(const BackwardParams p) {
+__global__ void __launch_bounds__(kThreads) attn_bwd_dkv_mma_kernel(const BackwardParams p,
+                                                                    const float* __restrict__ delta) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int TB = kRows * D * 2;
   constexpr int NT = DC / 8;            // 8-channel n-tiles of this CTA's output channels
   constexpr int kSplit = D / DC;
   const uint32_t sK = smem_u32(smem), sV = sK + TB, sQ = sK + 2 * TB, sG = sK + 4 * TB;
-  int* m_pos = reinterpret_cast<int*>(smem + 6 * TB);            // [2][64]
-  float* m_lse2 = reinterpret_cast<float*>(m_pos + 2 * kRows);   // [2][64]
-  float* m_delta = m_lse2 + 2 * kRows;                           // [2][64]
+  int* m_pos = reinterpret_cast<int*>(smem + 6 * TB);           // [2][64]
+  float* m_lse = reinterpret_cast<float*>(m_pos + 2 * kRows);   // [2][64]
+  float* m_delta = m_lse + 2 * kRows;                           // [2][64]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, c = lane & 3;
   const int b = blockIdx.y;
@@ -338,21 +363,20 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_dkv_mma_kernel(const Backwa
 #pragma unroll
     for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.f;
 
-  // Row metadata of block rb into stage st: position (INT_MIN / 2 for rows
-  // that take no gradient), lse in log2 units and D. Two threads per row.
+  // Row metadata of block rb into stage st: the position (INT_MIN / 2 for
+  // rows past the block's tokens; a row whose forward saw no key sees none
+  // here either), and lse and D by cp.async (zero for those rows).
   auto load_meta = [&](int rb, int st) {
-    const int r = threadIdx.x >> 1, part = threadIdx.x & 1;
+    const int r = threadIdx.x & (kRows - 1);
     const int tk = r / G;
     const int tok = r_lo + rb * tpb + tk;
     const bool ok = tk < tpb && tok <= r_hi;
-    const size_t elt = ok ? ((size_t)(q0 + tok) * p.H + kvh * G + (r - tk * G)) * D : 0;
-    float dl = ok ? row_delta<D>(p, elt, part, 2) : 0.f;
-    dl += __shfl_xor_sync(0xffffffffu, dl, 1);
-    if (part == 0) {
-      const float l = ok ? p.lse[elt / D] : -INFINITY;
-      m_pos[st * kRows + r] = ok && l > -INFINITY ? tok + off : INT_MIN / 2;
-      m_lse2[st * kRows + r] = l * kLog2eMma;
-      m_delta[st * kRows + r] = dl;
+    const size_t row = ok ? (size_t)(q0 + tok) * p.H + kvh * G + (r - tk * G) : 0;
+    if (threadIdx.x < kRows) {
+      m_pos[st * kRows + r] = ok ? tok + off : INT_MIN / 2;
+      cp_async4(smem_u32(m_lse + st * kRows + r), p.lse + row, ok);
+    } else {
+      cp_async4(smem_u32(m_delta + st * kRows + r), delta + row, ok);
     }
   };
   auto load_block = [&](int rb, int st) {
@@ -366,14 +390,14 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_dkv_mma_kernel(const Backwa
   if (n_blocks > 0) {
     load_keys<D>(p, b, kvh, k_len, key0, sK, sV, false);
     load_block(0, 0);
-    cp_async_commit();
     load_meta(0, 0);
+    cp_async_commit();
     for (int rb = 0; rb < n_blocks; ++rb) {
       const int st = rb & 1;
       if (rb + 1 < n_blocks) {
         load_block(rb + 1, st ^ 1);
-        cp_async_commit();
         load_meta(rb + 1, st ^ 1);
+        cp_async_commit();
         cp_async_wait<1>();
       } else {
         cp_async_wait<0>();
@@ -381,7 +405,7 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_dkv_mma_kernel(const Backwa
       __syncthreads();
       const uint32_t q_t = sQ + st * TB, g_t = sG + st * TB;
       const int* mp = m_pos + st * kRows;
-      const float* ml = m_lse2 + st * kRows;
+      const float* ml = m_lse + st * kRows;
       const float* md = m_delta + st * kRows;
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
@@ -413,8 +437,9 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_dkv_mma_kernel(const Backwa
           for (int e = 0; e < 4; ++e) {
             const int col = half * 32 + n * 8 + 2 * c + (e & 1);
             const int j = key0 + warp * 16 + g + 8 * (e >> 1);
-            const float pr =
-                visible(j, mp[col], p.window, p.sinks) ? fast_exp2(s[n][e] * sl2 - ml[col]) : 0.f;
+            const float pr = visible(j, mp[col], p.window, p.sinks)
+                                 ? fast_exp2(fmaf(s[n][e], sl2, -ml[col] * kLog2eMma))
+                                 : 0.f;
             s[n][e] = pr;
             dp[n][e] = pr * (dp[n][e] - md[col]);
           }
@@ -475,16 +500,26 @@ cudaError_t launch_d(const BackwardParams& p, cudaStream_t stream) {
   e = cudaFuncSetAttribute(attn_bwd_dkv_mma_kernel<D, DC>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dkv_smem);
   if (e != cudaSuccess) return e;
+  // D of every row goes to the first T H floats of d_q, read by the dK / dV
+  // kernel; the dQ kernel, launched after it, computes D of its own rows and
+  // overwrites d_q.
+  if (p.max_kv_len > 0) {
+    float* delta = p.d_q;
+    const long long rows = (long long)p.T * p.H;
+    attn_bwd_delta_kernel<D><<<(unsigned)((rows * 8 + 255) / 256), 256, 0, stream>>>(p, delta);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const unsigned key_blocks = (unsigned)((p.max_kv_len + kKeys - 1) / kKeys);
+    attn_bwd_dkv_mma_kernel<D, DC><<<dim3(key_blocks, (unsigned)p.batch,
+                                          (unsigned)(p.Hk * (D / DC))),
+                                     kThreads, dkv_smem, stream>>>(p, delta);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   const int tpb = kRows / p.G;
   const unsigned row_blocks = (unsigned)max(1, (p.max_q_len + tpb - 1) / tpb);
   attn_bwd_dq_mma_kernel<D><<<dim3(row_blocks, (unsigned)p.batch, (unsigned)p.Hk), kThreads,
                               dq_smem, stream>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || p.max_kv_len == 0) return e;
-  const unsigned key_blocks = (unsigned)((p.max_kv_len + kKeys - 1) / kKeys);
-  attn_bwd_dkv_mma_kernel<D, DC><<<dim3(key_blocks, (unsigned)p.batch,
-                                        (unsigned)(p.Hk * (D / DC))),
-                                   kThreads, dkv_smem, stream>>>(p);
   return cudaGetLastError();
 }
 
