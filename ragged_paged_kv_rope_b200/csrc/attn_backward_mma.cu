@@ -238,6 +238,11 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_dq_mma_kernel(const Backwar
   float dq[NT][4];
 #pragma unroll
   for (int n = 0; n < NT; ++n) dq[n][0] = dq[n][1] = dq[n][2] = dq[n][3] = 0.f;
+  // Up to head_dim 128 the warp's Q and dO fragments stay in registers for the
+  // whole key walk; at 256 they are re-read from shared memory.
+  constexpr bool kFragRegs = D <= 128;
+  constexpr int KF = kFragRegs ? D / 16 : 1;
+  uint32_t qf[KF][4], gf[KF][4];
 
   const float sl2 = p.scale * kLog2eMma;
   if (kt <= hi_tile) {
@@ -256,6 +261,13 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_dq_mma_kernel(const Backwar
         cp_async_wait<0>();
       }
       __syncthreads();
+      if (kFragRegs && it == 0) {
+#pragma unroll
+        for (int ks = 0; ks < KF; ++ks) {
+          ldsm_x4(a_addr<D>(sQ, lane, warp * 16, ks), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+          ldsm_x4(a_addr<D>(sG, lane, warp * 16, ks), gf[ks][0], gf[ks][1], gf[ks][2], gf[ks][3]);
+        }
+      }
       const uint32_t k_t = sK + st * TB, v_t = sV + st * TB;
       const int key0 = kt * kKeys;
 #pragma unroll 1
@@ -268,8 +280,13 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_dq_mma_kernel(const Backwar
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           uint32_t aq[4], ag[4];
-          ldsm_x4(a_addr<D>(sQ, lane, warp * 16, ks), aq[0], aq[1], aq[2], aq[3]);
-          ldsm_x4(a_addr<D>(sG, lane, warp * 16, ks), ag[0], ag[1], ag[2], ag[3]);
+          if constexpr (kFragRegs) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) aq[i] = qf[ks][i], ag[i] = gf[ks][i];
+          } else {
+            ldsm_x4(a_addr<D>(sQ, lane, warp * 16, ks), aq[0], aq[1], aq[2], aq[3]);
+            ldsm_x4(a_addr<D>(sG, lane, warp * 16, ks), ag[0], ag[1], ag[2], ag[3]);
+          }
 #pragma unroll
           for (int np = 0; np < 2; ++np) {
             uint32_t b0, b1, b2, b3;
