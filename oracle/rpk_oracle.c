@@ -616,7 +616,7 @@ int rpko_attention_backward(const void* q, const void* d_out, int dtype, const i
     int32_t k_len = kv_lens[b];
     int32_t r = t - q_offsets[b];
     for (int32_t h = 0; h < n_heads && status == RPKO_OK; ++h) {
-      int kvh = h / group;
+      int kv_head = h / group;
       size_t qb = ((size_t)t * n_heads + h) * d;
       /* visible keys: scores, then weights */
       int64_t n = 0;
@@ -627,10 +627,10 @@ int rpko_attention_backward(const void* q, const void* d_out, int dtype, const i
         if (pi >= max_pages_per_seq) { status = RPKO_ERR_PAGE; break; }
         int32_t page = block_table[(size_t)b * max_pages_per_seq + pi];
         if (page < 0 || page >= num_pages) { status = RPKO_ERR_PAGE; break; }
-        base[n] = (((size_t)page * page_size + j % page_size) * n_kv_heads + kvh) * d;
+        base[n] = (((size_t)page * page_size + j % page_size) * n_kv_heads + kv_head) * d;
         double acc = 0.0;
         for (int c = 0; c < d; ++c)
-          acc += load_elt(q, dtype, qb + c) * load_cache(&J, k_pages, k_scale, kvh, base[n] + c);
+          acc += load_elt(q, dtype, qb + c) * load_cache(&J, k_pages, k_scale, kv_head, base[n] + c);
         p[n] = scale * acc;
         if (p[n] > m) m = p[n];
         ++n;
@@ -646,14 +646,14 @@ int rpko_attention_backward(const void* q, const void* d_out, int dtype, const i
         p[i] /= den;
         double acc = 0.0;
         for (int c = 0; c < d; ++c)
-          acc += load_elt(d_out, dtype, qb + c) * load_cache(&J, v_pages, v_scale, kvh, base[i] + c);
+          acc += load_elt(d_out, dtype, qb + c) * load_cache(&J, v_pages, v_scale, kv_head, base[i] + c);
         dp[i] = acc;
         D += p[i] * dp[i];
       }
       for (int64_t i = 0; i < n; ++i) {
         double ds = p[i] * (dp[i] - D);
         for (int c = 0; c < d; ++c) {
-          d_q[qb + c] += scale * ds * load_cache(&J, k_pages, k_scale, kvh, base[i] + c);
+          d_q[qb + c] += scale * ds * load_cache(&J, k_pages, k_scale, kv_head, base[i] + c);
           d_k[base[i] + c] += scale * ds * load_elt(q, dtype, qb + c);
           d_v[base[i] + c] += p[i] * load_elt(d_out, dtype, qb + c);
         }
