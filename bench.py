@@ -1,7 +1,7 @@
 """Benchmark of the fused RoPE + paged-KV + ragged-attention path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rpk|reference]
-                    [--workload NAME] [--no-prefill] [--no-cpu-baseline]
+                    [--workload NAME] [--no-prefill] [--no-backward] [--no-cpu-baseline]
 
 One step is one pass of the whole path over one batch: rope_qk_paged_ragged
 for the batch's new tokens (RoPE on Q and K, K/V written into the paged
@@ -10,7 +10,9 @@ workload is the Llama-3-8B-shaped decode batch (64 sequences, 1 new token
 each, cached contexts U[512, 8192], 32 q / 8 kv heads, d 128, page 64); its
 metric is the K/V bytes attention reads per second. Every run also measures
 the ragged causal prefill workload (16 sequences of U[128, 4096] tokens) in
-TFLOP/s of visible (query, key) pairs, reported under "prefill".
+TFLOP/s of visible (query, key) pairs, reported under "prefill", and the
+attention backward on that workload (query, key and value gradients from the
+forward's output and log-sum-exp), reported under "backward".
 
 Under torchrun each rank runs its own batch (a different seed): sequences are
 independent, so the path shards with no exchange (weak scaling); the time is
@@ -56,8 +58,8 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--backward", action="store_true",
-                    help="also time the attention backward on the ragged prefill workload")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip timing the attention backward on the ragged prefill workload")
     ap.add_argument("--cache-dtype", default=None, choices=["e4m3"],
                     help="hold the KV cache as e4m3 codes with per-head scales")
     return ap.parse_args()
@@ -604,7 +606,7 @@ def main():
                "note": "pinned host inputs copied in, output copied out, inside the timed region"}
 
     prefill = None if args.no_prefill else prefill_measure(device, world)
-    backward = backward_measure(device, world) if args.backward else None
+    backward = None if args.no_backward else backward_measure(device, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -285,7 +285,9 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
  *   out             the forward's output [total_q_tokens, n_heads, head_dim] dtype
  *   d_out           [total_q_tokens, n_heads, head_dim] dtype, the output gradient
  *   log_sum_exp     float32 [total_q_tokens, n_heads], the forward's log_sum_exp
- *   d_q             float32 [total_q_tokens, n_heads, head_dim] (written)
+ *   d_q             float32 [total_q_tokens, n_heads, head_dim] (written; on
+ *                   the tensor-core path its memory also holds each row's D_i
+ *                   between the call's kernels)
  *   d_k_pages,      float32, the shape of one layer's pools
  *   d_v_pages       [num_pages, page_size, n_kv_heads, head_dim]: the entry of
  *                   every key below kv_lens[b] of each sequence is written (the
@@ -293,9 +295,14 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
  *                   of its dequantised value); other entries are left as they
  *                   were, so a caller that sums over the pool zeroes them first.
  *
- * CUDA-core kernels in fp32 (a row-parallel one for d_q, a key-parallel one
- * for d_k and d_v; no atomics). Errors as ragged_paged_attention; every pointer
- * is 16-byte aligned device memory; buffers must not overlap.
+ * bf16 tensors over a bf16 cache with groups of at most 16 query heads run on
+ * warp-level tensor cores (bf16 operands, fp32 sums; P and dS are rounded to
+ * bf16 as operands of the second products). The kernels are: D_i of every
+ * row, a key-parallel one for d_k and d_v, then a row-parallel one for d_q.
+ * Other shapes (fp32 tensors, an e4m3 cache, larger groups) run on CUDA-core
+ * kernels in fp32. Neither path uses atomics, so results are deterministic.
+ * Errors as ragged_paged_attention; every pointer is 16-byte aligned device
+ * memory; buffers must not overlap.
  */
 rpk_status ragged_paged_attention_backward(
     const void* q, const int32_t* q_row_offsets, const int32_t* kv_lens,
