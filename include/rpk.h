@@ -220,6 +220,8 @@ size_t ragged_paged_attention_workspace_size(int32_t total_q_tokens, int32_t n_h
  *   page_table      the cache (host struct); cache_lens is not read
  *   scale           finite > 0 (1/sqrt(head_dim) for plain SDPA)
  *   window          <= 0: unbounded; w > 0: w keys including the row's own
+ *                   (w >= max_kv_len covers every key a row sees: unbounded,
+ *                   and sink_tokens then has no effect)
  *   out             [total_q_tokens, n_heads, head_dim] dtype
  *   batch, total_q_tokens, max_q_len, max_kv_len: sizes (host); max_q_len and
  *                   max_kv_len bound q_len[b] and kv_lens[b] (device data) and

@@ -250,7 +250,6 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
 
   rpk::AttnParams p;
   p.lse = log_sum_exp;
-  p.sinks = window > 0 ? sink_tokens : 0;
   p.q = q; p.out = out;
   {
     void *k, *v;
@@ -262,7 +261,9 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
   p.T = total_q_tokens; p.batch = batch; p.H = n_heads; p.Hk = n_kv_heads;
   p.G = n_heads / n_kv_heads; p.d = head_dim; p.P = page_table->page_size;
   p.num_pages = page_table->num_pages; p.max_pages = page_table->max_pages_per_seq;
-  p.window = window > 0 ? window : 0; p.max_q_len = max_q_len; p.max_kv_len = max_kv_len;
+  p.window = rpk::effective_window(window, max_kv_len);
+  p.sinks = p.window > 0 ? sink_tokens : 0;
+  p.max_q_len = max_q_len; p.max_kv_len = max_kv_len;
   p.scale = scale;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
   p.cache_fp8 = page_table->cache_dtype == RPK_E4M3;
@@ -366,8 +367,9 @@ rpk_status ragged_paged_attention_backward(
   p.T = total_q_tokens; p.batch = batch; p.H = n_heads; p.Hk = n_kv_heads;
   p.G = n_heads / n_kv_heads; p.d = head_dim; p.P = page_table->page_size;
   p.num_pages = page_table->num_pages; p.max_pages = page_table->max_pages_per_seq;
-  p.window = window > 0 ? window : 0; p.max_q_len = max_q_len; p.max_kv_len = max_kv_len;
-  p.sinks = window > 0 ? sink_tokens : 0;
+  p.window = rpk::effective_window(window, max_kv_len);
+  p.sinks = p.window > 0 ? sink_tokens : 0;
+  p.max_q_len = max_q_len; p.max_kv_len = max_kv_len;
   p.scale = scale;
   p.cache_fp8 = page_table->cache_dtype == RPK_E4M3;
   p.k_scale = page_table->k_scale;

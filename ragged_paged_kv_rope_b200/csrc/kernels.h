@@ -13,6 +13,13 @@ namespace rpk {
 // The pools of the layer a call uses: layer layer_idx of num_layers (0 means
 // one) layer-major copies of [num_pages, page_size, n_kv_heads, head_dim].
 // False when layer_idx is out of range.
+// The window a launch uses: 0 (unbounded) for window <= 0 and for a window of
+// at least max_kv_len keys, which already covers every key a row can see;
+// otherwise the window itself. Keeps the band arithmetic far from int overflow.
+inline int32_t effective_window(int32_t window, int32_t max_kv_len) {
+  return window > 0 && window < max_kv_len ? window : 0;
+}
+
 inline bool layer_pools(const rpk_paged_kv* c, void** k, void** v) {
   const int32_t layers = c->num_layers > 0 ? c->num_layers : 1;
   if (c->num_layers < 0 || c->layer_idx < 0 || c->layer_idx >= layers) return false;

@@ -138,6 +138,20 @@ def test_attention_sinks_ignored_without_window():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+def test_attention_window_covering_every_key_is_unbounded():
+    # a window of at least max_kv_len keys bounds nothing (sinks included), up to
+    # the largest int32 window: the result equals the unbounded one bit for bit
+    sp = W.spec("ragged_prefill", n_heads=8, n_kv_heads=2, batch=2)
+    wl = W.attention_only(sp, 52, [70, 1], [70, 500])
+    dev = to_device(wl)
+    a = gpu_attention(wl, dev, dev.q, window=0).cpu()
+    for w in (wl.max_kv_len, 2**31 - 1):
+        b = gpu_attention(wl, dev, dev.q, window=w, sinks=3).cpu()
+        torch.cuda.synchronize()
+        assert int(dev.error_word.item()) == 0
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), w
+
+
 @pytest.mark.slow
 def test_attention_gemma_window_with_sinks_sampled():
     # the Gemma-like sliding-window decode at full context, with 4 sink tokens
