@@ -355,13 +355,16 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_dkv_mma_kernel(const Backwa
   float* m_delta = m_lse + 2 * kRows;                           // [2][64]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, c = lane & 3;
+  // grid (KV head x channel half, sequence, key block): the key block varies
+  // slowest, so the first key blocks of every sequence (those the most rows
+  // see) are the first to run and the short ones fill the tail
   const int b = blockIdx.y;
-  const int kvh = blockIdx.z / kSplit, ch0 = (blockIdx.z % kSplit) * DC;
+  const int kvh = blockIdx.x / kSplit, ch0 = (blockIdx.x % kSplit) * DC;
   const int G = p.G, tpb = kRows / G;
   const int q0 = __ldg(p.offsets + b);
   const int q_len = __ldg(p.offsets + b + 1) - q0;
   const int k_len = __ldg(p.kv_lens + b);
-  const int key0 = blockIdx.x * kKeys;
+  const int key0 = blockIdx.z * kKeys;
   // bad lengths are reported by the dQ kernel
   if (k_len < 0 || k_len > p.max_kv_len || q_len > p.max_q_len || key0 >= k_len) return;
   const int off = k_len - q_len;
@@ -527,8 +530,8 @@ cudaError_t launch_d(const BackwardParams& p, cudaStream_t stream) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const unsigned key_blocks = (unsigned)((p.max_kv_len + kKeys - 1) / kKeys);
-    attn_bwd_dkv_mma_kernel<D, DC><<<dim3(key_blocks, (unsigned)p.batch,
-                                          (unsigned)(p.Hk * (D / DC))),
+    attn_bwd_dkv_mma_kernel<D, DC><<<dim3((unsigned)(p.Hk * (D / DC)), (unsigned)p.batch,
+                                          key_blocks),
                                      kThreads, dkv_smem, stream>>>(p, delta);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
