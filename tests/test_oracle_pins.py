@@ -27,8 +27,10 @@ def paged(k_dense, v_dense, page_size, seed=0, spare=3, dtype=np.float32):
     total = sum(n_pages) + spare
     perm = rng.permutation(total)
     Hk, d = k_dense[0].shape[1:]
-    kp = np.full((total, page_size, Hk, d), np.nan, dtype=dtype)
-    vp = np.full((total, page_size, Hk, d), np.nan, dtype=dtype)
+    # unused slots hold NaN (for e4m3 codes, 0x7F: the format's NaN)
+    fill = 0x7F if dtype == np.uint8 else np.nan
+    kp = np.full((total, page_size, Hk, d), fill, dtype=dtype)
+    vp = np.full((total, page_size, Hk, d), fill, dtype=dtype)
     bt = np.full((len(k_dense), max(1, max(n_pages))), -1, dtype=np.int32)
     cur = 0
     for b, (k, v) in enumerate(zip(k_dense, v_dense)):
