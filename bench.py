@@ -1,18 +1,24 @@
 """Benchmark of the fused RoPE + paged-KV + ragged-attention path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rpk|reference]
-                    [--workload NAME] [--no-prefill] [--no-backward] [--no-cpu-baseline]
+                    [--workload NAME] [--no-workloads] [--no-backward] [--no-cpu-baseline]
 
 One step is one pass of the whole path over one batch: rope_qk_paged_ragged
 for the batch's new tokens (RoPE on Q and K, K/V written into the paged
 cache) followed by ragged_paged_attention over the cache. The default
 workload is the Llama-3-8B-shaped decode batch (64 sequences, 1 new token
 each, cached contexts U[512, 8192], 32 q / 8 kv heads, d 128, page 64); its
-metric is the K/V bytes attention reads per second. Every run also measures
-the ragged causal prefill workload (16 sequences of U[128, 4096] tokens) in
-TFLOP/s of visible (query, key) pairs, reported under "prefill", and the
-attention backward on that workload (query, key and value gradients from the
-forward's output and log-sum-exp), reported under "backward".
+metric is the K/V bytes attention reads per second.
+
+Every run also measures the four other workloads, each on its own timed loop
+of at least 200 ms of device time, reported under "workloads" with its own
+roofline, RoPE + scatter bandwidth, clocks and oracle baseline: the fp32 tiny
+prefill (launch-bound), the Gemma-like sliding-window decode (K/V bytes of the
+window per second), the ragged causal prefill (16 sequences of U[128, 4096]
+tokens) and the mixed chunked M-RoPE prefill (TFLOP/s of visible (query, key)
+pairs). The attention backward on the ragged prefill workload (query, key and
+value gradients from the forward's output and log-sum-exp) is reported under
+"backward".
 
 Under torchrun each rank runs its own batch (a different seed): sequences are
 independent, so the path shards with no exchange (weak scaling); the time is
@@ -25,6 +31,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -55,7 +62,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
-    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-workloads", "--no-prefill", dest="no_workloads", action="store_true",
+                    help="time only the chosen workload (not the other four)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-backward", action="store_true",
@@ -388,30 +396,110 @@ def time_e2e(step: Step, steps: int, warmup: int, world: int):
     return a.elapsed_time(b) / steps, h2d, d2h
 
 
-def prefill_measure(device, world, steps=5, warmup=3):
-    wl = W.make("ragged_prefill", seed=0)
-    step = Step(wl, device)
-    total, rope_ms, attn_ms = time_steps(step, steps, warmup, world)
+def steps_for(ms_one: float, min_ms: float = 200.0, lo: int = 5, hi: int = 20000) -> int:
+    """Loop count whose timed region lasts at least min_ms of device time."""
+    return int(min(hi, max(lo, math.ceil(min_ms / max(ms_one, 1e-3)))))
+
+
+def one_step_ms(step: "Step") -> float:
+    """Device time of one warm step (RoPE + attention), to size a timed loop."""
+    stream = torch.cuda.current_stream()
+    for _ in range(2):
+        step.rope()
+        step.attention()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    step.rope()
+    step.attention()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
+def kernel_of(wl: W.Workload) -> tuple[str, str]:
+    """(traffic key prefix, description) of the kernel the attention call runs."""
     sp = wl.spec
-    flops = M.attention_flops(wl.q_lens, wl.kv_lens, sp.window, sp.n_heads, sp.head_dim)
+    if sp.dtype != "bf16":
+        return "attn_simt", "ragged_paged_attention (CUDA-core fp32 kernel)"
+    if is_decode(wl):
+        return "attn_decode", "ragged_paged_attention (split-KV decode + combine)"
+    if sp.head_dim in (64, 128) and sp.cache_dtype is None:
+        return "attn_prefill", "ragged_paged_attention (tcgen05 prefill)"
+    return "attn_simt", "ragged_paged_attention (CUDA-core kernel)"
+
+
+def measure_workload(name: str, device, world: int, local: int, rank: int, seed: int,
+                     cpu_s: float | None):
+    """One workload measured on its own: a timed loop of at least 200 ms of
+    device time (RoPE + attention per step, CUDA events on the launching
+    stream), its attention roofline, its RoPE + scatter bandwidth, the clocks
+    sampled during its timed loop and the oracle on a bounded sample."""
+    wl = W.make(name, seed=rank_seed(seed, rank))
+    sp = wl.spec
+    step = Step(wl, device)
+    metric, unit, amount, scale = metric_of(wl)
+    n = steps_for(one_step_ms(step))
+    with ClockSampler(local) as clocks:
+        total_ms, rope_ms, attn_ms = time_steps(step, n, 3, world, clocks)
+    clk = clocks.summary()
+    step_ms = max_over_ranks(total_ms / n, world)
     attn = max_over_ranks(statistics.mean(attn_ms), world)
-    peaks = load_peaks()
-    tflops = flops / (attn * 1e-3) / 1e12
-    rope_b = M.rope_bytes(wl.total_tokens, sp.n_heads, sp.n_kv_heads, sp.head_dim,
-                          sp.rotary_dim, 2)
     rope = max_over_ranks(statistics.mean(rope_ms), world)
-    return {
-        "workload": "ragged_prefill", "total_tokens": wl.total_tokens,
-        "attention_tflops": tflops, "tensor_peak_tflops": peaks["bf16_tflops"],
-        "frac": tflops / peaks["bf16_tflops"], "attention_ms": attn,
-        "visible_pair_flops": flops, "rope_ms": rope,
-        "rope_gbs": rope_b / (rope * 1e-3) / 1e9,
-        "tokens_per_s": whole_job_throughput(wl.total_tokens, total / steps * 1e-3, world),
+    peaks = load_peaks()
+    key, kdesc = kernel_of(wl)
+    achieved = amount / (attn * 1e-3) / scale
+    traffic = load_traffic(f"{key}@{name}")
+    if sp.dtype != "bf16":
+        roofline = {"bound": "launch", "kernel": kdesc, "achieved": achieved, "unit": unit,
+                    "note": "fp32 correctness workload of a few hundred kFLOP: the step is "
+                            "launch latency, no roofline applies"}
+    elif is_decode(wl):
+        roofline = {"bound": "hbm", "kernel": kdesc, "achieved": achieved,
+                    "peak": peaks["hbm_gbs"], "unit": unit, "frac": achieved / peaks["hbm_gbs"],
+                    "traffic": None if traffic is None else traffic["bytes_per_launch"],
+                    "algorithmic_bytes_per_launch": amount,
+                    "peak_source": f"{peaks['source']} hbm_gbs"}
+    else:
+        roofline = {"bound": "tensor", "kernel": kdesc, "achieved": achieved,
+                    "peak": peaks["bf16_tflops"], "unit": unit,
+                    "frac": achieved / peaks["bf16_tflops"],
+                    "traffic": None if traffic is None else traffic["bytes_per_launch"],
+                    "algorithmic_flops_per_launch": amount,
+                    "peak_source": f"{peaks['source']} bf16_tflops (burst: kernel timed alone)"}
+    elt = 4 if sp.dtype == "f32" else 2
+    rope_b = M.rope_bytes(wl.total_tokens, sp.n_heads, sp.n_kv_heads, sp.head_dim,
+                          sp.rotary_dim, elt)
+    rope_traffic = load_traffic(f"rope@{name}")
+    rope_gbs = rope_b / (rope * 1e-3) / 1e9
+    entry = {
+        "metric": metric, "value": sum_over_ranks(amount, world) / (step_ms * 1e-3) / scale,
+        "unit": unit, "steps": n, "warmup": 3, "ms_per_step": step_ms,
+        "description": sp.description, "new_tokens_per_step": wl.total_tokens,
+        "tokens_per_s": sum_over_ranks(wl.total_tokens, world) / (step_ms * 1e-3),
+        "breakdown_ms": {"rope_qk_paged_ragged": rope, "ragged_paged_attention": attn},
+        "roofline": roofline,
+        "rope_roofline": {"bound": "hbm", "kernel": "rope_scatter_kernel", "achieved": rope_gbs,
+                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": rope_gbs / peaks["hbm_gbs"],
+                          "traffic": None if rope_traffic is None
+                          else rope_traffic["bytes_per_launch"],
+                          "algorithmic_bytes_per_launch": rope_b},
+        "clocks": clk,
+        "gpu_launches": step.launches_per_step() * n,
         "error_word": int(step.error_word.item()),
+        "l2": "inputs larger than L2" if (wl.k_pages.numel() * wl.k_pages.element_size() * 2
+                                          + wl.q.numel() * wl.q.element_size() * 3
+                                          > L2_BYTES) else "inputs fit in L2 (launch-bound case)",
     }
+    if cpu_s is not None and rank == 0 and world == 1:
+        entry["cpu_baseline"] = cpu_baseline(wl, unit, scale, budget_s=cpu_s,
+                                             per_pass_s=cpu_s / 2)
+    del step
+    torch.cuda.empty_cache()
+    return entry
 
 
-def backward_measure(device, world, steps=5, warmup=3):
+def backward_measure(device, world, warmup=3):
     """The attention backward (its two kernels) on the ragged prefill workload:
     the forward runs once for the output and log-sum-exp, then the backward is
     timed with a seeded N(0, 1) output gradient. Algorithmic FLOPs are 2.5x the
@@ -444,6 +532,12 @@ def backward_measure(device, world, steps=5, warmup=3):
     for _ in range(warmup):
         run()
     torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    run()
+    b.record()
+    torch.cuda.synchronize()
+    steps = steps_for(a.elapsed_time(b))
     barrier(world)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
@@ -459,7 +553,7 @@ def backward_measure(device, world, steps=5, warmup=3):
     kernel = ("tensor-core (mma.sync) dQ and dK/dV kernels"
               if sp.dtype == "bf16" and sp.n_heads // sp.n_kv_heads <= 16
               else "CUDA-core dQ and dK/dV kernels")
-    return {"workload": "ragged_prefill", "kernel": kernel, "backward_ms": ms,
+    return {"workload": "ragged_prefill", "kernel": kernel, "backward_ms": ms, "steps": steps,
             "algorithmic_flops": flops, "tflops": tflops,
             "tensor_peak_tflops": peaks["bf16_tflops"], "frac": tflops / peaks["bf16_tflops"],
             "error_word": int(step.error_word.item())}
@@ -497,10 +591,23 @@ def metric_of(wl: W.Workload):
 
 # -------------------------------------------------------- the oracle on CPU
 
-def oracle_sample_time(wl: W.Workload, max_seconds: float = 20.0):
+def _row_visible(wl: W.Workload, b: int) -> np.ndarray:
+    """Visible keys of each row (token) of sequence b under the workload's band."""
+    sp = wl.spec
+    lo, hi = M._bands(int(wl.q_lens[b]), int(wl.kv_lens[b]), sp.window)
+    return np.maximum(hi - lo + 1, 0)
+
+
+def oracle_sample_time(wl: W.Workload, max_seconds: float = 20.0, chunk_tokens: int = 128):
     """Time the fp64 oracle (RoPE, cache image, attention) on a bounded sample
-    of the workload's sequences; returns (seconds, amount, tokens, sample,
-    threads), amount in the workload's unit (K/V bytes or visible-pair FLOPs)."""
+    of the workload; returns (seconds, amount, tokens, sample, threads), amount
+    in the workload's unit (K/V bytes or visible-pair FLOPs).
+
+    RoPE and the cache image run over the whole batch and are charged in
+    proportion to the rows sampled. Attention runs sequence by sequence, all
+    query heads of `chunk_tokens` tokens at a time, until the time budget is
+    used: a decode sequence counts its K/V bytes once all its rows are done,
+    a prefill chunk counts 4 d FLOPs per visible (row, key) pair."""
     import oracle as O
     sp = wl.spec
     table = O.freqs_cis(wl.max_position, sp.rotary_dim, sp.theta)
@@ -517,31 +624,54 @@ def oracle_sample_time(wl: W.Workload, max_seconds: float = 20.0):
                   inplace=True)
     qr = O.round_to(q_rot, code)
     t_rope = time.perf_counter() - t0
-    # attention one sequence at a time until the time budget is used
-    done_b, kv_bytes, flops, toks = 0, 0, 0, 0
-    t1 = time.perf_counter()
+    decode = is_decode(wl)
     elt = cache_elt(wl)
+    H = sp.n_heads
+    done_seq, done_tok, amount = 0, 0, 0
+    t1 = time.perf_counter()
+    out_of_time = False
     for b in range(sp.batch):
         lo, hi = int(wl.q_offsets[b]), int(wl.q_offsets[b + 1])
-        rows = np.array([[t, h] for t in range(lo, hi) for h in range(sp.n_heads)], np.int32)
-        if len(rows):
+        vis = _row_visible(wl, b)
+        step = (hi - lo) if decode else chunk_tokens
+        for t0_ in range(lo, hi, max(1, step)):
+            t1_ = min(hi, t0_ + max(1, step))
+            rows = np.array([[t, h] for t in range(t0_, t1_) for h in range(H)], np.int32)
             O.attention(qr, wl.q_offsets, wl.kv_lens, kp, vp, wl.block_table, sp.n_kv_heads,
                         sp.softmax_scale, sp.window, rows=rows, n_threads=threads)
-        done_b += 1
-        kv_bytes += M.attention_kv_bytes(wl.q_lens[b:b + 1], wl.kv_lens[b:b + 1], sp.window,
-                                         sp.n_kv_heads, sp.head_dim, elt)
-        flops += M.attention_flops(wl.q_lens[b:b + 1], wl.kv_lens[b:b + 1], sp.window,
-                                   sp.n_heads, sp.head_dim)
-        toks += hi - lo
-        if time.perf_counter() - t1 > max_seconds:
+            done_tok += t1_ - t0_
+            if not decode:
+                amount += 4 * H * sp.head_dim * int(vis[t0_ - lo:t1_ - lo].sum())
+            if time.perf_counter() - t1 > max_seconds:
+                out_of_time = True
+                break
+        if decode and not out_of_time:
+            amount += M.attention_kv_bytes(wl.q_lens[b:b + 1], wl.kv_lens[b:b + 1], sp.window,
+                                           sp.n_kv_heads, sp.head_dim, elt)
+            done_seq += 1
+        if out_of_time:
             break
     t_attn = time.perf_counter() - t1
-    # RoPE ran over the whole batch; charge the sampled sequences their share
-    share = done_b / sp.batch
+    share = done_tok / max(1, wl.total_tokens)
     seconds = t_attn + t_rope * share
-    amount = kv_bytes if is_decode(wl) else flops
-    return seconds, amount, toks, f"{done_b} of {sp.batch} sequences (all rows), " \
-                                  f"RoPE + cache image + attention", threads
+    if decode:
+        sample = f"{done_seq} of {sp.batch} sequences (all rows), RoPE + cache image + attention"
+    else:
+        sample = (f"{done_tok} of {wl.total_tokens} query tokens (all heads, the first "
+                  f"sequences in order), RoPE + cache image + attention")
+    return seconds, amount, done_tok, sample, threads
+
+
+def cpu_baseline(wl: W.Workload, unit: str, scale: float, budget_s: float, per_pass_s: float):
+    """Whole passes of the oracle over a bounded sample, about budget_s seconds."""
+    total_s, total_amount, passes, t_all = 0.0, 0, 0, time.perf_counter()
+    while passes < 1 or (time.perf_counter() - t_all < budget_s and passes < 50):
+        secs, amount, toks, sample, threads = oracle_sample_time(wl, max_seconds=per_pass_s)
+        total_s += secs
+        total_amount += amount
+        passes += 1
+    return {"value": total_amount / total_s / scale, "unit": unit, "cores": threads,
+            "kind": "oracle", "sample": f"{sample}; {passes} passes", "seconds": total_s}
 
 
 # --------------------------------------------------------------------- main
@@ -605,20 +735,25 @@ def main():
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "note": "pinned host inputs copied in, output copied out, inside the timed region"}
 
-    prefill = None if args.no_prefill else prefill_measure(device, world)
+    launches = step.launches_per_step() * args.steps
+    del step
+    torch.cuda.empty_cache()
+    workloads = {}
+    if not args.no_workloads:
+        # every other workload, each measured on its own timed loop
+        for name in ("tiny_prefill_f32", "gemma_swa_decode", "ragged_prefill",
+                     "mixed_chunked_mrope"):
+            if name == args.workload:
+                continue
+            workloads[name] = measure_workload(
+                name, device, world, local, rank, args.seed,
+                None if args.no_cpu_baseline else 4.0)
     backward = None if args.no_backward else backward_measure(device, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # whole passes of the oracle over (a bounded sample of) the batch, ~10-30 s in all
-        total_s, total_b, passes, t_all = 0.0, 0, 0, time.perf_counter()
-        while passes < 1 or (time.perf_counter() - t_all < 10.0 and passes < 50):
-            secs, kvb, toks, sample, threads = oracle_sample_time(wl)
-            total_s += secs
-            total_b += kvb
-            passes += 1
-        cpu = {"value": total_b / total_s / scale, "unit": unit, "cores": threads,
-               "kind": "oracle", "sample": f"{sample}; {passes} passes", "seconds": total_s}
+        cpu = cpu_baseline(wl, unit, scale, budget_s=10.0, per_pass_s=20.0)
 
     line = {
         "metric": metric, "value": value, "unit": unit,
@@ -638,9 +773,9 @@ def main():
         "roofline": roofline,
         "clocks": clk,
         "e2e": e2e,
-        "gpu_launches": step.launches_per_step() * args.steps,
+        "gpu_launches": launches,
         "error_word": err,
-        "prefill": prefill,
+        "workloads": workloads,
         "backward": backward,
         "cpu_baseline": cpu,
     }

@@ -324,10 +324,12 @@ rpk_status ragged_paged_attention_backward(
  * implicit synchronisation of cudaMalloc. They cannot supply the workspace
  * that ragged_paged_attention takes.
  *
- * Arguments and results are those of ragged_paged_attention, without the
- * workspace. It runs the same split-KV decode kernels, so it takes only the
- * decode shapes: dtype RPK_BF16 and max_q_len * (n_heads / n_kv_heads) <= 16.
- * Other shapes return RPK_ERR_UNSUPPORTED.
+ * Arguments and results are those of ragged_paged_attention without the
+ * workspace, the log_sum_exp output and the sink_tokens band (this entry point
+ * takes none of the three; sinks are off). It runs the same split-KV decode
+ * kernels, so it takes only the decode shapes: dtype RPK_BF16 over a bf16
+ * cache and max_q_len * (n_heads / n_kv_heads) <= 16. Other shapes return
+ * RPK_ERR_UNSUPPORTED.
  *
  * Scratch: the kernels' fp32 partials go to one array inside the library,
  * RPK_NOALLOC_SCRATCH_BYTES (32 MiB) per GPU, held from the moment the
@@ -338,6 +340,9 @@ rpk_status ragged_paged_attention_backward(
  *
  * The first call on each device looks up the array's device address and
  * caches it; make that first call before any stream capture on that device.
+ * The cached address belongs to the device's context: after cudaDeviceReset
+ * (or any destruction of the primary context) the address is stale, so do not
+ * call this entry point again in that process.
  *
  * All calls on a device share the one array, and it keeps whatever the last
  * call left in it. Nothing in it needs to start at zero. Calls whose kernels
@@ -353,6 +358,24 @@ rpk_status ragged_paged_attention_noalloc(const void* q, const int32_t* q_row_of
                                           int32_t window, void* out, int32_t batch,
                                           int32_t total_q_tokens, int32_t max_q_len,
                                           int32_t max_kv_len, rpk_dtype dtype, void* stream);
+
+/*
+ * rpk_set_wait_limit_ns -- the bound, in nanoseconds of the GPU's global
+ * timer, that every later attention launch gives each of its device-side
+ * waits (a stage of K/V tiles, a score tile, a work item). A wait that runs
+ * out makes its CTA give up: it ORs RPK_DEVERR_TIMEOUT into
+ * page_table->error_word, lets the copies and tensor-core operations it has
+ * already issued finish, frees its tensor memory and returns, so the context
+ * stays usable and later calls on the stream run normally (a kernel that finds
+ * RPK_DEVERR_TIMEOUT already set in the error word also stops early, so clear
+ * the word before relying on later results). The pages have no counterpart;
+ * this is the library's failure detection (no wait is unbounded, nothing
+ * traps). 0 restores the default of 2 seconds. The setting is process-wide
+ * and read when a call is made; waits for copies already in flight during a
+ * give-up keep the default bound.
+ */
+void rpk_set_wait_limit_ns(uint64_t limit_ns);
+uint64_t rpk_wait_limit_ns(void);
 
 /* Static text for a status code. */
 const char* rpk_status_string(rpk_status status);

@@ -23,4 +23,6 @@ from .binding import (  # noqa: F401
     ragged_paged_attention_backward,
     ragged_paged_attention_workspace_size,
     rope_qk_paged_ragged,
+    set_wait_limit_ns,
+    wait_limit_ns,
 )

@@ -13,6 +13,8 @@ Entry points keep the C names:
 * ``ragged_paged_attention_workspace_size``
 * ``freqs_cis``             builds the fp32 (cos, sin) table with ``rope_freqs_cis``
 * ``freqs_cis_proportional`` builds the p-RoPE table with ``rope_freqs_cis_proportional``
+* ``ragged_paged_attention_noalloc`` the decode path with library-owned scratch
+* ``set_wait_limit_ns`` / ``wait_limit_ns`` the bound of the kernels' device-side waits
 """
 
 from __future__ import annotations
@@ -87,6 +89,10 @@ def lib():
         L.rpk_status_string.restype = C.c_char_p
         L.rpk_last_cuda_error.argtypes = []
         L.rpk_last_cuda_error.restype = C.c_char_p
+        L.rpk_set_wait_limit_ns.argtypes = [C.c_uint64]
+        L.rpk_set_wait_limit_ns.restype = None
+        L.rpk_wait_limit_ns.argtypes = []
+        L.rpk_wait_limit_ns.restype = C.c_uint64
         _lib = L
     return _lib
 
@@ -95,7 +101,8 @@ def header_symbols() -> list[str]:
     """Names of the functions include/rpk.h declares."""
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return re.findall(r"^\s*(?:rpk_status|size_t|const char\*)\s+(\w+)\s*\(", text, flags=re.M)
+    return re.findall(r"^\s*(?:rpk_status|size_t|const char\*|void|uint64_t)\s+(\w+)\s*\(", text,
+                      flags=re.M)
 
 
 def _check(status: int):
@@ -348,6 +355,16 @@ def ragged_paged_attention_backward(q, q_row_offsets, kv_lens, page_table: Paged
               float(scale), int(window), op, gp, lp, dq, d_k_pages.data_ptr(),
               d_v_pages.data_ptr(), int(kv_lens.shape[0]), T, int(max_q_len), int(max_kv_len),
               _dtype_code(q.dtype), int(sink_tokens), _stream(stream)))
+
+
+def set_wait_limit_ns(limit_ns: int) -> None:
+    """Bound (ns of the GPU timer) of every device-side wait of later attention
+    launches (``rpk_set_wait_limit_ns``); 0 restores the 2 s default."""
+    lib().rpk_set_wait_limit_ns(int(limit_ns))
+
+
+def wait_limit_ns() -> int:
+    return int(lib().rpk_wait_limit_ns())
 
 
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024

@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
       bool ok = true;
       for (int i = 0; i < n_tiles && ok; ++i) {
         const int s = i % S;
-        if (!mbar_wait(&empty_bar[s], ((i / S) & 1) ^ 1)) { ok = false; break; }
+        if (!mbar_wait(&empty_bar[s], ((i / S) & 1) ^ 1, p.wait_ns)) { ok = false; break; }
         const int key0 = ss.tile_at(v_begin + i) * kDecodeTile;
         // Count the boxes to load (pages wholly past k_len or invalid are skipped).
         uint32_t bytes = 0;
@@ -423,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
 
   for (int i = 0; i < n_tiles; ++i) {
     const int s = i % S;
-    if (!mbar_wait(&full_bar[s], (i / S) & 1)) { ok = false; break; }
+    if (!mbar_wait(&full_bar[s], (i / S) & 1, p.wait_ns)) { ok = false; break; }
     const int key0 = ss.tile_at(v_begin + i) * kDecodeTile + warp * 16;  // this warp's 16 keys
     uint32_t kbase = smem_u32(k_stage(s));
     uint32_t vbase = smem_u32(v_stage(s));

@@ -19,7 +19,6 @@
 // allocator.
 #include <cuda.h>
 #include <cuda_runtime.h>
-#include <cudaTypedefs.h>
 
 #include <cmath>
 #include <mutex>
@@ -40,44 +39,22 @@ void* g_scratch_addr[kMaxDevices] = {};
 // Device address of g_decode_scratch on the current device; looked up once per device.
 rpk_status scratch_address(void** out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return RPK_ERR_CUDA;
-  if (dev >= kMaxDevices) return RPK_ERR_UNSUPPORTED;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return rpk::cuda_status(e);
+  if (dev < 0 || dev >= kMaxDevices) return RPK_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
   if (g_scratch_addr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr)
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return rpk::cuda_status(e);
+    if (p == nullptr) {
+      rpk::set_last_error_text("cudaGetSymbolAddress returned no address");
       return RPK_ERR_CUDA;
+    }
     g_scratch_addr[dev] = p;
   }
   *out = g_scratch_addr[dev];
   return RPK_OK;
-}
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-// 3-D bf16 tensor map over the pool viewed as [pages * page_size, heads, d]
-// with box (64, 1, box_rows) and 128-byte swizzle, as the decode kernel reads it.
-rpk_status pool_map(CUtensorMap* map, const void* base, int32_t d, int32_t heads, int64_t rows,
-                    int32_t box_rows) {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  if (!fn) return RPK_ERR_CUDA;
-  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
-  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
-  cuuint32_t box[3] = {64u, 1u, (cuuint32_t)box_rows};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? RPK_OK : RPK_ERR_CUDA;
 }
 
 }  // namespace
@@ -87,30 +64,24 @@ extern "C" rpk_status ragged_paged_attention_noalloc(
     const rpk_paged_kv* page_table, int32_t n_heads, int32_t n_kv_heads, int32_t head_dim,
     float scale, int32_t window, void* out, int32_t batch, int32_t total_q_tokens,
     int32_t max_q_len, int32_t max_kv_len, rpk_dtype dtype, void* stream) {
-  // Host-side checks, the same as ragged_paged_attention's.
-  if (!q || !q_row_offsets || !kv_lens || !out || !page_table) return RPK_ERR_NULL;
+  // Host-side checks, the same as ragged_paged_attention's (shared code).
+  if (!q || !q_row_offsets || !kv_lens || !out) return RPK_ERR_NULL;
+  rpk_status st = rpk::check_cache(page_table);
+  if (st != RPK_OK) return st;
   const rpk_paged_kv* c = page_table;
-  if (!c->k_pages || !c->v_pages || !c->block_table) return RPK_ERR_NULL;
-  if (c->cache_dtype != RPK_BF16 && c->cache_dtype != RPK_F32) return RPK_ERR_DTYPE;
   if (dtype != RPK_BF16 && dtype != RPK_F32) return RPK_ERR_DTYPE;
   if (dtype != c->cache_dtype) return RPK_ERR_DTYPE;
-  if (c->num_pages <= 0 || c->n_kv_heads <= 0 || c->max_pages_per_seq <= 0 || c->batch <= 0)
-    return RPK_ERR_SHAPE;
-  if (!(c->page_size == 16 || c->page_size == 32 || c->page_size == 64 || c->page_size == 128))
-    return RPK_ERR_UNSUPPORTED;
-  if (!(head_dim == 64 || head_dim == 128 || head_dim == 256)) return RPK_ERR_UNSUPPORTED;
   if (n_kv_heads != c->n_kv_heads || head_dim != c->head_dim) return RPK_ERR_SHAPE;
   if (n_heads <= 0 || n_heads % n_kv_heads != 0) return RPK_ERR_SHAPE;
   if (batch <= 0 || batch != c->batch || batch > 65535) return RPK_ERR_SHAPE;
   if (total_q_tokens < 0 || max_q_len < 0 || max_kv_len < 0) return RPK_ERR_SHAPE;
   if (!(scale > 0.f) || !std::isfinite(scale)) return RPK_ERR_SHAPE;
-  if (!aligned16(q) || !aligned16(out) || !aligned16(c->k_pages) || !aligned16(c->v_pages))
+  if ((reinterpret_cast<uintptr_t>(q) & 15u) != 0 || (reinterpret_cast<uintptr_t>(out) & 15u) != 0)
     return RPK_ERR_SHAPE;
-  if ((long long)c->num_pages * c->page_size > INT32_MAX) return RPK_ERR_UNSUPPORTED;
-  void *k_layer, *v_layer;
-  if (!rpk::layer_pools(c, &k_layer, &v_layer)) return RPK_ERR_SHAPE;
   if ((long long)max_kv_len > (long long)c->max_pages_per_seq * c->page_size)
     return RPK_ERR_SHAPE;
+  void *k_layer, *v_layer;
+  rpk::layer_pools(c, &k_layer, &v_layer);
   const int32_t group = n_heads / n_kv_heads;
   // Only the split-KV decode path uses scratch; this entry point runs nothing else.
   if (dtype != RPK_BF16 || (long long)max_q_len * group > rpk::kDecodeMaxRows)
@@ -121,7 +92,7 @@ extern "C" rpk_status ragged_paged_attention_noalloc(
   if (need > (size_t)RPK_NOALLOC_SCRATCH_BYTES) return RPK_ERR_WORKSPACE;
 
   void* scratch = nullptr;
-  rpk_status st = scratch_address(&scratch);
+  st = scratch_address(&scratch);
   if (st != RPK_OK) return st;
 
   rpk::AttnParams p;
@@ -130,9 +101,13 @@ extern "C" rpk_status ragged_paged_attention_noalloc(
   p.error_word = c->error_word;
   p.T = total_q_tokens; p.batch = batch; p.H = n_heads; p.Hk = n_kv_heads; p.G = group;
   p.d = head_dim; p.P = c->page_size; p.num_pages = c->num_pages;
-  p.max_pages = c->max_pages_per_seq; p.window = window > 0 ? window : 0;
+  p.max_pages = c->max_pages_per_seq;
+  // As in ragged_paged_attention: a window covering every key is unbounded,
+  // which keeps the band arithmetic far from int overflow.
+  p.window = rpk::effective_window(window, max_kv_len);
   p.max_q_len = max_q_len; p.max_kv_len = max_kv_len; p.scale = scale;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  p.wait_ns = rpk::wait_limit_ns();
 
   // Partials layout inside the scratch: O [splits, T, H, d] fp32, then (m, l).
   const rpk::DecodePlan plan = rpk::decode_launch_plan(max_kv_len, batch * n_kv_heads, head_dim,
@@ -146,11 +121,10 @@ extern "C" rpk_status ragged_paged_attention_noalloc(
   CUtensorMap k_map, v_map;
   const int32_t box_rows = p.P < rpk::kDecodeTile ? p.P : rpk::kDecodeTile;
   const int64_t pool_rows = (int64_t)p.num_pages * p.P;
-  st = pool_map(&k_map, p.k_pages, head_dim, n_kv_heads, pool_rows, box_rows);
+  st = rpk::encode_rows_map(&k_map, p.k_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
   if (st != RPK_OK) return st;
-  st = pool_map(&v_map, p.v_pages, head_dim, n_kv_heads, pool_rows, box_rows);
+  st = rpk::encode_rows_map(&v_map, p.v_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
   if (st != RPK_OK) return st;
-  const cudaError_t e =
-      rpk::launch_attn_decode(p, k_map, v_map, plan, ws, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? RPK_OK : RPK_ERR_CUDA;
+  return rpk::cuda_status(
+      rpk::launch_attn_decode(p, k_map, v_map, plan, ws, static_cast<cudaStream_t>(stream)));
 }

@@ -158,22 +158,25 @@ __device__ __forceinline__ bool timed_out_elsewhere(const int32_t* error_word) {
          (*reinterpret_cast<const volatile int32_t*>(error_word) & (int32_t)RPK_DEVERR_TIMEOUT);
 }
 
-// Bounded wait by one thread; false on timeout or abort. The thread sleeps in
-// try_wait (woken when the phase completes, at most 0.2 ms per try), so
+// Bounded wait by one thread; false on timeout (after `limit_ns`) or abort.
+// The first test does not block; then the thread sleeps in try_wait (woken
+// when the phase completes, at most 0.2 ms or the limit per try), so
 // waiting warps leave the issue slots to the warps that compute; between
 // tries it looks at the abort flag, the timer and, once the wait has lasted
 // longer than any healthy one (50 us), the global error word.
 __device__ __forceinline__ bool thread_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                            const int32_t* error_word) {
+                                            const int32_t* error_word,
+                                            unsigned long long limit_ns) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
+  if (mbar_test_wait(a, parity)) return true;
+  const uint32_t hint = wait_hint_ns(limit_ns);
   const unsigned long long t0 = global_timer_ns();
 #pragma unroll 1
   while (true) {
-    if (mbar_try_wait_suspend(a, parity, 200000u)) return true;
+    if (mbar_try_wait_suspend(a, parity, hint)) return true;
     if (*abort) return false;
     const unsigned long long dt = global_timer_ns() - t0;
-    if (dt > kWaitTimeoutNs) return false;
+    if (dt > limit_ns) return false;
     if (dt > 50000ull && timed_out_elsewhere(error_word)) return false;
   }
 }
@@ -181,8 +184,9 @@ __device__ __forceinline__ bool thread_wait(uint64_t* bar, uint32_t parity, vola
 // Bounded wait shared by the whole warp: every lane polls (so each lane has
 // acquired the phase) and the lanes agree on the outcome.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          const int32_t* error_word) {
-  const bool ok = thread_wait(bar, parity, abort, error_word);
+                                          const int32_t* error_word,
+                                          unsigned long long limit_ns) {
+  const bool ok = thread_wait(bar, parity, abort, error_word, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -191,20 +195,21 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 // complete pays one barrier round trip, not two.
 __device__ __forceinline__ bool warp_wait2(uint64_t* bar_a, uint32_t par_a, uint64_t* bar_b,
                                            uint32_t par_b, bool need_b, volatile int* abort,
-                                           const int32_t* error_word) {
+                                           const int32_t* error_word,
+                                           unsigned long long limit_ns) {
   uint32_t ok_a, ok_b;
   asm volatile(
       "{\n\t.reg .pred pa, pb;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 pa, [%2], %3;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 pb, [%4], %5;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 pa, [%2], %3;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 pb, [%4], %5;\n\t"
       "selp.u32 %0, 1, 0, pa;\n\t"
       "selp.u32 %1, 1, 0, pb;\n\t}"
       : "=r"(ok_a), "=r"(ok_b)
       : "r"(smem_u32(bar_a)), "r"(par_a), "r"(smem_u32(need_b ? bar_b : bar_a)),
         "r"(need_b ? par_b : par_a)
       : "memory");
-  bool ok = (ok_a != 0 || thread_wait(bar_a, par_a, abort, error_word)) &&
-            (!need_b || ok_b != 0 || thread_wait(bar_b, par_b, abort, error_word));
+  bool ok = (ok_a != 0 || thread_wait(bar_a, par_a, abort, error_word, limit_ns)) &&
+            (!need_b || ok_b != 0 || thread_wait(bar_b, par_b, abort, error_word, limit_ns));
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -357,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto publish = [&](int seq, int w) -> bool {
         const int slot = seq & 1;
         if (seq >= 2 &&
-            !thread_wait(&bars.item_empty[slot], ((seq >> 1) & 1) ^ 1, abort, p.error_word))
+            !thread_wait(&bars.item_empty[slot], ((seq >> 1) & 1) ^ 1, abort, p.error_word, p.wait_ns))
           return false;
         *reinterpret_cast<volatile int*>(&item_slot[slot]) = w;
         mbar_arrive(&bars.item_full[slot]);
@@ -366,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The two Q tiles of an item, once the previous item's S MMAs that read
       // them have completed. Rows past the last token read the fill value.
       auto load_q = [&](const Item& it) -> bool {
-        if (q_loads > 0 && !thread_wait(&bars.q_empty, (q_loads - 1) & 1, abort, p.error_word))
+        if (q_loads > 0 && !thread_wait(&bars.q_empty, (q_loads - 1) & 1, abort, p.error_word, p.wait_ns))
           return false;
         mbar_arrive_expect_tx(&bars.q_full, 2 * C::kBoxes * q_box_bytes);
         for (int t = 0; t < 2; ++t)
@@ -385,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = gi % S;
         const int key0 = tile_of(it, i) * kBN;
         if (gi >= S &&
-            !thread_wait(&bars.kv_empty[st], ((gi / S) & 1) ^ 1, abort, p.error_word))
+            !thread_wait(&bars.kv_empty[st], ((gi / S) & 1) ^ 1, abort, p.error_word, p.wait_ns))
           return false;
         uint32_t bytes = 0;
         for (int r = 0; r < kBN; r += box_rows) {
@@ -503,13 +508,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     };
     auto wait_stage = [&]() -> bool {
-      if (!warp_wait(&bars.kv_full[g_kv % S], (g_kv / S) & 1, abort, p.error_word)) return false;
+      if (!warp_wait(&bars.kv_full[g_kv % S], (g_kv / S) & 1, abort, p.error_word, p.wait_ns)) return false;
       ++g_kv;
       return true;
     };
     for (int seq = 0; ok; ++seq) {
       const int slot = seq & 1;
-      if (!warp_wait(&bars.item_full[slot], (seq >> 1) & 1, abort, p.error_word)) {
+      if (!warp_wait(&bars.item_full[slot], (seq >> 1) & 1, abort, p.error_word, p.wait_ns)) {
         ok = false;
         break;
       }
@@ -520,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       Item it;
       if (!decode_item(p, w, n_qpairs, tpt, false, it) || it.n_tiles == 0) continue;
       const int n = it.n_tiles;
-      ok = warp_wait(&bars.q_full, q_seen & 1, abort, p.error_word);
+      ok = warp_wait(&bars.q_full, q_seen & 1, abort, p.error_word, p.wait_ns);
       ++q_seen;
       // S(0), S(1)
       for (int j = 0; ok && j < n && j < 2; ++j) {
@@ -537,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool more_s = i + 2 < n;
         const int kst = more_s ? g_kv % S : -1;
         if (!warp_wait2(&bars.p_full[pb], (g_pv >> 1) & 1, &bars.kv_full[g_kv % S],
-                        (g_kv / S) & 1, more_s, abort, p.error_word)) {
+                        (g_kv / S) & 1, more_s, abort, p.error_word, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -561,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (i == 0 && o_commits > 0) {
           // O of the previous item has been read by its epilogue.
-          if (!warp_wait(&bars.o_empty, (o_commits - 1) & 1, abort, p.error_word)) {
+          if (!warp_wait(&bars.o_empty, (o_commits - 1) & 1, abort, p.error_word, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -586,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok) do_abort(abort, p.error_word);
     // Drain: every MMA issued above has completed before TMEM is freed.
     commit_to(&bars.drain);
-    if (!warp_wait(&bars.drain, 0, abort, p.error_word)) mbar_wait(&bars.drain, 0);
+    if (!warp_wait(&bars.drain, 0, abort, p.error_word, p.wait_ns)) mbar_wait(&bars.drain, 0);
   } else if (warp < 4) {
     // idle warps of the first warpgroup
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
@@ -606,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
     for (int seq = 0; ok; ++seq) {
       const int slot = seq & 1;
-      if (!warp_wait(&bars.item_full[slot], (seq >> 1) & 1, abort, p.error_word)) {
+      if (!warp_wait(&bars.item_full[slot], (seq >> 1) & 1, abort, p.error_word, p.wait_ns)) {
         ok = false;
         break;
       }
@@ -630,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float v[kBN];
         for (int i = 0; i < n; ++i) {
           const int b = s_seen & 1;
-          if (!warp_wait(&bars.s_full[b], (s_seen >> 1) & 1, abort, p.error_word)) {
+          if (!warp_wait(&bars.s_full[b], (s_seen >> 1) & 1, abort, p.error_word, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -712,9 +717,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool waited =
                 i + 1 < n
                     ? warp_wait(&bars.s_full[(gt + 1) & 1], ((gt + 1) >> 1) & 1, abort,
-                                p.error_word)
-                    : warp_wait(&bars.pv_item[0], pv_items & 1, abort, p.error_word);
+                                p.error_word, p.wait_ns)
+                    : warp_wait(&bars.pv_item[0], pv_items & 1, abort, p.error_word, p.wait_ns);
             if (!waited) {
+              tc::tmem_wait_st();  // no store of P may be in flight when TMEM is freed
               ok = false;
               break;
             }
@@ -742,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------- epilogue
       const bool have_o = n > 0;
       if (have_o) {
-        if (!warp_wait(&bars.o_final, o_seen & 1, abort, p.error_word)) { ok = false; break; }
+        if (!warp_wait(&bars.o_final, o_seen & 1, abort, p.error_word, p.wait_ns)) { ok = false; break; }
         ++o_seen;
         tc::fence_after_sync();
       }

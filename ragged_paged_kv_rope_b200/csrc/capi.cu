@@ -9,14 +9,19 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/rpk.h"
 #include "kernels.h"
 
 namespace {
-
 thread_local char g_last_cuda_error[256] = "";
+// Bound of every device-side wait of later launches (rpk_set_wait_limit_ns).
+std::atomic<unsigned long long> g_wait_limit_ns{rpk::kDefaultWaitLimitNs};
+}  // namespace
+
+namespace rpk {
 
 rpk_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return RPK_OK;
@@ -24,6 +29,12 @@ rpk_status cuda_status(cudaError_t e) {
            cudaGetErrorString(e));
   return RPK_ERR_CUDA;
 }
+
+void set_last_error_text(const char* text) {
+  snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s", text);
+}
+
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -75,7 +86,7 @@ rpk_status encode_rows_map_u8(CUtensorMap* map, const void* base, int32_t d, int
                               int64_t rows, int32_t box_rows) {
   auto fn = encode_fn();
   if (!fn) {
-    snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled unavailable");
+    set_last_error_text("cuTensorMapEncodeTiled unavailable");
     return RPK_ERR_CUDA;
   }
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
@@ -88,8 +99,9 @@ rpk_status encode_rows_map_u8(CUtensorMap* map, const void* base, int32_t d, int
                   swizzled ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
-    snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled failed (%d)",
-             (int)r);
+    char text[64];
+    snprintf(text, sizeof text, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    set_last_error_text(text);
     return RPK_ERR_CUDA;
   }
   return RPK_OK;
@@ -101,7 +113,7 @@ rpk_status encode_rows_map(CUtensorMap* map, const void* base, int32_t d, int32_
                            int64_t rows, int32_t box_heads, int32_t box_rows) {
   auto fn = encode_fn();
   if (!fn) {
-    snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled unavailable");
+    set_last_error_text("cuTensorMapEncodeTiled unavailable");
     return RPK_ERR_CUDA;
   }
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
@@ -112,14 +124,17 @@ rpk_status encode_rows_map(CUtensorMap* map, const void* base, int32_t d, int32_
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
-    snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled failed (%d)",
-             (int)r);
+    char text[64];
+    snprintf(text, sizeof text, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    set_last_error_text(text);
     return RPK_ERR_CUDA;
   }
   return RPK_OK;
 }
 
-}  // namespace
+}  // namespace rpk
+
+using namespace rpk;
 
 extern "C" {
 
@@ -137,6 +152,13 @@ const char* rpk_status_string(rpk_status s) {
 }
 
 const char* rpk_last_cuda_error(void) { return g_last_cuda_error; }
+
+void rpk_set_wait_limit_ns(uint64_t limit_ns) {
+  g_wait_limit_ns.store(limit_ns == 0 ? kDefaultWaitLimitNs : (unsigned long long)limit_ns,
+                        std::memory_order_relaxed);
+}
+
+uint64_t rpk_wait_limit_ns(void) { return (uint64_t)wait_limit_ns(); }
 
 rpk_status rope_qk_paged_ragged(const void* q_proj, const int32_t* input_row_offsets,
                                 const void* k_new, const void* v_new,
@@ -269,6 +291,7 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
   p.cache_fp8 = page_table->cache_dtype == RPK_E4M3;
   p.k_scale = page_table->k_scale;
   p.v_scale = page_table->v_scale;
+  p.wait_ns = wait_limit_ns();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   if (dtype == RPK_F32) return cuda_status(rpk::launch_attn_simt(p, dtype, s));

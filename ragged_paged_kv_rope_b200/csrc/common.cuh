@@ -20,7 +20,10 @@
 
 namespace rpk {
 
-// Upper bound of any single wait inside a kernel (nanoseconds of %globaltimer).
+// Default upper bound of a single wait inside a kernel (nanoseconds of
+// %globaltimer); launches take theirs from rpk_set_wait_limit_ns. Waits for
+// copies or tensor-core operations already in flight while a CTA gives up
+// always use this bound.
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
 
 __device__ __forceinline__ void raise_error(int32_t* error_word, unsigned bits) {
@@ -211,17 +214,38 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar_addr, uint32_
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Sleep hint of one try_wait inside a wait bounded by `limit_ns`.
+__device__ __forceinline__ uint32_t wait_hint_ns(unsigned long long limit_ns) {
+  return limit_ns < 200000ull ? (uint32_t)limit_ns : 200000u;
+}
+
+// Wait for the phase with the given parity to complete; false once more than
+// `limit_ns` have passed. The first test does not block, and each later try
+// sleeps at most the limit, so a limit of a few nanoseconds gives up on any
+// phase that is not complete when the wait starts.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          unsigned long long limit_ns = kWaitTimeoutNs) {
   const uint32_t a = smem_u32(bar);
-#pragma unroll 1
-  for (int i = 0; i < 32; ++i)
-    if (mbar_try_wait(a, parity)) return true;
+  if (mbar_test_wait(a, parity)) return true;
+  const uint32_t hint = wait_hint_ns(limit_ns);
   const unsigned long long t0 = global_timer_ns();
 #pragma unroll 1
   while (true) {
-    if (mbar_try_wait(a, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
+    if (mbar_try_wait_suspend(a, parity, hint)) return true;
+    if (global_timer_ns() - t0 > limit_ns) return false;
   }
 }
 

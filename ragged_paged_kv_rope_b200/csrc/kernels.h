@@ -10,6 +10,24 @@
 
 namespace rpk {
 
+// ------------------------------------------------ host helpers (capi.cu)
+
+// Default bound of every device-side wait (nanoseconds of %globaltimer).
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
+// The bound later launches give their device-side waits (rpk_set_wait_limit_ns).
+unsigned long long wait_limit_ns();
+// RPK_OK for cudaSuccess; otherwise records the error's text for
+// rpk_last_cuda_error() and returns RPK_ERR_CUDA.
+rpk_status cuda_status(cudaError_t e);
+// Records `text` for rpk_last_cuda_error() (this thread).
+void set_last_error_text(const char* text);
+// Host-side checks of a cache description shared by every entry point.
+rpk_status check_cache(const rpk_paged_kv* c);
+// 3-D bf16 tensor map over rows of [rows, heads, d]: dims (d, heads, rows),
+// box (64, box_heads, box_rows), 128-byte swizzle, no multicast.
+rpk_status encode_rows_map(CUtensorMap* map, const void* base, int32_t d, int32_t heads,
+                           int64_t rows, int32_t box_heads, int32_t box_rows);
+
 // The pools of the layer a call uses: layer layer_idx of num_layers (0 means
 // one) layer-major copies of [num_pages, page_size, n_kv_heads, head_dim].
 // False when layer_idx is out of range.
@@ -75,6 +93,7 @@ struct AttnParams {
   int32_t cache_fp8 = 0;       // the pools hold e4m3 codes; key = code * k_scale[kvh] etc.
   const float* k_scale = nullptr;
   const float* v_scale = nullptr;
+  unsigned long long wait_ns = kDefaultWaitLimitNs;  // bound of each mbarrier wait
 };
 
 // fp32 / bf16 CUDA-core attention: one warp per (token, head) row.

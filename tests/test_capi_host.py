@@ -215,3 +215,14 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(R.RpkError):
         R.rope_qk_paged_ragged(x, torch.zeros(2, dtype=torch.int32), x, x, c, torch.zeros(8, 64),
                                None, False, 64, x)
+
+
+def test_wait_limit_setting():
+    # process-wide bound of the kernels' device-side waits; 0 restores 2 s
+    from ragged_paged_kv_rope_b200 import binding as B
+    try:
+        B.set_wait_limit_ns(12345)
+        assert B.wait_limit_ns() == 12345
+    finally:
+        B.set_wait_limit_ns(0)
+    assert B.wait_limit_ns() == 2_000_000_000

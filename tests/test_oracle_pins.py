@@ -150,16 +150,17 @@ def test_two_pass_reproduces_online_worked_example(golden):
 
 
 def test_online_state_worked_example(golden):
-    # The printed o after key 1 is one fp64 ulp from the correctly rounded
-    # 10 + e^-1 * 20, hence the relative tolerance rather than equality.
+    # Every printed value is matched exactly: the page prints o after key 1
+    # with 17 significant digits (17.357588823428847), which parses to the same
+    # fp64 value as the shortest form 17.35758882342885 of 10 + e^-1 * 20.
     g = golden["online_softmax"]
     m, l, o = g["m0"], 0.0, 0.0
     for s, v, want in zip(g["scores"], g["values"], g["steps"]):
         m, l, o = O.flash_step(m, l, o, s, v)
         assert m == want["m"]
-        assert l == pytest.approx(want["l"], rel=1e-15)
-        assert o == pytest.approx(want["o"], rel=5e-16)
-    assert o / l == pytest.approx(g["final"], rel=1e-15)
+        assert l == want["l"]
+        assert o == want["o"]
+    assert o / l == g["final"]
 
 
 def test_online_state_agrees_with_two_pass_random():
