@@ -144,18 +144,26 @@ def load_peaks():
                 "source": "fallback"}
 
 
-def load_traffic(kernel: str):
-    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if the
-    kernel's source is unchanged since the capture (else None)."""
+def sources_digest(names) -> str:
+    """SHA-256 over the given csrc files (a kernel's .cu and the headers it includes)."""
     import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "ragged_paged_kv_rope_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def load_traffic(key: str):
+    """Per-launch DRAM bytes of a kernel on a workload ("kernel@workload") from
+    the committed ncu summary, if the kernel's sources are unchanged since the
+    capture (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             table = json.load(f)
-        ent = table[kernel]
-        src = os.path.join(ROOT, "ragged_paged_kv_rope_b200", "csrc", ent["source"])
-        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
-        if digest != ent["sha256"]:
+        ent = table[key]
+        if sources_digest(ent["sources"]) != ent["sha256"]:
             return None
         return ent
     except (OSError, KeyError, ValueError):
@@ -707,7 +715,7 @@ def main():
     value = job_amount / (step_ms * 1e-3) / scale
     achieved = amount / (attn_ms_mean * 1e-3) / scale
     # the committed DRAM capture is of the bf16-cache decode kernel
-    traffic = load_traffic("attn_decode") if decode and sp.cache_dtype is None else None
+    traffic = load_traffic(f"{kernel_of(wl)[0]}@{sp.name}") if sp.cache_dtype is None else None
     if decode:
         roofline = {"bound": "hbm", "kernel": "ragged_paged_attention (split-KV decode + combine)",
                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": unit,
@@ -722,7 +730,8 @@ def main():
                   else "ragged_paged_attention (CUDA-core kernel)")
         roofline = {"bound": "tensor", "kernel": kernel, "achieved": achieved,
                     "peak": peaks["bf16_tflops"], "unit": unit,
-                    "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                    "frac": achieved / peaks["bf16_tflops"],
+                    "traffic": None if traffic is None else traffic["bytes_per_launch"],
                     "peak_source": "measured (MEASURED_PEAKS.json bf16_tflops)"
                     if peaks["source"] == "measured" else "fallback 1.59 PFLOP/s",
                     "algorithmic_flops_per_launch": amount}
