@@ -370,7 +370,9 @@ rpk_status ragged_paged_attention_noalloc(const void* q, const int32_t* q_row_of
  * RPK_DEVERR_TIMEOUT already set in the error word also stops early, so clear
  * the word before relying on later results). The pages have no counterpart;
  * this is the library's failure detection (no wait is unbounded, nothing
- * traps). 0 restores the default of 2 seconds. The setting is process-wide
+ * traps). A limit under 1 microsecond, below the resolution of the GPU's
+ * global timer, makes a wait give up at its first test of a phase that is not
+ * already complete. 0 restores the default of 2 seconds. The setting is process-wide
  * and read when a call is made; waits for copies already in flight during a
  * give-up keep the default bound.
  */

@@ -397,7 +397,25 @@ rpk_status ragged_paged_attention_backward(
   p.cache_fp8 = page_table->cache_dtype == RPK_E4M3;
   p.k_scale = page_table->k_scale;
   p.v_scale = page_table->v_scale;
-  return cuda_status(rpk::launch_attn_backward(p, dtype, static_cast<cudaStream_t>(stream)));
+  p.wait_ns = wait_limit_ns();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (rpk::attn_backward_tc_supported(p, dtype)) {
+    // tcgen05 kernels: TMA maps over q, d_out and the layer's pools
+    CUtensorMap q_map, do_map, k_map, v_map;
+    const int32_t tpt = 128 / p.G;
+    const int32_t box_rows = p.P < 128 ? p.P : 128;
+    const int64_t pool_rows = (int64_t)p.num_pages * p.P;
+    st = encode_rows_map(&q_map, q, head_dim, n_heads, total_q_tokens, p.G, tpt);
+    if (st != RPK_OK) return st;
+    st = encode_rows_map(&do_map, d_out, head_dim, n_heads, total_q_tokens, p.G, tpt);
+    if (st != RPK_OK) return st;
+    st = encode_rows_map(&k_map, p.k_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
+    if (st != RPK_OK) return st;
+    st = encode_rows_map(&v_map, p.v_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
+    if (st != RPK_OK) return st;
+    return cuda_status(rpk::launch_attn_backward_tc(p, q_map, do_map, k_map, v_map, s));
+  }
+  return cuda_status(rpk::launch_attn_backward(p, dtype, s));
 }
 
 }  // extern "C"

@@ -232,14 +232,19 @@ __device__ __forceinline__ uint32_t wait_hint_ns(unsigned long long limit_ns) {
   return limit_ns < 200000ull ? (uint32_t)limit_ns : 200000u;
 }
 
+// Limits below this give up at the first test of a phase that is not
+// complete: the global timer does not resolve shorter intervals.
+constexpr unsigned long long kTimerResolutionNs = 1000ull;
+
 // Wait for the phase with the given parity to complete; false once more than
-// `limit_ns` have passed. The first test does not block, and each later try
-// sleeps at most the limit, so a limit of a few nanoseconds gives up on any
-// phase that is not complete when the wait starts.
+// `limit_ns` have passed. The first test does not block; a limit under
+// kTimerResolutionNs gives up right there when the phase is not complete, and
+// each later try sleeps at most the limit.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           unsigned long long limit_ns = kWaitTimeoutNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_test_wait(a, parity)) return true;
+  if (limit_ns < kTimerResolutionNs) return false;
   const uint32_t hint = wait_hint_ns(limit_ns);
   const unsigned long long t0 = global_timer_ns();
 #pragma unroll 1
@@ -276,6 +281,172 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // is 1024-byte aligned, so the XOR uses the row index within its 8-row group).
 __device__ __forceinline__ uint32_t swz128(uint32_t row, uint32_t chunk) {
   return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+// ------------------------------------------------- packed fp32 arithmetic
+
+// Packed and three-input fp32 instructions of sm_100: softmax-like passes over
+// tensor-memory tiles are bound by instruction issue and the exponential unit,
+// so two values per instruction where the hardware allows it.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// (d0, d1) = (a0, a1) * b + c
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %4};\n\t"
+      "mov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+// (s0, s1) += (a0, a1)
+__device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(s0), "=f"(s1)
+      : "f"(a0), "f"(a1), "f"(s0), "f"(s1));
+}
+
+// (d0, d1) = (a0, a1) + (b0, b1)
+__device__ __forceinline__ void add2_to(float& d0, float& d1, float a0, float a1, float b0,
+                                        float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// (d0, d1) = (a0, a1) * (b0, b1) + (c0, c1)
+__device__ __forceinline__ void fma2_v(float& d0, float& d1, float a0, float a1, float b0,
+                                       float b1, float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// (d0, d1) = (a0, a1) * (b0, b1)
+__device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, float b0,
+                                     float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// 2^x0, 2^x1 on the FMA pipe, for x <= 2^8 (x below -127, -inf included,
+// gives +0). Range reduction x = n + f with n = round(x) and |f| <= 1/2:
+// adding 1.5 * 2^23 rounds x to an integer held in the low mantissa bits of
+// the sum. 2^f comes from a cubic fitted here to 2^f on [-1/2, 1/2] by
+// iteratively reweighted least squares in relative error (constant term 1
+// exactly; largest relative error 1.3e-4 after fp32 evaluation, far inside
+// the bf16 rounding of P), and 2^n is added to its exponent field.
+__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c1 = 0.6932254433631897f, c2 = 0.2422972172498703f,
+                  c3 = 0.0553351491689682f;
+  x0 = fmaxf(x0, -127.0f);
+  x1 = fmaxf(x1, -127.0f);
+  float t0, t1, n0, n1, f0, f1, q0, q1;
+  add2_to(t0, t1, x0, x1, kMagic, kMagic);       // round(x) in the low mantissa bits
+  add2_to(n0, n1, t0, t1, -kMagic, -kMagic);     // round(x) as a float
+  fma2_v(f0, f1, n0, n1, -1.0f, -1.0f, x0, x1);  // f = x - n
+  fma2_v(q0, q1, f0, f1, c3, c3, c2, c2);
+  fma2_v(q0, q1, q0, q1, f0, f1, c1, c1);
+  fma2_v(q0, q1, q0, q1, f0, f1, 1.0f, 1.0f);
+  y0 = __int_as_float(__float_as_int(q0) + (int)((uint32_t)__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(q1) + (int)((uint32_t)__float_as_int(t1) << 23));
+}
+
+// ------------------------------------- bounded waits of persistent kernels
+
+// A CTA that gives up on a wait publishes RPK_DEVERR_TIMEOUT in the error
+// word; every other CTA of the launch (and of later launches, until the caller
+// clears the word) sees it and stops early instead of waiting out its own
+// bound, so a broken launch ends in about one bound, not one per CTA.
+__device__ __forceinline__ bool timed_out_elsewhere(const int32_t* error_word) {
+  return error_word &&
+         (*reinterpret_cast<const volatile int32_t*>(error_word) & (int32_t)RPK_DEVERR_TIMEOUT);
+}
+
+// Bounded wait by one thread; false on timeout (after `limit_ns`; at the first
+// incomplete test for a limit under kTimerResolutionNs) or abort.
+// The first test does not block; then the thread sleeps in try_wait (woken
+// when the phase completes, at most 0.2 ms or the limit per try), so
+// waiting warps leave the issue slots to the warps that compute; between
+// tries it looks at the abort flag, the timer and, once the wait has lasted
+// longer than any healthy one (50 us), the global error word.
+__device__ __forceinline__ bool thread_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                            const int32_t* error_word,
+                                            unsigned long long limit_ns) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_test_wait(a, parity)) return true;
+  if (limit_ns < kTimerResolutionNs) return false;
+  const uint32_t hint = wait_hint_ns(limit_ns);
+  const unsigned long long t0 = global_timer_ns();
+#pragma unroll 1
+  while (true) {
+    if (mbar_try_wait_suspend(a, parity, hint)) return true;
+    if (*abort) return false;
+    const unsigned long long dt = global_timer_ns() - t0;
+    if (dt > limit_ns) return false;
+    if (dt > 50000ull && timed_out_elsewhere(error_word)) return false;
+  }
+}
+
+// Bounded wait shared by the whole warp: every lane polls (so each lane has
+// acquired the phase) and the lanes agree on the outcome.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          const int32_t* error_word,
+                                          unsigned long long limit_ns) {
+  const bool ok = thread_wait(bar, parity, abort, error_word, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait for two barriers at once: the two tests are issued back to
+// back, so a warp that finds both phases complete pays one barrier round
+// trip, not two.
+__device__ __forceinline__ bool warp_wait2(uint64_t* bar_a, uint32_t par_a, uint64_t* bar_b,
+                                           uint32_t par_b, volatile int* abort,
+                                           const int32_t* error_word,
+                                           unsigned long long limit_ns) {
+  uint32_t ok_a, ok_b;
+  asm volatile(
+      "{\n\t.reg .pred pa, pb;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 pa, [%2], %3;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 pb, [%4], %5;\n\t"
+      "selp.u32 %0, 1, 0, pa;\n\t"
+      "selp.u32 %1, 1, 0, pb;\n\t}"
+      : "=r"(ok_a), "=r"(ok_b)
+      : "r"(smem_u32(bar_a)), "r"(par_a), "r"(smem_u32(bar_b)), "r"(par_b)
+      : "memory");
+  bool ok = (ok_a != 0 || thread_wait(bar_a, par_a, abort, error_word, limit_ns)) &&
+            (ok_b != 0 || thread_wait(bar_b, par_b, abort, error_word, limit_ns));
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void do_abort(volatile int* abort, int32_t* error_word) {
+  if (!*abort) {
+    *abort = 1;
+    raise_error(error_word, RPK_DEVERR_TIMEOUT);
+  }
 }
 
 }  // namespace rpk

@@ -130,7 +130,7 @@ cudaError_t launch_attn_decode(const AttnParams& p, const CUtensorMap& k_map,
 // items from `work_counter` (device int, zeroed by the launch; one per
 // concurrently running launch).
 constexpr size_t kPrefillWorkspaceBytes = 256;
-constexpr int kPrefillKeyTile = 64;   // keys per tcgen05 prefill key tile (K/V box rows <= this)
+constexpr int kPrefillKeyTile = 128;  // keys per tcgen05 prefill key tile (K/V box rows <= this)
 cudaError_t launch_attn_prefill(const AttnParams& p, const CUtensorMap& q_map,
                                 const CUtensorMap& k_map, const CUtensorMap& v_map,
                                 int* work_counter, cudaStream_t stream);
@@ -156,8 +156,17 @@ struct BackwardParams {
   int32_t cache_fp8;
   const float* k_scale;
   const float* v_scale;
+  unsigned long long wait_ns = kDefaultWaitLimitNs;  // bound of each mbarrier wait
 };
 cudaError_t launch_attn_backward(const BackwardParams& p, rpk_dtype dtype, cudaStream_t stream);
+// tcgen05 kernels: bf16 tensors over a bf16 cache, head_dim 64 / 128, groups of
+// up to 128 query heads. Maps: q and d_out as [T, H, d] with box (64, G,
+// 128 / G); the pools as [pages * page_size, n_kv_heads, d] with box
+// (64, 1, min(page_size, 128)); all 128-byte swizzled.
+bool attn_backward_tc_supported(const BackwardParams& p, rpk_dtype dtype);
+cudaError_t launch_attn_backward_tc(const BackwardParams& p, const CUtensorMap& q_map,
+                                    const CUtensorMap& do_map, const CUtensorMap& k_map,
+                                    const CUtensorMap& v_map, cudaStream_t stream);
 // Tensor-core (mma.sync) kernels: bf16 tensors over a bf16 cache, groups of at
 // most 16 query heads, head_dim 64 / 128 / 256.
 bool attn_backward_mma_supported(const BackwardParams& p, rpk_dtype dtype);

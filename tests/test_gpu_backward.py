@@ -71,6 +71,13 @@ CASES = [
      0, 0),
     ("head_dim 256 prefill, window and sinks", "gemma_swa_decode",
      dict(n_heads=4, n_kv_heads=2), [100, 1], [300, 77], 128, 4),
+    ("many 128-key and 128-row blocks", "ragged_prefill",
+     dict(n_heads=8, n_kv_heads=2, page_size=64), [700, 129, 3], [900, 129, 260], 0, 0),
+    ("group of 8, chunked rows, window", "mixed_chunked_mrope",
+     dict(n_heads=16, n_kv_heads=2, mrope_section=None), [150, 1, 40], [1000, 300, 41], 300, 0),
+    ("group of 128, one token per row block", "ragged_prefill",
+     dict(n_heads=128, n_kv_heads=1, head_dim=64, rotary_dim=64, page_size=128), [5, 2],
+     [300, 2], 0, 0),
 ]
 
 

@@ -26,7 +26,7 @@ from parity import check_attention, gpu_attention, to_device
 
 pytestmark = pytest.mark.gpu
 
-SHORT_NS = 20
+SHORT_NS = 20  # under the timer resolution: waits give up at their first incomplete test
 
 
 def _timeout_then_healthy(sp: W.Spec, q_lens, kv_lens, seed: int):
