@@ -507,14 +507,14 @@ def measure_workload(name: str, device, world: int, local: int, rank: int, seed:
     return entry
 
 
-def backward_measure(device, world, warmup=3):
+def backward_measure(device, world, warmup=3, batch=None):
     """The attention backward (its two kernels) on the ragged prefill workload:
     the forward runs once for the output and log-sum-exp, then the backward is
     timed with a seeded N(0, 1) output gradient. Algorithmic FLOPs are 2.5x the
     forward's visible-pair FLOPs: five products of 2 d FLOP per visible (row,
     key) pair and head (S, dP, dQ, dK, dV); the kernels recompute S and dP in
     each of their two passes, which is not counted."""
-    wl = W.make("ragged_prefill", seed=0)
+    wl = W.make("ragged_prefill", seed=0, **({} if batch is None else {"batch": batch}))
     sp = wl.spec
     step = Step(wl, device)
     step.rope()
@@ -558,9 +558,13 @@ def backward_measure(device, world, warmup=3):
     flops = 2.5 * M.attention_flops(wl.q_lens, wl.kv_lens, sp.window, sp.n_heads, sp.head_dim)
     peaks = load_peaks()
     tflops = flops / (ms * 1e-3) / 1e12
-    kernel = ("tensor-core (mma.sync) dQ and dK/dV kernels"
-              if sp.dtype == "bf16" and sp.n_heads // sp.n_kv_heads <= 16
-              else "CUDA-core dQ and dK/dV kernels")
+    G = sp.n_heads // sp.n_kv_heads
+    if sp.dtype == "bf16" and sp.cache_dtype is None and sp.head_dim in (64, 128) and G <= 128:
+        kernel = "tcgen05 dK/dV and dQ kernels (attn_bwd_dkv_tc_kernel, attn_bwd_dq_tc_kernel)"
+    elif sp.dtype == "bf16" and sp.cache_dtype is None and G <= 16:
+        kernel = "warp-level tensor-core (mma.sync) dQ and dK/dV kernels"
+    else:
+        kernel = "CUDA-core dQ and dK/dV kernels"
     return {"workload": "ragged_prefill", "kernel": kernel, "backward_ms": ms, "steps": steps,
             "algorithmic_flops": flops, "tflops": tflops,
             "tensor_peak_tflops": peaks["bf16_tflops"], "frac": tflops / peaks["bf16_tflops"],
@@ -757,7 +761,8 @@ def main():
             workloads[name] = measure_workload(
                 name, device, world, local, rank, args.seed,
                 None if args.no_cpu_baseline else 4.0)
-    backward = None if args.no_backward else backward_measure(device, world)
+    backward = None if args.no_backward else backward_measure(
+        device, world, batch=args.batch if args.workload == "ragged_prefill" else None)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
