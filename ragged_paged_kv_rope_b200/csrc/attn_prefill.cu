@@ -9,12 +9,10 @@
 // running sum and output rescaled by e^(m_old - m_new), final divide).
 //
 // Work unit (item): two query tiles A and B of 128 rows each of one
-// (sequence, KV head), against key tiles of 128 keys. The 128 rows of a tile
+// (sequence, KV head), against key tiles of 64 keys. The 128 rows of a tile
 // are the (token, query head) pairs of one KV head's group, token-major
 // (tokens_per_tile = 128 / G), so the G query heads that share a KV head share
 // every K/V tile; tile B holds the next tokens_per_tile tokens after tile A.
-// Both tiles run every key tile of the item (tile B's rows past the sequence
-// are masked and never stored).
 //
 // Persistent launch: one CTA per SM claims items from a counter in the
 // caller's workspace (zeroed by the launch). Items run sequence by sequence,
@@ -22,30 +20,29 @@
 // sequence at the same time read the same K/V tiles in the same order, so a
 // tile read from HBM for one of them is an L2 hit for the others.
 //
-// Tensor memory (512 columns): one score tile S_t (128 fp32 columns) and one
-// output accumulator O_t (head_dim columns) per query tile t. P_t(i) (packed
-// bf16 pairs) is written over the first 64 columns of S_t(i). The two tiles
-// ping-pong: the tensor core issues, in order,
-//     S_A(0) S_B(0) | P_A(0)V_0 S_A(1) | P_B(0)V_0 S_B(1) | P_A(1)V_1 S_A(2) | ...
-// so while the softmax of tile A turns S_A(i) into P_A(i), the tensor core
-// runs P_B(i-1)V_{i-1} and S_B(i), and the other way round. Every MMA is
-// 128 x 128 x 16 (N = 128 keys for the scores, N = head_dim 128 for P V), the
-// shape at which the tensor core runs at its full rate from shared memory.
-// S_t(i) is committed after P_t(i-1)V_{i-1} (issued before it, and tensor-core
-// operations of one thread complete in order), so once the softmax of tile t
-// sees S_t(i), no MMA writes O_t until it has handed over P_t(i): that window
-// is where it rescales O_t.
+// Tensor memory (512 columns): two score buffers of 64 columns per query
+// tile (S_t[0], S_t[1]) and one 128-row output accumulator per tile (O_A,
+// O_B). Score tile i of both query tiles lives in buffer i mod 2, and P_t(i)
+// (packed bf16 pairs) is written over the first 32 columns of S_t(i). The MMA
+// issuer computes S(i+2) right after issuing P(i) V_i, so while the softmax
+// warpgroups turn S(i) into P(i), the tensor core has already computed S(i+1):
+// the softmax does not wait for the tensor core in the steady state, and the
+// two softmax warpgroups keep the exponential unit busy together. Every item
+// runs both query tiles (tile B's rows past the sequence are masked and never
+// stored), so the two tiles share every barrier phase.
 //
 // Warp roles (384 threads, three warpgroups):
 //   warp 0     TMA producer: claims the next item, hands its index to the
 //              other roles through a two-slot ring in shared memory, loads the
-//              item's two Q tiles, then K(0), V(0), K(1), V(1), ... into a ring
-//              of 32 KB slots (3-D map over the pool [pages * page_size,
-//              kv_heads, d], one box per page segment, 128-byte swizzle, no
-//              multicast). The tensor core frees the slots in the order they
-//              were loaded (K(i) after S_B(i), V(i) after P_B(i)V_i, and P_B(i)V_i
-//              is issued before S_B(i+1)), so one ring suffices.
-//   warp 1     allocates TMEM and issues every MMA from one thread.
+//              item's two Q tiles, then each key tile's K and V into one stage
+//              of a ring (3-D map over the pool [pages * page_size, kv_heads,
+//              d], one box per page segment, 128-byte swizzle, no multicast)
+//   warp 1     allocates TMEM and issues the MMAs from one thread: per item
+//              S(0), S(1), then per key tile i one burst of O_A += P_A(i) V_i,
+//              O_B += P_B(i) V_i (P from TMEM, V an MN-major operand in shared
+//              memory), S_A(i+2) and S_B(i+2) (Q_t K^T, both operands in shared
+//              memory); the next item's first S MMAs follow the last P V of the
+//              current one
 //   warps 2-3  idle (they complete the first warpgroup)
 //   warps 4-7  softmax of tile A, warps 8-11 softmax of tile B: thread r owns
 //              row r (TMEM lane r); loads S_t(i), masks the band, keeps (m, l)
@@ -53,6 +50,12 @@
 //              when the running max grew by more than 2^8 (the final O / l
 //              uses the same max, so this is exact); then normalises O_t and
 //              stores the rows.
+// A rescale of O_t during tile i must fall between P(i-1) V_{i-1} and
+// P(i) V_i. For i < n - 1 the softmax waits for S(i+1), which the issuer
+// placed after P(i-1) V_{i-1}; for the item's last tile it waits for a
+// barrier the issuer commits once per item after P(n-2) V_{n-2}. Either
+// barrier can be at most one phase short of the one waited for (P(i) V_i
+// needs this warp's own P(i)), so the phase parity is unambiguous.
 // Registers: the first warpgroup gives registers back (setmaxnreg 56) and the
 // two softmax warpgroups take them (setmaxnreg 224);
 // 4*32*56 + 8*32*224 = 64512 registers, the 384 * 168 the CTA is launched with.
@@ -74,52 +77,45 @@ int prefill_rows_per_tile(int group) { return group >= 1 && group <= 128 ? (128 
 namespace {
 
 constexpr int kBM = 128;              // rows per tile (MMA M)
-constexpr int kBN = kPrefillKeyTile;  // keys per tile (128)
+constexpr int kBN = kPrefillKeyTile;  // keys per tile (64)
 constexpr int kThreads = 384;
 constexpr int kRegsControl = 56;    // warpgroup 0: producer, MMA issuer, 2 idle warps
 constexpr int kRegsSoftmax = 224;   // warpgroups 1 and 2: softmax
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows > 2^8
-constexpr int kMaxSlots = 10;
-#ifndef RPK_PREFILL_POLY_OF8
-#define RPK_PREFILL_POLY_OF8 0
-#endif
-// Of every 8 pairs of scores of a row, this many take 2^x on the FMA pipe
-// (exp2_poly2) and the rest on the exponential unit, which both softmax
-// warps of a sub-partition share.
-constexpr int kPolyOf8 = RPK_PREFILL_POLY_OF8;
 
 template <int D>
 struct Cfg {
   static constexpr int kBoxes = D / 64;
+  static constexpr int kStages = D == 128 ? 5 : 10;  // K/V ring depth (key tiles)
   static constexpr int kQBytes = kBM * D * 2;         // one query tile
-  static constexpr int kSlotBytes = kBN * D * 2;      // one K or V tile
-  static constexpr int kSlots = D == 128 ? 5 : 10;    // ring of K / V tiles
+  static constexpr int kKVBytes = kBN * D * 2;        // one K or V tile
+  static constexpr int kStageBytes = 2 * kKVBytes;    // K then V of one key tile
   static constexpr int kQOff = 0;
-  static constexpr int kSlotOff = kQOff + 2 * kQBytes;
-  static constexpr int kEnd = kSlotOff + kSlots * kSlotBytes + 1024;
+  static constexpr int kKVOff = kQOff + 2 * kQBytes;
+  static constexpr int kEnd = kKVOff + kStages * kStageBytes + 1024;
   // At least half the SM's shared memory, so that one CTA holds the SM's TMEM.
   static constexpr int kSmemBytes = kEnd > 118 * 1024 ? kEnd : 118 * 1024;
-  // TMEM columns: S_t (fp32, kBN each) at t * kBN, then O_A, O_B.
-  static constexpr uint32_t kOCol = 2 * kBN;
+  // TMEM columns: S_t[b] (fp32, 64 each) at (2t + b) * 64, then O_A, O_B.
+  static constexpr uint32_t kOCol = 4 * kBN;
   static_assert(kOCol + 2 * D <= kTmemCols, "TMEM budget");
-  static_assert(kSmemBytes <= 232448 - 1024, "shared memory budget");
-  static_assert(kSlots <= kMaxSlots, "slot barriers");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
-__host__ __device__ constexpr uint32_t s_col(int t) { return (uint32_t)(t * kBN); }
+__host__ __device__ constexpr uint32_t s_col(int t, int b) { return (uint32_t)((2 * t + b) * kBN); }
 
 struct Bars {
-  uint64_t q_full;                // both query tiles loaded
-  uint64_t q_empty;               // the item's last S MMA reading them has completed
-  uint64_t full[kMaxSlots];       // per slot: its K or V tile loaded
-  uint64_t empty[kMaxSlots];      // per slot: the last MMA reading it has completed
-  uint64_t s_full[2];             // per query tile: S_t(i) computed
-  uint64_t p_full[2];             // per query tile: P_t(i) written (one arrival per warp)
-  uint64_t o_final[2];            // per query tile: the item's last P V has completed
-  uint64_t o_empty[2];            // per query tile: the epilogue has read O_t (per warp)
-  uint64_t item_full[2];          // work-item ring: index written by the producer
-  uint64_t item_empty[2];         // work-item ring: index read by the MMA and softmax warps
+  uint64_t q_full;       // both query tiles loaded
+  uint64_t q_empty;      // the item's last S MMAs reading them have completed
+  uint64_t kv_full[10];  // per stage: K and V of one key tile loaded
+  uint64_t kv_empty[10]; // per stage: its last P V has completed
+  uint64_t s_full[2];    // per score buffer: S_A and S_B computed
+  uint64_t p_full[2];    // per score buffer: P_A and P_B written (one arrival per softmax warp)
+  uint64_t pv_item[1];   // one phase per item with two or more key tiles: P(n-2) V done
+  uint64_t o_final;      // the item's last P V has completed
+  uint64_t o_empty;      // the epilogue has read O (one arrival per softmax warp)
+  uint64_t item_full[2];   // work-item ring: index written by the producer
+  uint64_t item_empty[2];  // work-item ring: index read by the MMA and softmax warps
   uint64_t drain;
 };
 
@@ -180,9 +176,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap v_map, const int tpt,
                         const int n_qpairs, int* __restrict__ work_counter) {
   using C = Cfg<D>;
-  constexpr int S = C::kSlots;
+  constexpr int S = C::kStages;
   constexpr int kItemReaders = 9;  // MMA warp + 8 softmax warps
-  constexpr int kTileWarps = 4;    // softmax warps per query tile
+  constexpr int kSoftmaxWarps = 8;
   extern __shared__ uint8_t smem_raw[];
   __shared__ Bars bars;
   __shared__ int item_slot[2];
@@ -200,21 +196,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const uint32_t sbase = smem_u32(smem);
   auto q_s = [&](int t) { return sbase + C::kQOff + t * C::kQBytes; };
-  auto slot_s = [&](int s) { return sbase + C::kSlotOff + s * C::kSlotBytes; };
+  auto k_s = [&](int st) { return sbase + C::kKVOff + st * C::kStageBytes; };
+  auto v_s = [&](int st) { return sbase + C::kKVOff + st * C::kStageBytes + C::kKVBytes; };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&bars.full[s], 1);
-      mbar_init(&bars.empty[s], 1);
+    for (int st = 0; st < S; ++st) {
+      mbar_init(&bars.kv_full[st], 1);
+      mbar_init(&bars.kv_empty[st], 1);
     }
     mbar_init(&bars.q_full, 1);
     mbar_init(&bars.q_empty, 1);
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&bars.s_full[t], 1);
-      mbar_init(&bars.p_full[t], kTileWarps);
-      mbar_init(&bars.o_final[t], 1);
-      mbar_init(&bars.o_empty[t], kTileWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars.s_full[b], 1);
+      mbar_init(&bars.p_full[b], kSoftmaxWarps);
     }
+    mbar_init(&bars.pv_item[0], 1);
+    mbar_init(&bars.o_final, 1);
+    mbar_init(&bars.o_empty, kSoftmaxWarps);
     for (int k = 0; k < 2; ++k) {
       mbar_init(&bars.item_full[k], 1);
       mbar_init(&bars.item_empty[k], kItemReaders);
@@ -246,12 +244,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_box_bytes = 128u * (uint32_t)rows_used;
       const int box_rows = p.P < kBN ? p.P : kBN;
       const uint32_t seg_bytes = (uint32_t)box_rows * 128u * C::kBoxes;
-      int loads = 0;     // K / V tiles loaded over all items (slot = loads % S)
-      int q_loads = 0;   // Q loads over all items
+      int kv_issued = 0;  // key tiles loaded over all items
+      int q_loads = 0;    // Q loads over all items
       bool ok = true;
       // Claim a non-empty work item and hand its index to the MMA and softmax
       // warps through the ring. The next item is claimed after the current
-      // one's Q and first key tile are in flight, so the claim's latency hides
+      // one's Q and first key tiles are in flight, so the claim's latency hides
       // behind real work.
       auto claim = [&](Item& it) -> int {
         int w;
@@ -262,8 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto publish = [&](int seq, int w) -> bool {
         const int slot = seq & 1;
-        if (seq >= 2 && !thread_wait(&bars.item_empty[slot], ((seq >> 1) & 1) ^ 1, abort,
-                                     p.error_word, p.wait_ns))
+        if (seq >= 2 &&
+            !thread_wait(&bars.item_empty[slot], ((seq >> 1) & 1) ^ 1, abort, p.error_word, p.wait_ns))
           return false;
         *reinterpret_cast<volatile int*>(&item_slot[slot]) = w;
         mbar_arrive(&bars.item_full[slot]);
@@ -272,8 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The two Q tiles of an item, once the previous item's S MMAs that read
       // them have completed. Rows past the last token read the fill value.
       auto load_q = [&](const Item& it) -> bool {
-        if (q_loads > 0 &&
-            !thread_wait(&bars.q_empty, (q_loads - 1) & 1, abort, p.error_word, p.wait_ns))
+        if (q_loads > 0 && !thread_wait(&bars.q_empty, (q_loads - 1) & 1, abort, p.error_word, p.wait_ns))
           return false;
         mbar_arrive_expect_tx(&bars.q_full, 2 * C::kBoxes * q_box_bytes);
         for (int t = 0; t < 2; ++t)
@@ -284,17 +281,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++q_loads;
         return true;
       };
-      // The K (kind 0) or V (kind 1) rows of key tile i of an item into the
-      // next slot of the ring, once the MMAs that read its previous tile have
-      // completed. Page segments wholly past k_len or with an invalid page id
-      // are not loaded.
-      auto load_tile = [&](const Item& it, int i, int kind) -> bool {
+      // K and V of key tile i of an item into the next stage of the ring; a
+      // stage frees once the P V MMAs that read its V have completed.
+      auto load_stage = [&](const Item& it, int i) -> bool {
         const int32_t* bt = p.block_table + (size_t)it.b * p.max_pages;
-        const int gi = loads;
-        const int s = gi % S;
+        const int gi = kv_issued;
+        const int st = gi % S;
         const int key0 = tile_of(it, i) * kBN;
         if (gi >= S &&
-            !thread_wait(&bars.empty[s], ((gi / S) & 1) ^ 1, abort, p.error_word, p.wait_ns))
+            !thread_wait(&bars.kv_empty[st], ((gi / S) & 1) ^ 1, abort, p.error_word, p.wait_ns))
           return false;
         uint32_t bytes = 0;
         for (int r = 0; r < kBN; r += box_rows) {
@@ -302,26 +297,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (key >= it.k_len) break;
           const int pi = key / p.P;
           const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
-          if (page >= 0 && page < p.num_pages) bytes += seg_bytes;
+          if (page >= 0 && page < p.num_pages) bytes += 2 * seg_bytes;
         }
-        mbar_arrive_expect_tx(&bars.full[s], bytes);
-        const CUtensorMap* map = kind == 0 ? &k_map : &v_map;
+        mbar_arrive_expect_tx(&bars.kv_full[st], bytes);
         for (int r = 0; r < kBN; r += box_rows) {
           const int key = key0 + r;
           if (key >= it.k_len) break;
           const int pi = key / p.P;
           const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
           if (page < 0 || page >= p.num_pages) {
-            if (kind == 0) raise_error(p.error_word, RPK_DEVERR_PAGE);
+            raise_error(p.error_word, RPK_DEVERR_PAGE);
             continue;
           }
           const int grow = page * p.P + (key - pi * p.P);
-          uint8_t* dst = smem + C::kSlotOff + s * C::kSlotBytes + r * 128;
+          uint8_t* kb = smem + C::kKVOff + st * C::kStageBytes + r * 128;
 #pragma unroll
-          for (int bx = 0; bx < C::kBoxes; ++bx)
-            tma_load_3d(dst + bx * (kBN * 128), map, bx * 64, it.kvh, grow, &bars.full[s]);
+          for (int bx = 0; bx < C::kBoxes; ++bx) {
+            tma_load_3d(kb + bx * (kBN * 128), &k_map, bx * 64, it.kvh, grow, &bars.kv_full[st]);
+            tma_load_3d(kb + C::kKVBytes + bx * (kBN * 128), &v_map, bx * 64, it.kvh, grow,
+                        &bars.kv_full[st]);
+          }
         }
-        ++loads;
+        ++kv_issued;
         return true;
       };
       Item cur;
@@ -330,13 +327,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int seq = 0; ok && cur_w >= 0; ++seq) {
         const int n = cur.n_tiles;
         if (n > 0) {
-          ok = load_q(cur) && load_tile(cur, 0, 0) && load_tile(cur, 0, 1);
+          ok = load_q(cur);
+          for (int i = 0; ok && i < n && i < 2; ++i) ok = load_stage(cur, i);
         }
         if (!ok) break;
         Item next;
         const int next_w = claim(next);
         if (!publish(seq + 1, next_w)) { ok = false; break; }
-        for (int i = 1; ok && i < n; ++i) ok = load_tile(cur, i, 0) && load_tile(cur, i, 1);
+        for (int i = 2; ok && i < n; ++i) ok = load_stage(cur, i);
         if (!ok) break;
         cur = next;
         cur_w = next_w;
@@ -344,17 +342,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) do_abort(abort, p.error_word);
       // Never leave with copies in flight.
       if (q_loads > 0) mbar_wait(&bars.q_full, (q_loads - 1) & 1);
-      for (int gi = max(0, loads - S); gi < loads; ++gi) mbar_wait(&bars.full[gi % S], (gi / S) & 1);
+      for (int gi = max(0, kv_issued - S); gi < kv_issued; ++gi)
+        mbar_wait(&bars.kv_full[gi % S], (gi / S) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
     constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(kBM, kBN, 0);
     constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(kBM, D, 1);
-    int base = 0;        // slot loads consumed before the current item (K and V)
-    int tiles = 0;       // key tiles over all items (phase of p_full)
+    int g_kv = 0;        // key tiles whose stage has been waited for, over all items
+    int g_pv = 0;        // key tiles whose P V has been issued, over all items
     int q_seen = 0;      // Q loads consumed
-    int o_items = 0;     // items with keys (phases of o_final / o_empty)
+    int s_issued = 0;    // S tile pairs issued (buffer = count mod 2)
+    int o_commits = 0;   // o_final commits
     bool ok = true;
     // Shared-memory descriptors: the start address is the low field of the
     // low word (address >> 4, 14 bits; every operand lies below 256 KB), so
@@ -362,44 +362,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     // offset >> 4; the high word (stride offset, swizzle) is common.
     const uint64_t q_desc0 = tc::smem_desc_sw128(q_s(0), 16, 1024);
     const uint32_t q_lo0 = (uint32_t)q_desc0;
-    const uint32_t k_lo0 = (uint32_t)tc::smem_desc_sw128(slot_s(0), 16, 1024);
-    const uint32_t v_lo0 = (uint32_t)tc::smem_desc_sw128(slot_s(0), kBN * 128, 1024);
+    const uint32_t k_lo0 = (uint32_t)tc::smem_desc_sw128(k_s(0), 16, 1024);
+    const uint32_t v_lo0 = (uint32_t)tc::smem_desc_sw128(v_s(0), kBN * 128, 1024);
     const uint32_t desc_hi = (uint32_t)(q_desc0 >> 32);
+    // S_A and S_B of the key tile in stage kst into the next score buffer.
+    auto issue_s = [&](int kst) {
+      const int b = s_issued & 1;
+      if (lane == 0) {
+        const uint32_t kd = k_lo0 + (uint32_t)((kst * C::kStageBytes) >> 4);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t d_tmem = tmem + s_col(t, b);
+          const uint32_t qd = q_lo0 + (uint32_t)((t * C::kQBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t qoff = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
+            const uint32_t koff = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
+            tc::mma_ss_lo(d_tmem, qd + (qoff >> 4), kd + (koff >> 4), desc_hi, idesc_qk, kk > 0);
+          }
+        }
+        tc::commit(smem_u32(&bars.s_full[b]));
+      }
+      __syncwarp();
+      ++s_issued;
+    };
+    // O_t (+)= P_t V for both tiles, P_t in the first 32 columns of buffer b.
+    auto issue_pv = [&](int vst, int b, bool first) {
+      if (lane == 0) {
+        const uint32_t vd = v_lo0 + (uint32_t)((vst * C::kStageBytes) >> 4);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t d_tmem = tmem + C::kOCol + (uint32_t)(t * D);
+          const uint32_t a_tmem = tmem + s_col(t, b);
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            tc::mma_ts_lo(d_tmem, a_tmem + kk * 8, vd + (uint32_t)((kk * (16 * 128)) >> 4),
+                          desc_hi, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+        }
+      }
+      __syncwarp();
+    };
     auto commit_to = [&](uint64_t* bar) {
       if (lane == 0) tc::commit(smem_u32(bar));
       __syncwarp();
     };
-    // S_t = Q_t K^T for the K tile in slot ks, then commit s_full[t].
-    auto issue_s = [&](int t, int ks) {
-      if (lane == 0) {
-        const uint32_t kd = k_lo0 + (uint32_t)((ks * C::kSlotBytes) >> 4);
-        const uint32_t d_tmem = tmem + s_col(t);
-        const uint32_t qd = q_lo0 + (uint32_t)((t * C::kQBytes) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qoff = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-          const uint32_t koff = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-          tc::mma_ss_lo(d_tmem, qd + (qoff >> 4), kd + (koff >> 4), desc_hi, idesc_qk, kk > 0);
-        }
-        tc::commit(smem_u32(&bars.s_full[t]));
-      }
-      __syncwarp();
-    };
-    // O_t (+)= P_t V for the V tile in slot vs, P_t in the first 64 columns of S_t.
-    auto issue_pv = [&](int t, int vs, bool first) {
-      if (lane == 0) {
-        const uint32_t vd = v_lo0 + (uint32_t)((vs * C::kSlotBytes) >> 4);
-        const uint32_t d_tmem = tmem + C::kOCol + (uint32_t)(t * D);
-        const uint32_t a_tmem = tmem + s_col(t);
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          tc::mma_ts_lo(d_tmem, a_tmem + kk * 8, vd + (uint32_t)((kk * (16 * 128)) >> 4), desc_hi,
-                        idesc_pv, (!first || kk > 0) ? 1u : 0u);
-      }
-      __syncwarp();
-    };
-    auto wait_slot = [&](int gi) -> bool {
-      return warp_wait(&bars.full[gi % S], (gi / S) & 1, abort, p.error_word, p.wait_ns);
+    auto wait_stage = [&]() -> bool {
+      if (!warp_wait(&bars.kv_full[g_kv % S], (g_kv / S) & 1, abort, p.error_word, p.wait_ns)) return false;
+      ++g_kv;
+      return true;
     };
     for (int seq = 0; ok; ++seq) {
       const int slot = seq & 1;
@@ -414,37 +424,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       Item it;
       if (!decode_item(p, w, n_qpairs, tpt, false, it) || it.n_tiles == 0) continue;
       const int n = it.n_tiles;
-      // K(i) is load base + 2i, V(i) is base + 2i + 1
-      if (!warp_wait(&bars.q_full, q_seen & 1, abort, p.error_word, p.wait_ns) ||
-          !wait_slot(base)) {
-        ok = false;
-        break;
-      }
+      ok = warp_wait(&bars.q_full, q_seen & 1, abort, p.error_word, p.wait_ns);
       ++q_seen;
-      tc::fence_after_sync();
-      issue_s(0, base % S);
-      issue_s(1, base % S);
-      commit_to(&bars.empty[base % S]);  // K(0) read by both tiles
-      if (n == 1) commit_to(&bars.q_empty);
+      // S(0), S(1)
+      for (int j = 0; ok && j < n && j < 2; ++j) {
+        const int kst = g_kv % S;
+        if (!wait_stage()) { ok = false; break; }
+        tc::fence_after_sync();
+        issue_s(kst);
+        if (j + 1 == n) commit_to(&bars.q_empty);  // last S of this item
+      }
       for (int i = 0; ok && i < n; ++i) {
-        const int kg = base + 2 * i + 2;  // K(i+1)
-        const int vg = base + 2 * i + 1;  // V(i)
-        const int vs = vg % S;
-        const bool more = i + 1 < n;
-        // ---- tile A: P_A(i) written and V(i) loaded
-        if (!warp_wait2(&bars.p_full[0], tiles & 1, &bars.full[vs], (vg / S) & 1, abort,
-                        p.error_word, p.wait_ns)) {
+        const int vst = g_pv % S;
+        const int pb = g_pv & 1;
+        // P_A(i) and P_B(i) written, and the stage of key tile i+2 (for S(i+2)) loaded
+        const bool more_s = i + 2 < n;
+        const int kst = more_s ? g_kv % S : -1;
+        const bool waited =
+            more_s ? warp_wait2(&bars.p_full[pb], (g_pv >> 1) & 1, &bars.kv_full[g_kv % S],
+                                (g_kv / S) & 1, abort, p.error_word, p.wait_ns)
+                   : warp_wait(&bars.p_full[pb], (g_pv >> 1) & 1, abort, p.error_word, p.wait_ns);
+        if (!waited) {
           ok = false;
           break;
         }
-        if (i == 0 && o_items > 0 &&
-            !warp_wait(&bars.o_empty[0], (o_items - 1) & 1, abort, p.error_word, p.wait_ns)) {
-          ok = false;
-          break;
-        }
+        if (more_s) ++g_kv;
         const int key0 = tile_of(it, i) * kBN;
         if (key0 + kBN > it.k_len) {
-          // zero value rows at or past k_len before the first P V reads them
+          // zero value rows at or past k_len (the stage was waited for with S(i))
           const int r0 = max(0, it.k_len - key0);
           const int chunks = (kBN - r0) * C::kBoxes * 8;
           for (int idx = lane; idx < chunks; idx += 32) {
@@ -452,47 +459,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int rb = idx >> 3;
             const int bx = rb % C::kBoxes;
             const int r = r0 + rb / C::kBoxes;
-            uint8_t* dst = smem + C::kSlotOff + vs * C::kSlotBytes + bx * (kBN * 128) + r * 128 +
-                           ch * 16;
+            uint8_t* dst = smem + C::kKVOff + vst * C::kStageBytes + C::kKVBytes +
+                           bx * (kBN * 128) + r * 128 + ch * 16;
             *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
           }
           fence_proxy_async_smem();
           __syncwarp();
         }
-        tc::fence_after_sync();
-        issue_pv(0, vs, i == 0);
-        if (more) {
-          if (!wait_slot(kg)) { ok = false; break; }
-          tc::fence_after_sync();
-          issue_s(0, kg % S);
-        } else {
-          commit_to(&bars.o_final[0]);
-        }
-        // ---- tile B: P_B(i) written
-        if (!warp_wait(&bars.p_full[1], tiles & 1, abort, p.error_word, p.wait_ns)) {
-          ok = false;
-          break;
-        }
-        if (i == 0 && o_items > 0 &&
-            !warp_wait(&bars.o_empty[1], (o_items - 1) & 1, abort, p.error_word, p.wait_ns)) {
-          ok = false;
-          break;
+        if (i == 0 && o_commits > 0) {
+          // O of the previous item has been read by its epilogue.
+          if (!warp_wait(&bars.o_empty, (o_commits - 1) & 1, abort, p.error_word, p.wait_ns)) {
+            ok = false;
+            break;
+          }
         }
         tc::fence_after_sync();
-        issue_pv(1, vs, i == 0);
-        commit_to(&bars.empty[vs]);  // V(i) read by both tiles
-        if (more) {
-          issue_s(1, kg % S);
-          commit_to(&bars.empty[kg % S]);  // K(i+1) read by both tiles
-          if (i + 2 == n) commit_to(&bars.q_empty);  // last S of this item
-        } else {
-          commit_to(&bars.o_final[1]);
+        issue_pv(vst, pb, i == 0);
+        ++g_pv;
+        if (i + 2 == n) commit_to(&bars.pv_item[0]);  // P(n-2) V done: last-tile rescales
+        if (i + 1 == n) {
+          commit_to(&bars.o_final);
+          ++o_commits;
         }
-        ++tiles;
+        commit_to(&bars.kv_empty[vst]);
+        if (kst >= 0) {
+          // S(i+2) overwrites the buffer P(i) lives in; the MMAs run in issue
+          // order, so P(i) V_i has read it by then.
+          issue_s(kst);
+          if (i + 3 == n) commit_to(&bars.q_empty);  // last S of this item
+        }
       }
-      if (!ok) break;
-      base += 2 * n;
-      ++o_items;
     }
     if (!ok) do_abort(abort, p.error_word);
     // Drain: every MMA issued above has completed before TMEM is freed.
@@ -509,10 +505,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = qw * 32 + lane;        // row of this thread
     const uint32_t lane_base = (uint32_t)(qw * 32) << 16;
     const uint32_t o_col = tmem + lane_base + C::kOCol + (uint32_t)(t * D);
-    const uint32_t sc = tmem + lane_base + s_col(t);
     const float sl2 = p.scale_log2;
     int s_seen = 0;      // score tiles consumed over all items
     int o_seen = 0;      // items with keys consumed
+    int pv_items = 0;    // items with two or more key tiles consumed
     bool ok = true;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
     for (int seq = 0; ok; ++seq) {
@@ -540,12 +536,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr bool kSinks = decltype(with_sinks)::value;
         float v[kBN];
         for (int i = 0; i < n; ++i) {
-          if (!warp_wait(&bars.s_full[t], s_seen & 1, abort, p.error_word, p.wait_ns)) {
+          const int b = s_seen & 1;
+          if (!warp_wait(&bars.s_full[b], (s_seen >> 1) & 1, abort, p.error_word, p.wait_ns)) {
             ok = false;
             break;
           }
-          ++s_seen;
+          const int gt = s_seen++;  // this tile's index over all items
           tc::fence_after_sync();
+          const uint32_t sc = tmem + lane_base + s_col(t, b);
 #pragma unroll
           for (int c = 0; c < kBN / 32; ++c) tc::tmem_ld32(sc + c * 32, v + c * 32);
           tc::tmem_wait_ld();
@@ -599,9 +597,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             rescale = true;
           }
           l *= alpha;
-          // O_t is stable here: P_t(i-1) V_{i-1} completed before S_t(i), and
-          // P_t(i) V_i waits for this warp's P.
-          if (__any_sync(0xffffffffu, rescale)) {
+          const float neg_m = m == -INFINITY ? 0.f : -m;  // an empty row keeps P = 0
+          float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
+          uint32_t pk[kBN / 2];
+#pragma unroll
+          for (int c = 0; c < kBN; c += 2) {
+            float x0, x1;
+            fma2(x0, x1, v[c], v[c + 1], sl2, neg_m);
+            const float w0 = fast_exp2(x0);
+            const float w1 = fast_exp2(x1);
+            const int k = (c >> 1) & 3;
+            add2(rs[2 * k], rs[2 * k + 1], w0, w1);
+            pk[c >> 1] = pack_bf16x2(w0, w1);
+          }
+          tc::tmem_st32(sc, reinterpret_cast<const float*>(pk));
+          l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+          // Rescale O_t after P(i-1) V_{i-1} has completed and before P(i) V_i
+          // is issued (before p_full): proven by S(i+1), or for the item's
+          // last tile by the per-item barrier (see the header).
+          if (i > 0 && __any_sync(0xffffffffu, rescale)) {
+            const bool waited =
+                i + 1 < n
+                    ? warp_wait(&bars.s_full[(gt + 1) & 1], ((gt + 1) >> 1) & 1, abort,
+                                p.error_word, p.wait_ns)
+                    : warp_wait(&bars.pv_item[0], pv_items & 1, abort, p.error_word, p.wait_ns);
+            if (!waited) {
+              tc::tmem_wait_st();  // no store of P may be in flight when TMEM is freed
+              ok = false;
+              break;
+            }
+            tc::fence_after_sync();
             float o[32];
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
@@ -612,44 +637,20 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc::tmem_st32(o_col + c * 32, o);
             }
           }
-          const float neg_m = m == -INFINITY ? 0.f : -m;  // an empty row keeps P = 0
-          float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
-#pragma unroll
-          for (int h = 0; h < kBN / 32; ++h) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              float x0, x1, w0, w1;
-              fma2(x0, x1, v[h * 32 + c], v[h * 32 + c + 1], sl2, neg_m);
-              if (((c >> 1) & 7) < kPolyOf8) {
-                exp2_poly2(w0, w1, x0, x1);
-              } else {
-                w0 = fast_exp2(x0);
-                w1 = fast_exp2(x1);
-              }
-              const int k = (c >> 1) & 3;
-              add2(rs[2 * k], rs[2 * k + 1], w0, w1);
-              pk[c >> 1] = pack_bf16x2(w0, w1);
-            }
-            tc::tmem_st16(sc + h * 16, pk);
-          }
-          l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
           tc::tmem_wait_st();
           tc::fence_before_sync();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bars.p_full[t]);
+          if (lane == 0) mbar_arrive(&bars.p_full[b]);
         }
       };
       if (p.sinks > 0) tile_loop(std::true_type{});
       else tile_loop(std::false_type{});
       if (!ok) break;
+      if (n >= 2) ++pv_items;
       // ---------------------------------------------------------- epilogue
       const bool have_o = n > 0;
       if (have_o) {
-        if (!warp_wait(&bars.o_final[t], o_seen & 1, abort, p.error_word, p.wait_ns)) {
-          ok = false;
-          break;
-        }
+        if (!warp_wait(&bars.o_final, o_seen & 1, abort, p.error_word, p.wait_ns)) { ok = false; break; }
         ++o_seen;
         tc::fence_after_sync();
       }
@@ -665,10 +666,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tmem_ld32(o_col + c * 32, o);
           tc::tmem_wait_ld();
           if (c + 1 == D / 32) {
-            // O_t may now be overwritten by the next item's first P V.
+            // O may now be overwritten by the next item's first P V.
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.o_empty[t]);
+            if (lane == 0) mbar_arrive(&bars.o_empty);
           }
         }
         if (row_ok) {
@@ -688,10 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (!ok) {
-      tc::tmem_wait_st();  // no store of P or O may be in flight when TMEM is freed
-      do_abort(abort, p.error_word);
-    }
+    if (!ok) do_abort(abort, p.error_word);
   }
 
   tc::fence_before_sync();

@@ -130,7 +130,7 @@ cudaError_t launch_attn_decode(const AttnParams& p, const CUtensorMap& k_map,
 // items from `work_counter` (device int, zeroed by the launch; one per
 // concurrently running launch).
 constexpr size_t kPrefillWorkspaceBytes = 256;
-constexpr int kPrefillKeyTile = 128;  // keys per tcgen05 prefill key tile (K/V box rows <= this)
+constexpr int kPrefillKeyTile = 64;   // keys per tcgen05 prefill key tile (K/V box rows <= this)
 cudaError_t launch_attn_prefill(const AttnParams& p, const CUtensorMap& q_map,
                                 const CUtensorMap& k_map, const CUtensorMap& v_map,
                                 int* work_counter, cudaStream_t stream);
