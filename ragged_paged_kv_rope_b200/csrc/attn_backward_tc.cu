@@ -459,11 +459,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok) {
       tc::tmem_wait_st();
       do_abort(abort, p.error_word);
-    } else if (key_ok) {
+    } else {
+      // tcgen05.ld is warp-collective: every lane loads, only keys below
+      // k_len on a valid page are stored
       const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
-      const int pi = key / p.P;
-      const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
-      const bool page_ok = page >= 0 && page < p.num_pages;
+      const int pi = key_ok ? key / p.P : 0;
+      const int page = key_ok && pi < p.max_pages ? __ldg(bt + pi) : -1;
+      const bool page_ok = key_ok && page >= 0 && page < p.num_pages;
       const size_t base = ((size_t)(page_ok ? page : 0) * p.P + (key - pi * p.P)) * p.Hk + kvh;
       float* dk = p.d_k + base * D + hh * (D / 2);
       float* dvp = p.d_v + base * D + hh * (D / 2);
@@ -781,7 +783,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok) {
       tc::tmem_wait_st();
       do_abort(abort, p.error_word);
-    } else if (row_ok) {
+    } else {
+      // tcgen05.ld is warp-collective: every lane loads, only valid rows store
       float* dq = p.d_q + hrow * D + hh * (D / 2);
       tc::fence_after_sync();
 #pragma unroll 1
@@ -794,11 +797,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) qv[e] = 0.f;
         }
+        if (row_ok) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dq + c + e) =
-              make_float4(qv[e] * p.scale, qv[e + 1] * p.scale, qv[e + 2] * p.scale,
-                          qv[e + 3] * p.scale);
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dq + c + e) =
+                make_float4(qv[e] * p.scale, qv[e + 1] * p.scale, qv[e + 2] * p.scale,
+                            qv[e + 3] * p.scale);
+        }
       }
     }
   }

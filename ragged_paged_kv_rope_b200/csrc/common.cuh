@@ -117,6 +117,17 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Two non-negative finite fp32 values -> bf16x2 (lo in bits 0-15) rounded to
+// nearest even with integer operations and one byte permute: adding 0x7FFF
+// plus the lowest kept bit to the fp32 bits and keeping the top half rounds
+// the dropped 16 bits to nearest, ties to even.
+__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
+  uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+  a += 0x7FFFu + ((a >> 16) & 1u);
+  b += 0x7FFFu + ((b >> 16) & 1u);
+  return __byte_perm(a, b, 0x7632);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
