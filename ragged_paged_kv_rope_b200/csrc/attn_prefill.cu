@@ -84,19 +84,6 @@ constexpr int kRegsSoftmax = 224;   // warpgroups 1 and 2: softmax
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows > 2^8
 
-#ifndef RPK_PREFILL_POLY_OF8
-#define RPK_PREFILL_POLY_OF8 0
-#endif
-#ifndef RPK_PREFILL_PACK_ALU
-#define RPK_PREFILL_PACK_ALU 0
-#endif
-// Of every 8 pairs of scores of a row, this many take 2^x on the FMA pipe
-// (exp2_poly2) and the rest on the exponential unit.
-constexpr int kPolyOf8 = RPK_PREFILL_POLY_OF8;
-// P is narrowed to bf16 by integer round-to-nearest-even on the ALU instead
-// of the conversion instruction.
-constexpr bool kPackAlu = RPK_PREFILL_PACK_ALU != 0;
-
 template <int D>
 struct Cfg {
   static constexpr int kBoxes = D / 64;
@@ -615,17 +602,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[kBN / 2];
 #pragma unroll
           for (int c = 0; c < kBN; c += 2) {
-            float x0, x1, w0, w1;
+            float x0, x1;
             fma2(x0, x1, v[c], v[c + 1], sl2, neg_m);
-            if (((c >> 1) & 7) < kPolyOf8) {
-              exp2_poly2(w0, w1, x0, x1);
-            } else {
-              w0 = fast_exp2(x0);
-              w1 = fast_exp2(x1);
-            }
+            const float w0 = fast_exp2(x0);
+            const float w1 = fast_exp2(x1);
             const int k = (c >> 1) & 3;
             add2(rs[2 * k], rs[2 * k + 1], w0, w1);
-            pk[c >> 1] = kPackAlu ? pack_bf16x2_alu(w0, w1) : pack_bf16x2(w0, w1);
+            pk[c >> 1] = pack_bf16x2(w0, w1);
           }
           tc::tmem_st32(sc, reinterpret_cast<const float*>(pk));
           l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));

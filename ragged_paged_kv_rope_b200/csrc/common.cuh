@@ -117,17 +117,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// Two non-negative finite fp32 values -> bf16x2 (lo in bits 0-15) rounded to
-// nearest even with integer operations and one byte permute: adding 0x7FFF
-// plus the lowest kept bit to the fp32 bits and keeping the top half rounds
-// the dropped 16 bits to nearest, ties to even.
-__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
-  uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
-  a += 0x7FFFu + ((a >> 16) & 1u);
-  b += 0x7FFFu + ((b >> 16) & 1u);
-  return __byte_perm(a, b, 0x7632);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -360,30 +349,6 @@ __device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, f
       "mov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-
-// 2^x0, 2^x1 on the FMA pipe, for x <= 2^8 (x below -127, -inf included,
-// gives +0). Range reduction x = n + f with n = round(x) and |f| <= 1/2:
-// adding 1.5 * 2^23 rounds x to an integer held in the low mantissa bits of
-// the sum. 2^f comes from a cubic fitted here to 2^f on [-1/2, 1/2] by
-// iteratively reweighted least squares in relative error (constant term 1
-// exactly; largest relative error 1.3e-4 after fp32 evaluation, far inside
-// the bf16 rounding of P), and 2^n is added to its exponent field.
-__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c1 = 0.6932254433631897f, c2 = 0.2422972172498703f,
-                  c3 = 0.0553351491689682f;
-  x0 = fmaxf(x0, -127.0f);
-  x1 = fmaxf(x1, -127.0f);
-  float t0, t1, n0, n1, f0, f1, q0, q1;
-  add2_to(t0, t1, x0, x1, kMagic, kMagic);       // round(x) in the low mantissa bits
-  add2_to(n0, n1, t0, t1, -kMagic, -kMagic);     // round(x) as a float
-  fma2_v(f0, f1, n0, n1, -1.0f, -1.0f, x0, x1);  // f = x - n
-  fma2_v(q0, q1, f0, f1, c3, c3, c2, c2);
-  fma2_v(q0, q1, q0, q1, f0, f1, c1, c1);
-  fma2_v(q0, q1, q0, q1, f0, f1, 1.0f, 1.0f);
-  y0 = __int_as_float(__float_as_int(q0) + (int)((uint32_t)__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(q1) + (int)((uint32_t)__float_as_int(t1) << 23));
 }
 
 // ------------------------------------- bounded waits of persistent kernels
