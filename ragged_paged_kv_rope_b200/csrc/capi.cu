@@ -401,19 +401,23 @@ rpk_status ragged_paged_attention_backward(
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (rpk::attn_backward_tc_supported(p, dtype)) {
     // tcgen05 kernels: TMA maps over q, d_out and the layer's pools
-    CUtensorMap q_map, do_map, k_map, v_map;
-    const int32_t tpt = 128 / p.G;
+    CUtensorMap q64, do64, q128, do128, k_map, v_map;
     const int32_t box_rows = p.P < 128 ? p.P : 128;
     const int64_t pool_rows = (int64_t)p.num_pages * p.P;
-    st = encode_rows_map(&q_map, q, head_dim, n_heads, total_q_tokens, p.G, tpt);
+    st = encode_rows_map(&q64, q, head_dim, n_heads, total_q_tokens, p.G, 64 / p.G);
     if (st != RPK_OK) return st;
-    st = encode_rows_map(&do_map, d_out, head_dim, n_heads, total_q_tokens, p.G, tpt);
+    st = encode_rows_map(&do64, d_out, head_dim, n_heads, total_q_tokens, p.G, 64 / p.G);
+    if (st != RPK_OK) return st;
+    st = encode_rows_map(&q128, q, head_dim, n_heads, total_q_tokens, p.G, 128 / p.G);
+    if (st != RPK_OK) return st;
+    st = encode_rows_map(&do128, d_out, head_dim, n_heads, total_q_tokens, p.G, 128 / p.G);
     if (st != RPK_OK) return st;
     st = encode_rows_map(&k_map, p.k_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
     if (st != RPK_OK) return st;
     st = encode_rows_map(&v_map, p.v_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
     if (st != RPK_OK) return st;
-    return cuda_status(rpk::launch_attn_backward_tc(p, q_map, do_map, k_map, v_map, s));
+    return cuda_status(
+        rpk::launch_attn_backward_tc(p, q64, do64, q128, do128, k_map, v_map, s));
   }
   return cuda_status(rpk::launch_attn_backward(p, dtype, s));
 }

@@ -160,12 +160,14 @@ struct BackwardParams {
 };
 cudaError_t launch_attn_backward(const BackwardParams& p, rpk_dtype dtype, cudaStream_t stream);
 // tcgen05 kernels: bf16 tensors over a bf16 cache, head_dim 64 / 128, groups of
-// up to 128 query heads. Maps: q and d_out as [T, H, d] with box (64, G,
-// 128 / G); the pools as [pages * page_size, n_kv_heads, d] with box
-// (64, 1, min(page_size, 128)); all 128-byte swizzled.
+// up to 64 query heads. Maps: q and d_out as [T, H, d] with box (64, G, 64 / G)
+// (the dK / dV kernel's 64-row blocks) and box (64, G, 128 / G) (the dQ
+// kernel's 128-row blocks); the pools as [pages * page_size, n_kv_heads, d]
+// with box (64, 1, min(page_size, 128)); all 128-byte swizzled.
 bool attn_backward_tc_supported(const BackwardParams& p, rpk_dtype dtype);
-cudaError_t launch_attn_backward_tc(const BackwardParams& p, const CUtensorMap& q_map,
-                                    const CUtensorMap& do_map, const CUtensorMap& k_map,
+cudaError_t launch_attn_backward_tc(const BackwardParams& p, const CUtensorMap& q_map64,
+                                    const CUtensorMap& do_map64, const CUtensorMap& q_map128,
+                                    const CUtensorMap& do_map128, const CUtensorMap& k_map,
                                     const CUtensorMap& v_map, cudaStream_t stream);
 // Tensor-core (mma.sync) kernels: bf16 tensors over a bf16 cache, groups of at
 // most 16 query heads, head_dim 64 / 128 / 256.
