@@ -26,7 +26,9 @@
 //        written back over the first half of each warp's own columns); then
 //        dV += P^T_j dO_j and dK += dS^T_j Q_j with P^T / dS^T read from
 //        tensor memory.
-//   dQ   one CTA per 128-row block. Q and dO stay in shared memory; the key
+//   dQ   one CTA per 128-row block, launched as a programmatic dependent of
+//        dK/dV (it waits for that grid only before storing, since d_q holds
+//        D until then). Q and dO stay in shared memory; the key
 //        blocks of the rows' band stream through rings of K (three deep) and
 //        V (two deep). Per key block i: S_i = Q K_i^T and dP_i = dO V_i^T
 //        (128 x 128, fp32); the compute warps (thread = row) load them and
@@ -225,6 +227,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (p.window > 0 && key0 >= p.sinks) i_hi = min(i_hi, key_hi + p.window - 1 - off);
   const int j_lo = i_lo / tpr;
   const int n_rb = i_lo <= i_hi ? i_hi / tpr - j_lo + 1 : 0;
+
+  // The dQ grid may start on SMs this grid's last CTAs leave idle; it waits
+  // for this grid's completion before its first store (griddepcontrol.wait).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -856,6 +862,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tmem_wait_st();
       do_abort(abort, p.error_word);
     } else {
+      // d_q holds D of every row until the dK / dV grid (launched before this
+      // one, as its programmatic dependent) has completed
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       // every lane loads (tcgen05.ld is warp-collective); valid rows store
       float* dq = p.d_q + hrow * D + hh * (D / 2);
       tc::fence_after_sync();
@@ -921,9 +930,20 @@ cudaError_t launch_d(const BackwardParams& p, const CUtensorMap& q_map64,
   const int tpt = 128 / p.G;
   const int n_rb = std::max(1, (p.max_q_len + tpt - 1) / tpt);
   const long long blocks = (long long)((n_rb + kGroup - 1) / kGroup) * units * kGroup;
-  attn_bwd_dq_tc_kernel<D><<<(unsigned)blocks, kThreads, kDqSmem, stream>>>(
-      p, q_map128, do_map128, k_map, v_map, n_rb);
-  return cudaGetLastError();
+  // A programmatic dependent of the dK / dV grid: its CTAs start as SMs free
+  // up and wait for that grid only before storing into d_q.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kDqSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = p.max_kv_len > 0 ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_bwd_dq_tc_kernel<D>, p, q_map128, do_map128, k_map, v_map,
+                            n_rb);
 }
 
 }  // namespace
