@@ -15,7 +15,9 @@
 // are deterministic:
 //   D    D_i of every row into the first T H floats of d_q (read by dK/dV; the
 //        dQ kernel computes D of its own rows and then overwrites d_q).
-//   dKV  one CTA per 128-key block of one (sequence, KV head). K and V stay in
+//   dKV  one CTA per 128-key block of one (sequence, KV head), launched as a
+//        programmatic dependent of D (its loader warp waits for D; the other
+//        warps start loading and multiplying at once). K and V stay in
 //        shared memory; the 64-row blocks that see the keys stream through a
 //        four-stage ring (Q and dO by TMA, -lse log2 e and -D by a loader warp).
 //        Per row block j the tensor core computes S^T_j = K Q_j^T and
@@ -134,6 +136,8 @@ __device__ __forceinline__ void bf16_pack8(uint32_t* out, const float* a) {
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_tc_delta_kernel(const BackwardParams p,
                                                                 float* __restrict__ delta) {
+  // the dK / dV grid may start at once; it reads D only after this grid completes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const long long row = ((long long)blockIdx.x * 256 + threadIdx.x) >> 3;
   const bool ok = row < (long long)p.T * p.H;
   const int part = threadIdx.x & 7;
@@ -214,10 +218,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kb = gidx * kGroup + rem % kGroup;
   const int b = unit / p.Hk, kvh = unit - (unit / p.Hk) * p.Hk;
   int q0, q_len, k_len;
-  if (kb >= n_kb || !seq_lengths(p, b, threadIdx.x == 0 && kvh == 0 && kb == 0, q0, q_len, k_len))
-    return;
+  const bool have_seq =
+      kb < n_kb && seq_lengths(p, b, threadIdx.x == 0 && kvh == 0 && kb == 0, q0, q_len, k_len);
   const int key0 = kb * 128;
-  if (key0 >= k_len) return;
+  if (!have_seq || key0 >= k_len) {
+    // Block 0 always waits for the D grid, so that this grid's completion
+    // (which the dQ grid waits for before overwriting D) implies D's.
+    if (blockIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+    return;
+  }
   const int key_hi = min(key0 + 128, k_len) - 1;
   const int off = k_len - q_len;  // row (token) i sits at position i + off
   // Tokens that see a key of the block: position >= key0, and under a window
@@ -312,6 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 2) {
     // --------------------------------------- loader: -lse log2 e and -D per row
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
+    // D comes from the D grid, of which this grid is a programmatic dependent
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     bool ok = true;
     for (int j = 0; j < n_rb && ok; ++j) {
       const int s = j % S;
@@ -922,9 +933,20 @@ cudaError_t launch_d(const BackwardParams& p, const CUtensorMap& q_map64,
     if (e != cudaSuccess) return e;
     const int n_kb = (p.max_kv_len + 127) / 128;
     const long long blocks = (long long)((n_kb + kGroup - 1) / kGroup) * units * kGroup;
-    attn_bwd_dkv_tc_kernel<D><<<(unsigned)blocks, kThreads, kDkvSmem, stream>>>(
-        p, q_map64, do_map64, k_map, v_map, delta, n_kb);
-    e = cudaGetLastError();
+    // A programmatic dependent of the D grid: only its loader warp reads D,
+    // after griddepcontrol.wait.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kDkvSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, attn_bwd_dkv_tc_kernel<D>, p, q_map64, do_map64, k_map, v_map,
+                           (const float*)delta, n_kb);
     if (e != cudaSuccess) return e;
   }
   const int tpt = 128 / p.G;
