@@ -251,9 +251,9 @@ size_t ragged_paged_attention_workspace_size(int32_t total_q_tokens, int32_t n_h
  * Paths (chosen from the host sizes, never from device data):
  *   dtype f32                      -> fp32 CUDA-core kernel
  *   bf16, max_q_len * group <= 16  -> split-KV decode kernel + combine kernel
- *   bf16, otherwise                -> tcgen05 prefill kernel (head_dim 64/128,
- *                                     group <= 128; other shapes run on the
- *                                     CUDA-core kernel)
+ *   bf16, otherwise                -> tcgen05 prefill kernel (head_dim 64, 128
+ *                                     and 256, group <= 128; larger groups run
+ *                                     on the CUDA-core kernel)
  * An RPK_E4M3 cache takes the same decode path (the kernel widens each tile
  * to f16 in shared memory, exactly, and folds k_scale into the score scale and
  * v_scale into the output); its other shapes run on the CUDA-core kernel.
@@ -297,12 +297,15 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
  *                   of its dequantised value); other entries are left as they
  *                   were, so a caller that sums over the pool zeroes them first.
  *
- * bf16 tensors over a bf16 cache with groups of at most 16 query heads run on
- * warp-level tensor cores (bf16 operands, fp32 sums; P and dS are rounded to
- * bf16 as operands of the second products). The kernels are: D_i of every
- * row, a key-parallel one for d_k and d_v, then a row-parallel one for d_q.
- * Other shapes (fp32 tensors, an e4m3 cache, larger groups) run on CUDA-core
- * kernels in fp32. Neither path uses atomics, so results are deterministic.
+ * bf16 tensors over a bf16 cache run on tensor cores (bf16 operands, fp32
+ * sums; P and dS are rounded to bf16 as operands of the second products):
+ * the 5th-generation ones (tcgen05, accumulators in tensor memory) for
+ * head_dim 64 and 128 with groups of at most 64 query heads, warp-level ones
+ * (mma.sync) for head_dim 256 with groups of at most 16. The kernels are: D_i
+ * of every row, a key-parallel one for d_k and d_v, then a row-parallel one for
+ * d_q. Other shapes (fp32 tensors, an e4m3 cache, larger groups) run on
+ * CUDA-core kernels in fp32. No path uses atomics, so results are
+ * deterministic.
  * Errors as ragged_paged_attention; every pointer is 16-byte aligned device
  * memory; buffers must not overlap.
  */

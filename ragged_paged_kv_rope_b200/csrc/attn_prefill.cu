@@ -8,48 +8,52 @@
 // online-softmax running state (algenta flash_attention: running max,
 // running sum and output rescaled by e^(m_old - m_new), final divide).
 //
-// Work unit (item): two query tiles A and B of 128 rows each of one
-// (sequence, KV head), against key tiles of 64 keys. The 128 rows of a tile
-// are the (token, query head) pairs of one KV head's group, token-major
-// (tokens_per_tile = 128 / G), so the G query heads that share a KV head share
-// every K/V tile; tile B holds the next tokens_per_tile tokens after tile A.
+// Work unit (item): NT query tiles of 128 rows each of one (sequence, KV
+// head), against key tiles of 64 keys; NT = 2 (tiles A and B) for head_dim 64
+// and 128, NT = 1 for head_dim 256. The 128 rows of a tile are the (token,
+// query head) pairs of one KV head's group, token-major (tokens_per_tile =
+// 128 / G), so the G query heads that share a KV head share every K/V tile;
+// tile B holds the next tokens_per_tile tokens after tile A.
 //
 // Persistent launch: one CTA per SM claims items from a counter in the
 // caller's workspace (zeroed by the launch). Items run sequence by sequence,
-// the last (longest) query pair of a sequence first: the CTAs that work on one
-// sequence at the same time read the same K/V tiles in the same order, so a
-// tile read from HBM for one of them is an L2 hit for the others.
+// the last (longest) query group of a sequence first: the CTAs that work on
+// one sequence at the same time read the same K/V tiles in the same order, so
+// a tile read from HBM for one of them is an L2 hit for the others.
 //
 // Tensor memory (512 columns): two score buffers of 64 columns per query
-// tile (S_t[0], S_t[1]) and one 128-row output accumulator per tile (O_A,
-// O_B). Score tile i of both query tiles lives in buffer i mod 2, and P_t(i)
-// (packed bf16 pairs) is written over the first 32 columns of S_t(i). The MMA
-// issuer computes S(i+2) right after issuing P(i) V_i, so while the softmax
-// warpgroups turn S(i) into P(i), the tensor core has already computed S(i+1):
-// the softmax does not wait for the tensor core in the steady state, and the
-// two softmax warpgroups keep the exponential unit busy together. Every item
-// runs both query tiles (tile B's rows past the sequence are masked and never
-// stored), so the two tiles share every barrier phase.
+// tile (S_t[0], S_t[1]) and one 128-row output accumulator per tile (O_t,
+// head_dim columns). Score tile i of every query tile lives in buffer i mod 2,
+// and P_t(i) (packed bf16 pairs) is written over the first 32 columns of
+// S_t(i). The MMA issuer computes S(i+2) right after issuing P(i) V_i, so
+// while the softmax warpgroups turn S(i) into P(i), the tensor core has
+// already computed S(i+1): the softmax does not wait for the tensor core in
+// the steady state. Every item runs all its query tiles (rows past the
+// sequence are masked and never stored), so the tiles share every barrier
+// phase.
 //
 // Warp roles (384 threads, three warpgroups):
 //   warp 0     TMA producer: claims the next item, hands its index to the
 //              other roles through a two-slot ring in shared memory, loads the
-//              item's two Q tiles, then each key tile's K and V into one stage
-//              of a ring (3-D map over the pool [pages * page_size, kv_heads,
-//              d], one box per page segment, 128-byte swizzle, no multicast)
+//              item's Q tiles, then each key tile's K into a ring of K slots
+//              and its V into a ring of V slots (3-D map over the pool
+//              [pages * page_size, kv_heads, d], one box per page segment,
+//              128-byte swizzle, no multicast). A K slot frees when the S MMAs
+//              that read it complete, a V slot when its P V MMAs do, so the K
+//              of tile i+2 never waits for the V of tile i.
 //   warp 1     allocates TMEM and issues the MMAs from one thread: per item
-//              S(0), S(1), then per key tile i one burst of O_A += P_A(i) V_i,
-//              O_B += P_B(i) V_i (P from TMEM, V an MN-major operand in shared
-//              memory), S_A(i+2) and S_B(i+2) (Q_t K^T, both operands in shared
-//              memory); the next item's first S MMAs follow the last P V of the
+//              S(0), S(1), then per key tile i one burst of O_t += P_t(i) V_i
+//              (P from TMEM, V an MN-major operand in shared memory) and
+//              S_t(i+2) (Q_t K^T, both operands in shared memory) for every
+//              tile t; the next item's first S MMAs follow the last P V of the
 //              current one
 //   warps 2-3  idle (they complete the first warpgroup)
-//   warps 4-7  softmax of tile A, warps 8-11 softmax of tile B: thread r owns
-//              row r (TMEM lane r); loads S_t(i), masks the band, keeps (m, l)
-//              in log2 units, writes P_t(i), and rescales O_t in TMEM only
-//              when the running max grew by more than 2^8 (the final O / l
-//              uses the same max, so this is exact); then normalises O_t and
-//              stores the rows.
+//   warps 4-7  softmax of tile A, warps 8-11 softmax of tile B (idle when
+//              NT = 1): thread r owns row r (TMEM lane r); loads S_t(i), masks
+//              the band, keeps (m, l) in log2 units, writes P_t(i), and
+//              rescales O_t in TMEM only when the running max grew by more
+//              than 2^8 (the final O / l uses the same max, so this is exact);
+//              then normalises O_t and stores the rows.
 // A rescale of O_t during tile i must fall between P(i-1) V_{i-1} and
 // P(i) V_i. For i < n - 1 the softmax waits for S(i+1), which the issuer
 // placed after P(i-1) V_{i-1}; for the item's last tile it waits for a
@@ -84,22 +88,29 @@ constexpr int kRegsSoftmax = 224;   // warpgroups 1 and 2: softmax
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows > 2^8
 
-template <int D>
+// NT query tiles of 128 rows per work item: two for head_dim 64 and 128, one
+// for head_dim 256 (whose 256-column output accumulator leaves tensor memory
+// for one tile's double-buffered scores only).
+template <int D, int NT>
 struct Cfg {
   static constexpr int kBoxes = D / 64;
-  static constexpr int kStages = D == 128 ? 5 : 10;  // K/V ring depth (key tiles)
+  // K and V rings (key tiles): K is freed once its S MMAs complete, V once its
+  // P V MMAs do, so S(i+2) never waits for the stage P(i) V_i is reading.
+  static constexpr int kKStages = D == 64 ? 10 : (D == 128 ? 5 : 3);
+  static constexpr int kVStages = D == 64 ? 10 : (D == 128 ? 4 : 2);
   static constexpr int kQBytes = kBM * D * 2;         // one query tile
   static constexpr int kKVBytes = kBN * D * 2;        // one K or V tile
-  static constexpr int kStageBytes = 2 * kKVBytes;    // K then V of one key tile
   static constexpr int kQOff = 0;
-  static constexpr int kKVOff = kQOff + 2 * kQBytes;
-  static constexpr int kEnd = kKVOff + kStages * kStageBytes + 1024;
+  static constexpr int kKOff = kQOff + NT * kQBytes;
+  static constexpr int kVOff = kKOff + kKStages * kKVBytes;
+  static constexpr int kEnd = kVOff + kVStages * kKVBytes + 1024;
   // At least half the SM's shared memory, so that one CTA holds the SM's TMEM.
   static constexpr int kSmemBytes = kEnd > 118 * 1024 ? kEnd : 118 * 1024;
-  // TMEM columns: S_t[b] (fp32, 64 each) at (2t + b) * 64, then O_A, O_B.
-  static constexpr uint32_t kOCol = 4 * kBN;
-  static_assert(kOCol + 2 * D <= kTmemCols, "TMEM budget");
-  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  // TMEM columns: S_t[b] (fp32, 64 each) at (2t + b) * 64, then O_t.
+  static constexpr uint32_t kOCol = 2 * NT * kBN;
+  static_assert(kOCol + NT * D <= kTmemCols, "TMEM budget");
+  static_assert(kSmemBytes <= 232448 - 1024, "shared memory budget");
+  static_assert(kKStages <= 10 && kVStages <= 10, "ring barriers");
 };
 
 __host__ __device__ constexpr uint32_t s_col(int t, int b) { return (uint32_t)((2 * t + b) * kBN); }
@@ -107,10 +118,12 @@ __host__ __device__ constexpr uint32_t s_col(int t, int b) { return (uint32_t)((
 struct Bars {
   uint64_t q_full;       // both query tiles loaded
   uint64_t q_empty;      // the item's last S MMAs reading them have completed
-  uint64_t kv_full[10];  // per stage: K and V of one key tile loaded
-  uint64_t kv_empty[10]; // per stage: its last P V has completed
-  uint64_t s_full[2];    // per score buffer: S_A and S_B computed
-  uint64_t p_full[2];    // per score buffer: P_A and P_B written (one arrival per softmax warp)
+  uint64_t k_full[10];   // per K slot: K of one key tile loaded
+  uint64_t k_empty[10];  // per K slot: its S MMAs have completed
+  uint64_t v_full[10];   // per V slot: V of one key tile loaded
+  uint64_t v_empty[10];  // per V slot: its P V MMAs have completed
+  uint64_t s_full[2];    // per score buffer: S of every query tile computed
+  uint64_t p_full[2];    // per score buffer: P of every tile written (per softmax warp)
   uint64_t pv_item[1];   // one phase per item with two or more key tiles: P(n-2) V done
   uint64_t o_final;      // the item's last P V has completed
   uint64_t o_empty;      // the epilogue has read O (one arrival per softmax warp)
@@ -136,7 +149,7 @@ __device__ __forceinline__ int tile_of(const Item& it, int i) {
 // Decode work item w (items ordered by sequence, then query-pair index
 // descending, then KV head). False when the item is empty or the sequence's
 // lengths are out of bounds (then RPK_DEVERR_LENGTH is raised once).
-__device__ __forceinline__ bool decode_item(const AttnParams& p, int w, int n_qpairs, int tpt,
+__device__ __forceinline__ bool decode_item(const AttnParams& p, int w, int n_qpairs, int span,
                                             bool report, Item& it) {
   const int per_seq = n_qpairs * p.Hk;
   it.b = w / per_seq;
@@ -150,9 +163,9 @@ __device__ __forceinline__ bool decode_item(const AttnParams& p, int w, int n_qp
     if (report && rem == 0) raise_error(p.error_word, RPK_DEVERR_LENGTH);
     return false;
   }
-  it.t_begin = qt * 2 * tpt;
+  it.t_begin = qt * span;
   if (it.t_begin >= it.q_len) return false;
-  const int t_end = min(it.q_len, it.t_begin + 2 * tpt);
+  const int t_end = min(it.q_len, it.t_begin + span);
   const int p_first = it.t_begin + it.k_len - it.q_len;
   const int p_last = (t_end - 1) + it.k_len - it.q_len;
   const int lo_first = p.window > 0 ? max(0, p_first - p.window + 1) : 0;
@@ -169,16 +182,16 @@ __device__ __forceinline__ bool decode_item(const AttnParams& p, int w, int n_qp
   return true;
 }
 
-template <int D>
+template <int D, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_prefill_kernel(const AttnParams p, const __grid_constant__ CUtensorMap q_map,
                         const __grid_constant__ CUtensorMap k_map,
                         const __grid_constant__ CUtensorMap v_map, const int tpt,
                         const int n_qpairs, int* __restrict__ work_counter) {
-  using C = Cfg<D>;
-  constexpr int S = C::kStages;
-  constexpr int kItemReaders = 9;  // MMA warp + 8 softmax warps
-  constexpr int kSoftmaxWarps = 8;
+  using C = Cfg<D, NT>;
+  constexpr int KS = C::kKStages, VS = C::kVStages;
+  constexpr int kSoftmaxWarps = 4 * NT;
+  constexpr int kItemReaders = 1 + kSoftmaxWarps;  // MMA warp + softmax warps
   extern __shared__ uint8_t smem_raw[];
   __shared__ Bars bars;
   __shared__ int item_slot[2];
@@ -191,18 +204,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_items = n_qpairs * p.batch * p.Hk;
   const int G = p.G;
   const int rows_used = tpt * G;
+  const int span = NT * tpt;  // tokens per work item
 
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const uint32_t sbase = smem_u32(smem);
   auto q_s = [&](int t) { return sbase + C::kQOff + t * C::kQBytes; };
-  auto k_s = [&](int st) { return sbase + C::kKVOff + st * C::kStageBytes; };
-  auto v_s = [&](int st) { return sbase + C::kKVOff + st * C::kStageBytes + C::kKVBytes; };
+  auto k_s = [&](int st) { return sbase + C::kKOff + st * C::kKVBytes; };
+  auto v_s = [&](int st) { return sbase + C::kVOff + st * C::kKVBytes; };
 
   if (threadIdx.x == 0) {
-    for (int st = 0; st < S; ++st) {
-      mbar_init(&bars.kv_full[st], 1);
-      mbar_init(&bars.kv_empty[st], 1);
+    for (int st = 0; st < KS; ++st) {
+      mbar_init(&bars.k_full[st], 1);
+      mbar_init(&bars.k_empty[st], 1);
+    }
+    for (int st = 0; st < VS; ++st) {
+      mbar_init(&bars.v_full[st], 1);
+      mbar_init(&bars.v_empty[st], 1);
     }
     mbar_init(&bars.q_full, 1);
     mbar_init(&bars.q_empty, 1);
@@ -244,7 +262,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_box_bytes = 128u * (uint32_t)rows_used;
       const int box_rows = p.P < kBN ? p.P : kBN;
       const uint32_t seg_bytes = (uint32_t)box_rows * 128u * C::kBoxes;
-      int kv_issued = 0;  // key tiles loaded over all items
+      int kv_issued = 0;  // key tiles whose K and V were loaded, over all items
+      int k_issued = 0, v_issued = 0;  // K and V tiles in flight or landed
       int q_loads = 0;    // Q loads over all items
       bool ok = true;
       // Claim a non-empty work item and hand its index to the MMA and softmax
@@ -255,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int w;
         do {
           w = atomicAdd(work_counter, 1);
-        } while (w < n_items && !decode_item(p, w, n_qpairs, tpt, true, it));
+        } while (w < n_items && !decode_item(p, w, n_qpairs, span, true, it));
         return w < n_items ? w : -1;
       };
       auto publish = [&](int seq, int w) -> bool {
@@ -267,13 +286,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&bars.item_full[slot]);
         return true;
       };
-      // The two Q tiles of an item, once the previous item's S MMAs that read
+      // The Q tiles of an item, once the previous item's S MMAs that read
       // them have completed. Rows past the last token read the fill value.
       auto load_q = [&](const Item& it) -> bool {
         if (q_loads > 0 && !thread_wait(&bars.q_empty, (q_loads - 1) & 1, abort, p.error_word, p.wait_ns))
           return false;
-        mbar_arrive_expect_tx(&bars.q_full, 2 * C::kBoxes * q_box_bytes);
-        for (int t = 0; t < 2; ++t)
+        mbar_arrive_expect_tx(&bars.q_full, NT * C::kBoxes * q_box_bytes);
+        for (int t = 0; t < NT; ++t)
 #pragma unroll
           for (int bx = 0; bx < C::kBoxes; ++bx)
             tma_load_3d(smem + C::kQOff + t * C::kQBytes + bx * (kBM * 128), &q_map, bx * 64,
@@ -281,42 +300,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++q_loads;
         return true;
       };
-      // K and V of key tile i of an item into the next stage of the ring; a
-      // stage frees once the P V MMAs that read its V have completed.
+      // K and V of key tile i of an item into the next slots of their rings;
+      // a K slot frees once the S MMAs that read it have completed, a V slot
+      // once the P V MMAs that read it have.
       auto load_stage = [&](const Item& it, int i) -> bool {
         const int32_t* bt = p.block_table + (size_t)it.b * p.max_pages;
         const int gi = kv_issued;
-        const int st = gi % S;
+        const int ks = gi % KS, vs = gi % VS;
         const int key0 = tile_of(it, i) * kBN;
-        if (gi >= S &&
-            !thread_wait(&bars.kv_empty[st], ((gi / S) & 1) ^ 1, abort, p.error_word, p.wait_ns))
-          return false;
         uint32_t bytes = 0;
         for (int r = 0; r < kBN; r += box_rows) {
           const int key = key0 + r;
           if (key >= it.k_len) break;
           const int pi = key / p.P;
           const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
-          if (page >= 0 && page < p.num_pages) bytes += 2 * seg_bytes;
+          if (page >= 0 && page < p.num_pages) bytes += seg_bytes;
         }
-        mbar_arrive_expect_tx(&bars.kv_full[st], bytes);
-        for (int r = 0; r < kBN; r += box_rows) {
-          const int key = key0 + r;
-          if (key >= it.k_len) break;
-          const int pi = key / p.P;
-          const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
-          if (page < 0 || page >= p.num_pages) {
-            raise_error(p.error_word, RPK_DEVERR_PAGE);
-            continue;
-          }
-          const int grow = page * p.P + (key - pi * p.P);
-          uint8_t* kb = smem + C::kKVOff + st * C::kStageBytes + r * 128;
+        for (int kind = 0; kind < 2; ++kind) {
+          const int st = kind == 0 ? ks : vs;
+          const int ring = kind == 0 ? KS : VS;
+          uint64_t* full = kind == 0 ? &bars.k_full[st] : &bars.v_full[st];
+          uint64_t* empty = kind == 0 ? &bars.k_empty[st] : &bars.v_empty[st];
+          if (gi >= ring &&
+              !thread_wait(empty, ((gi / ring) & 1) ^ 1, abort, p.error_word, p.wait_ns))
+            return false;
+          mbar_arrive_expect_tx(full, bytes);
+          const CUtensorMap* map = kind == 0 ? &k_map : &v_map;
+          uint8_t* base = smem + (kind == 0 ? C::kKOff : C::kVOff) + st * C::kKVBytes;
+          for (int r = 0; r < kBN; r += box_rows) {
+            const int key = key0 + r;
+            if (key >= it.k_len) break;
+            const int pi = key / p.P;
+            const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
+            if (page < 0 || page >= p.num_pages) {
+              if (kind == 0) raise_error(p.error_word, RPK_DEVERR_PAGE);
+              continue;
+            }
+            const int grow = page * p.P + (key - pi * p.P);
 #pragma unroll
-          for (int bx = 0; bx < C::kBoxes; ++bx) {
-            tma_load_3d(kb + bx * (kBN * 128), &k_map, bx * 64, it.kvh, grow, &bars.kv_full[st]);
-            tma_load_3d(kb + C::kKVBytes + bx * (kBN * 128), &v_map, bx * 64, it.kvh, grow,
-                        &bars.kv_full[st]);
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+              tma_load_3d(base + r * 128 + bx * (kBN * 128), map, bx * 64, it.kvh, grow, full);
           }
+          ++(kind == 0 ? k_issued : v_issued);
         }
         ++kv_issued;
         return true;
@@ -342,15 +367,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) do_abort(abort, p.error_word);
       // Never leave with copies in flight.
       if (q_loads > 0) mbar_wait(&bars.q_full, (q_loads - 1) & 1);
-      for (int gi = max(0, kv_issued - S); gi < kv_issued; ++gi)
-        mbar_wait(&bars.kv_full[gi % S], (gi / S) & 1);
+      for (int gi = max(0, k_issued - KS); gi < k_issued; ++gi)
+        mbar_wait(&bars.k_full[gi % KS], (gi / KS) & 1);
+      for (int gi = max(0, v_issued - VS); gi < v_issued; ++gi)
+        mbar_wait(&bars.v_full[gi % VS], (gi / VS) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
     constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(kBM, kBN, 0);
     constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(kBM, D, 1);
-    int g_kv = 0;        // key tiles whose stage has been waited for, over all items
+    int g_kv = 0;        // key tiles whose K slot has been waited for, over all items
     int g_pv = 0;        // key tiles whose P V has been issued, over all items
     int q_seen = 0;      // Q loads consumed
     int s_issued = 0;    // S tile pairs issued (buffer = count mod 2)
@@ -365,13 +392,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t k_lo0 = (uint32_t)tc::smem_desc_sw128(k_s(0), 16, 1024);
     const uint32_t v_lo0 = (uint32_t)tc::smem_desc_sw128(v_s(0), kBN * 128, 1024);
     const uint32_t desc_hi = (uint32_t)(q_desc0 >> 32);
-    // S_A and S_B of the key tile in stage kst into the next score buffer.
+    // S of every query tile for the K tile in slot kst into the next score
+    // buffer; the K slot is free once these MMAs complete.
     auto issue_s = [&](int kst) {
       const int b = s_issued & 1;
       if (lane == 0) {
-        const uint32_t kd = k_lo0 + (uint32_t)((kst * C::kStageBytes) >> 4);
+        const uint32_t kd = k_lo0 + (uint32_t)((kst * C::kKVBytes) >> 4);
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
+        for (int t = 0; t < NT; ++t) {
           const uint32_t d_tmem = tmem + s_col(t, b);
           const uint32_t qd = q_lo0 + (uint32_t)((t * C::kQBytes) >> 4);
 #pragma unroll
@@ -382,16 +410,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tc::commit(smem_u32(&bars.s_full[b]));
+        tc::commit(smem_u32(&bars.k_empty[kst]));
       }
       __syncwarp();
       ++s_issued;
     };
-    // O_t (+)= P_t V for both tiles, P_t in the first 32 columns of buffer b.
+    // O_t (+)= P_t V for every tile, P_t in the first 32 columns of buffer b.
     auto issue_pv = [&](int vst, int b, bool first) {
       if (lane == 0) {
-        const uint32_t vd = v_lo0 + (uint32_t)((vst * C::kStageBytes) >> 4);
+        const uint32_t vd = v_lo0 + (uint32_t)((vst * C::kKVBytes) >> 4);
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
+        for (int t = 0; t < NT; ++t) {
           const uint32_t d_tmem = tmem + C::kOCol + (uint32_t)(t * D);
           const uint32_t a_tmem = tmem + s_col(t, b);
 #pragma unroll
@@ -407,7 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     };
     auto wait_stage = [&]() -> bool {
-      if (!warp_wait(&bars.kv_full[g_kv % S], (g_kv / S) & 1, abort, p.error_word, p.wait_ns)) return false;
+      if (!warp_wait(&bars.k_full[g_kv % KS], (g_kv / KS) & 1, abort, p.error_word, p.wait_ns))
+        return false;
       ++g_kv;
       return true;
     };
@@ -422,28 +452,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&bars.item_empty[slot]);
       if (w < 0) break;
       Item it;
-      if (!decode_item(p, w, n_qpairs, tpt, false, it) || it.n_tiles == 0) continue;
+      if (!decode_item(p, w, n_qpairs, span, false, it) || it.n_tiles == 0) continue;
       const int n = it.n_tiles;
       ok = warp_wait(&bars.q_full, q_seen & 1, abort, p.error_word, p.wait_ns);
       ++q_seen;
       // S(0), S(1)
       for (int j = 0; ok && j < n && j < 2; ++j) {
-        const int kst = g_kv % S;
+        const int kst = g_kv % KS;
         if (!wait_stage()) { ok = false; break; }
         tc::fence_after_sync();
         issue_s(kst);
         if (j + 1 == n) commit_to(&bars.q_empty);  // last S of this item
       }
       for (int i = 0; ok && i < n; ++i) {
-        const int vst = g_pv % S;
+        const int vst = g_pv % VS;
         const int pb = g_pv & 1;
-        // P_A(i) and P_B(i) written, and the stage of key tile i+2 (for S(i+2)) loaded
+        // P(i) of every tile written, the K of key tile i+2 (for S(i+2)) and
+        // the V of key tile i loaded
         const bool more_s = i + 2 < n;
-        const int kst = more_s ? g_kv % S : -1;
+        const int kst = more_s ? g_kv % KS : -1;
         const bool waited =
-            more_s ? warp_wait2(&bars.p_full[pb], (g_pv >> 1) & 1, &bars.kv_full[g_kv % S],
-                                (g_kv / S) & 1, abort, p.error_word, p.wait_ns)
-                   : warp_wait(&bars.p_full[pb], (g_pv >> 1) & 1, abort, p.error_word, p.wait_ns);
+            (more_s ? warp_wait2(&bars.p_full[pb], (g_pv >> 1) & 1, &bars.k_full[g_kv % KS],
+                                 (g_kv / KS) & 1, abort, p.error_word, p.wait_ns)
+                    : warp_wait(&bars.p_full[pb], (g_pv >> 1) & 1, abort, p.error_word,
+                                p.wait_ns)) &&
+            warp_wait(&bars.v_full[vst], (g_pv / VS) & 1, abort, p.error_word, p.wait_ns);
         if (!waited) {
           ok = false;
           break;
@@ -451,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (more_s) ++g_kv;
         const int key0 = tile_of(it, i) * kBN;
         if (key0 + kBN > it.k_len) {
-          // zero value rows at or past k_len (the stage was waited for with S(i))
+          // zero value rows at or past k_len (the V slot was waited for above)
           const int r0 = max(0, it.k_len - key0);
           const int chunks = (kBN - r0) * C::kBoxes * 8;
           for (int idx = lane; idx < chunks; idx += 32) {
@@ -459,8 +492,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int rb = idx >> 3;
             const int bx = rb % C::kBoxes;
             const int r = r0 + rb / C::kBoxes;
-            uint8_t* dst = smem + C::kKVOff + vst * C::kStageBytes + C::kKVBytes +
-                           bx * (kBN * 128) + r * 128 + ch * 16;
+            uint8_t* dst = smem + C::kVOff + vst * C::kKVBytes + bx * (kBN * 128) + r * 128 +
+                           ch * 16;
             *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
           }
           fence_proxy_async_smem();
@@ -481,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           commit_to(&bars.o_final);
           ++o_commits;
         }
-        commit_to(&bars.kv_empty[vst]);
+        commit_to(&bars.v_empty[vst]);
         if (kst >= 0) {
           // S(i+2) overwrites the buffer P(i) lives in; the MMAs run in issue
           // order, so P(i) V_i has read it by then.
@@ -500,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------- softmax
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-    const int t = (warp - 4) >> 2;       // query tile: warps 4-7 -> A, 8-11 -> B
+    const int t = (warp - 4) >> 2;       // query tile: warps 4-7 -> A, 8-11 -> B (if NT == 2)
     const int qw = warp & 3;             // TMEM lane quarter of this warp
     const int r = qw * 32 + lane;        // row of this thread
     const uint32_t lane_base = (uint32_t)(qw * 32) << 16;
@@ -511,7 +544,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int pv_items = 0;    // items with two or more key tiles consumed
     bool ok = true;
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-    for (int seq = 0; ok; ++seq) {
+    // With one query tile per item the second softmax warpgroup has no rows.
+    for (int seq = 0; ok && t < NT; ++seq) {
       const int slot = seq & 1;
       if (!warp_wait(&bars.item_full[slot], (seq >> 1) & 1, abort, p.error_word, p.wait_ns)) {
         ok = false;
@@ -522,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&bars.item_empty[slot]);
       if (w < 0) break;
       Item it;
-      if (!decode_item(p, w, n_qpairs, tpt, false, it)) continue;
+      if (!decode_item(p, w, n_qpairs, span, false, it)) continue;
       const int tok = it.t_begin + t * tpt + r / G;
       const bool row_ok = r < rows_used && tok < it.q_len;
       const int pos = tok + it.k_len - it.q_len;
@@ -713,15 +747,15 @@ int sm_count() {
   return n[dev];
 }
 
-template <int D>
+template <int D, int NT>
 cudaError_t launch_d(const AttnParams& p, const CUtensorMap& q_map, const CUtensorMap& k_map,
                      const CUtensorMap& v_map, int* work_counter, cudaStream_t stream) {
-  using C = Cfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<D>,
+  using C = Cfg<D, NT>;
+  cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<D, NT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int tpt = prefill_rows_per_tile(p.G);
-  const int n_qpairs = (p.max_q_len + 2 * tpt - 1) / (2 * tpt);  // pairs of query tiles
+  const int n_qpairs = (p.max_q_len + NT * tpt - 1) / (NT * tpt);  // work items per (seq, head)
   const long long n_items = (long long)n_qpairs * p.batch * p.Hk;
   if (n_items == 0) return cudaSuccess;
   // Every CTA claims once past the last item, so the counter reaches n_items + grid.
@@ -730,8 +764,8 @@ cudaError_t launch_d(const AttnParams& p, const CUtensorMap& q_map, const CUtens
   e = cudaMemsetAsync(work_counter, 0, sizeof(int), stream);
   if (e != cudaSuccess) return e;
   const int grid = (int)std::min<long long>(n_items, sm_count());
-  attn_prefill_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(p, q_map, k_map, v_map, tpt,
-                                                                     n_qpairs, work_counter);
+  attn_prefill_kernel<D, NT><<<grid, kThreads, C::kSmemBytes, stream>>>(
+      p, q_map, k_map, v_map, tpt, n_qpairs, work_counter);
   return cudaGetLastError();
 }
 
@@ -743,8 +777,9 @@ cudaError_t launch_attn_prefill(const AttnParams& p, const CUtensorMap& q_map,
   if ((long long)p.T * p.H == 0 || p.batch == 0) return cudaSuccess;
   if (work_counter == nullptr) return cudaErrorInvalidValue;
   switch (p.d) {
-    case 64: return launch_d<64>(p, q_map, k_map, v_map, work_counter, stream);
-    case 128: return launch_d<128>(p, q_map, k_map, v_map, work_counter, stream);
+    case 64: return launch_d<64, 2>(p, q_map, k_map, v_map, work_counter, stream);
+    case 128: return launch_d<128, 2>(p, q_map, k_map, v_map, work_counter, stream);
+    case 256: return launch_d<256, 1>(p, q_map, k_map, v_map, work_counter, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -328,9 +328,9 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
   // An e4m3 cache under prefill shapes: CUDA-core kernel.
   if (p.cache_fp8) return cuda_status(rpk::launch_attn_simt(p, dtype, s));
 
-  // Prefill shapes: tcgen05 kernel for head_dim 64 / 128 and groups up to 128.
+  // Prefill shapes: tcgen05 kernel for head_dim 64 / 128 / 256 and groups up to 128.
   const int tpt = rpk::prefill_rows_per_tile(p.G);
-  if ((head_dim == 64 || head_dim == 128) && tpt > 0) {
+  if (tpt > 0) {
     if (!workspace || workspace_bytes < rpk::kPrefillWorkspaceBytes) return RPK_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return RPK_ERR_WORKSPACE;
     CUtensorMap q_map, k_map, v_map;
@@ -345,7 +345,7 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
     return cuda_status(
         rpk::launch_attn_prefill(p, q_map, k_map, v_map, static_cast<int*>(workspace), s));
   }
-  // head_dim 256 (or groups above 128): CUDA-core kernel.
+  // groups above 128 query heads per KV head: CUDA-core kernel.
   return cuda_status(rpk::launch_attn_simt(p, dtype, s));
 }
 

@@ -126,7 +126,7 @@ cudaError_t launch_attn_decode(const AttnParams& p, const CUtensorMap& k_map,
                                const CUtensorMap& v_map, const DecodePlan& plan,
                                const DecodeWorkspace& ws, cudaStream_t stream);
 
-// tcgen05 prefill (bf16, head_dim 64 or 128), persistent: its CTAs claim work
+// tcgen05 prefill (bf16, head_dim 64, 128 or 256), persistent: its CTAs claim work
 // items from `work_counter` (device int, zeroed by the launch; one per
 // concurrently running launch).
 constexpr size_t kPrefillWorkspaceBytes = 256;

@@ -160,6 +160,15 @@ def test_attention_gemma_window_with_sinks_sampled():
     _attn_case(sp, [1] * sp.batch, [32769] * sp.batch, seed=51, rows=rng_rows, sinks=4)
 
 
+@pytest.mark.parametrize("window", [0, 200])
+def test_attention_prefill_head_dim_256(window):
+    # Gemma-like layout (16 query heads over 8 KV heads, head_dim 256): one
+    # query tile per work item, several 64-key tiles, ragged tails, a chunked
+    # row block and a short sequence
+    sp = W.spec("gemma_swa_decode", batch=3, page_size=64)
+    _attn_case(sp, [300, 129, 7], [300, 700, 7], seed=16, window=window)
+
+
 def test_attention_prefill_shapes_bf16():
     sp = W.spec("ragged_prefill", n_heads=8, n_kv_heads=2)
     _attn_case(sp, [130, 64, 1, 257], [130, 64, 400, 300], seed=11)
