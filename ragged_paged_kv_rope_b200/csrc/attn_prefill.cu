@@ -94,16 +94,24 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max
 template <int D, int NT>
 struct Cfg {
   static constexpr int kBoxes = D / 64;
-  // K and V rings (key tiles): K is freed once its S MMAs complete, V once its
-  // P V MMAs do, so S(i+2) never waits for the stage P(i) V_i is reading.
-  static constexpr int kKStages = D == 64 ? 10 : (D == 128 ? 5 : 3);
-  static constexpr int kVStages = D == 64 ? 10 : (D == 128 ? 4 : 2);
+  // head_dim 64 / 128: one ring of stages, each the K and V of one key tile,
+  // freed when its P V MMAs complete. head_dim 256: a ring of K slots, freed
+  // when their S MMAs complete, and a ring of V slots, freed when their P V
+  // MMAs do; with one 64 KB stage per tile only two would fit, and S(i+2),
+  // issued right after P(i) V_i, would wait for the stage P(i) V_i reads.
+  static constexpr bool kSplit = D == 256;
+  static constexpr int kKStages = D == 64 ? 10 : (D == 128 ? 5 : 3);  // stages / K slots
+  static constexpr int kVStages = kSplit ? 2 : kKStages;              // V slots
   static constexpr int kQBytes = kBM * D * 2;         // one query tile
   static constexpr int kKVBytes = kBN * D * 2;        // one K or V tile
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + NT * kQBytes;
-  static constexpr int kVOff = kKOff + kKStages * kKVBytes;
-  static constexpr int kEnd = kVOff + kVStages * kKVBytes + 1024;
+  // unified stage st: K at kKOff + 2 st kKVBytes, V right after it
+  static constexpr int kKStride = kSplit ? kKVBytes : 2 * kKVBytes;
+  static constexpr int kVOff = kSplit ? kKOff + kKStages * kKVBytes : kKOff + kKVBytes;
+  static constexpr int kVStride = kKStride;
+  static constexpr int kEnd =
+      (kSplit ? kVOff + kVStages * kKVBytes : kKOff + kKStages * 2 * kKVBytes) + 1024;
   // At least half the SM's shared memory, so that one CTA holds the SM's TMEM.
   static constexpr int kSmemBytes = kEnd > 118 * 1024 ? kEnd : 118 * 1024;
   // TMEM columns: S_t[b] (fp32, 64 each) at (2t + b) * 64, then O_t.
@@ -210,8 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const uint32_t sbase = smem_u32(smem);
   auto q_s = [&](int t) { return sbase + C::kQOff + t * C::kQBytes; };
-  auto k_s = [&](int st) { return sbase + C::kKOff + st * C::kKVBytes; };
-  auto v_s = [&](int st) { return sbase + C::kVOff + st * C::kKVBytes; };
+  auto k_s = [&](int st) { return sbase + C::kKOff + st * C::kKStride; };
+  auto v_s = [&](int st) { return sbase + C::kVOff + st * C::kVStride; };
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < KS; ++st) {
@@ -317,16 +325,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (page >= 0 && page < p.num_pages) bytes += seg_bytes;
         }
         for (int kind = 0; kind < 2; ++kind) {
+          // unified stages: K and V share the stage's barriers (kind 0 waits
+          // and expects both tiles' bytes)
           const int st = kind == 0 ? ks : vs;
           const int ring = kind == 0 ? KS : VS;
-          uint64_t* full = kind == 0 ? &bars.k_full[st] : &bars.v_full[st];
+          uint64_t* full = (kind == 0 || !C::kSplit) ? &bars.k_full[st] : &bars.v_full[st];
           uint64_t* empty = kind == 0 ? &bars.k_empty[st] : &bars.v_empty[st];
-          if (gi >= ring &&
-              !thread_wait(empty, ((gi / ring) & 1) ^ 1, abort, p.error_word, p.wait_ns))
-            return false;
-          mbar_arrive_expect_tx(full, bytes);
+          if (kind == 0 || C::kSplit) {
+            if (gi >= ring &&
+                !thread_wait(empty, ((gi / ring) & 1) ^ 1, abort, p.error_word, p.wait_ns))
+              return false;
+            mbar_arrive_expect_tx(full, C::kSplit ? bytes : 2 * bytes);
+          }
           const CUtensorMap* map = kind == 0 ? &k_map : &v_map;
-          uint8_t* base = smem + (kind == 0 ? C::kKOff : C::kVOff) + st * C::kKVBytes;
+          uint8_t* base = smem + (kind == 0 ? C::kKOff + st * C::kKStride
+                                            : C::kVOff + st * C::kVStride);
           for (int r = 0; r < kBN; r += box_rows) {
             const int key = key0 + r;
             if (key >= it.k_len) break;
@@ -369,8 +382,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (q_loads > 0) mbar_wait(&bars.q_full, (q_loads - 1) & 1);
       for (int gi = max(0, k_issued - KS); gi < k_issued; ++gi)
         mbar_wait(&bars.k_full[gi % KS], (gi / KS) & 1);
-      for (int gi = max(0, v_issued - VS); gi < v_issued; ++gi)
-        mbar_wait(&bars.v_full[gi % VS], (gi / VS) & 1);
+      if constexpr (C::kSplit)
+        for (int gi = max(0, v_issued - VS); gi < v_issued; ++gi)
+          mbar_wait(&bars.v_full[gi % VS], (gi / VS) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
@@ -397,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_s = [&](int kst) {
       const int b = s_issued & 1;
       if (lane == 0) {
-        const uint32_t kd = k_lo0 + (uint32_t)((kst * C::kKVBytes) >> 4);
+        const uint32_t kd = k_lo0 + (uint32_t)((kst * C::kKStride) >> 4);
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
           const uint32_t d_tmem = tmem + s_col(t, b);
@@ -410,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tc::commit(smem_u32(&bars.s_full[b]));
-        tc::commit(smem_u32(&bars.k_empty[kst]));
+        if constexpr (C::kSplit) tc::commit(smem_u32(&bars.k_empty[kst]));
       }
       __syncwarp();
       ++s_issued;
@@ -418,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // O_t (+)= P_t V for every tile, P_t in the first 32 columns of buffer b.
     auto issue_pv = [&](int vst, int b, bool first) {
       if (lane == 0) {
-        const uint32_t vd = v_lo0 + (uint32_t)((vst * C::kKVBytes) >> 4);
+        const uint32_t vd = v_lo0 + (uint32_t)((vst * C::kVStride) >> 4);
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
           const uint32_t d_tmem = tmem + C::kOCol + (uint32_t)(t * D);
@@ -467,16 +481,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; ok && i < n; ++i) {
         const int vst = g_pv % VS;
         const int pb = g_pv & 1;
-        // P(i) of every tile written, the K of key tile i+2 (for S(i+2)) and
-        // the V of key tile i loaded
+        // P(i) of every tile written and the K (unified: the stage) of key
+        // tile i+2 (for S(i+2)) loaded; split rings also wait for the V of
+        // key tile i here (a unified stage was waited for with its S)
         const bool more_s = i + 2 < n;
         const int kst = more_s ? g_kv % KS : -1;
-        const bool waited =
-            (more_s ? warp_wait2(&bars.p_full[pb], (g_pv >> 1) & 1, &bars.k_full[g_kv % KS],
-                                 (g_kv / KS) & 1, abort, p.error_word, p.wait_ns)
-                    : warp_wait(&bars.p_full[pb], (g_pv >> 1) & 1, abort, p.error_word,
-                                p.wait_ns)) &&
-            warp_wait(&bars.v_full[vst], (g_pv / VS) & 1, abort, p.error_word, p.wait_ns);
+        bool waited =
+            more_s ? warp_wait2(&bars.p_full[pb], (g_pv >> 1) & 1, &bars.k_full[g_kv % KS],
+                                (g_kv / KS) & 1, abort, p.error_word, p.wait_ns)
+                   : warp_wait(&bars.p_full[pb], (g_pv >> 1) & 1, abort, p.error_word,
+                               p.wait_ns);
+        if constexpr (C::kSplit)
+          waited = waited &&
+                   warp_wait(&bars.v_full[vst], (g_pv / VS) & 1, abort, p.error_word, p.wait_ns);
         if (!waited) {
           ok = false;
           break;
@@ -492,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int rb = idx >> 3;
             const int bx = rb % C::kBoxes;
             const int r = r0 + rb / C::kBoxes;
-            uint8_t* dst = smem + C::kVOff + vst * C::kKVBytes + bx * (kBN * 128) + r * 128 +
+            uint8_t* dst = smem + C::kVOff + vst * C::kVStride + bx * (kBN * 128) + r * 128 +
                            ch * 16;
             *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
           }
@@ -514,7 +531,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           commit_to(&bars.o_final);
           ++o_commits;
         }
-        commit_to(&bars.v_empty[vst]);
+        // the V slot (unified: the whole stage) is free once P(i) V_i completes
+        commit_to(C::kSplit ? &bars.v_empty[vst] : &bars.k_empty[vst]);
         if (kst >= 0) {
           // S(i+2) overwrites the buffer P(i) lives in; the MMAs run in issue
           // order, so P(i) V_i has read it by then.
