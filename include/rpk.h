@@ -256,7 +256,11 @@ size_t ragged_paged_attention_workspace_size(int32_t total_q_tokens, int32_t n_h
  *                                     on the CUDA-core kernel)
  * An RPK_E4M3 cache takes the same decode path (the kernel widens each tile
  * to f16 in shared memory, exactly, and folds k_scale into the score scale and
- * v_scale into the output); its other shapes run on the CUDA-core kernel.
+ * v_scale into the output) and, for head_dim 64 and 128, the same tcgen05
+ * prefill path (two warps widen each key tile's codes to f16 in shared memory;
+ * each query row is narrowed to f16 under a power-of-two scale that is folded
+ * back into its scores); e4m3 prefill shapes of head_dim 256 run on the
+ * CUDA-core kernel.
  */
 rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
                                   const int32_t* kv_lens, const rpk_paged_kv* page_table,

@@ -80,7 +80,7 @@ extern "C" rpk_status ragged_paged_attention_noalloc(
     return RPK_ERR_SHAPE;
   if ((long long)max_kv_len > (long long)c->max_pages_per_seq * c->page_size)
     return RPK_ERR_SHAPE;
-  void *k_layer, *v_layer;
+  void *k_layer = nullptr, *v_layer = nullptr;
   rpk::layer_pools(c, &k_layer, &v_layer);
   const int32_t group = n_heads / n_kv_heads;
   // Only the split-KV decode path uses scratch; this entry point runs nothing else.

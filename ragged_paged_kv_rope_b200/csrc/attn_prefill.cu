@@ -90,8 +90,10 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max
 
 // NT query tiles of 128 rows per work item: two for head_dim 64 and 128, one
 // for head_dim 256 (whose 256-column output accumulator leaves tensor memory
-// for one tile's double-buffered scores only).
-template <int D, int NT>
+// for one tile's double-buffered scores only). F8: the pools hold e4m3 codes;
+// TMA brings each key tile's codes into a small raw ring and two converter
+// warps widen them to f16 in the stages the MMAs read.
+template <int D, int NT, bool F8 = false>
 struct Cfg {
   static constexpr int kBoxes = D / 64;
   // head_dim 64 / 128: one ring of stages, each the K and V of one key tile,
@@ -100,7 +102,10 @@ struct Cfg {
   // MMAs do; with one 64 KB stage per tile only two would fit, and S(i+2),
   // issued right after P(i) V_i, would wait for the stage P(i) V_i reads.
   static constexpr bool kSplit = D == 256;
-  static constexpr int kKStages = D == 64 ? 10 : (D == 128 ? 5 : 3);  // stages / K slots
+  static_assert(!(F8 && kSplit), "e4m3 prefill takes head_dim 64 / 128");
+  static_assert(!F8 || NT == 2, "e4m3: one converter warp narrows each query tile");
+  static constexpr int kKStages =
+      D == 64 ? (F8 ? 8 : 10) : (D == 128 ? (F8 ? 4 : 5) : 3);  // stages / K slots
   static constexpr int kVStages = kSplit ? 2 : kKStages;              // V slots
   static constexpr int kQBytes = kBM * D * 2;         // one query tile
   static constexpr int kKVBytes = kBN * D * 2;        // one K or V tile
@@ -110,8 +115,11 @@ struct Cfg {
   static constexpr int kKStride = kSplit ? kKVBytes : 2 * kKVBytes;
   static constexpr int kVOff = kSplit ? kKOff + kKStages * kKVBytes : kKOff + kKVBytes;
   static constexpr int kVStride = kKStride;
-  static constexpr int kEnd =
-      (kSplit ? kVOff + kVStages * kKVBytes : kKOff + kKStages * 2 * kKVBytes) + 1024;
+  static constexpr int kRawStages = F8 ? 2 : 0;         // raw ring: K then V codes of a tile
+  static constexpr int kRawBytes = kBN * D;             // codes of one K or V tile
+  static constexpr int kRawOff =
+      kSplit ? kVOff + kVStages * kKVBytes : kKOff + kKStages * 2 * kKVBytes;
+  static constexpr int kEnd = kRawOff + kRawStages * 2 * kRawBytes + 1024;
   // At least half the SM's shared memory, so that one CTA holds the SM's TMEM.
   static constexpr int kSmemBytes = kEnd > 118 * 1024 ? kEnd : 118 * 1024;
   // TMEM columns: S_t[b] (fp32, 64 each) at (2t + b) * 64, then O_t.
@@ -133,6 +141,10 @@ struct Bars {
   uint64_t s_full[2];    // per score buffer: S of every query tile computed
   uint64_t p_full[2];    // per score buffer: P of every tile written (per softmax warp)
   uint64_t pv_item[1];   // one phase per item with two or more key tiles: P(n-2) V done
+  uint64_t raw_full[2];  // e4m3: per raw stage, the codes of one key tile loaded
+  uint64_t raw_empty[2]; // e4m3: per raw stage, both converter warps done with it
+  uint64_t q_ready[2];   // e4m3, per Q load parity: the Q tiles narrowed to f16 and their
+                         // row scales written (one arrival per converter warp)
   uint64_t o_final;      // the item's last P V has completed
   uint64_t o_empty;      // the epilogue has read O (one arrival per softmax warp)
   uint64_t item_full[2];   // work-item ring: index written by the producer
@@ -190,22 +202,27 @@ __device__ __forceinline__ bool decode_item(const AttnParams& p, int w, int n_qp
   return true;
 }
 
-template <int D, int NT>
+template <int D, int NT, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_prefill_kernel(const AttnParams p, const __grid_constant__ CUtensorMap q_map,
                         const __grid_constant__ CUtensorMap k_map,
                         const __grid_constant__ CUtensorMap v_map, const int tpt,
                         const int n_qpairs, int* __restrict__ work_counter) {
-  using C = Cfg<D, NT>;
+  using C = Cfg<D, NT, F8>;
   constexpr int KS = C::kKStages, VS = C::kVStages;
+  constexpr int RS = C::kRawStages;
   constexpr int kSoftmaxWarps = 4 * NT;
-  constexpr int kItemReaders = 1 + kSoftmaxWarps;  // MMA warp + softmax warps
+  // MMA warp, softmax warps and, for an e4m3 cache, the two converter warps
+  constexpr int kItemReaders = 1 + kSoftmaxWarps + (F8 ? 2 : 0);
   extern __shared__ uint8_t smem_raw[];
   __shared__ Bars bars;
   __shared__ int item_slot[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   __shared__ int skip_sh;
+  // e4m3: per Q load parity and row, the power-of-two exponent k2 its query
+  // row was scaled by when narrowed to f16
+  __shared__ int8_t q_k2_sh[F8 ? 2 * NT * kBM : 1];
   volatile int* abort = &abort_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -223,9 +240,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < KS; ++st) {
-      mbar_init(&bars.k_full[st], 1);
+      mbar_init(&bars.k_full[st], F8 ? 2 : 1);  // e4m3: one arrival per converter warp
       mbar_init(&bars.k_empty[st], 1);
     }
+    for (int st = 0; st < RS; ++st) {
+      mbar_init(&bars.raw_full[st], 1);
+      mbar_init(&bars.raw_empty[st], 2);
+    }
+    for (int k = 0; k < 2; ++k) mbar_init(&bars.q_ready[k], 2);
     for (int st = 0; st < VS; ++st) {
       mbar_init(&bars.v_full[st], 1);
       mbar_init(&bars.v_empty[st], 1);
@@ -316,6 +338,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int gi = kv_issued;
         const int ks = gi % KS, vs = gi % VS;
         const int key0 = tile_of(it, i) * kBN;
+        if constexpr (F8) {
+          // e4m3 codes of K then V into the next raw stage, rows of D bytes
+          const int rs = gi % RS;
+          if (gi >= RS && !thread_wait(&bars.raw_empty[rs], ((gi / RS) & 1) ^ 1, abort,
+                                       p.error_word, p.wait_ns))
+            return false;
+          uint32_t cbytes = 0;
+          for (int r = 0; r < kBN; r += box_rows) {
+            const int key = key0 + r;
+            if (key >= it.k_len) break;
+            const int pi = key / p.P;
+            const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
+            if (page >= 0 && page < p.num_pages) cbytes += (uint32_t)box_rows * D;
+          }
+          mbar_arrive_expect_tx(&bars.raw_full[rs], 2 * cbytes);
+          uint8_t* raw = smem + C::kRawOff + rs * 2 * C::kRawBytes;
+          for (int r = 0; r < kBN; r += box_rows) {
+            const int key = key0 + r;
+            if (key >= it.k_len) break;
+            const int pi = key / p.P;
+            const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
+            if (page < 0 || page >= p.num_pages) {
+              raise_error(p.error_word, RPK_DEVERR_PAGE);
+              continue;
+            }
+            const int grow = page * p.P + (key - pi * p.P);
+            tma_load_3d(raw + r * D, &k_map, 0, it.kvh, grow, &bars.raw_full[rs]);
+            tma_load_3d(raw + C::kRawBytes + r * D, &v_map, 0, it.kvh, grow,
+                        &bars.raw_full[rs]);
+          }
+          ++kv_issued;
+          ++k_issued;
+          return true;
+        }
         uint32_t bytes = 0;
         for (int r = 0; r < kBN; r += box_rows) {
           const int key = key0 + r;
@@ -380,8 +436,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) do_abort(abort, p.error_word);
       // Never leave with copies in flight.
       if (q_loads > 0) mbar_wait(&bars.q_full, (q_loads - 1) & 1);
-      for (int gi = max(0, k_issued - KS); gi < k_issued; ++gi)
-        mbar_wait(&bars.k_full[gi % KS], (gi / KS) & 1);
+      if constexpr (F8) {
+        for (int gi = max(0, k_issued - RS); gi < k_issued; ++gi)
+          mbar_wait(&bars.raw_full[gi % RS], (gi / RS) & 1);
+      } else {
+        for (int gi = max(0, k_issued - KS); gi < k_issued; ++gi)
+          mbar_wait(&bars.k_full[gi % KS], (gi / KS) & 1);
+      }
       if constexpr (C::kSplit)
         for (int gi = max(0, v_issued - VS); gi < v_issued; ++gi)
           mbar_wait(&bars.v_full[gi % VS], (gi / VS) & 1);
@@ -389,8 +450,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
-    constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(kBM, kBN, 0);
-    constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(kBM, D, 1);
+    // e4m3 caches: K, V, Q and P are f16 (K and V widened exactly, Q scaled
+    // per row by a power of two), bf16 otherwise
+    constexpr uint32_t idesc_qk =
+        F8 ? tc::idesc_f16_f32(kBM, kBN, 0) : tc::idesc_bf16_f32(kBM, kBN, 0);
+    constexpr uint32_t idesc_pv = F8 ? tc::idesc_f16_f32(kBM, D, 1) : tc::idesc_bf16_f32(kBM, D, 1);
     int g_kv = 0;        // key tiles whose K slot has been waited for, over all items
     int g_pv = 0;        // key tiles whose P V has been issued, over all items
     int q_seen = 0;      // Q loads consumed
@@ -468,7 +532,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       Item it;
       if (!decode_item(p, w, n_qpairs, span, false, it) || it.n_tiles == 0) continue;
       const int n = it.n_tiles;
-      ok = warp_wait(&bars.q_full, q_seen & 1, abort, p.error_word, p.wait_ns);
+      ok = F8 ? warp_wait(&bars.q_ready[q_seen & 1], (q_seen >> 1) & 1, abort, p.error_word,
+                          p.wait_ns)
+              : warp_wait(&bars.q_full, q_seen & 1, abort, p.error_word, p.wait_ns);
       ++q_seen;
       // S(0), S(1)
       for (int j = 0; ok && j < n && j < 2; ++j) {
@@ -546,8 +612,118 @@ __global__ void __launch_bounds__(kThreads, 1)
     commit_to(&bars.drain);
     if (!warp_wait(&bars.drain, 0, abort, p.error_word, p.wait_ns)) mbar_wait(&bars.drain, 0);
   } else if (warp < 4) {
-    // idle warps of the first warpgroup
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
+    if constexpr (F8) {
+      // ---------------------------------------------- e4m3 converter warps
+      // Warp 2 widens the K codes, warp 3 the V codes of each key tile from
+      // its raw stage into the f16 stage the MMAs read (every e4m3 value is
+      // exact in f16), in the 128-byte-swizzled layout TMA would have written.
+      // At the start of each item with keys, warp 2 + t first narrows query
+      // tile t to f16 in place: each row is scaled by the power of two 2^k2
+      // that brings its largest magnitude into [2^14, 2^15) (exact for every
+      // element above f16's normal range floor: bf16 has 8 significant bits,
+      // f16 11), and k2 is left for the softmax warps, which fold 2^-k2 and
+      // k_scale into the score scale and v_scale into the output.
+      const int kind = warp - 2;  // 0: K, 1: V
+      int gi = 0;                 // key tiles converted over all items
+      int ql = 0;                 // Q loads narrowed
+      bool ok = true;
+      auto narrow_q = [&]() {
+        uint8_t* qtile = smem + C::kQOff + kind * C::kQBytes;
+        int8_t* k2s = q_k2_sh + (ql & 1) * (NT * kBM) + kind * kBM;
+        for (int r = lane; r < rows_used; r += 32) {
+          float mx = 0.f;
+#pragma unroll
+          for (int ch = 0; ch < D / 8; ++ch) {
+            const uint4 w4 = *reinterpret_cast<const uint4*>(
+                qtile + (ch >> 3) * (kBM * 128) + swz128((uint32_t)r, (uint32_t)(ch & 7)));
+            const uint32_t wds[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float2 f =
+                  __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wds[k]));
+              mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+          }
+          const int e = (int)((__float_as_uint(mx) >> 23) & 0xFFu) - 127;  // floor(log2 mx)
+          int k2 = (mx > 0.f && mx < INFINITY) ? 14 - e : 0;
+          k2 = max(-126, min(126, k2));
+          k2s[r] = (int8_t)k2;
+          const float up = __uint_as_float((uint32_t)(127 + k2) << 23);
+#pragma unroll
+          for (int ch = 0; ch < D / 8; ++ch) {
+            uint4* cp = reinterpret_cast<uint4*>(
+                qtile + (ch >> 3) * (kBM * 128) + swz128((uint32_t)r, (uint32_t)(ch & 7)));
+            const uint4 w4 = *cp;
+            const uint32_t wds[4] = {w4.x, w4.y, w4.z, w4.w};
+            uint32_t o4[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float2 f =
+                  __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wds[k]));
+              o4[k] = pack_f16x2(f.x * up, f.y * up);
+            }
+            *cp = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+          }
+        }
+        fence_proxy_async_smem();  // generic writes before the MMAs read Q
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.q_ready[ql & 1]);
+        ++ql;
+      };
+      for (int seq = 0; ok; ++seq) {
+        const int slot = seq & 1;
+        if (!warp_wait(&bars.item_full[slot], (seq >> 1) & 1, abort, p.error_word, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        const int w = *reinterpret_cast<volatile int*>(&item_slot[slot]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.item_empty[slot]);
+        if (w < 0) break;
+        Item it;
+        if (!decode_item(p, w, n_qpairs, span, false, it)) continue;
+        if (it.n_tiles > 0) {
+          if (!warp_wait(&bars.q_full, ql & 1, abort, p.error_word, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          narrow_q();
+        }
+        for (int i = 0; ok && i < it.n_tiles; ++i, ++gi) {
+          const int rs = gi % RS, st = gi % KS;
+          if (!warp_wait(&bars.raw_full[rs], (gi / RS) & 1, abort, p.error_word, p.wait_ns) ||
+              (gi >= KS && !warp_wait(&bars.k_empty[st], ((gi / KS) & 1) ^ 1, abort,
+                                      p.error_word, p.wait_ns))) {
+            ok = false;
+            break;
+          }
+          const uint8_t* raw = smem + C::kRawOff + rs * 2 * C::kRawBytes + kind * C::kRawBytes;
+          uint8_t* dst = smem + (kind == 0 ? C::kKOff + st * C::kKStride
+                                           : C::kVOff + st * C::kVStride);
+          constexpr int kChunks = kBN * (D / 8);  // 8 codes -> 16 bytes of f16
+#pragma unroll 4
+          for (int c = lane; c < kChunks; c += 32) {
+            const int row = c / (D / 8), c8 = c % (D / 8);
+            const uint2 w8 = *reinterpret_cast<const uint2*>(raw + row * D + c8 * 8);
+            uint4 h;
+            h.x = f16x2_from_e4m3x2(w8.x & 0xFFFFu);
+            h.y = f16x2_from_e4m3x2(w8.x >> 16);
+            h.z = f16x2_from_e4m3x2(w8.y & 0xFFFFu);
+            h.w = f16x2_from_e4m3x2(w8.y >> 16);
+            *reinterpret_cast<uint4*>(dst + (c8 >> 3) * (kBN * 128) +
+                                      swz128((uint32_t)row, (uint32_t)(c8 & 7))) = h;
+          }
+          fence_proxy_async_smem();  // generic writes before the MMAs read them
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&bars.k_full[st]);
+            mbar_arrive(&bars.raw_empty[rs]);
+          }
+        }
+      }
+      if (!ok) do_abort(abort, p.error_word);
+    }
   } else {
     // ------------------------------------------------------------- softmax
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
@@ -556,7 +732,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = qw * 32 + lane;        // row of this thread
     const uint32_t lane_base = (uint32_t)(qw * 32) << 16;
     const uint32_t o_col = tmem + lane_base + C::kOCol + (uint32_t)(t * D);
-    const float sl2 = p.scale_log2;
+    float sl2 = p.scale_log2;  // e4m3: times k_scale and the row's Q scale, per item
+    int q_seen_sm = 0;         // e4m3: Q loads consumed
     int s_seen = 0;      // score tiles consumed over all items
     int o_seen = 0;      // items with keys consumed
     int pv_items = 0;    // items with two or more key tiles consumed
@@ -582,6 +759,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int hi = pos;
       const int n = it.n_tiles;
       float m = -INFINITY, l = 0.f;      // running max (log2 units) and sum
+      float v_mul = 1.f;                 // e4m3: v_scale of the item's KV head
+      if constexpr (F8) {
+        if (n > 0) {
+          // The converter warps narrowed this row's query to f16 under 2^k2.
+          const int qs = q_seen_sm++;
+          if (!warp_wait(&bars.q_ready[qs & 1], (qs >> 1) & 1, abort, p.error_word, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          const int k2 = r < rows_used ? (int)q_k2_sh[(qs & 1) * (NT * kBM) + t * kBM + r] : 0;
+          const float down = __uint_as_float((uint32_t)(127 - k2) << 23);
+          sl2 = p.scale_log2 * __ldg(p.k_scale + it.kvh) * down;
+          v_mul = __ldg(p.v_scale + it.kvh);
+        }
+      }
       // The tile loop, compiled twice: without attention sinks (the common
       // case keeps the plain single-interval mask) and with them.
       auto tile_loop = [&](auto with_sinks) {
@@ -660,7 +852,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float w1 = fast_exp2(x1);
             const int k = (c >> 1) & 3;
             add2(rs[2 * k], rs[2 * k + 1], w0, w1);
-            pk[c >> 1] = pack_bf16x2(w0, w1);
+            pk[c >> 1] = F8 ? pack_f16x2(w0, w1) : pack_bf16x2(w0, w1);
           }
           tc::tmem_st32(sc, reinterpret_cast<const float*>(pk));
           l += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
@@ -706,7 +898,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++o_seen;
         tc::fence_after_sync();
       }
-      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      const float inv = (l > 0.f) ? v_mul / l : 0.f;
       const size_t hrow = (size_t)(it.q0 + tok) * p.H + (size_t)it.kvh * G + (r % G);
       const size_t orow = hrow * D;
       // l is relative to the (possibly stale) running max m, so m + log2 l is exact.
@@ -765,11 +957,11 @@ int sm_count() {
   return n[dev];
 }
 
-template <int D, int NT>
+template <int D, int NT, bool F8>
 cudaError_t launch_d(const AttnParams& p, const CUtensorMap& q_map, const CUtensorMap& k_map,
                      const CUtensorMap& v_map, int* work_counter, cudaStream_t stream) {
-  using C = Cfg<D, NT>;
-  cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<D, NT>,
+  using C = Cfg<D, NT, F8>;
+  cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<D, NT, F8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int tpt = prefill_rows_per_tile(p.G);
@@ -782,7 +974,7 @@ cudaError_t launch_d(const AttnParams& p, const CUtensorMap& q_map, const CUtens
   e = cudaMemsetAsync(work_counter, 0, sizeof(int), stream);
   if (e != cudaSuccess) return e;
   const int grid = (int)std::min<long long>(n_items, sm_count());
-  attn_prefill_kernel<D, NT><<<grid, kThreads, C::kSmemBytes, stream>>>(
+  attn_prefill_kernel<D, NT, F8><<<grid, kThreads, C::kSmemBytes, stream>>>(
       p, q_map, k_map, v_map, tpt, n_qpairs, work_counter);
   return cudaGetLastError();
 }
@@ -794,10 +986,17 @@ cudaError_t launch_attn_prefill(const AttnParams& p, const CUtensorMap& q_map,
                                 int* work_counter, cudaStream_t stream) {
   if ((long long)p.T * p.H == 0 || p.batch == 0) return cudaSuccess;
   if (work_counter == nullptr) return cudaErrorInvalidValue;
+  if (p.cache_fp8) {
+    switch (p.d) {
+      case 64: return launch_d<64, 2, true>(p, q_map, k_map, v_map, work_counter, stream);
+      case 128: return launch_d<128, 2, true>(p, q_map, k_map, v_map, work_counter, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (p.d) {
-    case 64: return launch_d<64, 2>(p, q_map, k_map, v_map, work_counter, stream);
-    case 128: return launch_d<128, 2>(p, q_map, k_map, v_map, work_counter, stream);
-    case 256: return launch_d<256, 1>(p, q_map, k_map, v_map, work_counter, stream);
+    case 64: return launch_d<64, 2, false>(p, q_map, k_map, v_map, work_counter, stream);
+    case 128: return launch_d<128, 2, false>(p, q_map, k_map, v_map, work_counter, stream);
+    case 256: return launch_d<256, 1, false>(p, q_map, k_map, v_map, work_counter, stream);
     default: return cudaErrorInvalidValue;
   }
 }

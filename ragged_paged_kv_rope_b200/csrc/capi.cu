@@ -78,12 +78,13 @@ bool cache_dtype_ok(rpk_dtype dtype, rpk_dtype cache) {
   return cache == dtype || cache == RPK_E4M3;
 }
 
-// 3-D byte map over rows of an e4m3 pool [rows, heads, d]: for head_dim >= 128
-// boxes of (128 codes, 1, box_rows) with the 128-byte swizzle (the decode
-// kernel reads K fragments straight from them), for head_dim 64 whole rows,
-// no swizzle.
+// 3-D byte map over rows of an e4m3 pool [rows, heads, d]. Decode layout
+// (whole_rows false): for head_dim >= 128 boxes of (128 codes, 1, box_rows)
+// with the 128-byte swizzle (the decode kernel reads K fragments straight from
+// them), for head_dim 64 whole rows, no swizzle. whole_rows true: whole rows of
+// d codes, no swizzle (the prefill kernel's raw ring, which it widens to f16).
 rpk_status encode_rows_map_u8(CUtensorMap* map, const void* base, int32_t d, int32_t heads,
-                              int64_t rows, int32_t box_rows) {
+                              int64_t rows, int32_t box_rows, bool whole_rows = false) {
   auto fn = encode_fn();
   if (!fn) {
     set_last_error_text("cuTensorMapEncodeTiled unavailable");
@@ -91,7 +92,7 @@ rpk_status encode_rows_map_u8(CUtensorMap* map, const void* base, int32_t d, int
   }
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)heads * d};
-  const bool swizzled = d >= 128;
+  const bool swizzled = d >= 128 && !whole_rows;
   cuuint32_t box[3] = {swizzled ? 128u : (cuuint32_t)d, 1u, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
@@ -325,12 +326,10 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
     if (st != RPK_OK) return st;
     return cuda_status(rpk::launch_attn_decode(p, k_map, v_map, plan, ws, s));
   }
-  // An e4m3 cache under prefill shapes: CUDA-core kernel.
-  if (p.cache_fp8) return cuda_status(rpk::launch_attn_simt(p, dtype, s));
-
-  // Prefill shapes: tcgen05 kernel for head_dim 64 / 128 / 256 and groups up to 128.
+  // Prefill shapes: tcgen05 kernel for head_dim 64 / 128 / 256 and groups up
+  // to 128 (an e4m3 cache: head_dim 64 / 128, its codes widened to f16 on chip).
   const int tpt = rpk::prefill_rows_per_tile(p.G);
-  if (tpt > 0) {
+  if (tpt > 0 && (!p.cache_fp8 || head_dim <= 128)) {
     if (!workspace || workspace_bytes < rpk::kPrefillWorkspaceBytes) return RPK_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return RPK_ERR_WORKSPACE;
     CUtensorMap q_map, k_map, v_map;
@@ -338,14 +337,21 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
     const int64_t pool_rows = (int64_t)p.num_pages * p.P;
     st = encode_rows_map(&q_map, q, head_dim, n_heads, total_q_tokens, p.G, tpt);
     if (st != RPK_OK) return st;
-    st = encode_rows_map(&k_map, p.k_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
-    if (st != RPK_OK) return st;
-    st = encode_rows_map(&v_map, p.v_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
+    if (p.cache_fp8) {
+      st = encode_rows_map_u8(&k_map, p.k_pages, head_dim, n_kv_heads, pool_rows, box_rows, true);
+      if (st != RPK_OK) return st;
+      st = encode_rows_map_u8(&v_map, p.v_pages, head_dim, n_kv_heads, pool_rows, box_rows, true);
+    } else {
+      st = encode_rows_map(&k_map, p.k_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
+      if (st != RPK_OK) return st;
+      st = encode_rows_map(&v_map, p.v_pages, head_dim, n_kv_heads, pool_rows, 1, box_rows);
+    }
     if (st != RPK_OK) return st;
     return cuda_status(
         rpk::launch_attn_prefill(p, q_map, k_map, v_map, static_cast<int*>(workspace), s));
   }
-  // groups above 128 query heads per KV head: CUDA-core kernel.
+  // groups above 128 query heads per KV head, or an e4m3 cache of head_dim
+  // 256: CUDA-core kernel.
   return cuda_status(rpk::launch_attn_simt(p, dtype, s));
 }
 

@@ -67,6 +67,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn_maj
          | ((uint32_t)(M >> 4) << 24);    // M / 16
 }
 
+// The same for f16 x f16 -> f32 (A and B both f16).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int b_mn_major) {
+  return (1u << 4)                        // D format: f32
+         | (0u << 7)                      // A format: f16
+         | (0u << 10)                     // B format: f16
+         | (0u << 15)                     // A K-major
+         | ((uint32_t)b_mn_major << 16)   // B major
+         | ((uint32_t)(N >> 3) << 17)     // N / 8
+         | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
 // --------------------------------------------------------------- MMA
 
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.

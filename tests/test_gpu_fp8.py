@@ -191,3 +191,56 @@ def test_end_to_end_decode_step_e4m3():
                       dev.cache.v_pages.cpu(), wl.block_table, sp.n_kv_heads, sp.softmax_scale,
                       sp.window, k_scale=wl.k_scale, v_scale=wl.v_scale)
     check_attention(out.cpu(), ref, "bf16", "decode step e4m3")
+
+
+# ------------------------------------------- prefill shapes over an e4m3 cache
+# The tcgen05 prefill kernel widens each key tile's codes to f16 on chip (exact)
+# and narrows each Q row to f16 under a power-of-two scale, so the products are
+# those of the bf16 path up to f16's extra mantissa bits.
+
+def _e4m3_prefill_case(sp, q_lens, kv_lens, seed, window=0, sinks=0, q_mul=None):
+    wl = W.attention_only(sp, seed, q_lens, kv_lens)
+    if q_mul is not None:
+        wl.q = (wl.q.float() * q_mul).to(torch.bfloat16)
+    dev = to_device(wl)
+    lse = torch.full((wl.total_tokens, sp.n_heads), float("nan"), device="cuda")
+    out = gpu_attention(wl, dev, dev.q, window=window, lse=lse, sinks=sinks)
+    torch.cuda.synchronize()
+    assert int(dev.error_word.item()) == 0
+    ref, ref_lse = O.attention(wl.q, wl.q_offsets, wl.kv_lens, wl.k_pages, wl.v_pages,
+                               wl.block_table, sp.n_kv_heads, sp.softmax_scale, window,
+                               with_lse=True, sinks=sinks, k_scale=wl.k_scale,
+                               v_scale=wl.v_scale)
+    what = f"e4m3 prefill d={sp.head_dim} q={list(q_lens)} window={window} sinks={sinks}"
+    check_lse(lse.cpu(), ref_lse, what)
+    check_attention(out.cpu(), ref, "bf16", what)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("window,sinks", [(0, 0), (150, 0), (129, 70)])
+def test_prefill_over_e4m3_cache(d, window, sinks):
+    # two query tiles per item, several key tiles, ragged tails, a chunk whose
+    # first token sits deep in its sequence and a one-token sequence
+    sp = W.spec("ragged_prefill", cache_dtype="e4m3", head_dim=d, rotary_dim=d, batch=4,
+                n_heads=8, n_kv_heads=2)
+    _e4m3_prefill_case(sp, [300, 129, 1, 77], [300, 700, 64, 77], seed=21, window=window,
+                       sinks=sinks)
+
+
+def test_prefill_over_e4m3_cache_page_16_group_8():
+    # pages of 16 tokens (a key tile spans four pages) and eight query heads per
+    # KV head (16 tokens per query tile)
+    sp = W.spec("llama3_8b_decode", cache_dtype="e4m3", batch=3, n_heads=16, n_kv_heads=2,
+                page_size=16)
+    _e4m3_prefill_case(sp, [100, 33, 250], [400, 33, 250], seed=22)
+
+
+def test_prefill_e4m3_large_and_small_queries():
+    # Q rows far outside f16's range in both directions: each row's
+    # power-of-two pre-scale keeps its scores right.
+    sp = W.spec("ragged_prefill", cache_dtype="e4m3", batch=3, n_heads=8, n_kv_heads=2)
+    wl = W.attention_only(sp, 23, [200, 70, 130], [200, 300, 130])
+    mul = torch.ones(wl.total_tokens, 1, 1)
+    mul[:200] = 1e6
+    mul[200:270] = 1e-7
+    _e4m3_prefill_case(sp, [200, 70, 130], [200, 300, 130], seed=23, q_mul=mul)
