@@ -431,8 +431,12 @@ def kernel_of(wl: W.Workload) -> tuple[str, str]:
         return "attn_simt", "ragged_paged_attention (CUDA-core fp32 kernel)"
     if is_decode(wl):
         return "attn_decode", "ragged_paged_attention (split-KV decode + combine)"
-    if sp.head_dim in (64, 128) and sp.cache_dtype is None:
-        return "attn_prefill", "ragged_paged_attention (tcgen05 prefill)"
+    if sp.n_heads // sp.n_kv_heads <= 128:
+        if sp.cache_dtype is None and sp.head_dim in (64, 128, 256):
+            return "attn_prefill", "ragged_paged_attention (tcgen05 prefill)"
+        if sp.cache_dtype == "e4m3" and sp.head_dim in (64, 128):
+            return ("attn_prefill_e4m3",
+                    "ragged_paged_attention (tcgen05 prefill, e4m3 codes widened to f16 on chip)")
     return "attn_simt", "ragged_paged_attention (CUDA-core kernel)"
 
 
@@ -718,10 +722,12 @@ def main():
     peaks = load_peaks()
     value = job_amount / (step_ms * 1e-3) / scale
     achieved = amount / (attn_ms_mean * 1e-3) / scale
-    # the committed DRAM capture is of the bf16-cache decode kernel
-    traffic = load_traffic(f"{kernel_of(wl)[0]}@{sp.name}") if sp.cache_dtype is None else None
+    key, kdesc = kernel_of(wl)
+    if decode and sp.cache_dtype is not None:
+        key = f"{key}_{sp.cache_dtype}"
+    traffic = load_traffic(f"{key}@{sp.name}")
     if decode:
-        roofline = {"bound": "hbm", "kernel": "ragged_paged_attention (split-KV decode + combine)",
+        roofline = {"bound": "hbm", "kernel": kdesc,
                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": unit,
                     "frac": achieved / peaks["hbm_gbs"],
                     "traffic": None if traffic is None else traffic["bytes_per_launch"],
@@ -729,10 +735,7 @@ def main():
                     if peaks["source"] == "measured" else "fallback 6.65 TB/s",
                     "algorithmic_bytes_per_launch": kv_bytes}
     else:
-        kernel = ("ragged_paged_attention (tcgen05 prefill)"
-                  if sp.dtype == "bf16" and sp.head_dim in (64, 128)
-                  else "ragged_paged_attention (CUDA-core kernel)")
-        roofline = {"bound": "tensor", "kernel": kernel, "achieved": achieved,
+        roofline = {"bound": "tensor", "kernel": kdesc, "achieved": achieved,
                     "peak": peaks["bf16_tflops"], "unit": unit,
                     "frac": achieved / peaks["bf16_tflops"],
                     "traffic": None if traffic is None else traffic["bytes_per_launch"],

@@ -79,13 +79,14 @@ DecodePlan decode_plan(int32_t max_kv_len) {
 }
 
 DecodePlan decode_launch_plan(int32_t max_kv_len, int32_t units, int32_t head_dim, int32_t window,
-                              int32_t max_q_len, int32_t sinks) {
+                              int32_t max_q_len, int32_t sinks, bool cache_fp8) {
   // Longer splits stream more bytes per CTA for the same start-up and merge,
   // but a launch needs enough CTAs to fill the GPU, and a last wave with few
   // CTAs cannot keep HBM busy. When every (sequence, KV head) unit fits in one
   // wave (two CTAs per SM for head_dim <= 128, one for 256), the splits fill
   // exactly one wave. Otherwise aim at two waves and keep splits between the
-  // sizing plan's and 24 tiles (16 for head_dim 256). Then even out the splits
+  // sizing plan's and 24 tiles (16 for head_dim 256; three times that for
+  // e4m3 codes, whose tiles hold half the bytes). Then even out the splits
   // of the longest band.
   const DecodePlan most = decode_plan(max_kv_len);
   // Keys a sequence's rows can see: under a window at most window + max_q_len - 1
@@ -106,7 +107,10 @@ DecodePlan decode_launch_plan(int32_t max_kv_len, int32_t units, int32_t head_di
     const long long slots = 2 * wave;
     const long long per_unit = std::max(1LL, (slots + n_units - 1) / n_units);
     tps = (max_tiles + per_unit - 1) / per_unit;
-    const int32_t cap = std::max(head_dim <= 128 ? 24 : 16, most.tiles_per_split);
+    // e4m3 tiles are half the bytes: longer splits (three times the tiles
+  // measured best on the Llama-3-8B and Gemma-like decodes)
+    const int32_t cap = std::max((head_dim <= 128 ? 24 : 16) * (cache_fp8 ? 3 : 1),
+                                 most.tiles_per_split);
     tps = std::min<long long>(std::max<long long>(tps, most.tiles_per_split), cap);
   }
   const int32_t splits = (int32_t)((max_tiles + tps - 1) / tps);
@@ -188,9 +192,9 @@ struct DecodeCfg {
   static_assert(kConsumerWarps * 16 * D * 4 <= kStages * kStageBytes, "merge buffer");
 };
 
-// e4m3 cache: stages of raw codes [64 keys][D bytes] for K then V, and one
-// f16 tile of 16 rows (kBoxes 128-byte swizzled boxes) for K and for V per
-// consumer warp.
+// e4m3 cache: stages of raw codes [64 keys][D bytes] for K then V, and per
+// consumer warp one f16 tile of 16 rows (kBoxes 128-byte swizzled boxes) for V
+// and, for head_dim 64 (whose K is widened too), one for K.
 template <int D>
 struct DecodeCfg<D, true> {
   static constexpr int kBoxes = D / 64;
@@ -198,8 +202,10 @@ struct DecodeCfg<D, true> {
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kStages = D == 256 ? 4 : (D == 128 ? 4 : 8);
   static constexpr int kConvTileBytes = 16 * D * 2;           // 16 rows of f16
+  static constexpr int kConvTiles = D >= 128 ? 1 : 2;         // V, and K for head_dim 64
   static constexpr int kConvOff = kStages * kStageBytes;
-  static constexpr int kSmemBytes = kConvOff + kConsumerWarps * 2 * kConvTileBytes + 1024;
+  static constexpr int kSmemBytes =
+      kConvOff + kConsumerWarps * kConvTiles * kConvTileBytes + 1024;
   static_assert(kConsumerWarps * 16 * D * 4 <= kSmemBytes - 1024, "merge buffer");
 };
 
@@ -433,8 +439,8 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
     if constexpr (kFp8) {
       // Widen this warp's 16 rows of K and V from e4m3 codes to f16 in its own
       // tiles (value rows at or past k_len become zeros), then release the stage.
-      uint8_t* ck = smem + Cfg::kConvOff + warp * 2 * Cfg::kConvTileBytes;
-      uint8_t* cv = ck + Cfg::kConvTileBytes;
+      uint8_t* ck = smem + Cfg::kConvOff + warp * Cfg::kConvTiles * Cfg::kConvTileBytes;
+      uint8_t* cv = ck + (Cfg::kConvTiles - 1) * Cfg::kConvTileBytes;  // == ck when K is read raw
       constexpr int kChunks = D / 16;  // 16-code chunks per row
       // K, then V (one tile at a time keeps fewer registers live under the
       // 168-register cap; head_dim 256 runs one CTA per SM and unrolls both)
@@ -454,20 +460,22 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
                        : raw + (wrow0 + kr) * D + j * 16;
           uint4 r4 = *reinterpret_cast<const uint4*>(src);
           if (kv && key0 + kr >= k_len) r4 = make_uint4(0, 0, 0, 0);
-          const uint32_t w[4] = {r4.x, r4.y, r4.z, r4.w};
-          uint32_t h[8];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            h[2 * q] = f16x2_from_e4m3x2(w[q] & 0xFFFFu);
-            h[2 * q + 1] = f16x2_from_e4m3x2(w[q] >> 16);
-          }
-          // f16 channels 16j .. 16j+15 are the 16-byte chunks 2j and 2j+1 of the row.
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int ch = 2 * j + hh;
-            *reinterpret_cast<uint4*>(conv + (ch >> 3) * kBoxStride + swz128(kr, ch & 7)) =
-                make_uint4(h[4 * hh], h[4 * hh + 1], h[4 * hh + 2], h[4 * hh + 3]);
-          }
+          // f16 channels 16j .. 16j+7 and 16j+8 .. 16j+15 are the 16-byte
+          // chunks 2j and 2j+1 of the row, in one 64-channel box. A 16-byte
+          // store is served eight lanes at a time; for head_dim >= 128 those
+          // eight lanes are chunks 0-7 of one row, whose first units fall on
+          // four bank groups only, so odd groups of four store their second
+          // unit first: eight distinct bank groups per store.
+          const int sw = (j >> 2) & 1;
+          uint4 a, b;  // a to chunk 2j + sw, b to chunk 2j + 1 - sw
+          f16x4_from_e4m3x4(sw ? r4.z : r4.x, a.x, a.y);
+          f16x4_from_e4m3x4(sw ? r4.w : r4.y, a.z, a.w);
+          f16x4_from_e4m3x4(sw ? r4.x : r4.z, b.x, b.y);
+          f16x4_from_e4m3x4(sw ? r4.y : r4.w, b.z, b.w);
+          const int ch = 2 * j;
+          uint8_t* row_box = conv + (ch >> 3) * kBoxStride;
+          *reinterpret_cast<uint4*>(row_box + swz128(kr, (ch & 7) + sw)) = a;
+          *reinterpret_cast<uint4*>(row_box + swz128(kr, (ch & 7) + 1 - sw)) = b;
         }
       }
       __syncwarp();

@@ -300,7 +300,8 @@ rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
   if ((long long)max_q_len * p.G <= rpk::kDecodeMaxRows) {
     const size_t need = rpk::decode_workspace_bytes(total_q_tokens, n_heads, head_dim, max_kv_len);
     const rpk::DecodePlan plan = rpk::decode_launch_plan(max_kv_len, batch * n_kv_heads, head_dim,
-                                                         p.window, max_q_len, p.sinks);
+                                                         p.window, max_q_len, p.sinks,
+                                                         p.cache_fp8);
     if (plan.max_splits > 1) {
       if (!workspace || workspace_bytes < need) return RPK_ERR_WORKSPACE;
       if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return RPK_ERR_WORKSPACE;

@@ -91,6 +91,16 @@ __device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint32_t codes) {
   return r;
 }
 
+// Four e4m3 codes (bytes 0-3) -> four f16 values: bytes 0-1 into lo, 2-3 into hi.
+__device__ __forceinline__ void f16x4_from_e4m3x4(uint32_t codes, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 c0, c1;\n\t"
+      "mov.b32 {c0, c1}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, c0;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, c1;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(codes));
+}
+
 // One e4m3 code -> fp32 (exact).
 __device__ __forceinline__ float f32_from_e4m3(uint8_t code) {
   const uint32_t h2 = f16x2_from_e4m3x2(code);

@@ -111,9 +111,9 @@ struct DecodePlan {
 // The plan with the most splits any launch uses (sizes the workspace).
 DecodePlan decode_plan(int32_t max_kv_len);
 // The plan a launch uses for `units` (sequence, KV head) pairs: never more
-// splits than decode_plan.
+// splits than decode_plan. cache_fp8: the pools hold 1-byte e4m3 codes.
 DecodePlan decode_launch_plan(int32_t max_kv_len, int32_t units, int32_t head_dim, int32_t window,
-                              int32_t max_q_len, int32_t sinks);
+                              int32_t max_q_len, int32_t sinks, bool cache_fp8 = false);
 size_t decode_workspace_bytes(int32_t total_q_tokens, int32_t n_heads, int32_t head_dim,
                               int32_t max_kv_len);
 
