@@ -380,37 +380,63 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
           if (page >= 0 && page < p.num_pages) bytes += seg_bytes;
         }
-        for (int kind = 0; kind < 2; ++kind) {
-          // unified stages: K and V share the stage's barriers (kind 0 waits
-          // and expects both tiles' bytes)
-          const int st = kind == 0 ? ks : vs;
-          const int ring = kind == 0 ? KS : VS;
-          uint64_t* full = (kind == 0 || !C::kSplit) ? &bars.k_full[st] : &bars.v_full[st];
-          uint64_t* empty = kind == 0 ? &bars.k_empty[st] : &bars.v_empty[st];
-          if (kind == 0 || C::kSplit) {
-            if (gi >= ring &&
-                !thread_wait(empty, ((gi / ring) & 1) ^ 1, abort, p.error_word, p.wait_ns))
-              return false;
-            mbar_arrive_expect_tx(full, C::kSplit ? bytes : 2 * bytes);
-          }
-          const CUtensorMap* map = kind == 0 ? &k_map : &v_map;
-          uint8_t* base = smem + (kind == 0 ? C::kKOff + st * C::kKStride
-                                            : C::kVOff + st * C::kVStride);
+        if constexpr (!C::kSplit) {
+          // One stage for the tile's K and V: the copies go out box by box as
+          // K, V pairs (measured 3% faster than all K boxes, then all V).
+          if (gi >= KS &&
+              !thread_wait(&bars.k_empty[ks], ((gi / KS) & 1) ^ 1, abort, p.error_word, p.wait_ns))
+            return false;
+          mbar_arrive_expect_tx(&bars.k_full[ks], 2 * bytes);
+          uint8_t* kb = smem + C::kKOff + ks * C::kKStride;
+          uint8_t* vb = smem + C::kVOff + ks * C::kVStride;
           for (int r = 0; r < kBN; r += box_rows) {
             const int key = key0 + r;
             if (key >= it.k_len) break;
             const int pi = key / p.P;
             const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
             if (page < 0 || page >= p.num_pages) {
-              if (kind == 0) raise_error(p.error_word, RPK_DEVERR_PAGE);
+              raise_error(p.error_word, RPK_DEVERR_PAGE);
               continue;
             }
             const int grow = page * p.P + (key - pi * p.P);
 #pragma unroll
-            for (int bx = 0; bx < C::kBoxes; ++bx)
-              tma_load_3d(base + r * 128 + bx * (kBN * 128), map, bx * 64, it.kvh, grow, full);
+            for (int bx = 0; bx < C::kBoxes; ++bx) {
+              tma_load_3d(kb + r * 128 + bx * (kBN * 128), &k_map, bx * 64, it.kvh, grow,
+                          &bars.k_full[ks]);
+              tma_load_3d(vb + r * 128 + bx * (kBN * 128), &v_map, bx * 64, it.kvh, grow,
+                          &bars.k_full[ks]);
+            }
           }
-          ++(kind == 0 ? k_issued : v_issued);
+          ++k_issued;
+        } else {
+          for (int kind = 0; kind < 2; ++kind) {
+            const int st = kind == 0 ? ks : vs;
+            const int ring = kind == 0 ? KS : VS;
+            uint64_t* full = kind == 0 ? &bars.k_full[st] : &bars.v_full[st];
+            uint64_t* empty = kind == 0 ? &bars.k_empty[st] : &bars.v_empty[st];
+            if (gi >= ring &&
+                !thread_wait(empty, ((gi / ring) & 1) ^ 1, abort, p.error_word, p.wait_ns))
+              return false;
+            mbar_arrive_expect_tx(full, bytes);
+            const CUtensorMap* map = kind == 0 ? &k_map : &v_map;
+            uint8_t* base = smem + (kind == 0 ? C::kKOff + st * C::kKStride
+                                              : C::kVOff + st * C::kVStride);
+            for (int r = 0; r < kBN; r += box_rows) {
+              const int key = key0 + r;
+              if (key >= it.k_len) break;
+              const int pi = key / p.P;
+              const int page = pi < p.max_pages ? __ldg(bt + pi) : -1;
+              if (page < 0 || page >= p.num_pages) {
+                if (kind == 0) raise_error(p.error_word, RPK_DEVERR_PAGE);
+                continue;
+              }
+              const int grow = page * p.P + (key - pi * p.P);
+#pragma unroll
+              for (int bx = 0; bx < C::kBoxes; ++bx)
+                tma_load_3d(base + r * 128 + bx * (kBN * 128), map, bx * 64, it.kvh, grow, full);
+            }
+            ++(kind == 0 ? k_issued : v_issued);
+          }
         }
         ++kv_issued;
         return true;
