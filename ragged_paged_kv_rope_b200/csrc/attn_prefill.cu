@@ -82,9 +82,7 @@ namespace {
 
 constexpr int kBM = 128;              // rows per tile (MMA M)
 constexpr int kBN = kPrefillKeyTile;  // keys per tile (64)
-constexpr int kThreads = 384;
-constexpr int kRegsControl = 56;    // warpgroup 0: producer, MMA issuer, 2 idle warps
-constexpr int kRegsSoftmax = 224;   // warpgroups 1 and 2: softmax
+constexpr int kRegsControl = 56;    // warpgroup 0 (and 3): producer, MMA issuer, helpers
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows > 2^8
 
@@ -96,6 +94,15 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max
 template <int D, int NT, bool F8 = false>
 struct Cfg {
   static constexpr int kBoxes = D / 64;
+  // Warpgroup 0: producer, MMA issuer and two warps that, for an e4m3 cache,
+  // narrow Q; warpgroups 1 and 2: softmax; for an e4m3 cache a fourth
+  // warpgroup widens the key tiles. Registers: 56 per thread in warpgroups 0
+  // and 3, the rest of the launch allocation to the softmax.
+  static constexpr int kThreads = F8 ? 512 : 384;
+  static constexpr int kRegsSoftmax = F8 ? 200 : 224;
+  static_assert(4 * 32 * kRegsControl * (F8 ? 2 : 1) + 8 * 32 * kRegsSoftmax ==
+                    kThreads * ((65536 / kThreads) & ~7),
+                "register split");
   // head_dim 64 / 128: one ring of stages, each the K and V of one key tile,
   // freed when its P V MMAs complete. head_dim 256: a ring of K slots, freed
   // when their S MMAs complete, and a ring of V slots, freed when their P V
@@ -203,7 +210,7 @@ __device__ __forceinline__ bool decode_item(const AttnParams& p, int w, int n_qp
 }
 
 template <int D, int NT, bool F8>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<D, NT, F8>::kThreads, 1)
     attn_prefill_kernel(const AttnParams p, const __grid_constant__ CUtensorMap q_map,
                         const __grid_constant__ CUtensorMap k_map,
                         const __grid_constant__ CUtensorMap v_map, const int tpt,
@@ -212,8 +219,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int KS = C::kKStages, VS = C::kVStages;
   constexpr int RS = C::kRawStages;
   constexpr int kSoftmaxWarps = 4 * NT;
-  // MMA warp, softmax warps and, for an e4m3 cache, the two converter warps
-  constexpr int kItemReaders = 1 + kSoftmaxWarps + (F8 ? 2 : 0);
+  // MMA warp, softmax warps and, for an e4m3 cache, two Q warps and four
+  // converter warps
+  constexpr int kItemReaders = 1 + kSoftmaxWarps + (F8 ? 6 : 0);
   extern __shared__ uint8_t smem_raw[];
   __shared__ Bars bars;
   __shared__ int item_slot[2];
@@ -240,12 +248,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < KS; ++st) {
-      mbar_init(&bars.k_full[st], F8 ? 2 : 1);  // e4m3: one arrival per converter warp
+      mbar_init(&bars.k_full[st], F8 ? 4 : 1);  // e4m3: one arrival per converter warp
       mbar_init(&bars.k_empty[st], 1);
     }
     for (int st = 0; st < RS; ++st) {
       mbar_init(&bars.raw_full[st], 1);
-      mbar_init(&bars.raw_empty[st], 2);
+      mbar_init(&bars.raw_empty[st], 4);
     }
     for (int k = 0; k < 2; ++k) mbar_init(&bars.q_ready[k], 2);
     for (int st = 0; st < VS; ++st) {
@@ -637,26 +645,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Drain: every MMA issued above has completed before TMEM is freed.
     commit_to(&bars.drain);
     if (!warp_wait(&bars.drain, 0, abort, p.error_word, p.wait_ns)) mbar_wait(&bars.drain, 0);
-  } else if (warp < 4) {
+  } else if (warp < 4 || warp >= 12) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
     if constexpr (F8) {
-      // ---------------------------------------------- e4m3 converter warps
-      // Warp 2 widens the K codes, warp 3 the V codes of each key tile from
-      // its raw stage into the f16 stage the MMAs read (every e4m3 value is
-      // exact in f16), in the 128-byte-swizzled layout TMA would have written.
-      // At the start of each item with keys, warp 2 + t first narrows query
-      // tile t to f16 in place: each row is scaled by the power of two 2^k2
-      // that brings its largest magnitude into [2^14, 2^15) (exact for every
-      // element above f16's normal range floor: bf16 has 8 significant bits,
-      // f16 11), and k2 is left for the softmax warps, which fold 2^-k2 and
-      // k_scale into the score scale and v_scale into the output.
-      const int kind = warp - 2;  // 0: K, 1: V
+      // --------------------------------------- e4m3: Q warps and converters
+      // Warps 2 and 3: at the start of each item with keys, warp 2 + t
+      // narrows query tile t to f16 in place. Each row is scaled by the power
+      // of two 2^k2 that brings its largest magnitude into [2^14, 2^15) (exact
+      // for every element above f16's normal range floor: bf16 has 8
+      // significant bits, f16 11), and k2 is left for the softmax warps, which
+      // fold 2^-k2 and k_scale into the score scale and v_scale into the output.
+      // Warps 12-15: warp 12 + 2 kind + h widens rows [32 h, 32 h + 32) of
+      // the K (kind 0) or V (kind 1) codes of each key tile from its raw stage
+      // into the f16 stage the MMAs read (every e4m3 value is exact in f16),
+      // in the 128-byte-swizzled layout TMA would have written.
+      const bool q_warp = warp < 4;
+      const int role = q_warp ? warp - 2 : warp - 12;
       int gi = 0;                 // key tiles converted over all items
       int ql = 0;                 // Q loads narrowed
       bool ok = true;
       auto narrow_q = [&]() {
-        uint8_t* qtile = smem + C::kQOff + kind * C::kQBytes;
-        int8_t* k2s = q_k2_sh + (ql & 1) * (NT * kBM) + kind * kBM;
+        uint8_t* qtile = smem + C::kQOff + role * C::kQBytes;
+        int8_t* k2s = q_k2_sh + (ql & 1) * (NT * kBM) + role * kBM;
         for (int r = lane; r < rows_used; r += 32) {
           float mx = 0.f;
 #pragma unroll
@@ -697,6 +707,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&bars.q_ready[ql & 1]);
         ++ql;
       };
+      // Rows [32 h, 32 h + 32) of the K or V codes of key tile gi.
+      auto widen = [&](int kind, int h) {
+        const int rs = gi % RS, st = gi % KS;
+        const uint8_t* raw = smem + C::kRawOff + rs * 2 * C::kRawBytes + kind * C::kRawBytes;
+        uint8_t* dst = smem + (kind == 0 ? C::kKOff + st * C::kKStride
+                                         : C::kVOff + st * C::kVStride);
+        constexpr int kChunks = (kBN / 2) * (D / 8);  // 8 codes -> 16 bytes of f16
+#pragma unroll 4
+        for (int c = lane; c < kChunks; c += 32) {
+          const int row = 32 * h + c / (D / 8), c8 = c % (D / 8);
+          const uint2 w8 = *reinterpret_cast<const uint2*>(raw + row * D + c8 * 8);
+          uint4 hv;
+          hv.x = f16x2_from_e4m3x2(w8.x & 0xFFFFu);
+          hv.y = f16x2_from_e4m3x2(w8.x >> 16);
+          hv.z = f16x2_from_e4m3x2(w8.y & 0xFFFFu);
+          hv.w = f16x2_from_e4m3x2(w8.y >> 16);
+          *reinterpret_cast<uint4*>(dst + (c8 >> 3) * (kBN * 128) +
+                                    swz128((uint32_t)row, (uint32_t)(c8 & 7))) = hv;
+        }
+        fence_proxy_async_smem();  // generic writes before the MMAs read them
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bars.k_full[st]);
+          mbar_arrive(&bars.raw_empty[rs]);
+        }
+      };
       for (int seq = 0; ok; ++seq) {
         const int slot = seq & 1;
         if (!warp_wait(&bars.item_full[slot], (seq >> 1) & 1, abort, p.error_word, p.wait_ns)) {
@@ -709,12 +745,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (w < 0) break;
         Item it;
         if (!decode_item(p, w, n_qpairs, span, false, it)) continue;
-        if (it.n_tiles > 0) {
-          if (!warp_wait(&bars.q_full, ql & 1, abort, p.error_word, p.wait_ns)) {
-            ok = false;
-            break;
+        if (q_warp) {
+          if (it.n_tiles > 0) {
+            if (!warp_wait(&bars.q_full, ql & 1, abort, p.error_word, p.wait_ns)) {
+              ok = false;
+              break;
+            }
+            narrow_q();
           }
-          narrow_q();
+          continue;
         }
         for (int i = 0; ok && i < it.n_tiles; ++i, ++gi) {
           const int rs = gi % RS, st = gi % KS;
@@ -724,35 +763,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          const uint8_t* raw = smem + C::kRawOff + rs * 2 * C::kRawBytes + kind * C::kRawBytes;
-          uint8_t* dst = smem + (kind == 0 ? C::kKOff + st * C::kKStride
-                                           : C::kVOff + st * C::kVStride);
-          constexpr int kChunks = kBN * (D / 8);  // 8 codes -> 16 bytes of f16
-#pragma unroll 4
-          for (int c = lane; c < kChunks; c += 32) {
-            const int row = c / (D / 8), c8 = c % (D / 8);
-            const uint2 w8 = *reinterpret_cast<const uint2*>(raw + row * D + c8 * 8);
-            uint4 h;
-            h.x = f16x2_from_e4m3x2(w8.x & 0xFFFFu);
-            h.y = f16x2_from_e4m3x2(w8.x >> 16);
-            h.z = f16x2_from_e4m3x2(w8.y & 0xFFFFu);
-            h.w = f16x2_from_e4m3x2(w8.y >> 16);
-            *reinterpret_cast<uint4*>(dst + (c8 >> 3) * (kBN * 128) +
-                                      swz128((uint32_t)row, (uint32_t)(c8 & 7))) = h;
-          }
-          fence_proxy_async_smem();  // generic writes before the MMAs read them
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&bars.k_full[st]);
-            mbar_arrive(&bars.raw_empty[rs]);
-          }
+          widen(role >> 1, role & 1);
         }
       }
       if (!ok) do_abort(abort, p.error_word);
     }
   } else {
     // ------------------------------------------------------------- softmax
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kRegsSoftmax));
     const int t = (warp - 4) >> 2;       // query tile: warps 4-7 -> A, 8-11 -> B (if NT == 2)
     const int qw = warp & 3;             // TMEM lane quarter of this warp
     const int r = qw * 32 + lane;        // row of this thread
@@ -1000,7 +1018,7 @@ cudaError_t launch_d(const AttnParams& p, const CUtensorMap& q_map, const CUtens
   e = cudaMemsetAsync(work_counter, 0, sizeof(int), stream);
   if (e != cudaSuccess) return e;
   const int grid = (int)std::min<long long>(n_items, sm_count());
-  attn_prefill_kernel<D, NT, F8><<<grid, kThreads, C::kSmemBytes, stream>>>(
+  attn_prefill_kernel<D, NT, F8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(
       p, q_map, k_map, v_map, tpt, n_qpairs, work_counter);
   return cudaGetLastError();
 }
