@@ -192,17 +192,17 @@ struct DecodeCfg {
   static_assert(kConsumerWarps * 16 * D * 4 <= kStages * kStageBytes, "merge buffer");
 };
 
-// e4m3 cache: stages of raw codes [64 keys][D bytes] for K then V, and per
-// consumer warp one f16 tile of 16 rows (kBoxes 128-byte swizzled boxes) for V
-// and, for head_dim 64 (whose K is widened too), one for K.
+// e4m3 cache: stages of raw codes [64 keys][D bytes] for K then V. head_dim
+// >= 128 reads both straight from the codes; head_dim 64 widens its 16 rows of
+// K and V into two f16 tiles (kBoxes 128-byte swizzled boxes) per consumer warp.
 template <int D>
 struct DecodeCfg<D, true> {
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = kDecodeTile * D;          // raw codes of K or V
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = D == 256 ? 4 : (D == 128 ? 4 : 8);
+  static constexpr int kStages = D == 256 ? 6 : (D == 128 ? 4 : 8);
   static constexpr int kConvTileBytes = 16 * D * 2;           // 16 rows of f16
-  static constexpr int kConvTiles = D >= 128 ? 1 : 2;         // V, and K for head_dim 64
+  static constexpr int kConvTiles = D >= 128 ? 0 : 2;         // K and V for head_dim 64
   static constexpr int kConvOff = kStages * kStageBytes;
   static constexpr int kSmemBytes =
       kConvOff + kConsumerWarps * kConvTiles * kConvTileBytes + 1024;
@@ -221,6 +221,9 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
   constexpr int S = Cfg::kStages;
   // e4m3 with head_dim >= 128: K fragments straight from the swizzled raw codes
   constexpr bool kKDirect = kFp8 && D >= 128;
+  // ... and V fragments too: each lane widens the codes of its A fragment's
+  // 8x8 blocks in registers and transposes them with movmatrix.
+  constexpr bool kVDirect = kKDirect;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t full_bar[S], empty_bar[S];
   __shared__ float m_part[kConsumerWarps][kDecodeMaxRows];
@@ -436,11 +439,11 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
     const int wrow0 = warp * 16;  // row of this warp's first key inside the tile
     constexpr int kBoxStride = (kFp8 ? 16 : kDecodeTile) * 128;  // bytes between 64-channel boxes
     const bool tail = key0 + 15 >= k_len;
-    if constexpr (kFp8) {
+    if constexpr (kFp8 && !kVDirect) {
       // Widen this warp's 16 rows of K and V from e4m3 codes to f16 in its own
       // tiles (value rows at or past k_len become zeros), then release the stage.
       uint8_t* ck = smem + Cfg::kConvOff + warp * Cfg::kConvTiles * Cfg::kConvTileBytes;
-      uint8_t* cv = ck + (Cfg::kConvTiles - 1) * Cfg::kConvTileBytes;  // == ck when K is read raw
+      uint8_t* cv = ck + Cfg::kConvTileBytes;
       constexpr int kChunks = D / 16;  // 16-code chunks per row
       // K, then V (one tile at a time keeps fewer registers live under the
       // 168-register cap; head_dim 256 runs one CTA per SM and unrolls both)
@@ -484,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
         kbase = smem_u32(ck);
       }
       vbase = smem_u32(cv);
-    } else if (tail) {
+    } else if (!kFp8 && tail) {
       // Zero value rows at or past k_len (stale or never written bytes).
       for (int idx = lane; idx < 16 * (D / 8); idx += 32) {
         const int kr = idx / (D / 8);
@@ -529,10 +532,6 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
       }
     }
 
-    if constexpr (kKDirect) {
-      __syncwarp();  // every lane has read its K codes and V is widened
-      if (lane == 0) mbar_arrive(&empty_bar[s]);
-    }
 
     // Mask, scale to log2 units, online-softmax update of this lane's rows;
     // the 16 keys of a row sit on the 8 lanes that share c.
@@ -595,17 +594,40 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
         o[dc][nt][2] *= alpha[nt][0]; o[dc][nt][3] *= alpha[nt][1];
       }
 
-    // O^T += V^T P^T: A = V^T (16 channels x 16 keys) by a transposing load.
+    // O^T += V^T P^T: A = V^T (16 channels x 16 keys).
 #pragma unroll
     for (int dc = 0; dc < D / 16; ++dc) {
-      // matrices (transposed): (keys 0-7, d lo), (keys 0-7, d hi), (keys 8-15, d lo),
-      // (keys 8-15, d hi)
-      const int mi = lane >> 3;
-      const int vrow = (kFp8 ? 0 : wrow0) + (mi >> 1) * 8 + (lane & 7);
-      const int chunk = dc * 2 + (mi & 1);
-      const uint32_t addr = vbase + (chunk >> 3) * kBoxStride + swz128(vrow, chunk & 7);
       uint32_t a[4];
-      ldsm_x4_t(addr, a[0], a[1], a[2], a[3]);
+      if constexpr (kVDirect) {
+        // Codes of channels 16 dc + 4c .. 4c+3 of keys g and g + 8 (value
+        // rows at or past k_len read as zeros): widened, they are the 8x8
+        // blocks (keys 0-7 | 8-15) x (channel pairs lo | hi) in row layout;
+        // movmatrix turns each into its transpose, a block of the A fragment.
+        // Output row m of the step is channel 4 (m/2) + m%2 (m < 8) or
+        // 4 ((m-8)/2) + 2 + m%2 (m >= 8) of the 16; the merge puts it back.
+        const uint8_t* vb = v_stage(s) + (dc >> 3) * (kDecodeTile * 128) + 4 * c;
+        uint32_t w0 = *reinterpret_cast<const uint32_t*>(vb + swz128(wrow0 + g, dc & 7));
+        uint32_t w1 = *reinterpret_cast<const uint32_t*>(vb + swz128(wrow0 + g + 8, dc & 7));
+        if (tail) {
+          if (key0 + g >= k_len) w0 = 0u;
+          if (key0 + g + 8 >= k_len) w1 = 0u;
+        }
+        uint32_t x0, x1, y0, y1;
+        f16x4_from_e4m3x4(w0, x0, x1);
+        f16x4_from_e4m3x4(w1, y0, y1);
+        a[0] = movmatrix_trans(x0);  // channels lo, keys 0-7
+        a[1] = movmatrix_trans(x1);  // channels hi, keys 0-7
+        a[2] = movmatrix_trans(y0);  // channels lo, keys 8-15
+        a[3] = movmatrix_trans(y1);  // channels hi, keys 8-15
+      } else {
+        // by a transposing load; matrices (transposed): (keys 0-7, d lo),
+        // (keys 0-7, d hi), (keys 8-15, d lo), (keys 8-15, d hi)
+        const int mi = lane >> 3;
+        const int vrow = (kFp8 ? 0 : wrow0) + (mi >> 1) * 8 + (lane & 7);
+        const int chunk = dc * 2 + (mi & 1);
+        const uint32_t addr = vbase + (chunk >> 3) * kBoxStride + swz128(vrow, chunk & 7);
+        ldsm_x4_t(addr, a[0], a[1], a[2], a[3]);
+      }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         if constexpr (kFp8) mma_f16(o[dc][nt], a, pb[nt][0], pb[nt][1]);
@@ -614,8 +636,10 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
     }
 
     __syncwarp();
-    if constexpr (!kFp8) {
-      if (tail) fence_proxy_async_smem();  // generic zero-writes before the next TMA into s
+    if constexpr (!kFp8 || kVDirect) {
+      if constexpr (!kFp8) {
+        if (tail) fence_proxy_async_smem();  // generic zero-writes before the next TMA into s
+      }
       if (lane == 0) mbar_arrive(&empty_bar[s]);
     }
   }
@@ -657,11 +681,15 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__(D <= 128 ? 168 : 255)
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) mx = fmaxf(mx, m_part[w][rr]);
       const float f = m_run[nt][j] == -INFINITY ? 0.f : fast_exp2(m_run[nt][j] - mx);
-      float* orow = obuf + ((size_t)warp * 16 + rr) * D + g;
+      // output rows g and g + 8 of each 16-channel step: channels g and g + 8,
+      // or, with V read from the codes, 4 (g/2) + g%2 and that + 2
+      const int ch_lo = kVDirect ? 4 * (g >> 1) + (g & 1) : g;
+      const int ch_hi = kVDirect ? ch_lo + 2 : g + 8;
+      float* orow = obuf + ((size_t)warp * 16 + rr) * D;
 #pragma unroll
       for (int dc = 0; dc < D / 16; ++dc) {
-        orow[dc * 16] = o[dc][nt][j] * f;
-        orow[dc * 16 + 8] = o[dc][nt][2 + j] * f;
+        orow[dc * 16 + ch_lo] = o[dc][nt][j] * f;
+        orow[dc * 16 + ch_hi] = o[dc][nt][2 + j] * f;
       }
     }
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
