@@ -569,9 +569,20 @@ def backward_measure(device, world, warmup=3, batch=None):
         kernel = "warp-level tensor-core (mma.sync) dQ and dK/dV kernels"
     else:
         kernel = "CUDA-core dQ and dK/dV kernels"
+    # DRAM bytes per launch of the two tcgen05 kernels (committed small-case
+    # captures scaled to this workload) beside the bytes of their inputs.
+    kv_tokens = int(np.sum(wl.kv_lens))
+    inputs = {"q_and_d_out": 2 * T * H * d * 2,
+              "k_and_v": 2 * kv_tokens * sp.n_kv_heads * d * 2,
+              "lse_and_delta": 2 * T * H * 4}
+    traffic = {}
+    for key in ("attn_bwd_dkv", "attn_bwd_dq"):
+        ent = load_traffic(f"{key}@ragged_prefill") if batch is None else None
+        traffic[key] = None if ent is None else ent["bytes_per_launch"]
     return {"workload": "ragged_prefill", "kernel": kernel, "backward_ms": ms, "steps": steps,
             "algorithmic_flops": flops, "tflops": tflops,
             "tensor_peak_tflops": peaks["bf16_tflops"], "frac": tflops / peaks["bf16_tflops"],
+            "traffic": traffic, "input_bytes": inputs,
             "error_word": int(step.error_word.item())}
 
 
