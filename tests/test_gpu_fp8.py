@@ -198,7 +198,7 @@ def test_end_to_end_decode_step_e4m3():
 # and narrows each Q row to f16 under a power-of-two scale, so the products are
 # those of the bf16 path up to f16's extra mantissa bits.
 
-def _e4m3_prefill_case(sp, q_lens, kv_lens, seed, window=0, sinks=0, q_mul=None):
+def _e4m3_case(sp, q_lens, kv_lens, seed, window=0, sinks=0, q_mul=None):
     wl = W.attention_only(sp, seed, q_lens, kv_lens)
     if q_mul is not None:
         wl.q = (wl.q.float() * q_mul).to(torch.bfloat16)
@@ -211,7 +211,7 @@ def _e4m3_prefill_case(sp, q_lens, kv_lens, seed, window=0, sinks=0, q_mul=None)
                                wl.block_table, sp.n_kv_heads, sp.softmax_scale, window,
                                with_lse=True, sinks=sinks, k_scale=wl.k_scale,
                                v_scale=wl.v_scale)
-    what = f"e4m3 prefill d={sp.head_dim} q={list(q_lens)} window={window} sinks={sinks}"
+    what = f"e4m3 d={sp.head_dim} q={list(q_lens)} window={window} sinks={sinks}"
     check_lse(lse.cpu(), ref_lse, what)
     check_attention(out.cpu(), ref, "bf16", what)
 
@@ -223,7 +223,7 @@ def test_prefill_over_e4m3_cache(d, window, sinks):
     # first token sits deep in its sequence and a one-token sequence
     sp = W.spec("ragged_prefill", cache_dtype="e4m3", head_dim=d, rotary_dim=d, batch=4,
                 n_heads=8, n_kv_heads=2)
-    _e4m3_prefill_case(sp, [300, 129, 1, 77], [300, 700, 64, 77], seed=21, window=window,
+    _e4m3_case(sp, [300, 129, 1, 77], [300, 700, 64, 77], seed=21, window=window,
                        sinks=sinks)
 
 
@@ -232,7 +232,7 @@ def test_prefill_over_e4m3_cache_page_16_group_8():
     # KV head (16 tokens per query tile)
     sp = W.spec("llama3_8b_decode", cache_dtype="e4m3", batch=3, n_heads=16, n_kv_heads=2,
                 page_size=16)
-    _e4m3_prefill_case(sp, [100, 33, 250], [400, 33, 250], seed=22)
+    _e4m3_case(sp, [100, 33, 250], [400, 33, 250], seed=22)
 
 
 def test_prefill_e4m3_large_and_small_queries():
@@ -243,4 +243,13 @@ def test_prefill_e4m3_large_and_small_queries():
     mul = torch.ones(wl.total_tokens, 1, 1)
     mul[:200] = 1e6
     mul[200:270] = 1e-7
-    _e4m3_prefill_case(sp, [200, 70, 130], [200, 300, 130], seed=23, q_mul=mul)
+    _e4m3_case(sp, [200, 70, 130], [200, 300, 130], seed=23, q_mul=mul)
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_decode_over_e4m3_cache_window_and_sinks(d):
+    # decode rows (one and two tokens) under a window with attention sinks: the
+    # sink tile and the band's tiles, a band whose first tile is partial and a
+    # sequence shorter than the window
+    sp = W.spec("llama3_8b_decode", cache_dtype="e4m3", head_dim=d, rotary_dim=d, batch=4)
+    _e4m3_case(sp, [1, 1, 1, 2], [5000, 300, 70, 2000], seed=24, window=1000, sinks=4)
