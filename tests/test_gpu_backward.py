@@ -11,11 +11,12 @@ D_i and so every dS_ij; the tensor-core kernels also round P_ij and dS_ij to
 bf16, relative 2^-9, as operands of their second products); for fp32,
 1e-4 max|ref|.
 
-bf16 shapes with groups of up to 16 query heads run on the tensor-core
-kernels, the others (fp32, an e4m3 cache, larger groups) on the CUDA-core
-ones; the cases cover both, several 64-key tiles and 64-row blocks with
-ragged tails, windows with sinks across tiles, groups that do not divide 64,
-and rows that see no key.
+bf16 shapes run on the tensor-core kernels: tcgen05 for head_dim 64 / 128
+with groups of up to 64 query heads, warp-level mma.sync for head_dim 256
+with groups of up to 16. The others (fp32, an e4m3 cache, larger groups)
+run on the CUDA-core ones. The cases cover all three, several key tiles and
+row blocks with ragged tails, windows with sinks across tiles, groups that
+do not divide 64, and rows that see no key.
 """
 
 import numpy as np
@@ -65,7 +66,7 @@ CASES = [
     ("group of 3", "ragged_prefill", dict(n_heads=6, n_kv_heads=2), [50, 7], [120, 7], 0, 0),
     ("group of 16", "ragged_prefill",
      dict(n_heads=16, n_kv_heads=1, head_dim=64, rotary_dim=64), [9, 20], [70, 20], 0, 0),
-    ("group of 32 (CUDA cores)", "ragged_prefill",
+    ("group of 32", "ragged_prefill",
      dict(n_heads=32, n_kv_heads=1, head_dim=64, rotary_dim=64), [3, 5], [50, 5], 0, 0),
     ("rows without keys", "ragged_prefill", dict(n_heads=4, n_kv_heads=2), [12, 3], [5, 40],
      0, 0),
@@ -75,7 +76,7 @@ CASES = [
      dict(n_heads=8, n_kv_heads=2, page_size=64), [700, 129, 3], [900, 129, 260], 0, 0),
     ("group of 8, chunked rows, window", "mixed_chunked_mrope",
      dict(n_heads=16, n_kv_heads=2, mrope_section=None), [150, 1, 40], [1000, 300, 41], 300, 0),
-    ("group of 128, one token per row block", "ragged_prefill",
+    ("group of 128 (CUDA cores), one token per row block", "ragged_prefill",
      dict(n_heads=128, n_kv_heads=1, head_dim=64, rotary_dim=64, page_size=128), [5, 2],
      [300, 2], 0, 0),
 ]
