@@ -144,13 +144,39 @@ def load_peaks():
                 "source": "fallback"}
 
 
+def strip_comments(src: str) -> str:
+    """C/C++ source without its comments and blank lines (string and character
+    literals kept), so that an edit to comments alone leaves the digest as is."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (line.rstrip() for line in "".join(out).split("\n"))
+    return "\n".join(line for line in lines if line)
+
+
 def sources_digest(names) -> str:
-    """SHA-256 over the given csrc files (a kernel's .cu and the headers it includes)."""
+    """SHA-256 over the given csrc files (a kernel's .cu and the headers it
+    includes), comments and blank lines left out."""
     import hashlib
     h = hashlib.sha256()
     for n in names:
-        with open(os.path.join(ROOT, "ragged_paged_kv_rope_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "ragged_paged_kv_rope_b200", "csrc", n)) as f:
+            h.update(strip_comments(f.read()).encode())
     return h.hexdigest()
 
 

@@ -47,7 +47,9 @@
 //              S_t(i+2) (Q_t K^T, both operands in shared memory) for every
 //              tile t; the next item's first S MMAs follow the last P V of the
 //              current one
-//   warps 2-3  idle (they complete the first warpgroup)
+//   warps 2-3  idle (they complete the first warpgroup); over an e4m3 cache
+//              they narrow the query tiles to f16, and a fourth warpgroup
+//              (warps 12-15) widens the key tiles' codes to f16
 //   warps 4-7  softmax of tile A, warps 8-11 softmax of tile B (idle when
 //              NT = 1): thread r owns row r (TMEM lane r); loads S_t(i), masks
 //              the band, keeps (m, l) in log2 units, writes P_t(i), and
@@ -62,7 +64,8 @@
 // needs this warp's own P(i)), so the phase parity is unambiguous.
 // Registers: the first warpgroup gives registers back (setmaxnreg 56) and the
 // two softmax warpgroups take them (setmaxnreg 224);
-// 4*32*56 + 8*32*224 = 64512 registers, the 384 * 168 the CTA is launched with.
+// 4*32*56 + 8*32*224 = 64512 registers, the 384 * 168 the CTA is launched with
+// (e4m3: 512 threads, warpgroups 0 and 3 at 56, the softmax at 200, 512 * 128).
 // Value rows at or past k_len are zeroed in shared memory before P V, so the
 // NaN sentinels of unused slots never meet a zero weight. Every mbarrier wait
 // is bounded; on a timeout the CTA raises RPK_DEVERR_TIMEOUT, drains its copies
@@ -89,7 +92,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max
 // NT query tiles of 128 rows per work item: two for head_dim 64 and 128, one
 // for head_dim 256 (whose 256-column output accumulator leaves tensor memory
 // for one tile's double-buffered scores only). F8: the pools hold e4m3 codes;
-// TMA brings each key tile's codes into a small raw ring and two converter
+// TMA brings each key tile's codes into a small raw ring and four converter
 // warps widen them to f16 in the stages the MMAs read.
 template <int D, int NT, bool F8 = false>
 struct Cfg {
@@ -149,9 +152,9 @@ struct Bars {
   uint64_t p_full[2];    // per score buffer: P of every tile written (per softmax warp)
   uint64_t pv_item[1];   // one phase per item with two or more key tiles: P(n-2) V done
   uint64_t raw_full[2];  // e4m3: per raw stage, the codes of one key tile loaded
-  uint64_t raw_empty[2]; // e4m3: per raw stage, both converter warps done with it
+  uint64_t raw_empty[2]; // e4m3: per raw stage, the four converter warps done with it
   uint64_t q_ready[2];   // e4m3, per Q load parity: the Q tiles narrowed to f16 and their
-                         // row scales written (one arrival per converter warp)
+                         // row scales written (one arrival per Q warp)
   uint64_t o_final;      // the item's last P V has completed
   uint64_t o_empty;      // the epilogue has read O (one arrival per softmax warp)
   uint64_t item_full[2];   // work-item ring: index written by the producer
@@ -806,7 +809,7 @@ __global__ void __launch_bounds__(Cfg<D, NT, F8>::kThreads, 1)
       float v_mul = 1.f;                 // e4m3: v_scale of the item's KV head
       if constexpr (F8) {
         if (n > 0) {
-          // The converter warps narrowed this row's query to f16 under 2^k2.
+          // A Q warp narrowed this row's query to f16 under 2^k2.
           const int qs = q_seen_sm++;
           if (!warp_wait(&bars.q_ready[qs & 1], (qs >> 1) & 1, abort, p.error_word, p.wait_ns)) {
             ok = false;

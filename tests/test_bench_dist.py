@@ -63,3 +63,15 @@ def test_single_rank_needs_no_group():
     assert bench.dist_setup() == (1, 0, 0)
     assert bench.max_over_ranks(3.0, 1) == 3.0
     assert bench.whole_job_throughput(50.0, 2.0, 1) == 25.0
+
+
+def test_traffic_digest_ignores_comments_only():
+    # The DRAM capture of a kernel stays valid through edits to its comments
+    # and blank lines, and not through any edit to its code.
+    sys.path.insert(0, ROOT)
+    import bench
+    src = 'int a = 1; // count\n/* block\n comment */ const char* s = "x//y\\"z";\n\n  a++;\n'
+    assert bench.strip_comments(src) == 'int a = 1;\n const char* s = "x//y\\"z";\n  a++;'
+    assert bench.strip_comments(src.replace("count", "number")) == bench.strip_comments(src)
+    assert bench.strip_comments(src.replace("a++", "a--")) != bench.strip_comments(src)
+
