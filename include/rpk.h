@@ -254,13 +254,14 @@ size_t ragged_paged_attention_workspace_size(int32_t total_q_tokens, int32_t n_h
  *   bf16, otherwise                -> tcgen05 prefill kernel (head_dim 64, 128
  *                                     and 256, group <= 128; larger groups run
  *                                     on the CUDA-core kernel)
- * An RPK_E4M3 cache takes the same decode path (the kernel widens each tile
- * to f16 in shared memory, exactly, and folds k_scale into the score scale and
- * v_scale into the output) and, for head_dim 64 and 128, the same tcgen05
- * prefill path (two warps widen each key tile's codes to f16 in shared memory;
- * each query row is narrowed to f16 under a power-of-two scale that is folded
- * back into its scores); e4m3 prefill shapes of head_dim 256 run on the
- * CUDA-core kernel.
+ * An RPK_E4M3 cache takes the same decode path and, for head_dim 64 and 128,
+ * the same tcgen05 prefill path. Codes are widened to f16, which is exact
+ * (decode: in registers for head_dim >= 128, in shared memory for 64;
+ * prefill: by a warpgroup of its own into shared memory). The query is
+ * narrowed to f16 under a power-of-two scale, per row in the prefill and per
+ * group in the decode, and that scale and k_scale are folded into the score
+ * scale, v_scale into the output. e4m3 prefill shapes of head_dim 256 run on
+ * the CUDA-core kernel.
  */
 rpk_status ragged_paged_attention(const void* q, const int32_t* q_row_offsets,
                                   const int32_t* kv_lens, const rpk_paged_kv* page_table,
