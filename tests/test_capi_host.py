@@ -138,6 +138,22 @@ def test_e4m3_cache_needs_both_scales(L):
 
 
 @host_only
+def test_e4m3_prefill_routes(L):
+    # Prefill shapes over an e4m3 cache take the tcgen05 kernel for head_dim 64
+    # and 128, which keeps its work counter in the workspace; head_dim 256 runs
+    # the CUDA-core kernel, which needs none (on a host without a GPU its launch
+    # then fails with a CUDA error, never a workspace error).
+    for d in (64, 128):
+        c = cache(cache_dtype=B.RPK_E4M3, k_scale=FAKE, v_scale=FAKE, head_dim=d,
+                  max_pages_per_seq=16)
+        assert attn(L, c, d=d, mq=5, ws=None, wsb=0) == 6
+        assert attn(L, c, d=d, mq=5, ws=FAKE, wsb=128) == 6
+    c = cache(cache_dtype=B.RPK_E4M3, k_scale=FAKE, v_scale=FAKE, head_dim=256,
+              max_pages_per_seq=16)
+    assert attn(L, c, d=256, mq=5, ws=None, wsb=0) == 5
+
+
+@host_only
 def test_e4m3_cache_takes_bf16_and_f32_tensors_only(L):
     c = cache(cache_dtype=B.RPK_E4M3, k_scale=FAKE, v_scale=FAKE, max_pages_per_seq=16)
     assert rope(L, c, dtype=B.RPK_E4M3) == 3       # e4m3 is a cache dtype only
